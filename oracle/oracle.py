@@ -1,0 +1,334 @@
+"""CPU oracle for the SpinQuant W4A4 + online-Hadamard inference path.
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, obviously correct
+statement of what the CUDA library computes.  Only ``tests/``, the smoke check
+in ``__graft_entry__.py`` and the ``cpu_baseline`` / reference arm of
+``bench.py`` may import it.  The product (``rotation_ptq_b200``) never imports
+it, and it never imports the product: the two share no code, tables or
+constants.  Inputs for both sides come from ``workloads.synthetic``.
+
+Arithmetic: float64 for every linear step (numpy matmul is the one library
+primitive used), with a cast to float32 where a quantizer decision is taken,
+because the CUDA path takes those decisions in float32 ("where floating point
+decides an integer, both sides decide in the same precision").
+
+Citations name the page and section they restate:
+  * "SpinQuant, Reproduced", Q1-Q13: the third-party reproduction page.
+  * "SpinQuant abstract": the arXiv abstract reproduced on several pages.
+
+Readings of points the pages leave open (each listed in the design doc):
+  * Hadamard matrices: Sylvester H_{2^k}[a][b] = (-1)^popcount(a&b) in natural
+    order; Paley-I H12 from the quadratic residues mod 11; H12 (x) H_{2^k} with
+    H12 on the outer channel index; row-vector convention y = x H.
+  * Activation / weight quantizer: symmetric INT4, scale = clip*absmax/7,
+    codes clamp(round_half_even(y/scale), -8, 7); an all-zero row gets scale 1.
+  * INT4 packing: two codes per byte, even element in the low nibble,
+    two's complement for signed codes.
+  * KV quantizer: asymmetric 4-bit per (token, head) group of 128 with an
+    integer zero point; the range is widened to include 0.
+  * RoPE: half-split ("rotate_half") convention, host tables in float64 rounded
+    to float32, theta 1e6.
+
+Parity pins: every function below is checked in tests/test_oracle_pins.py
+against closed forms, brute force or invariants that do not reuse it.
+"""
+from __future__ import annotations
+
+import functools
+import math
+
+import numpy as np
+
+F32 = np.float32
+
+# ---------------------------------------------------------------------------
+# Hadamard matrices ("SpinQuant, Reproduced", Q5: R3 and R4 "stay Hadamard"
+# because they must be applied quickly online; the orders come from the
+# Qwen3-8B widths in the same section: head dim 128, MLP width 12,288).
+# ---------------------------------------------------------------------------
+
+
+def sylvester(n: int) -> np.ndarray:
+    """Sylvester Hadamard of order n = 2^k, natural order: H[a][b] = (-1)^popcount(a & b)."""
+    assert n >= 1 and n & (n - 1) == 0, n
+    a = np.arange(n, dtype=np.int64)
+    parity = (np.bitwise_count(a[:, None] & a[None, :]) & 1).astype(np.int64)
+    return 1 - 2 * parity
+
+
+def quadratic_character(r: int, q: int) -> int:
+    """Legendre symbol chi(r) mod prime q: 0 at 0, +1 on nonzero squares, -1 otherwise."""
+    r %= q
+    if r == 0:
+        return 0
+    squares = {(t * t) % q for t in range(1, q)}
+    return 1 if r in squares else -1
+
+
+def paley1(q: int = 11) -> np.ndarray:
+    """Paley construction I for a prime q = 3 (mod 4): order q + 1.
+
+    Q[i][j] = chi(j - i); S = [[0, 1^T], [-1, Q]]; H = I + S.
+    For q = 11 this is the order-12 Hadamard used for the non-power-of-two
+    factor of the 12,288-wide R4 rotation.
+    """
+    assert q % 4 == 3
+    n = q + 1
+    Q = np.array([[quadratic_character(j - i, q) for j in range(q)] for i in range(q)],
+                 dtype=np.int64)
+    S = np.zeros((n, n), dtype=np.int64)
+    S[0, 1:] = 1
+    S[1:, 0] = -1
+    S[1:, 1:] = Q
+    return np.eye(n, dtype=np.int64) + S
+
+
+def kron(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """Kronecker product (A (x) B)[i*nB + j][k*nB + l] = A[i][k] * B[j][l] (library primitive)."""
+    return np.kron(A, B)
+
+
+def small_hadamard(n_small: int) -> np.ndarray:
+    if n_small == 1:
+        return np.ones((1, 1), dtype=np.int64)
+    if n_small == 12:
+        return paley1(11)
+    if n_small & (n_small - 1) == 0:
+        return sylvester(n_small)
+    raise ValueError("no Hadamard construction pinned for order %d" % n_small)
+
+
+@functools.lru_cache(maxsize=4)
+def hadamard(n_small: int, n_pow2: int) -> np.ndarray:
+    """Dense float64 H = H_small (x) H_pow2 (entries +-1, unnormalised)."""
+    return kron(small_hadamard(n_small), sylvester(n_pow2)).astype(np.float64)
+
+
+def rotate(x: np.ndarray, n_small: int, n_pow2: int) -> np.ndarray:
+    """Online rotation y = x H / sqrt(g), block-diagonal on each group of g channels.
+
+    g = n_small * n_pow2; the row-vector convention y_c = sum_k x_k H[k][c] is
+    used.  Computed in float64 by one dense matmul, returned in float32 (the
+    precision in which the quantizer then decides).  With g = 1 this is the
+    identity (the R1-folded projections have no online rotation).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    M, K = x.shape
+    g = n_small * n_pow2
+    assert K % g == 0
+    if g == 1:
+        return x.astype(F32)
+    H = hadamard(n_small, n_pow2)
+    y = (x.reshape(M * (K // g), g) @ H) / math.sqrt(g)
+    return y.reshape(M, K).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Symmetric INT4 quantizer (SpinQuant abstract: 4-bit weights and
+# activations; "SpinQuant, Reproduced", Q2: W4A4).  Per token for
+# activations, per output channel for weights.
+# ---------------------------------------------------------------------------
+
+
+def quant_sym_int4(y: np.ndarray, clip: float = 1.0):
+    """Per-row symmetric INT4 round-to-nearest.
+
+    scale = clip * max_k |y_k| / 7 (float32), scale := 1 for an all-zero row;
+    v = y / scale (float32 IEEE division); code = clamp(rint(v), -8, 7) with
+    round-half-to-even.  Returns (codes int8 [M,K], scale f32 [M], v f32 [M,K]).
+    """
+    y = np.asarray(y, dtype=F32)
+    assert np.all(np.isfinite(y))
+    absmax = np.max(np.abs(y), axis=1)
+    scale = (F32(clip) * absmax) / F32(7.0)
+    scale = np.where(scale == 0, F32(1.0), scale).astype(F32)
+    v = (y / scale[:, None]).astype(F32)
+    codes = np.clip(np.rint(v), -8, 7).astype(np.int8)
+    return codes, scale, v
+
+
+def pack_int4(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte: element 2j in bits 0-3, element 2j+1 in bits 4-7."""
+    c = np.asarray(codes).astype(np.int64)
+    assert c.shape[-1] % 2 == 0
+    lo = c[..., 0::2] & 0xF
+    hi = c[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed: np.ndarray, signed: bool = True) -> np.ndarray:
+    """Inverse of pack_int4 (two's complement nibbles when signed)."""
+    p = np.asarray(packed).astype(np.int64)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    if signed:
+        out = np.where(out >= 8, out - 16, out)
+    return out.astype(np.int8 if signed else np.uint8)
+
+
+def rotate_quant(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
+    """Online rotation followed by per-token INT4 quantization and packing.
+
+    "SpinQuant, Reproduced", Q5: R4 sits before down_proj and cannot be merged,
+    so it runs online as a Hadamard; the rotated activations are then
+    quantized to 4 bits (SpinQuant abstract).
+    Returns (packed uint8 [M, K/2], scale f32 [M], codes int8, v f32).
+    """
+    y = rotate(x, n_small, n_pow2)
+    codes, scale, v = quant_sym_int4(y, clip)
+    return pack_int4(codes), scale, codes, v
+
+
+def quantize_weights(w: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
+    """Offline fold of the rotation into the weights, then per-channel RTN INT4.
+
+    W' = W H / sqrt(g) in float64, cast to float32, quantized per output row.
+    With y = x H / sqrt(g) this keeps y W'^T = x W^T in full precision
+    ("SpinQuant, Reproduced", Q1: the rotation is free at full precision).
+    Returns (packed uint8 [N, K/2], scale f32 [N], codes int8 [N, K]).
+    """
+    wr = rotate(w, n_small, n_pow2)
+    codes, scale, _ = quant_sym_int4(wr, clip)
+    return pack_int4(codes), scale, codes
+
+
+# ---------------------------------------------------------------------------
+# W4A4 GEMM with per-token x per-channel dequantization.
+# ---------------------------------------------------------------------------
+
+
+def gemm_int(a_codes: np.ndarray, w_codes: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k a[m, k] * w[n, k], exact, returned as int64.
+
+    Uses a float64 BLAS matmul on integer-valued matrices: every partial sum is
+    an integer below 2^53 in magnitude (|a|,|w| <= 8, K < 2^40), so the result
+    is exact whatever order the library sums in.
+    """
+    a = np.asarray(a_codes, dtype=np.float64)
+    w = np.asarray(w_codes, dtype=np.float64)
+    assert a.shape[1] == w.shape[1] and a.shape[1] * 64 < 2 ** 53
+    return (a @ w.T).astype(np.int64)
+
+
+def dequant(acc: np.ndarray, a_scale: np.ndarray, w_scale: np.ndarray) -> np.ndarray:
+    """out[m, n] = acc[m, n] * a_scale[m] * w_scale[n] in float64."""
+    return acc.astype(np.float64) * np.asarray(a_scale, np.float64)[:, None] \
+        * np.asarray(w_scale, np.float64)[None, :]
+
+
+def w4a4_linear(a_packed, a_scale, w_packed, w_scale):
+    """Packed-code W4A4 linear: returns (int64 acc, float64 dequantized output)."""
+    acc = gemm_int(unpack_int4(a_packed), unpack_int4(w_packed))
+    return acc, dequant(acc, a_scale, w_scale)
+
+
+# ---------------------------------------------------------------------------
+# R3 KV path ("SpinQuant, Reproduced", Q5: R3 in the KV path stays an online
+# Hadamard; SpinQuant abstract: 4-bit KV cache).
+# ---------------------------------------------------------------------------
+
+
+def rope_tables(theta: float, max_pos: int, d: int):
+    """cos/sin tables [max_pos, d/2]: angle(p, i) = p * theta^(-2i/d), float64 rounded to f32."""
+    i = np.arange(d // 2, dtype=np.float64)
+    inv_freq = theta ** (-2.0 * i / d)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+    return np.cos(ang).astype(F32), np.sin(ang).astype(F32)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Half-split rotary embedding, float64.
+
+    For i < d/2: out_i = x_i c - x_{i+d/2} s and out_{i+d/2} = x_{i+d/2} c + x_i s,
+    with c, s the table entries at (pos, i).  x: [T, h, d], pos: [T].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    h = x.shape[-1] // 2
+    c = np.asarray(cos, np.float64)[pos][:, None, :]
+    s = np.asarray(sin, np.float64)[pos][:, None, :]
+    x1, x2 = x[..., :h], x[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def headwise_hadamard(x: np.ndarray) -> np.ndarray:
+    """y = x H_d / sqrt(d) on the last axis (head vectors), float64."""
+    d = x.shape[-1]
+    H = sylvester(d).astype(np.float64)
+    return (np.asarray(x, np.float64) @ H) / math.sqrt(d)
+
+
+def quant_asym_uint4(x: np.ndarray):
+    """Asymmetric 4-bit quantizer over the last axis, decisions in float32.
+
+    lo = min(min x, 0), hi = max(max x, 0); scale = (hi - lo) / 15 (1 if 0);
+    zero = clamp(rint(-lo / scale), 0, 15);
+    code = clamp(rint(x / scale) + zero, 0, 15).
+    Returns (codes uint8 [..., d], scale f32 [...], zero uint8 [...], v f32 = x/scale).
+    """
+    x = np.asarray(x, dtype=F32)
+    lo = np.minimum(np.min(x, axis=-1), F32(0))
+    hi = np.maximum(np.max(x, axis=-1), F32(0))
+    scale = ((hi - lo) / F32(15.0)).astype(F32)
+    scale = np.where(scale == 0, F32(1.0), scale).astype(F32)
+    zero = np.clip(np.rint((-lo) / scale), 0, 15).astype(F32)
+    v = (x / scale[..., None]).astype(F32)
+    codes = np.clip(np.rint(v) + zero[..., None], 0, 15).astype(np.uint8)
+    return codes, scale, zero.astype(np.uint8), v
+
+
+def dequant_asym(codes: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
+    """x_hat = (code - zero) * scale, float64."""
+    return (np.asarray(codes, np.float64) - np.asarray(zero, np.float64)[..., None]) \
+        * np.asarray(scale, np.float64)[..., None]
+
+
+def kv_rotate_quant(q, k, v, pos, cos, sin):
+    """RoPE on Q and K, head-wise H_d on Q and K, asymmetric 4-bit K/V caches.
+
+    q: [T, hq, d], k, v: [T, hkv, d] (any float dtype), pos: [T].  cos/sin may be
+    None, meaning the inputs already carry their rotary embedding.
+    Returns a dict with q_rot (f32, the value the bf16 output rounds), the
+    packed caches, scales, zeros, and the pre-round values v_k / v_v.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    if cos is not None:
+        q = rope(q, pos, cos, sin)
+        k = rope(k, pos, cos, sin)
+    q_rot = headwise_hadamard(q).astype(F32)
+    k_rot = headwise_hadamard(k).astype(F32)
+    kc, ks, kz, kv_ = quant_asym_uint4(k_rot)
+    vc, vs, vz, vv_ = quant_asym_uint4(np.asarray(v, F32))
+    return dict(q_rot=q_rot, k_rot=k_rot,
+                k_cache=pack_int4(kc), k_codes=kc, k_scale=ks, k_zero=kz, k_v=kv_,
+                v_cache=pack_int4(vc), v_codes=vc, v_scale=vs, v_zero=vz, v_v=vv_)
+
+
+def kv_dequant(cache: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
+    """Read-back of a packed asymmetric cache to float64 values."""
+    return dequant_asym(unpack_int4(cache, signed=False), scale, zero)
+
+
+# ---------------------------------------------------------------------------
+# Statistics ("SpinQuant, Reproduced", Q3: kurtosis across channels within a
+# token, averaged over tokens; 3 is a Gaussian).
+# ---------------------------------------------------------------------------
+
+
+def kurtosis(x: np.ndarray) -> float:
+    """Mean over rows of the Pearson (non-excess) kurtosis m4 / m2^2 across columns."""
+    x = np.asarray(x, np.float64)
+    c = x - x.mean(axis=1, keepdims=True)
+    m2 = np.mean(c * c, axis=1)
+    m4 = np.mean(c ** 4, axis=1)
+    return float(np.mean(m4 / (m2 * m2)))
+
+
+def rel_fro(a: np.ndarray, ref: np.ndarray) -> float:
+    """||a - ref||_F / ||ref||_F in float64."""
+    a = np.asarray(a, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), 1e-300))

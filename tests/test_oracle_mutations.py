@@ -1,0 +1,164 @@
+"""Plant plausible mistakes in the CPU oracle and check that the pins catch them.
+
+Each mutation replaces one oracle function (on the CPU, inside this process
+only) with a subtly wrong variant; at least one pin of tests/test_oracle_pins.py
+must then fail.  This is evidence that the pins constrain the oracle rather
+than restate it.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from tests import test_oracle_pins as P
+
+F32 = np.float32
+
+
+def _transposed_paley(q=11):
+    return _orig["paley1"](q).T.copy()
+
+
+def _kron_swapped(A, B):
+    return np.kron(B, A)
+
+
+def _rotate_unnormalised(x, n_small, n_pow2):
+    x = np.asarray(x, np.float64)
+    M, K = x.shape
+    g = n_small * n_pow2
+    if g == 1:
+        return x.astype(F32)
+    H = O.hadamard(n_small, n_pow2)
+    return (x.reshape(-1, g) @ H).reshape(M, K).astype(F32)
+
+
+def _quant_div8(y, clip=1.0):
+    y = np.asarray(y, F32)
+    s = (F32(clip) * np.max(np.abs(y), axis=1)) / F32(8.0)
+    s = np.where(s == 0, F32(1), s).astype(F32)
+    v = (y / s[:, None]).astype(F32)
+    return np.clip(np.rint(v), -8, 7).astype(np.int8), s, v
+
+
+def _quant_floor(y, clip=1.0):
+    y = np.asarray(y, F32)
+    s = (F32(clip) * np.max(np.abs(y), axis=1)) / F32(7.0)
+    s = np.where(s == 0, F32(1), s).astype(F32)
+    v = (y / s[:, None]).astype(F32)
+    return np.clip(np.floor(v + F32(0.5)), -8, 7).astype(np.int8), s, v
+
+
+def _pack_swapped(codes):
+    c = np.asarray(codes).astype(np.int64)
+    return ((c[..., 1::2] & 0xF) | ((c[..., 0::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def _rope_sign(x, pos, cos, sin):
+    x = np.asarray(x, np.float64)
+    h = x.shape[-1] // 2
+    c = np.asarray(cos, np.float64)[pos][:, None, :]
+    s = np.asarray(sin, np.float64)[pos][:, None, :]
+    x1, x2 = x[..., :h], x[..., h:]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
+
+
+def _rope_interleaved(x, pos, cos, sin):
+    x = np.asarray(x, np.float64)
+    c = np.asarray(cos, np.float64)[pos][:, None, :]
+    s = np.asarray(sin, np.float64)[pos][:, None, :]
+    x1, x2 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x1 * c - x2 * s
+    out[..., 1::2] = x2 * c + x1 * s
+    return out
+
+
+def _asym_zero_sign(x):
+    x = np.asarray(x, F32)
+    lo = np.minimum(np.min(x, -1), F32(0))
+    hi = np.maximum(np.max(x, -1), F32(0))
+    s = ((hi - lo) / F32(15)).astype(F32)
+    s = np.where(s == 0, F32(1), s).astype(F32)
+    z = np.clip(np.rint(lo / s), 0, 15).astype(F32)
+    v = (x / s[..., None]).astype(F32)
+    return np.clip(np.rint(v) + z[..., None], 0, 15).astype(np.uint8), s, z.astype(np.uint8), v
+
+
+def _dequant_swapped(acc, a_scale, w_scale):
+    n = acc.shape[1]
+    m = acc.shape[0]
+    sa = np.resize(np.asarray(a_scale, np.float64), n)
+    sw = np.resize(np.asarray(w_scale, np.float64), m)
+    return acc.astype(np.float64) * sw[:, None] * sa[None, :]
+
+
+def _sylvester_walsh_order(n):
+    # sequency (Walsh) ordering instead of natural order
+    H = _orig["sylvester"](n)
+    changes = (np.diff(H, axis=1) != 0).sum(axis=1)
+    return H[np.argsort(changes, kind="stable")]
+
+
+_orig = {name: getattr(O, name) for name in
+         ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
+          "quant_asym_uint4", "dequant", "sylvester"]}
+
+MUTATIONS = {
+    "paley_transposed": ("paley1", _transposed_paley),
+    "kron_order_swapped": ("kron", _kron_swapped),
+    "rotation_missing_1_over_sqrt_g": ("rotate", _rotate_unnormalised),
+    "quant_divisor_8": ("quant_sym_int4", _quant_div8),
+    "quant_round_half_up": ("quant_sym_int4", _quant_floor),
+    "pack_nibbles_swapped": ("pack_int4", _pack_swapped),
+    "rope_sign_flipped": ("rope", _rope_sign),
+    "rope_interleaved_pairs": ("rope", _rope_interleaved),
+    "asym_zero_point_sign": ("quant_asym_uint4", _asym_zero_sign),
+    "dequant_scales_swapped": ("dequant", _dequant_swapped),
+    "sylvester_walsh_order": ("sylvester", _sylvester_walsh_order),
+}
+
+PIN_TESTS = [
+    lambda: [P.test_sylvester_is_hadamard(n) for n in (2, 8, 64)],
+    P.test_sylvester_matches_textbook_recursion,
+    lambda: [P.test_dense_sylvester_equals_butterfly(n) for n in (4, 16)],
+    P.test_paley_h12_properties,
+    P.test_paley_h12_golden,
+    P.test_kron_definition,
+    P.test_kron_h12_outer_index,
+    lambda: P.test_rotation_of_one_hot_is_scaled_row(12, 16),
+    P.test_rotation_is_row_vector_convention,
+    lambda: P.test_computational_invariance(1, 256, 256, 256),
+    P.test_quant_bruteforce_nearest_grid_point,
+    P.test_quant_divisor_and_special_rows,
+    P.test_quant_clip_clamps,
+    P.test_pack_golden_bytes,
+    P.test_dequant_scales_index_rows_and_columns,
+    P.test_rope_matches_complex_rotation_and_rotate_half,
+    P.test_headwise_hadamard_matches_butterfly,
+    P.test_asym_quant_bounds_and_zero_point,
+    P.test_asym_quant_constant_and_zero_rows,
+]
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(mutation, monkeypatch):
+    name, fn = MUTATIONS[mutation]
+    monkeypatch.setattr(O, name, fn)
+    O.hadamard.cache_clear()
+    caught = []
+    try:
+        for t in PIN_TESTS:
+            try:
+                t()
+            except AssertionError:
+                caught.append(t)
+    finally:
+        O.hadamard.cache_clear()
+    assert caught, "no pin caught mutation %s" % mutation
+
+
+def test_unmutated_oracle_passes_the_same_pins():
+    for t in PIN_TESTS:
+        t()

@@ -1,0 +1,456 @@
+"""Pins of the CPU oracle against facts fixed by mathematics and by the pages.
+
+Nothing here calls the CUDA library.  Each test checks an oracle function
+against something other than itself: a closed form, a textbook recursion,
+brute force on tiny inputs, an invariant, or a stored fixture under
+tests/golden/ whose provenance is stated in the fixture.  The checks are
+chosen so that a plausible slip (a dropped term, a wrong sign or index, a
+transposed operand, a wrong divisor or nibble order) fails at least one;
+tests/test_oracle_mutations.py plants such slips and confirms that.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from workloads import synthetic as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append([int(t, 0) for t in line.replace(",", " ").split()])
+    return rows
+
+
+# --------------------------------------------------------------------------
+# Hadamard constructions
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024])
+def test_sylvester_is_hadamard(n):
+    H = O.sylvester(n)
+    assert set(np.unique(H)) <= {-1, 1}
+    assert np.array_equal(H @ H.T, n * np.eye(n, dtype=np.int64))
+    assert np.array_equal(H, H.T)           # Sylvester matrices are symmetric
+    assert np.all(H[0] == 1) and np.all(H[:, 0] == 1)
+
+
+def test_sylvester_matches_textbook_recursion():
+    # H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]: the classical construction.
+    H = np.ones((1, 1), dtype=np.int64)
+    for k in range(1, 11):
+        H = np.block([[H, H], [H, -H]])
+        assert np.array_equal(O.sylvester(2 ** k), H)
+
+
+def fwht_butterfly(x):
+    """Iterative in-place Walsh-Hadamard butterfly (natural order), written independently."""
+    x = np.array(x, dtype=np.int64, copy=True)
+    n = x.shape[-1]
+    h = 1
+    while h < n:
+        for start in range(0, n, 2 * h):
+            a = x[..., start:start + h].copy()
+            b = x[..., start + h:start + 2 * h].copy()
+            x[..., start:start + h] = a + b
+            x[..., start + h:start + 2 * h] = a - b
+        h *= 2
+    return x
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
+def test_dense_sylvester_equals_butterfly(n):
+    rng = np.random.default_rng(n)
+    x = rng.integers(-100, 100, size=(7, n))
+    assert np.array_equal(x @ O.sylvester(n), fwht_butterfly(x))
+
+
+def test_quadratic_residues_mod_11():
+    # The nonzero squares mod 11 are 1, 4, 9, 5 (=16), 3 (=25).
+    res = {r for r in range(1, 11) if O.quadratic_character(r, 11) == 1}
+    assert res == {1, 3, 4, 5, 9}
+    assert O.quadratic_character(0, 11) == 0
+    assert sum(O.quadratic_character(r, 11) for r in range(11)) == 0
+
+
+def test_paley_h12_properties():
+    H = O.paley1(11)
+    assert H.shape == (12, 12)
+    assert np.array_equal(H @ H.T, 12 * np.eye(12, dtype=np.int64))
+    S = H - np.eye(12, dtype=np.int64)
+    # Paley construction I yields a skew Hadamard matrix: H = I + S, S^T = -S.
+    assert np.array_equal(S.T, -S)
+    assert np.all(H[0] == 1)
+    assert np.all((H[1:] == -1).sum(axis=1) == 6)
+
+
+def test_paley_h12_golden():
+    # Fixture written out from the construction's definition (see its header).
+    G = np.array(load_golden("paley_h12.txt"), dtype=np.int64)
+    assert np.array_equal(O.paley1(11), G)
+
+
+def test_kron_definition():
+    rng = np.random.default_rng(1)
+    A = rng.integers(-3, 4, size=(3, 4))
+    B = rng.integers(-3, 4, size=(2, 5))
+    K = O.kron(A, B)
+    for i in range(3):
+        for j in range(2):
+            for k in range(4):
+                for l in range(5):
+                    assert K[i * 2 + j, k * 5 + l] == A[i, k] * B[j, l]
+
+
+def test_kron_h12_outer_index():
+    H = O.hadamard(12, 64)
+    assert H.shape == (768, 768)
+    assert np.array_equal(H @ H.T, 768 * np.eye(768))
+    # channel c = i*64 + j with H12 on the outer index i
+    H12 = O.paley1(11)
+    assert np.array_equal(H[::64, ::64], H12)
+    assert np.array_equal(H[:64, :64], O.sylvester(64))
+
+
+# --------------------------------------------------------------------------
+# Rotation
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("ns,np2", [(1, 256), (12, 16), (1, 128)])
+def test_rotation_of_one_hot_is_scaled_row(ns, np2):
+    g = ns * np2
+    H = O.kron(O.small_hadamard(ns), O.sylvester(np2))
+    for k in [0, 1, g // 2 + 3, g - 1]:
+        e = np.zeros((1, g))
+        e[0, k] = 1.0
+        y = O.rotate(e, ns, np2)
+        assert np.allclose(y[0], H[k] / math.sqrt(g), rtol=0, atol=1e-7)
+
+
+def test_rotation_is_row_vector_convention():
+    # y = x H (not H x): with the non-symmetric Paley factor these differ.
+    x = np.zeros((1, 12 * 2))
+    x[0, 2] = 1.0                         # i = 1, j = 0
+    y = O.rotate(x, 12, 2)[0] * math.sqrt(24)
+    H12 = O.paley1(11)
+    expect = np.kron(H12[1], [1, 1])      # row 1 of H12, spread over j
+    assert np.allclose(y, expect, atol=1e-6)
+    assert not np.allclose(np.kron(H12[:, 1], [1, 1]), expect)
+
+
+def test_rotation_is_block_diagonal_over_groups():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 3 * 256))
+    y = O.rotate(x, 1, 256)
+    for b in range(3):
+        yb = O.rotate(x[:, b * 256:(b + 1) * 256], 1, 256)
+        assert np.array_equal(y[:, b * 256:(b + 1) * 256], yb)
+
+
+def test_rotation_identity_when_g_is_1():
+    x = np.random.default_rng(0).standard_normal((3, 16)).astype(np.float32)
+    assert np.array_equal(O.rotate(x, 1, 1), x)
+
+
+def test_rotation_orthogonal_norm_preserved():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((3, 12288))
+    y = O.rotate(x, 12, 1024).astype(np.float64)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-6)
+
+
+@pytest.mark.parametrize("ns,np2,K,N", [(1, 256, 256, 256), (12, 1024, 12288, 8), (1, 1, 64, 32)])
+def test_computational_invariance(ns, np2, K, N):
+    # (x H)(W H)^T / g = x W^T: the full-precision invariance that makes the
+    # rotation free ("SpinQuant, Reproduced", Q1), to 1e-4 relative in fp32.
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, K)).astype(np.float32)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    y = O.rotate(x, ns, np2).astype(np.float64)
+    wr = O.rotate(w, ns, np2).astype(np.float64)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T
+    assert O.rel_fro(y @ wr.T, ref) < 1e-4
+
+
+def test_invariance_through_r1_fold():
+    # r1-folded workload: x = x_raw R1 and W' = W R1 keep x W'^T = x_raw W^T.
+    rng = np.random.default_rng(6)
+    R = W.random_orthogonal(rng, 64)
+    assert np.abs(R.T @ R - np.eye(64)).max() < 1e-12
+    x = rng.standard_normal((5, 64))
+    w = rng.standard_normal((7, 64))
+    assert np.allclose((x @ R) @ (w @ R).T, x @ w.T, atol=1e-10)
+
+
+def test_kurtosis_definition():
+    rng = np.random.default_rng(7)
+    g = rng.standard_normal((64, 20000))
+    assert abs(O.kurtosis(g) - 3.0) < 0.05                 # Gaussian: 3
+    u = rng.uniform(-1, 1, (64, 20000))
+    assert abs(O.kurtosis(u) - 1.8) < 0.02                 # uniform: 9/5
+
+
+def test_kurtosis_collapses_after_rotation():
+    # "SpinQuant, Reproduced", Q3: per-token kurtosis in the hundreds before
+    # rotation falls to about 3 after it (210-472 -> 2.8-2.9 on Qwen3-8B).
+    # The SwiGLU product of two Student-t(3) draws reproduces that collapse.
+    rng = np.random.default_rng(8)
+    a = rng.standard_t(3.0, (32, 12288))
+    b = rng.standard_t(3.0, (32, 12288))
+    h = a / (1.0 + np.exp(-a)) * b
+    before = O.kurtosis(h)
+    after = O.kurtosis(O.rotate(h, 12, 1024))
+    assert before > 100, before
+    assert 2.7 <= after <= 3.3, after
+
+
+def test_kurtosis_with_planted_outlier_channels():
+    # With a few channels scaled x100 they dominate every rotated coordinate,
+    # which becomes a +-1-weighted sum of those few values: a sub-Gaussian
+    # (Rademacher-sum) law whose kurtosis lies in [1, 3].
+    x = W.swiglu_acts(np.random.default_rng(8), 32, 12288)
+    before = O.kurtosis(x)
+    after = O.kurtosis(O.rotate(x, 12, 1024))
+    assert before > 1000, before
+    assert 1.0 <= after <= 3.0, after
+
+
+# --------------------------------------------------------------------------
+# Symmetric INT4 quantizer and packing
+# --------------------------------------------------------------------------
+
+def test_quant_error_bound():
+    rng = np.random.default_rng(9)
+    y = (rng.standard_t(3, (50, 256)) * 3).astype(np.float32)
+    q, s, v = O.quant_sym_int4(y)
+    recon = q.astype(np.float64) * s[:, None]
+    err = np.abs(y - recon)
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-6))
+    assert q.min() >= -8 and q.max() <= 7
+
+
+def test_quant_bruteforce_nearest_grid_point():
+    rng = np.random.default_rng(10)
+    for trial in range(200):
+        y = (rng.standard_normal(8) * rng.uniform(0.01, 10)).astype(np.float32)
+        if trial % 5 == 0:
+            y[rng.integers(8)] = 0.0
+        q, s, v = O.quant_sym_int4(y[None, :])
+        sf = np.float32(s[0])
+        for k in range(8):
+            vk = np.float32(y[k] / sf)
+            # exhaustive nearest point of the grid -8..7, ties to the even code
+            cands = np.arange(-8, 8)
+            d = np.abs(cands - np.float64(vk))
+            best = cands[d == d.min()]
+            pick = best[best % 2 == 0][0] if len(best) > 1 else best[0]
+            assert q[0, k] == pick
+
+
+def test_quant_divisor_and_special_rows():
+    # The largest-magnitude element lands exactly on +-7 (divisor 7, clip 1).
+    y = np.array([[0.5, -3.5, 1.0, 0.25]], dtype=np.float32)
+    q, s, _ = O.quant_sym_int4(y)
+    assert s[0] == np.float32(0.5) and list(q[0]) == [1, -7, 2, 0]   # 0.5 -> 1.0 -> 1; 0.25/0.5 = 0.5 -> 0 (even)
+    c = np.full((1, 16), -2.5, dtype=np.float32)
+    q, s, _ = O.quant_sym_int4(c)
+    assert np.all(q == -7) and np.isclose(s[0], 2.5 / 7)
+    z = np.zeros((1, 16), dtype=np.float32)
+    q, s, _ = O.quant_sym_int4(z)
+    assert np.all(q == 0) and s[0] == 1.0
+
+
+def test_quant_clip_clamps():
+    y = np.array([[7.0, -7.0, 3.0, 0.0]], dtype=np.float32)
+    q, s, v = O.quant_sym_int4(y, clip=0.5)
+    assert s[0] == np.float32(0.5)
+    assert list(q[0]) == [7, -8, 6, 0]
+
+
+def test_pack_golden_bytes():
+    rows = load_golden("int4_pack.txt")
+    codes = np.array(rows[0], dtype=np.int8)
+    packed = np.array(rows[1], dtype=np.uint8)
+    assert np.array_equal(O.pack_int4(codes), packed)
+    assert np.array_equal(O.unpack_int4(packed), codes)
+
+
+def test_pack_roundtrip_random():
+    rng = np.random.default_rng(11)
+    c = rng.integers(-8, 8, size=(5, 64)).astype(np.int8)
+    assert np.array_equal(O.unpack_int4(O.pack_int4(c)), c)
+    u = rng.integers(0, 16, size=(5, 64)).astype(np.uint8)
+    assert np.array_equal(O.unpack_int4(O.pack_int4(u), signed=False), u)
+
+
+# --------------------------------------------------------------------------
+# Integer GEMM and dequant
+# --------------------------------------------------------------------------
+
+def test_gemm_int_bruteforce():
+    rng = np.random.default_rng(12)
+    a = rng.integers(-8, 8, size=(5, 32))
+    w = rng.integers(-8, 8, size=(6, 32))
+    acc = O.gemm_int(a, w)
+    for m in range(5):
+        for n in range(6):
+            assert acc[m, n] == sum(int(a[m, k]) * int(w[n, k]) for k in range(32))
+
+
+def test_gemm_one_hot_rows_return_weight_codes():
+    rng = np.random.default_rng(13)
+    w = rng.integers(-8, 8, size=(16, 64))
+    a = np.zeros((64, 64), dtype=np.int64)
+    a[np.arange(64), np.arange(64)] = 1
+    assert np.array_equal(O.gemm_int(a, w), w.T)
+
+
+def test_gemm_extreme_codes_exact():
+    K = 12288
+    a = np.full((2, K), -8)
+    w = np.full((3, K), -8)
+    assert np.all(O.gemm_int(a, w) == 64 * K)
+    w[1] = 7
+    assert O.gemm_int(a, w)[0, 1] == -56 * K
+
+
+def test_dequant_scales_index_rows_and_columns():
+    acc = np.array([[1, 2, 3], [4, 5, 6]])
+    sa = np.array([2.0, 3.0])
+    sw = np.array([1.0, 10.0, 100.0])
+    out = O.dequant(acc, sa, sw)
+    assert np.array_equal(out, [[2, 40, 600], [12, 150, 1800]])
+
+
+def test_w4a4_end_to_end_error_is_quantization_sized():
+    # Context for the pages' W4A4 layer error ("SpinQuant, Reproduced", Q2):
+    # the dequantized W4A4 output approximates x W^T within INT4 noise.
+    wl = W.tiny_linear()
+    x = wl.x.numpy().astype(np.float64)
+    w = wl.w.numpy().astype(np.float64)
+    ap, sa, _, _ = O.rotate_quant(x, wl.n_small, wl.n_pow2)
+    wp, sw, _ = O.quantize_weights(w, wl.n_small, wl.n_pow2)
+    _, out = O.w4a4_linear(ap, sa, wp, sw)
+    err = O.rel_fro(out, x @ w.T)
+    assert 0.02 < err < 0.3, err
+    # rotation helps: without it the outlier channels wreck the per-token scale
+    ap0, sa0, _, _ = O.rotate_quant(x, 1, 1)
+    wp0, sw0, _ = O.quantize_weights(w, 1, 1)
+    _, out0 = O.w4a4_linear(ap0, sa0, wp0, sw0)
+    assert O.rel_fro(out0, x @ w.T) > 1.1 * err
+
+
+# --------------------------------------------------------------------------
+# RoPE, head-wise Hadamard and the asymmetric KV quantizer
+# --------------------------------------------------------------------------
+
+def test_rope_tables_closed_form():
+    cos, sin = O.rope_tables(1e6, 16, 128)
+    p = np.arange(16)
+    assert np.allclose(cos[:, 0], np.cos(p), atol=1e-7)       # inv_freq_0 = 1
+    assert np.allclose(sin[:, 0], np.sin(p), atol=1e-7)
+    f63 = 1e6 ** (-126 / 128)
+    assert np.allclose(sin[:, 63], np.sin(p * f63), atol=1e-9)
+    assert np.all(cos[0] == 1) and np.all(sin[0] == 0)
+    assert np.allclose(cos.astype(np.float64) ** 2 + sin.astype(np.float64) ** 2, 1, atol=1e-6)
+
+
+def test_rope_matches_complex_rotation_and_rotate_half():
+    rng = np.random.default_rng(14)
+    d = 128
+    cos, sin = O.rope_tables(1e6, 64, d)
+    x = rng.standard_normal((5, 3, d))
+    pos = np.array([0, 1, 7, 33, 63])
+    out = O.rope(x, pos, cos, sin)
+    h = d // 2
+    # complex form: (x_i + i x_{i+h}) * (c + i s)
+    z = (x[..., :h] + 1j * x[..., h:]) * (cos[pos].astype(np.float64) + 1j * sin[pos].astype(np.float64))[:, None, :]
+    assert np.allclose(out[..., :h], z.real, atol=1e-12)
+    assert np.allclose(out[..., h:], z.imag, atol=1e-12)
+    # rotate_half form: x * [c, c] + concat(-x2, x1) * [s, s]
+    c2 = np.concatenate([cos[pos], cos[pos]], -1).astype(np.float64)[:, None, :]
+    s2 = np.concatenate([sin[pos], sin[pos]], -1).astype(np.float64)[:, None, :]
+    rh = np.concatenate([-x[..., h:], x[..., :h]], -1)
+    assert np.allclose(out, x * c2 + rh * s2, atol=1e-12)
+    # position 0 is the identity; each (i, i+h) pair keeps its norm
+    assert np.array_equal(out[0], x[0])
+    n_in = x[..., :h] ** 2 + x[..., h:] ** 2
+    n_out = out[..., :h] ** 2 + out[..., h:] ** 2
+    assert np.allclose(n_in, n_out, rtol=1e-6)
+
+
+def test_headwise_hadamard_matches_butterfly():
+    rng = np.random.default_rng(15)
+    x = rng.integers(-50, 50, size=(4, 2, 128))
+    y = O.headwise_hadamard(x) * math.sqrt(128)
+    assert np.allclose(y, fwht_butterfly(x), atol=1e-9)
+
+
+def test_asym_quant_bounds_and_zero_point():
+    rng = np.random.default_rng(16)
+    x = (rng.standard_normal((200, 128)) * rng.uniform(0.1, 5, (200, 1))).astype(np.float32)
+    x[::7] = np.abs(x[::7])          # all non-negative rows
+    x[3::7] = -np.abs(x[3::7])       # all non-positive rows
+    codes, scale, zero, v = O.quant_asym_uint4(x)
+    assert codes.min() >= 0 and codes.max() <= 15
+    xh = O.dequant_asym(codes, scale, zero)
+    err = np.abs(xh - x)
+    assert np.all(err <= scale[:, None] * (0.5 + 1e-5) + 1e-12)
+    assert np.all(zero[::7] == 0)
+    assert np.all(zero[3::7] == 15)
+    # the integer zero point represents 0 exactly
+    c0, s0, z0, _ = O.quant_asym_uint4(np.concatenate([x, np.zeros((200, 1), np.float32)], 1))
+    assert np.all(O.dequant_asym(c0, s0, z0)[:, -1] == 0)
+
+
+def test_asym_quant_constant_and_zero_rows():
+    c, s, z, _ = O.quant_asym_uint4(np.zeros((1, 128), np.float32))
+    assert s[0] == 1 and z[0] == 0 and np.all(c == 0)
+    c, s, z, _ = O.quant_asym_uint4(np.full((1, 128), 3.0, np.float32))
+    assert np.isclose(s[0], 0.2) and z[0] == 0 and np.all(c == 15)
+
+
+def test_kv_rotate_quant_composition():
+    rng = np.random.default_rng(17)
+    T, hq, hkv, d = 6, 4, 2, 128
+    q = rng.standard_normal((T, hq, d))
+    k = rng.standard_normal((T, hkv, d))
+    v = rng.standard_normal((T, hkv, d)).astype(np.float32)
+    pos = np.arange(T)
+    cos, sin = O.rope_tables(1e6, 8, d)
+    r = O.kv_rotate_quant(q, k, v, pos, cos, sin)
+    # Q' is the head-wise Hadamard of the rotary-embedded Q; norms are preserved
+    assert np.allclose(np.linalg.norm(r["q_rot"], axis=-1), np.linalg.norm(q, axis=-1), rtol=1e-5)
+    # V is not rotated: its dequantized cache approximates V directly
+    vh = O.kv_dequant(r["v_cache"], r["v_scale"], r["v_zero"])
+    assert np.all(np.abs(vh - v) <= r["v_scale"][..., None] * 0.5 + 1e-6)
+    kh = O.kv_dequant(r["k_cache"], r["k_scale"], r["k_zero"])
+    assert np.all(np.abs(kh - r["k_rot"]) <= r["k_scale"][..., None] * 0.5 + 1e-6)
+    # undoing the Hadamard and the rotary embedding recovers K
+    k_back = O.headwise_hadamard(r["k_rot"].astype(np.float64))   # H/sqrt(d) is an involution
+    c = cos[pos].astype(np.float64)[:, None, :]
+    s = sin[pos].astype(np.float64)[:, None, :]
+    k1, k2 = k_back[..., :64], k_back[..., 64:]
+    k_unrope = np.concatenate([k1 * c + k2 * s, k2 * c - k1 * s], -1)
+    assert np.allclose(k_unrope, k, atol=1e-5)
+
+
+# --------------------------------------------------------------------------
+# Workload generators (shapes and distributions only)
+# --------------------------------------------------------------------------
+
+def test_workload_shapes_and_determinism():
+    a = W.tiny_linear()
+    b = W.tiny_linear()
+    assert a.x.shape == (16, 256) and a.w.shape == (256, 256)
+    assert np.array_equal(a.x.numpy(), b.x.numpy())
+    big = np.abs(a.x.numpy()).max(axis=0)
+    assert (big > 20).sum() >= 4                    # the x50 outlier channels
