@@ -1,0 +1,361 @@
+"""Benchmark of the SpinQuant W4A4 + online-Hadamard hot path on B200.
+
+One step = the down_proj path at Qwen3-8B shape ("SpinQuant, Reproduced",
+section Q5): online R4 rotation H12 (x) H1024 + per-token INT4 quantization of
+x [4096, 12288] (sq_rotate_quant), then the W4A4 GEMM against INT4 weights
+[4096, 12288] with the dequant epilogue to bf16 (sq_w4a4_linear).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs the full step on its own GPU (the path shards by tokens with no data
+exchange), and rank 0 prints one JSON line with the max-over-ranks time.
+
+metric  : W4A4 linear TOPS (2*M*N*K per step / step time), step inputs resident
+          in HBM; rotate+quant GB/s and the GEMM's own TOPS ride along.
+e2e     : the same metric through the public API with the step's input x in
+          pinned host memory and the bf16 result copied back each step.
+roofline: the GEMM against the int8 tensor peak (measured bf16 peak x 2, the
+          nominal int8/bf16 ratio); the rotate+quant kernel against HBM.
+cpu_baseline / --impl reference: the CPU oracle on a bounded sample of the
+          same workload, extrapolated to one full step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N = 4096, 12288, 4096
+N_SMALL, N_POW2 = 12, 1024
+OPS = 2.0 * M * N * K
+# algorithmic bytes of sq_rotate_quant per row: bf16 in, packed INT4 out, f32 scale
+RQ_BYTES = M * (2 * K + K // 2 + 4)
+KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
+METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
+WORKLOAD = "down_proj_M4096_K12288_N4096_R4_H12xH1024"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk["hbm_gbs"], pk["bf16_tflops"], pk.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.result = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v == "Active"})
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        self.result = {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
+                       "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import rotation_ptq_b200 as sq
+    from workloads import synthetic as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = W.down_proj(M=M, K=K, N=N)
+    hs = sq.paley_h12()
+    x = wl.x.to(dev)
+    w_q, w_s = sq.quantize_weights(wl.w.to(dev), hs, N_POW2)
+    del wl
+    a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    a_s = torch.empty((M,), dtype=torch.float32, device=dev)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 2x the 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sq.rotate_quant(x, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+        sq.w4a4_linear(a_q, a_s, w_q, w_s, out=out)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if sq.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # timed region: K steps, L2 flushed between steps (outside the events)
+    t_step, t_rq, t_gemm = [], [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            sq.rotate_quant(x, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+            e1.record(stream)
+            sq.w4a4_linear(a_q, a_s, w_q, w_s, out=out)
+            e2.record(stream)
+            t_step.append((e0, e2))
+            t_rq.append((e0, e1))
+            t_gemm.append((e1, e2))
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = lambda pairs: sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)  # noqa: E731
+    ms_step, ms_rq, ms_gemm = ms(t_step), ms(t_rq), ms(t_gemm)
+    status = sq.device_status()
+
+    # e2e: pinned host input, H2D + path + D2H every step, device-timed
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        sq.rotate_quant(x_dev, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+        sq.w4a4_linear(a_q, a_s, w_q, w_s, out=out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e = []
+    for _ in range(args.steps):
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        sq.rotate_quant(x_dev, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+        sq.w4a4_linear(a_q, a_s, w_q, w_s, out=out)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_e2e = ms(e2e)
+
+    # KV path (config of the R3 rows), timed alone for the record
+    kv_info = None
+    if not args.no_kv:
+        kvw = W.kv_path()
+        q, k, v, pos = kvw.q.to(dev), kvw.k.to(dev), kvw.v.to(dev), kvw.pos.to(dev)
+        cos, sin = sq.rope_tables(kvw.theta, kvw.max_pos, 128, device=dev)
+        kvo = sq.kv_rotate_quant(q, k, v, pos, cos, sin)
+        kdq = sq.kv_dequant(kvo["k_cache"], kvo["k_scale"], kvo["k_zero"])
+        vdq = sq.kv_dequant(kvo["v_cache"], kvo["v_scale"], kvo["v_zero"])
+        torch.cuda.synchronize()
+        tq, td = [], []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            sq.kv_rotate_quant(q, k, v, pos, cos, sin, out=kvo)
+            e1.record(stream)
+            sq.kv_dequant(kvo["k_cache"], kvo["k_scale"], kvo["k_zero"], out=kdq)
+            sq.kv_dequant(kvo["v_cache"], kvo["v_scale"], kvo["v_zero"], out=vdq)
+            e2.record(stream)
+            tq.append((e0, e1))
+            td.append((e1, e2))
+        torch.cuda.synchronize()
+        d = 128
+        kv_fwd_bytes = KV_T * (2 * (KV_HQ * d * 2) + 2 * (KV_HKV * d * 2) + 2 * KV_HKV * (d // 2 + 5))
+        kv_rb_bytes = 2 * KV_T * KV_HKV * ((d // 2 + 5) + d * 2)
+        mq, md = ms(tq), ms(td)
+        kv_info = {"workload": "kv_T65536_hq32_hkv8_d128", "rotate_quant_us": mq * 1e3,
+                   "rotate_quant_gbs": kv_fwd_bytes / (mq * 1e-3) / 1e9,
+                   "dequant_us": md * 1e3, "dequant_gbs": kv_rb_bytes / (md * 1e-3) / 1e9}
+        del q, k, v, kvo, kdq, vdq
+
+    # max over ranks
+    vals = torch.tensor([ms_step, ms_rq, ms_gemm, ms_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_step, ms_rq, ms_gemm, ms_e2e = vals.tolist()
+    return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
+                clocks=clk.result, kv=kv_info)
+
+
+# ------------------------------------------------------------ oracle arm
+
+def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
+    """Time the CPU oracle on rows x cols of the workload; extrapolate one full step.
+
+    The oracle's step is rotate+quant of x (cost per row) then the integer GEMM
+    and dequant (cost per row x column).  Weight codes are prepared offline and
+    not timed, as on the GPU side.
+    """
+    import numpy as np
+    from oracle import oracle as O
+    from workloads import synthetic as W
+
+    wl = W.down_proj(M=rows, K=K, N=cols, seed=1001)
+    x = wl.x.double().numpy()
+    wp, ws, _ = O.quantize_weights(wl.w.double().numpy(), N_SMALL, N_POW2)
+    O.rotate_quant(x[:2], N_SMALL, N_POW2)          # builds and caches the dense H
+    t_rot, t_gemm, n = 0.0, 0.0, 0
+    t_start = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        ap, sa, _, _ = O.rotate_quant(x, N_SMALL, N_POW2)
+        t1 = time.perf_counter()
+        O.w4a4_linear(ap, sa, wp, ws)
+        t2 = time.perf_counter()
+        t_rot += t1 - t0
+        t_gemm += t2 - t1
+        n += 1
+        if time.perf_counter() - t_start >= min_seconds or (max_steps and n >= max_steps):
+            break
+    per_row = t_rot / n / rows
+    per_cell = t_gemm / n / (rows * cols)
+    full_s = per_row * M + per_cell * M * N
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info()) if threadpool_info() else 1
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": OPS / full_s / 1e12, "unit": "TOPS", "cores": int(cores), "kind": "oracle",
+            "sample": "%d rows x %d cols of the workload, %d repetitions (%.1f s), extrapolated "
+                      "to one full step (rotation cost per row, GEMM cost per row x col)"
+                      % (rows, cols, n, t_rot + t_gemm), "full_step_s": full_s}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kv", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    hbm, bf16, bf16_sus, peak_src = load_peaks()
+    int8_peak = 2.0 * bf16            # nominal dense int8 : bf16 ratio is 2 (4.5 : 2.25 PFLOP/s)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = oracle_sample(min_seconds=max(10.0, 2.0 * args.steps), max_steps=None)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TOPS",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": cb["full_step_s"] * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded numpy; Qwen3-8B down_proj shape)",
+                "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N},
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "TOPS", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample()
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    tops_step = OPS / (r["ms_step"] * 1e-3) / 1e12
+    tops_gemm = OPS / (r["ms_gemm"] * 1e-3) / 1e12
+    gbs_rq = RQ_BYTES / (r["ms_rq"] * 1e-3) / 1e9
+    tops_e2e = OPS / (r["ms_e2e"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": world * tops_step, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic (seeded numpy; SwiGLU of Student-t(3) + 8 outlier channels, "
+                "W ~ N(0, 0.02); Qwen3-8B down_proj shape)",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "tokens_per_gpu": M,
+                   "parallelism": "replicas (token-sharded, no collective)" if world > 1 else "1 GPU",
+                   "l2": "flushed (256 MB write) between timed steps"},
+        "kernels": {
+            "rotate_quant": {"us": r["ms_rq"] * 1e3, "GB/s": gbs_rq,
+                             "frac_of_hbm": gbs_rq / hbm, "bytes": RQ_BYTES},
+            "w4a4_gemm": {"us": r["ms_gemm"] * 1e3, "TOPS": tops_gemm,
+                          "frac_of_int8_peak": tops_gemm * 1e12 / (int8_peak * 1e12)},
+            "kv_path": r["kv"],
+        },
+        "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
+                     "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": None,
+                     "kernel": "w4a4_gemm_kernel",
+                     "peak_source": "%s bf16 %.1f TFLOP/s x 2 (nominal int8/bf16)" % (peak_src, bf16)},
+        "roofline_rotate_quant": {"bound": "hbm", "achieved": gbs_rq, "peak": hbm, "unit": "GB/s",
+                                  "frac": gbs_rq / hbm, "traffic": None,
+                                  "peak_source": peak_src + " copy bandwidth"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
+                "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * sq.h -- C ABI of the B200 (sm_100a) SpinQuant W4A4 inference hot path.
+ *
+ * What the library computes, in the words of the sources it follows:
+ *   - "SpinQuant, Reproduced", section Q5: of the four rotations, R1 (residual
+ *     stream) and R2 (value path, head-wise) fold into the weights offline;
+ *     R3 (KV path, head-wise, after RoPE) and R4 (before down_proj) sit
+ *     between operations that do not commute, so they stay Hadamard matrices
+ *     applied online.  Qwen3-8B sizes: hidden 4,096, 32 heads of 128, MLP
+ *     width 12,288.
+ *   - SpinQuant abstract: weights, activations and the KV cache are
+ *     quantized to 4 bits (W4A4KV4).
+ * The quantizer formulas, the Hadamard constructions, the RoPE convention and
+ * all data layouts are readings of points the pages leave open; each is
+ * stated below at the call that uses it.
+ *
+ * Conventions for every call
+ *   - Plain C; nothing throws across the ABI.
+ *   - Every tensor pointer is caller-owned DEVICE memory unless the argument
+ *     says "host".  The library allocates no device memory.  Device pointers
+ *     must be 16-byte aligned (else SQ_ERR_MISALIGNED).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls enqueue work and return without synchronising.
+ *   - Arguments are validated before anything is launched; on any error
+ *     status nothing has been enqueued and no output has been written.
+ *   - All matrices are row-major.  M = tokens, K = input channels,
+ *     N = output channels.
+ *   - Packed INT4: two codes per byte, element 2j in bits 0-3 and element
+ *     2j+1 in bits 4-7; signed codes are two's complement.
+ *   - Kernels bound every wait they spin on.  A wait that runs out records
+ *     SQ_ERR_TIMEOUT in a device status word and the kernel returns; read and
+ *     clear it with sq_device_status().
+ *   - The calls are stateless and may be issued from several host threads.
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum, bad clip ratio */
+  SQ_ERR_UNSUPPORTED_SHAPE = 2,  /* a shape rule of the call is violated */
+  SQ_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned */
+  SQ_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed (see sq_last_error) */
+  SQ_ERR_TIMEOUT = 5,            /* a bounded device-side wait ran out (from sq_device_status) */
+  SQ_ERR_WORKSPACE = 6           /* workspace too small for the requested split */
+} sq_status;
+
+typedef enum { SQ_IN_F32 = 0, SQ_IN_BF16 = 1 } sq_in_dtype;
+
+/* SQ_OUT_BF16: dequantized bf16 result.  SQ_OUT_I32: the exact int32 sum of
+ * code products, before any scale (used to check the integer GEMM). */
+typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_I32 = 1 } sq_out_kind;
+
+/* Human-readable name of a status code (static storage). */
+const char* sq_status_string(sq_status s);
+
+/* Detail of the last error raised on the calling host thread (static or
+ * thread-local storage; empty string if none). */
+const char* sq_last_error(void);
+
+/* Library ABI version: (major << 16) | minor. */
+int sq_version(void);
+
+/* ---------------------------------------------------------------------------
+ * sq_rotate_quant -- online Hadamard rotation + per-token symmetric INT4.
+ *
+ * Source: "SpinQuant, Reproduced", Q5 (R4 before down_proj is an online
+ * Hadamard; with R1 folded, the other projections get no online rotation)
+ * and the SpinQuant abstract (4-bit activations).
+ *
+ * For every row m (token) and every group of g = n_small * n_pow2 consecutive
+ * channels (K % g == 0):
+ *     y = x_group . (H_small (x) H_pow2) / sqrt(g)          (row vector times H)
+ * where H_pow2 is the Sylvester Hadamard in natural order,
+ * H_pow2[a][b] = (-1)^popcount(a & b), and H_small is the caller's +-1
+ * matrix (e.g. the Paley H12); channel c of a group is i * n_pow2 + j with i
+ * indexing H_small.  Then, per row over all K channels:
+ *     scale[m] = clip_ratio * max_k |y[m][k]| / 7     (1.0 for an all-zero row)
+ *     code[m][k] = clamp(round_half_even(y[m][k] / scale[m]), -8, 7)
+ * computed in float32.  n_small = n_pow2 = 1 is plain quantization.
+ *
+ * x         device, [M][ld_x] elements of x_dtype (row stride ld_x >= K,
+ *           ld_x * elem_size a multiple of 16 bytes); read only.
+ * had_small HOST, [n_small][n_small] int8 entries +-1, row-major; copied into
+ *           the launch, so it may be freed on return.  May be NULL iff
+ *           n_small == 1.
+ * n_small   1 or any order 2..32 (12 for the Paley factor of a 12,288-wide R4).
+ * n_pow2    power of two, 1..1024.
+ * clip_ratio in (0, 1].
+ * a_q       device, [M][K/2] bytes, packed signed INT4 codes (written).
+ * a_scale   device, [M] float32 (written).
+ * Shape rules: M >= 0 (M == 0 is a no-op), K % 32 == 0, 32 <= K <= 32768,
+ * K % g == 0.
+ * The same call quantizes weights offline: pass W [N][K] as x (float32) to
+ * get per-output-channel codes and scales with the rotation folded in.
+ * ------------------------------------------------------------------------- */
+sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
+                          float clip_ratio, uint8_t* a_q, float* a_scale, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * sq_w4a4_linear -- INT4 x INT4 GEMM with the per-token x per-channel dequant
+ * fused into its epilogue.
+ *
+ * Source: SpinQuant abstract (4-bit weights and activations: W4A4) and
+ * "SpinQuant, Reproduced", Q2 (the W4A4 output of one linear layer).
+ *
+ *     acc[m][n] = sum_k a[m][k] * w[n][k]                    (exact, int32)
+ *     out[m][n] = bf16_round_nearest_even(float(acc) * a_scale[m] * w_scale[n])
+ *                 (SQ_OUT_BF16), or acc itself (SQ_OUT_I32)
+ *
+ * a_q       device, [M][K/2] packed signed INT4 (from sq_rotate_quant).
+ * a_scale   device, [M] float32.
+ * w_q       device, [N][K/2] packed signed INT4 (K-contiguous rows).
+ * w_scale   device, [N] float32.
+ * out       device, [M][N] bf16 or int32, row-major (written).
+ * workspace device scratch for split-K partial sums, or NULL.  When non-NULL
+ *           it must hold sq_w4a4_workspace_bytes(M, N, K) bytes and be
+ *           zero-filled before its first use; every call that returns SQ_OK
+ *           and whose kernel finishes leaves it zero-filled again.  After a
+ *           device timeout (SQ_ERR_TIMEOUT) zero it again.  Concurrent calls
+ *           must not share one workspace.  With NULL, no split-K is used.
+ * Shape rules: M >= 0 (0 is a no-op), N % 16 == 0, N >= 16, K % 128 == 0,
+ * 128 <= K <= 65536 (so |acc| < 2^31).
+ * ------------------------------------------------------------------------- */
+sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                         const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
+                         sq_out_kind kind, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Bytes of split-K workspace sq_w4a4_linear may use for this shape (0 if the
+ * shape never splits). */
+size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* ---------------------------------------------------------------------------
+ * sq_kv_rotate_quant -- RoPE, head-wise Hadamard R3 on Q and K, and the
+ * asymmetric 4-bit KV cache.
+ *
+ * Source: "SpinQuant, Reproduced", Q5 (R3 is a head-wise Hadamard in the KV
+ * path, after RoPE, applied online; R2 on the value path is folded offline,
+ * so V is not rotated here) and the SpinQuant abstract (4-bit KV cache).
+ *
+ * Per token t and head h, on the d = 128 values of one head:
+ *   RoPE (half-split, "rotate_half"): for i < 64, with c = rope_cos[pos[t]][i],
+ *   s = rope_sin[pos[t]][i]:  x'_i = x_i c - x_{i+64} s,  x'_{i+64} = x_{i+64} c + x_i s.
+ *   Q and K:  y = x' . H_128 / sqrt(128)  (Sylvester, natural order).
+ *   q_out = bf16(y_q).
+ *   K and V caches (y_k, and v unrotated), per (token, head) group of 128:
+ *     lo = min(min x, 0), hi = max(max x, 0), scale = (hi - lo) / 15 (1 if 0),
+ *     zero = clamp(rint(-lo / scale), 0, 15),
+ *     code = clamp(rint(x / scale) + zero, 0, 15)      (float32, unsigned codes)
+ *
+ * q         device, [T][hq][d] bf16.        k, v: device, [T][hkv][d] bf16.
+ * pos       device, [T] int32, 0 <= pos < max_pos (out-of-range positions set
+ *           SQ_ERR_INVALID_ARG in the device status and the token's outputs
+ *           are left unwritten).
+ * rope_cos, rope_sin  device, [max_pos][d/2] float32 (see sq_rope_tables), or
+ *           both NULL when q and k already carry their rotary embedding.
+ * q_out     device, [T][hq][d] bf16 (written; may not alias q).
+ * k_cache, v_cache  device, [T][hkv][d/2] packed unsigned 4-bit codes.
+ * k_scale, v_scale  device, [T][hkv] float32.
+ * k_zero, v_zero    device, [T][hkv] uint8 (need only 1-byte alignment).
+ * Shape rules: d == 128, 1 <= hq <= 256, 1 <= hkv <= 64, hq % hkv == 0, T >= 0.
+ * ------------------------------------------------------------------------- */
+sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
+                             int hkv, int d, const int32_t* pos, const float* rope_cos,
+                             const float* rope_sin, int max_pos, void* q_out,
+                             uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                             uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                             void* stream);
+
+/* sq_kv_dequant -- read-back of one packed asymmetric cache to bf16:
+ *     out[t][h][j] = bf16((code - zero[t][h]) * scale[t][h]).
+ * cache [T][h][d/2], scale [T][h] f32, zero [T][h] uint8, out [T][h][d] bf16.
+ * Shape rules: d == 128, h >= 1, T >= 0. */
+sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                        int64_t T, int h, int d, void* out_bf16, void* stream);
+
+/* sq_rope_tables -- the cos/sin tables the KV call reads:
+ *     angle(p, i) = p * theta^(-2i/d),  cos[p][i] = float(cos(angle)),
+ *     sin[p][i] = float(sin(angle)),  evaluated in double precision on the
+ * device.  cos, sin: device [max_pos][d/2] float32.  d even, 2 <= d <= 1024,
+ * theta > 1, max_pos >= 1. */
+sq_status sq_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,
+                         void* stream);
+
+/* sq_device_status -- synchronise `stream`, then read and clear the device
+ * status word that kernels set when a bounded wait runs out (SQ_ERR_TIMEOUT)
+ * or a device-side argument check fails (SQ_ERR_INVALID_ARG).  Returns SQ_OK
+ * if no kernel reported anything since the last call. */
+sq_status sq_device_status(void* stream);
+
+/* sq_debug_set_spin_limit -- test hook: the number of polls a device wait
+ * makes before giving up (0 restores the default, which is a few seconds of
+ * polling).  Applies to kernels launched afterwards from any thread. */
+void sq_debug_set_spin_limit(uint32_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

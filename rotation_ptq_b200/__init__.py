@@ -1,0 +1,34 @@
+"""B200 (sm_100a) SpinQuant W4A4 inference hot path: thin Python binding.
+
+The compute lives in the C-ABI library ``libsq.so`` (CUDA kernels for
+sm_100a); this module only marshals arguments.  Tensors are torch CUDA
+tensors; every call enqueues on torch's current CUDA stream of the tensor's
+device.  There is no CPU fallback: if the library is missing, importing this
+package raises.
+
+Entry points (same names as the C ABI without the ``sq_`` prefix):
+  rotate_quant, w4a4_linear, w4a4_workspace_bytes, kv_rotate_quant,
+  kv_dequant, rope_tables, device_status, debug_set_spin_limit.
+"""
+from __future__ import annotations
+
+from .binding import (  # noqa: F401
+    SQ_IN_BF16,
+    SQ_IN_F32,
+    SQ_OUT_BF16,
+    SQ_OUT_I32,
+    SqError,
+    debug_set_spin_limit,
+    device_status,
+    kv_dequant,
+    kv_rotate_quant,
+    lib,
+    library_path,
+    quantize_weights,
+    rope_tables,
+    rotate_quant,
+    version,
+    w4a4_linear,
+    w4a4_workspace_bytes,
+)
+from .hadamard import paley_h12  # noqa: F401

@@ -1,0 +1,245 @@
+"""ctypes marshalling for ``libsq.so``: torch CUDA tensors in, C-ABI calls out.
+
+Nothing here computes: shapes are read off the tensors, outputs are allocated
+with torch (device memory is the one service torch provides), and each call
+goes straight to the matching ``sq_*`` entry point on torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(HERE, "libsq.so")
+
+if not os.path.exists(library_path):
+    raise ImportError(
+        "rotation_ptq_b200: CUDA library %s is missing; build it with "
+        "`python -m rotation_ptq_b200.build` (there is no CPU fallback)" % library_path)
+
+lib = ctypes.CDLL(library_path)
+
+SQ_IN_F32, SQ_IN_BF16 = 0, 1
+SQ_OUT_BF16, SQ_OUT_I32 = 0, 1
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int
+_f32 = ctypes.c_float
+
+lib.sq_status_string.restype = ctypes.c_char_p
+lib.sq_status_string.argtypes = [_i32]
+lib.sq_last_error.restype = ctypes.c_char_p
+lib.sq_last_error.argtypes = []
+lib.sq_version.restype = _i32
+lib.sq_rotate_quant.restype = _i32
+lib.sq_rotate_quant.argtypes = [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
+lib.sq_w4a4_linear.restype = _i32
+lib.sq_w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp,
+                               ctypes.c_size_t, _vp]
+lib.sq_w4a4_workspace_bytes.restype = ctypes.c_size_t
+lib.sq_w4a4_workspace_bytes.argtypes = [_i64, _i64, _i64]
+lib.sq_kv_rotate_quant.restype = _i32
+lib.sq_kv_rotate_quant.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32,
+                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.sq_kv_dequant.restype = _i32
+lib.sq_kv_dequant.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]
+lib.sq_rope_tables.restype = _i32
+lib.sq_rope_tables.argtypes = [ctypes.c_double, _i32, _i32, _vp, _vp, _vp]
+lib.sq_device_status.restype = _i32
+lib.sq_device_status.argtypes = [_vp]
+lib.sq_debug_set_spin_limit.restype = None
+lib.sq_debug_set_spin_limit.argtypes = [ctypes.c_uint32]
+
+
+class SqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = lib.sq_status_string(status).decode()
+        detail = lib.sq_last_error().decode()
+        super().__init__("%s: %s (%s)" % (where, name, detail))
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SqError(status, where)
+
+
+def version() -> int:
+    return lib.sq_version()
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("rotation_ptq_b200 takes CUDA tensors (no CPU path)")
+
+
+def rotate_quant(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float = 1.0,
+                 a_q: torch.Tensor = None, a_scale: torch.Tensor = None):
+    """Online rotation + per-token INT4 (``sq_rotate_quant``).
+
+    x: CUDA [M, K] bf16 or float32 (unit stride along K).  had_small: None or a
+    host +-1 int8 matrix [n, n].  Returns (a_q uint8 [M, K/2], a_scale f32 [M]).
+    """
+    _need_cuda(x)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit stride along K")
+    if x.dtype == torch.bfloat16:
+        dt = SQ_IN_BF16
+    elif x.dtype == torch.float32:
+        dt = SQ_IN_F32
+    else:
+        raise ValueError("x must be bf16 or float32")
+    M, K = x.shape
+    if had_small is None:
+        hs, n_small, hs_ptr = None, 1, None
+    else:
+        hs = np.ascontiguousarray(np.asarray(had_small, dtype=np.int8))
+        n_small = hs.shape[0]
+        if hs.shape != (n_small, n_small):
+            raise ValueError("had_small must be square")
+        hs_ptr = hs.ctypes.data
+    if a_q is None:
+        a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if a_scale is None:
+        a_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    st = lib.sq_rotate_quant(x.data_ptr(), dt, M, K, x.stride(0), hs_ptr, n_small, n_pow2,
+                             float(clip), a_q.data_ptr(), a_scale.data_ptr(), _stream(x))
+    _check(st, "sq_rotate_quant")
+    return a_q, a_scale
+
+
+def quantize_weights(w: torch.Tensor, had_small=None, n_pow2: int = 1):
+    """Offline: fold the rotation into W [N, K] (float32) and RTN-quantize per channel.
+
+    The same kernel as ``rotate_quant`` (clip 1.0), applied to weight rows:
+    codes of W H / sqrt(g).  Returns (w_q uint8 [N, K/2], w_scale f32 [N]).
+    """
+    return rotate_quant(w.float().contiguous(), had_small, n_pow2, 1.0)
+
+
+_ws_lock = threading.Lock()
+_ws_cache = {}
+
+
+def _workspace(device: torch.device, stream: int, nbytes: int) -> torch.Tensor:
+    key = (device.index, stream)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            # zero-filled once; the library hands it back zero-filled after every call
+            buf = torch.zeros((max(nbytes, 256),), dtype=torch.uint8, device=device)
+            _ws_cache[key] = buf
+        return buf
+
+
+def w4a4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.sq_w4a4_workspace_bytes(M, N, K))
+
+
+def w4a4_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
+                w_scale: torch.Tensor, out_int32: bool = False, out: torch.Tensor = None,
+                workspace: torch.Tensor = None, use_workspace: bool = True):
+    """W4A4 GEMM with fused dequant (``sq_w4a4_linear``).
+
+    a_q [M, K/2], a_scale [M], w_q [N, K/2], w_scale [N] on one CUDA device.
+    Returns bf16 [M, N] (or int32 accumulators with out_int32=True).
+    """
+    _need_cuda(a_q, a_scale, w_q, w_scale)
+    M, Kh = a_q.shape
+    N = w_q.shape[0]
+    K = 2 * Kh
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if out_int32 else torch.bfloat16,
+                          device=a_q.device)
+    stream = _stream(a_q)
+    ws_ptr, ws_bytes = None, 0
+    if use_workspace:
+        need = w4a4_workspace_bytes(M, N, K)
+        if workspace is not None:
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+        elif need > 0:
+            ws = _workspace(a_q.device, stream, need)
+            ws_ptr, ws_bytes = ws.data_ptr(), ws.numel()
+    st = lib.sq_w4a4_linear(a_q.data_ptr(), a_scale.data_ptr(), w_q.data_ptr(),
+                            w_scale.data_ptr(), M, N, K, out.data_ptr(),
+                            SQ_OUT_I32 if out_int32 else SQ_OUT_BF16, ws_ptr, ws_bytes, stream)
+    _check(st, "sq_w4a4_linear")
+    return out
+
+
+def rope_tables(theta: float, max_pos: int, d: int = 128, device=None):
+    """cos/sin tables [max_pos, d/2] float32 computed on the device (``sq_rope_tables``)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    cos = torch.empty((max_pos, d // 2), dtype=torch.float32, device=device)
+    sin = torch.empty_like(cos)
+    st = lib.sq_rope_tables(float(theta), max_pos, d, cos.data_ptr(), sin.data_ptr(),
+                            _stream(cos))
+    _check(st, "sq_rope_tables")
+    return cos, sin
+
+
+def kv_rotate_quant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+                    cos: torch.Tensor = None, sin: torch.Tensor = None, out=None):
+    """RoPE + head-wise H128 on Q/K, asymmetric 4-bit K/V caches (``sq_kv_rotate_quant``).
+
+    q [T, hq, 128], k/v [T, hkv, 128] bf16; pos [T] int32.  Returns a dict with
+    q_out, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero.
+    """
+    _need_cuda(q, k, v, pos, cos, sin)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    dev = q.device
+    if out is None:
+        out = dict(
+            q_out=torch.empty_like(q),
+            k_cache=torch.empty((T, hkv, d // 2), dtype=torch.uint8, device=dev),
+            k_scale=torch.empty((T, hkv), dtype=torch.float32, device=dev),
+            k_zero=torch.empty((T, hkv), dtype=torch.uint8, device=dev),
+            v_cache=torch.empty((T, hkv, d // 2), dtype=torch.uint8, device=dev),
+            v_scale=torch.empty((T, hkv), dtype=torch.float32, device=dev),
+            v_zero=torch.empty((T, hkv), dtype=torch.uint8, device=dev))
+    max_pos = cos.shape[0] if cos is not None else 0
+    st = lib.sq_kv_rotate_quant(q.data_ptr(), k.data_ptr(), v.data_ptr(), T, hq, hkv, d,
+                                pos.data_ptr(), _ptr(cos), _ptr(sin), max_pos,
+                                out["q_out"].data_ptr(), out["k_cache"].data_ptr(),
+                                out["k_scale"].data_ptr(), out["k_zero"].data_ptr(),
+                                out["v_cache"].data_ptr(), out["v_scale"].data_ptr(),
+                                out["v_zero"].data_ptr(), _stream(q))
+    _check(st, "sq_kv_rotate_quant")
+    return out
+
+
+def kv_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out=None):
+    """Packed asymmetric cache [T, h, 64] -> bf16 [T, h, 128] (``sq_kv_dequant``)."""
+    _need_cuda(cache, scale, zero)
+    T, h, dh = cache.shape
+    if out is None:
+        out = torch.empty((T, h, 2 * dh), dtype=torch.bfloat16, device=cache.device)
+    st = lib.sq_kv_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, 2 * dh,
+                           out.data_ptr(), _stream(cache))
+    _check(st, "sq_kv_dequant")
+    return out
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(lib.sq_device_status(torch.cuda.current_stream(dev).cuda_stream))
+
+
+def debug_set_spin_limit(polls: int) -> None:
+    lib.sq_debug_set_spin_limit(int(polls))

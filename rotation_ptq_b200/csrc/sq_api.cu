@@ -1,0 +1,318 @@
+// C ABI of the library: argument validation, dispatch, status reporting.
+// Every check runs before anything is enqueued, so an error status means no
+// output was touched.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "sq_device.cuh"
+#include "sq_host.h"
+
+namespace sq {
+
+__device__ unsigned int g_status = 0;
+
+namespace host {
+
+static thread_local char t_err[512] = {0};
+static std::atomic<uint32_t> g_spin_limit{0};
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+}
+
+sq_status cuda_fail(const char* what, cudaError_t e) {
+  set_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+  return SQ_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!fn) set_error("cuTensorMapEncodeTiled is not available from the driver");
+  return fn;
+}
+
+int current_device() {
+  int d = -1;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) {
+    cuda_fail("cudaGetDevice", e);
+    return -1;
+  }
+  return d;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int d = current_device();
+  if (d < 0) return 0;
+  if (d < 64 && cache[d] > 0) return cache[d];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0)
+    n = 148;
+  if (d < 64) cache[d] = n;
+  return n;
+}
+
+uint32_t spin_limit() { return g_spin_limit.load(std::memory_order_relaxed); }
+
+}  // namespace host
+}  // namespace sq
+
+using sq::host::set_error;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sq_status precheck_device() {
+  if (sq::host::current_device() < 0) return SQ_ERR_CUDA;
+  return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG";
+    case SQ_ERR_UNSUPPORTED_SHAPE: return "SQ_ERR_UNSUPPORTED_SHAPE";
+    case SQ_ERR_MISALIGNED: return "SQ_ERR_MISALIGNED";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+    case SQ_ERR_WORKSPACE: return "SQ_ERR_WORKSPACE";
+  }
+  return "SQ_ERR_UNKNOWN";
+}
+
+const char* sq_last_error(void) { return sq::host::t_err; }
+
+int sq_version(void) { return (1 << 16) | 0; }
+
+void sq_debug_set_spin_limit(uint32_t polls) {
+  sq::host::g_spin_limit.store(polls, std::memory_order_relaxed);
+}
+
+sq_status sq_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return sq::host::cuda_fail("cudaStreamSynchronize", e);
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, sq::g_status, sizeof(v));
+  if (e != cudaSuccess) return sq::host::cuda_fail("read device status", e);
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(sq::g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return sq::host::cuda_fail("clear device status", e);
+    set_error("device reported %s", sq_status_string(static_cast<sq_status>(v)));
+    return static_cast<sq_status>(v);
+  }
+  return SQ_OK;
+}
+
+sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
+                          float clip_ratio, uint8_t* a_q, float* a_scale, void* stream) {
+  if (x_dtype != SQ_IN_F32 && x_dtype != SQ_IN_BF16) {
+    set_error("x_dtype %d is not SQ_IN_F32 or SQ_IN_BF16", static_cast<int>(x_dtype));
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (M < 0 || K < 0 || ld_x < K) {
+    set_error("bad sizes M=%lld K=%lld ld_x=%lld", (long long)M, (long long)K, (long long)ld_x);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!(clip_ratio > 0.f && clip_ratio <= 1.f)) {
+    set_error("clip_ratio %g is outside (0, 1]", static_cast<double>(clip_ratio));
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (n_small < 1 || n_small > 32 || n_pow2 < 1 || n_pow2 > 1024 || (n_pow2 & (n_pow2 - 1))) {
+    set_error("n_small=%d must be in 1..32 and n_pow2=%d a power of two in 1..1024", n_small,
+              n_pow2);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (n_small > 1 && had_small == nullptr) {
+    set_error("had_small is NULL with n_small=%d", n_small);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (n_small > 1) {
+    for (int i = 0; i < n_small * n_small; ++i) {
+      if (had_small[i] != 1 && had_small[i] != -1) {
+        set_error("had_small[%d] = %d is not +-1", i, had_small[i]);
+        return SQ_ERR_INVALID_ARG;
+      }
+    }
+  }
+  const int64_t g = static_cast<int64_t>(n_small) * n_pow2;
+  if (K % 32 != 0 || K < 32 || K > 65536 || K % g != 0) {
+    set_error("K=%lld must be a multiple of 32 in [32, 65536] and of the group %lld",
+              (long long)K, (long long)g);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (M > 0x7fffffff) {
+    set_error("M=%lld too large", (long long)M);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (M == 0) return SQ_OK;
+  if (!x || !a_q || !a_scale) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  const int64_t esz = x_dtype == SQ_IN_BF16 ? 2 : 4;
+  if (!aligned16(x) || !aligned16(a_q) || !aligned16(a_scale) || (ld_x * esz) % 16 != 0) {
+    set_error("x, a_q and a_scale must be 16-byte aligned and ld_x*elem a multiple of 16");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::rq::run(x, x_dtype == SQ_IN_BF16, M, K, ld_x, had_small, n_small, n_pow2,
+                     clip_ratio, a_q, a_scale, static_cast<cudaStream_t>(stream));
+}
+
+size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N < 16 || N % 16 || K < 128 || K % 128 || K > 65536) return 0;
+  if (sq::host::current_device() < 0) return 0;
+  return sq::gemm::workspace_bytes(M, N, K, sq::host::num_sms());
+}
+
+sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                         const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
+                         sq_out_kind kind, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (kind != SQ_OUT_BF16 && kind != SQ_OUT_I32) {
+    set_error("kind %d is not SQ_OUT_BF16 or SQ_OUT_I32", static_cast<int>(kind));
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (M < 0 || N < 0 || K < 0) {
+    set_error("negative size");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (N < 16 || N % 16 != 0 || K < 128 || K % 128 != 0 || K > 65536 || M > 0x7fffffff ||
+      N > 0x7fffffff) {
+    set_error("shape M=%lld N=%lld K=%lld: need N %% 16 == 0, K %% 128 == 0, 128 <= K <= 65536",
+              (long long)M, (long long)N, (long long)K);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (M == 0) return SQ_OK;
+  if (!a_q || !a_scale || !w_q || !w_scale || !out) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(a_q) || !aligned16(a_scale) || !aligned16(w_q) || !aligned16(w_scale) ||
+      !aligned16(out) || (workspace && !aligned16(workspace))) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::gemm::run(a_q, a_scale, w_q, w_scale, M, N, K, out, kind == SQ_OUT_I32, workspace,
+                       workspace_bytes, static_cast<cudaStream_t>(stream),
+                       sq::host::spin_limit(), sq::host::num_sms(), nullptr);
+}
+
+sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
+                             int hkv, int d, const int32_t* pos, const float* rope_cos,
+                             const float* rope_sin, int max_pos, void* q_out,
+                             uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                             uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                             void* stream) {
+  if (T < 0 || hq < 1 || hkv < 1) {
+    set_error("bad sizes T=%lld hq=%d hkv=%d", (long long)T, hq, hkv);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (d != 128 || hq > 256 || hkv > 64 || hq % hkv != 0 || T > 0x7fffffff) {
+    set_error("unsupported shape d=%d hq=%d hkv=%d (need d == 128, hq %% hkv == 0)", d, hq, hkv);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) {
+    set_error("rope_cos and rope_sin must both be set or both be NULL");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (rope_cos && max_pos < 1) {
+    set_error("max_pos=%d must be >= 1 with RoPE tables", max_pos);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (T == 0) return SQ_OK;
+  if (!q || !k || !v || !pos || !q_out || !k_cache || !k_scale || !k_zero || !v_cache ||
+      !v_scale || !v_zero) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (q_out == q) {
+    set_error("q_out may not alias q");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_out) ||
+      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_scale) || !aligned16(v_scale) ||
+      !aligned16(pos) || (rope_cos && (!aligned16(rope_cos) || !aligned16(rope_sin)))) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::kv::run_rotate_quant(q, k, v, T, hq, hkv, pos, rope_cos, rope_sin, max_pos, q_out,
+                                  k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                        int64_t T, int h, int d, void* out_bf16, void* stream) {
+  if (T < 0 || h < 1) {
+    set_error("bad sizes T=%lld h=%d", (long long)T, h);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (d != 128 || T > 0x7fffffff) {
+    set_error("unsupported head dim %d (need 128)", d);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (T == 0) return SQ_OK;
+  if (!cache || !scale || !zero || !out_bf16) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(cache) || !aligned16(scale) || !aligned16(out_bf16)) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::kv::run_dequant(cache, scale, zero, T, h, out_bf16,
+                             static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,
+                         void* stream) {
+  if (!(theta > 1.0) || max_pos < 1 || d < 2 || d > 1024 || (d & 1)) {
+    set_error("bad RoPE table arguments theta=%g max_pos=%d d=%d", theta, max_pos, d);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!cos || !sin) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(cos) || !aligned16(sin)) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::kv::run_rope_tables(theta, max_pos, d, cos, sin, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

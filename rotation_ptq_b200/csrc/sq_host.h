@@ -1,0 +1,65 @@
+// Host-side helpers shared by the C-ABI translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sq.h"
+
+namespace sq {
+namespace host {
+
+// Record a printf-style detail for sq_last_error() (thread-local).
+void set_error(const char* fmt, ...);
+// Record a CUDA runtime failure and return SQ_ERR_CUDA.
+sq_status cuda_fail(const char* what, cudaError_t e);
+// cuTensorMapEncodeTiled from the driver, resolved once (nullptr on failure).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+// Current device ordinal (-1 on failure, with the error recorded).
+int current_device();
+// Number of SMs of the current device (cached per device).
+int num_sms();
+// Poll limit for device waits set by sq_debug_set_spin_limit (0 = default).
+uint32_t spin_limit();
+
+}  // namespace host
+
+namespace gemm {
+
+struct Plan {
+  int swap;         // weights on the MMA M side (small M)
+  int bn;           // MMA N tile
+  int tilesA, tilesB, KT, splits, kps, units, grid;
+};
+
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms);
+size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
+              int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
+              size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
+              const Plan* forced);
+
+}  // namespace gemm
+
+namespace rq {
+sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
+              const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
+              float* a_scale, cudaStream_t stream);
+}  // namespace rq
+
+namespace kv {
+sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
+                           int hkv, const int32_t* pos, const float* cos, const float* sin,
+                           int max_pos, void* q_out, uint8_t* k_cache, float* k_scale,
+                           uint8_t* k_zero, uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                           cudaStream_t stream);
+sq_status run_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero, int64_t T,
+                      int h, void* out, cudaStream_t stream);
+sq_status run_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,
+                          cudaStream_t stream);
+}  // namespace kv
+
+}  // namespace sq

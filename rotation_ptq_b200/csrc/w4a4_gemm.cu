@@ -1,0 +1,580 @@
+// W4A4 GEMM with fused per-token x per-channel dequant, sm_100a.
+//
+// What it computes (SpinQuant abstract: 4-bit weights and activations;
+// "SpinQuant, Reproduced", Q2: the W4A4 output of one linear layer):
+//     acc[m][n] = sum_k a[m][k] * w[n][k]            (exact int32)
+//     out[m][n] = bf16(float(acc) * a_scale[m] * w_scale[n])   or acc itself.
+//
+// Blackwell has no INT4 tensor-core MMA, so the kernel streams packed INT4 and
+// widens it on chip:
+//   TMA warp     : 2-D tiled bulk loads of packed rows (64 B = 128 codes per
+//                  row per stage) into a packed ring; out-of-range rows are
+//                  zero-filled by the copy engine.
+//   unpack warps : packed ring -> int8 ring in the 128-byte-swizzled K-major
+//                  layout the tensor core reads.  A packed word w holding 8
+//                  codes becomes (w << 4) & 0xF0F0F0F0 (even codes x16) and
+//                  w & 0xF0F0F0F0 (odd codes x16): two ops per 8 codes.  Both
+//                  operands get the same K permutation, so the dot product is
+//                  unchanged and equals 256 x the true sum (exact; divided out
+//                  in the epilogue).
+//   MMA thread   : tcgen05.mma.kind::i8, M = 128, N = BN, K = 32, int32
+//                  accumulators in tensor memory (two buffers so the epilogue
+//                  of one tile overlaps the mainloop of the next).
+//   epilogue     : 4 warps, tcgen05.ld of their 32 TMEM lanes, scale, bf16.
+// Small M uses "swap" mode: weights on the MMA M side (128 channels per tile)
+// and tokens on the N side (16..128), with the K range split across CTAs and
+// the partial int32 sums reduced with red.add into a caller workspace; the
+// last CTA of a tile (arrival counter) applies the epilogue and re-zeroes the
+// workspace.  Integer addition is associative, so the result is
+// deterministic.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sq_device.cuh"
+#include "sq_host.h"
+
+namespace sq {
+namespace gemm {
+
+constexpr int BM = 128;          // MMA M: TMEM lanes
+constexpr int BK = 128;          // int8 K elements per stage (one 128-byte swizzle row)
+constexpr int KP = BK / 2;       // packed bytes per row per stage
+constexpr int UMMA_K = 32;       // K per tcgen05.mma kind::i8
+constexpr int EPI_WARPS = 4;
+constexpr int MMA_WARP = 4;
+constexpr int TMA_WARP = 5;
+constexpr int UNPACK_WARP0 = 6;
+constexpr int UNPACK_WARPS = 8;
+constexpr int NUM_THREADS = (UNPACK_WARP0 + UNPACK_WARPS) * 32;   // 448
+constexpr int NPT = UNPACK_WARPS * 32;                             // unpack threads
+
+struct Params {
+  int rowsA, rowsB;        // valid rows of the A-side / B-side operands
+  int tilesA, tilesB;      // tiles along A (128 rows) and B (BN rows)
+  int KT;                  // K / 128
+  int splits, kps;         // K splits and k-tiles per split
+  int units;               // tilesA * tilesB * splits
+  int swap;                // 0: A = tokens, B = channels; 1: A = channels, B = tokens
+  int M, N;
+  const float* a_scale;    // [M]
+  const float* w_scale;    // [N]
+  void* out;               // [M][N] bf16 or int32
+  int out_i32;
+  int* ws_acc;             // [M][N] int32 (split-K only; zero on entry and exit)
+  unsigned* ws_cnt;        // [tilesA * tilesB] (split-K only; zero on entry and exit)
+  uint32_t spin_limit;
+};
+
+template <int BN, int PST, int UST>
+struct Layout {
+  static constexpr int PA = BM * KP;                 // packed A bytes per stage
+  static constexpr int PB = BN * KP;
+  static constexpr int PSTAGE = PA + PB;
+  static constexpr int UA = BM * BK;                 // int8 A bytes per stage
+  static constexpr int UB = BN * BK;
+  static constexpr int USTAGE = UA + UB;
+  static constexpr int U_OFF = 0;                    // 1024-aligned rings first
+  static constexpr int P_OFF = UST * USTAGE;
+  static constexpr int BAR_OFF = P_OFF + PST * PSTAGE;
+  // barriers: pfull[PST], pempty[PST], ufull[UST], uempty[UST], tfull[2], tempty[2], drain
+  static constexpr int NBAR = 2 * PST + 2 * UST + 5;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = MISC_OFF + 32 + 1024;  // + slack to align the base
+  static constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulator buffers
+  static_assert(USTAGE % 1024 == 0 && UA % 1024 == 0, "swizzle atoms need 1 KB alignment");
+  static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
+                "TMEM allocation must be a power of two in [32, 512]");
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128B-swizzled
+// K-major tile whose rows are 128 bytes and whose 8-row groups are 1 KB apart.
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+struct Unit {
+  int ta, tb, s, kt0, kt1;
+};
+
+__device__ __forceinline__ Unit decompose(const Params& p, int u) {
+  Unit r;
+  r.s = u % p.splits;
+  int t = u / p.splits;
+  r.ta = t % p.tilesA;
+  r.tb = t / p.tilesA;
+  r.kt0 = r.s * p.kps;
+  r.kt1 = min(r.kt0 + p.kps, p.KT);
+  return r;
+}
+
+template <int BN, int PST, int UST>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
+                     const __grid_constant__ CUtensorMap mapB, const Params p) {
+  using L = Layout<BN, PST, UST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* pempty = pfull + PST;
+  uint64_t* ufull = pempty + PST;
+  uint64_t* uempty = ufull + UST;
+  uint64_t* tfull = uempty + UST;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PST; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], NPT);
+    }
+    for (int s = 0; s < UST; ++s) {
+      mbar_init(&ufull[s], NPT);
+      mbar_init(&uempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], EPI_WARPS * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp == TMA_WARP) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units && !*abort_flag; u += gridDim.x) {
+        const Unit w = decompose(p, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          const int ps = it % PST;
+          const uint32_t ph = (it / PST) & 1;
+          if (!mbar_wait(&pempty[ps], ph ^ 1, p.spin_limit)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* dst = smem + L::P_OFF + ps * L::PSTAGE;
+          mbar_arrive_expect_tx(&pfull[ps], L::PSTAGE);
+          tma_load_2d(dst, &mapA, kt * KP, w.ta * BM, &pfull[ps]);
+          tma_load_2d(dst + L::PA, &mapB, kt * KP, w.tb * BN, &pfull[ps]);
+        }
+      }
+      // Before the CTA may exit, every bulk copy it issued must have landed.
+      // The last PST stages are the only ones that can still be in flight;
+      // waiting on an already-completed phase returns at once.
+      for (uint32_t j = it > static_cast<uint32_t>(PST) ? it - PST : 0u; j < it; ++j)
+        mbar_wait(&pfull[j % PST], (j / PST) & 1, 0);
+    }
+  } else if (warp >= UNPACK_WARP0) {
+    // ------------------------------------------------ unpack: INT4 -> INT8
+    constexpr int ITEMS = (BM + BN) * 4;                 // 16-byte packed chunks per stage
+    constexpr int IPT = (ITEMS + NPT - 1) / NPT;
+    const int t = threadIdx.x - UNPACK_WARP0 * 32;
+    uint32_t src_off[IPT], dst_off0[IPT], dst_off1[IPT];
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const int idx = t + i * NPT;
+      const int row_all = idx >> 2, q = idx & 3;
+      // packed stage: rows of 64 bytes, A rows then B rows
+      src_off[i] = static_cast<uint32_t>(row_all * KP + q * 16);
+      const bool is_a = row_all < BM;
+      const int row = is_a ? row_all : row_all - BM;
+      const uint32_t base = is_a ? 0u : static_cast<uint32_t>(L::UA);
+      dst_off0[i] = base + sw128_off(row, 2 * q);
+      dst_off1[i] = base + sw128_off(row, 2 * q + 1);
+    }
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      const Unit w = decompose(p, u);
+      for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+        const int ps = it % PST, us = it % UST;
+        const uint32_t pph = (it / PST) & 1, uph = (it / UST) & 1;
+        if (!mbar_wait(&pfull[ps], pph, p.spin_limit) ||
+            !mbar_wait(&uempty[us], uph ^ 1, p.spin_limit) || *abort_flag) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
+        const uint32_t udst = smem_base + L::U_OFF + us * L::USTAGE;
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+          if (t + i * NPT < ITEMS) {
+            const uint4 v = lds128(psrc + src_off[i]);
+            const uint32_t m = 0xF0F0F0F0u;
+            sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+            sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&pempty[ps]);
+        mbar_arrive(&ufull[us]);
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_i8(BM, BN);
+      uint32_t it = 0, acc_it = 0;
+      for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++acc_it) {
+        const Unit w = decompose(p, u);
+        const int buf = acc_it & 1;
+        const uint32_t aph = (acc_it >> 1) & 1;
+        if (*abort_flag || !mbar_wait(&tempty[buf], aph ^ 1, p.spin_limit)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        bool ok = true;
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          const int us = it % UST;
+          const uint32_t uph = (it / UST) & 1;
+          if (!mbar_wait(&ufull[us], uph, p.spin_limit) || *abort_flag) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_base + L::U_OFF + us * L::USTAGE;
+          const uint32_t b_addr = a_addr + L::UA;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            mma_i8(d_tmem, desc_sw128(a_addr + kk * UMMA_K), desc_sw128(b_addr + kk * UMMA_K),
+                   IDESC, (kt > w.kt0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&uempty[us]);
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int row = warp * 32 + lane;                     // TMEM lane of this thread
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t acc_it = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++acc_it) {
+      const Unit w = decompose(p, u);
+      const int buf = acc_it & 1;
+      const uint32_t aph = (acc_it >> 1) & 1;
+      if (threadIdx.x == 0) {
+        const bool ok = !*abort_flag && mbar_wait(&tfull[buf], aph, p.spin_limit);
+        if (!ok) *abort_flag = 1;
+        bcast[0] = ok ? 1 : 0;
+      }
+      named_bar_sync(1, EPI_WARPS * 32);
+      const bool ok = bcast[0] != 0;
+      named_bar_sync(1, EPI_WARPS * 32);
+      if (!ok) break;
+      tc_fence_after();
+
+      // Coordinates: the TMEM lane indexes the A-side row, the column the B side.
+      const int a_row = w.ta * BM + row;
+      const bool a_valid = a_row < p.rowsA;
+      const bool split = p.splits > 1;
+      float lane_scale = 0.f;
+      if (a_valid) lane_scale = p.swap ? p.w_scale[a_row] : p.a_scale[a_row];
+#pragma unroll 1
+      for (int c = 0; c < BN / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(lane_addr + static_cast<uint32_t>(buf * BN + c * 16), v);
+        tmem_ld_wait();
+        const int b0 = w.tb * BN + c * 16;                 // first B-side index of chunk
+        if (!a_valid || b0 >= p.rowsB) continue;
+        if (!p.swap) {
+          // thread = token m, columns = channels n0..n0+15 (N % 16 == 0: all valid)
+          const int m = a_row, n0 = b0;
+          if (split) {
+            int* dst = p.ws_acc + static_cast<int64_t>(m) * p.N + n0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) atomicAdd(dst + j, static_cast<int>(v[j]) >> 8);
+          } else if (p.out_i32) {
+            int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
+                                                static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_int4(static_cast<int>(v[4 * j]) >> 8, static_cast<int>(v[4 * j + 1]) >> 8,
+                                 static_cast<int>(v[4 * j + 2]) >> 8,
+                                 static_cast<int>(v[4 * j + 3]) >> 8);
+          } else {
+            const float4* sw4 = reinterpret_cast<const float4*>(p.w_scale + n0);
+            uint32_t packed[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 s = __ldg(sw4 + j);
+              const float sj[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const int k = 4 * j + e;
+                const float f0 = static_cast<float>(static_cast<int>(v[k]) >> 8) * lane_scale * sj[e];
+                const float f1 =
+                    static_cast<float>(static_cast<int>(v[k + 1]) >> 8) * lane_scale * sj[e + 1];
+                __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+                packed[k / 2] = *reinterpret_cast<uint32_t*>(&h);
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                  static_cast<int64_t>(m) * p.N + n0);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          }
+        } else {
+          // thread = channel n, columns = tokens m0..m0+15
+          const int n = a_row;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = b0 + j;
+            if (m >= p.M) break;
+            const int acc = static_cast<int>(v[j]) >> 8;
+            const int64_t o = static_cast<int64_t>(m) * p.N + n;
+            if (split) {
+              atomicAdd(p.ws_acc + o, acc);
+            } else if (p.out_i32) {
+              static_cast<int*>(p.out)[o] = acc;
+            } else {
+              const float f = static_cast<float>(acc) * __ldg(p.a_scale + m) * lane_scale;
+              static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(f);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+
+      if (split) {
+        // Last of the p.splits CTAs of this tile applies the epilogue.
+        __threadfence();
+        named_bar_sync(1, EPI_WARPS * 32);
+        const int tile = w.tb * p.tilesA + w.ta;
+        if (threadIdx.x == 0) {
+          const unsigned old = atomicAdd(p.ws_cnt + tile, 1u);
+          bcast[1] = (old == static_cast<unsigned>(p.splits - 1)) ? 1 : 0;
+        }
+        named_bar_sync(1, EPI_WARPS * 32);
+        const bool last = bcast[1] != 0;
+        named_bar_sync(1, EPI_WARPS * 32);
+        if (last) {
+          __threadfence();
+          if (a_valid) {
+            for (int j = 0; j < BN; ++j) {
+              const int b = w.tb * BN + j;
+              if (b >= p.rowsB) break;
+              const int m = p.swap ? b : a_row;
+              const int n = p.swap ? a_row : b;
+              const int64_t o = static_cast<int64_t>(m) * p.N + n;
+              const int acc = __ldcg(p.ws_acc + o);
+              __stcg(p.ws_acc + o, 0);
+              if (p.out_i32) {
+                static_cast<int*>(p.out)[o] = acc;
+              } else {
+                const float f = static_cast<float>(acc) * __ldg(p.a_scale + m) * __ldg(p.w_scale + n);
+                static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(f);
+              }
+            }
+          }
+          if (threadIdx.x == 0) p.ws_cnt[tile] = 0u;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    if (lane == 0) {
+      mma_commit(drain);                 // completes once every issued MMA has
+      mbar_wait(drain, 0, 0);            // finished writing tensor memory
+    }
+    __syncwarp();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+static bool make_map(CUtensorMap* map, const uint8_t* base, int rows, int64_t K,
+                     int box_rows) {
+  auto encode = host::tensor_map_encoder();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(KP), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    host::set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+template <int BN, int PST, int UST>
+static sq_status launch(const Plan& plan, const uint8_t* opA, const uint8_t* opB, int64_t K,
+                        Params prm, cudaStream_t stream) {
+  using L = Layout<BN, PST, UST>;
+  CUtensorMap mapA, mapB;
+  if (!make_map(&mapA, opA, prm.rowsA, K, BM) || !make_map(&mapB, opB, prm.rowsB, K, BN))
+    return SQ_ERR_CUDA;
+  auto kfn = w4a4_gemm_kernel<BN, PST, UST>;
+  static bool attr_done[64] = {};
+  const int dev = host::current_device();
+  if (dev < 0) return SQ_ERR_CUDA;
+  if (!attr_done[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute", e);
+    attr_done[dev & 63] = true;
+  }
+  kfn<<<plan.grid, NUM_THREADS, L::BYTES, stream>>>(mapA, mapB, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return host::cuda_fail("w4a4_gemm launch", e);
+  return SQ_OK;
+}
+
+static int pick_bn_swap(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
+  Plan pl{};
+  pl.swap = M <= 128;
+  pl.bn = pl.swap ? pick_bn_swap(M) : 256;
+  const int64_t rowsA = pl.swap ? N : M, rowsB = pl.swap ? M : N;
+  pl.tilesA = static_cast<int>((rowsA + BM - 1) / BM);
+  pl.tilesB = static_cast<int>((rowsB + pl.bn - 1) / pl.bn);
+  pl.KT = static_cast<int>(K / BK);
+  const int64_t base = static_cast<int64_t>(pl.tilesA) * pl.tilesB;
+  int splits = 1;
+  if (have_ws && base < 2 * num_sms) {
+    // choose the split that best fills whole waves, with >= 4 k-tiles each
+    double best = -1.0;
+    for (int s = 1; s <= 16 && s <= pl.KT / 4; ++s) {
+      const int64_t units = base * s;
+      const int64_t waves = (units + num_sms - 1) / num_sms;
+      double eff = static_cast<double>(units) / static_cast<double>(waves * num_sms);
+      eff -= 0.01 * (s - 1);                       // mild preference for fewer splits
+      if (eff > best + 1e-9) {
+        best = eff;
+        splits = s;
+      }
+    }
+  }
+  pl.kps = (pl.KT + splits - 1) / splits;
+  pl.splits = (pl.KT + pl.kps - 1) / pl.kps;
+  pl.units = static_cast<int>(base * pl.splits);
+  pl.grid = static_cast<int>(pl.units < num_sms ? pl.units : num_sms);
+  return pl;
+}
+
+size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= 0 || N <= 0 || K < BK) return 0;
+  Plan pl = plan_gemm(M, N, K, true, num_sms);
+  if (pl.splits <= 1) return 0;
+  const size_t acc = static_cast<size_t>(M) * static_cast<size_t>(N) * 4;
+  const size_t cnt = static_cast<size_t>(pl.tilesA) * pl.tilesB * 4;
+  return ((acc + 255) & ~static_cast<size_t>(255)) + ((cnt + 255) & ~static_cast<size_t>(255));
+}
+
+sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
+              int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
+              size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
+              const Plan* forced) {
+  Plan pl = forced ? *forced : plan_gemm(M, N, K, ws != nullptr, num_sms);
+  Params prm{};
+  prm.swap = pl.swap;
+  prm.rowsA = static_cast<int>(pl.swap ? N : M);
+  prm.rowsB = static_cast<int>(pl.swap ? M : N);
+  prm.tilesA = pl.tilesA;
+  prm.tilesB = pl.tilesB;
+  prm.KT = pl.KT;
+  prm.splits = pl.splits;
+  prm.kps = pl.kps;
+  prm.units = pl.units;
+  prm.M = static_cast<int>(M);
+  prm.N = static_cast<int>(N);
+  prm.a_scale = a_scale;
+  prm.w_scale = w_scale;
+  prm.out = out;
+  prm.out_i32 = out_i32;
+  prm.spin_limit = spin_limit;
+  if (pl.splits > 1) {
+    const size_t acc = static_cast<size_t>(M) * static_cast<size_t>(N) * 4;
+    const size_t acc_al = (acc + 255) & ~static_cast<size_t>(255);
+    const size_t need = acc_al + ((static_cast<size_t>(pl.tilesA) * pl.tilesB * 4 + 255) &
+                                  ~static_cast<size_t>(255));
+    if (ws == nullptr || ws_bytes < need) {
+      host::set_error("split-K needs %zu workspace bytes, got %zu", need, ws_bytes);
+      return SQ_ERR_WORKSPACE;
+    }
+    prm.ws_acc = static_cast<int*>(ws);
+    prm.ws_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + acc_al);
+  }
+  const uint8_t* opA = pl.swap ? w_q : a_q;
+  const uint8_t* opB = pl.swap ? a_q : w_q;
+  switch (pl.bn) {
+    case 16: return launch<16, 8, 3>(pl, opA, opB, K, prm, stream);
+    case 32: return launch<32, 8, 3>(pl, opA, opB, K, prm, stream);
+    case 64: return launch<64, 6, 3>(pl, opA, opB, K, prm, stream);
+    case 128: return launch<128, 4, 3>(pl, opA, opB, K, prm, stream);
+    case 256: return launch<256, 4, 2>(pl, opA, opB, K, prm, stream);
+    default: break;
+  }
+  host::set_error("no kernel for tile width %d", pl.bn);
+  return SQ_ERR_UNSUPPORTED_SHAPE;
+}
+
+}  // namespace gemm
+}  // namespace sq

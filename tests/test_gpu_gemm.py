@@ -1,0 +1,141 @@
+"""GPU parity of sq_w4a4_linear against the oracle's exact integer GEMM.
+
+Operands are random packed bytes from the shared generator; both sides read
+the same bytes.  int32 accumulators must match bit for bit; the bf16 output
+must sit within the Frobenius bound of the oracle's float64 dequantized
+result.  Shapes cover the swap (small M, split-K) and the large-M paths, tile
+tails along M and N, and the full down_proj size on sampled rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests import parity as P
+from workloads import synthetic as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _operands(M, N, K, seed):
+    a = W.random_packed(seed, M, K)
+    w = W.random_packed(seed + 1, N, K)
+    sa = W.random_scales(seed + 2, M)
+    sw = W.random_scales(seed + 3, N)
+    return a, w, sa, sw
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 16, 128), (3, 48, 256), (16, 256, 256), (17, 272, 384), (64, 512, 1024),
+    (100, 4096, 12288), (128, 1024, 4096), (129, 272, 256), (256, 4096, 12288),
+    (300, 528, 1024), (1000, 768, 512), (2048, 1024, 4096),
+])
+def test_int32_bit_exact(cuda_ok, M, N, K):
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 100 + M + N)
+    acc = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True)
+    assert sq.device_status() == 0
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (33, 272, 512), (512, 768, 1024)])
+def test_bf16_epilogue(cuda_ok, M, N, K):
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 7 + M)
+    out = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw))
+    _, ref = O.w4a4_linear(a, sa, w, sw)
+    got = out.float().cpu().numpy()
+    P.check_fro(got, ref)
+    # each element is the bf16 rounding of the float32 product: within 2^-8 relative
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-30)
+
+
+def test_no_workspace_path_matches(cuda_ok):
+    import rotation_ptq_b200 as sq
+    M, N, K = 16, 1024, 4096
+    a, w, sa, sw = _operands(M, N, K, 55)
+    x = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True, use_workspace=False)
+    y = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True)
+    assert torch.equal(x, y)
+
+
+def test_workspace_left_zero_and_repeatable(cuda_ok):
+    import rotation_ptq_b200 as sq
+    M, N, K = 4, 4096, 12288
+    nbytes = sq.w4a4_workspace_bytes(M, N, K)
+    assert nbytes > 0
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    a, w, sa, sw = _operands(M, N, K, 77)
+    r1 = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True, workspace=ws)
+    r2 = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) == 0
+    assert torch.equal(r1, r2)
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    assert np.array_equal(r1.cpu().numpy().astype(np.int64), ref)
+
+
+def test_extreme_codes_full_k(cuda_ok):
+    # every code -8: acc = 64 K exactly (the largest magnitude the format allows)
+    import rotation_ptq_b200 as sq
+    M, N, K = 130, 48, 12288
+    a = np.full((M, K // 2), 0x88, np.uint8)
+    w = np.full((N, K // 2), 0x88, np.uint8)
+    w[1] = 0x77                                  # all +7
+    ones_m, ones_n = np.ones(M, np.float32), np.ones(N, np.float32)
+    acc = sq.w4a4_linear(_dev(a), _dev(ones_m), _dev(w), _dev(ones_n), out_int32=True)
+    got = acc.cpu().numpy()
+    assert np.all(got[:, 0] == 64 * K) and np.all(got[:, 1] == -56 * K)
+
+
+def test_down_proj_full_size_sampled_rows(cuda_ok):
+    import rotation_ptq_b200 as sq
+    M, N, K = 4096, 4096, 12288
+    a, w, sa, sw = _operands(M, N, K, 2024)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    acc = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True).cpu().numpy()
+    out = sq.w4a4_linear(da, dsa, dw, dsw).float().cpu().numpy()
+    rows = P.sample_rows(M, 48, seed=5)
+    wc = O.unpack_int4(w)
+    ref_acc = O.gemm_int(O.unpack_int4(a[rows]), wc)
+    assert np.array_equal(acc[rows].astype(np.int64), ref_acc)
+    P.check_fro(out[rows], O.dequant(ref_acc, sa[rows], sw))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 64, 256, 1024, 4096, 16384])
+@pytest.mark.parametrize("shape", ["down_proj", "gate_up"])
+def test_m_sweep_int32_sampled(cuda_ok, M, shape):
+    import rotation_ptq_b200 as sq
+    N, K = (4096, 12288) if shape == "down_proj" else (24576, 4096)
+    a, w, sa, sw = _operands(M, N, K, 9000 + M)
+    acc = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True)
+    rows = P.sample_rows(M, 16, seed=M)
+    got = acc[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64)
+    ref = O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w))
+    assert np.array_equal(got, ref)
+
+
+def test_forced_timeout_reports_status_and_recovers(cuda_ok):
+    # One poll per wait: the pipeline's first waits run out, every role
+    # returns, the kernel records SQ_ERR_TIMEOUT, and the context stays usable.
+    import rotation_ptq_b200 as sq
+    M, N, K = 256, 512, 1024
+    a, w, sa, sw = _operands(M, N, K, 31)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    assert sq.device_status() == 0
+    sq.debug_set_spin_limit(1)
+    try:
+        sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True, use_workspace=False)
+        status = sq.device_status()
+    finally:
+        sq.debug_set_spin_limit(0)
+    assert status == 5                      # SQ_ERR_TIMEOUT
+    acc = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+    assert sq.device_status() == 0
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)

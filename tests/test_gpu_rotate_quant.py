@@ -1,0 +1,112 @@
+"""GPU parity of sq_rotate_quant against the oracle (dense float64 Hadamard).
+
+Codes follow the graded rule (equal, or +-1 at a rounding boundary with a
+mismatch rate <= 1e-5); scales agree to 1e-5 relative; packing of equal codes
+is bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests import parity as P
+from workloads import synthetic as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(sq, x_cpu, ns, np2, clip=1.0):
+    hs = sq.paley_h12() if ns == 12 else (None if ns == 1 else O.sylvester(ns).astype(np.int8))
+    a_q, a_s = sq.rotate_quant(x_cpu.cuda(), hs, np2, clip)
+    assert sq.device_status() == 0
+    return a_q.cpu().numpy(), a_s.cpu().numpy()
+
+
+def _check(aq, asc, x64, ns, np2, clip=1.0):
+    ref_p, ref_s, ref_c, ref_v = O.rotate_quant(x64, ns, np2, clip)
+    P.check_scales(asc, ref_s)
+    got = O.unpack_int4(aq)
+    P.check_codes(got, ref_c, ref_v)
+    same = (got == ref_c).reshape(got.shape[0], -1, 2).all(axis=2)
+    assert np.array_equal(aq[same], ref_p[same])     # packing of equal codes is exact
+    return ref_c
+
+
+def test_tiny_fp32_sylvester256(cuda_ok):
+    import rotation_ptq_b200 as sq
+    wl = W.tiny_linear()
+    aq, asc = _run(sq, wl.x, 1, 256)
+    _check(aq, asc, wl.x.numpy().astype(np.float64), 1, 256)
+
+
+def test_down_proj_full_size_sampled_rows(cuda_ok):
+    import rotation_ptq_b200 as sq
+    wl = W.down_proj(with_weights=False)
+    aq, asc = _run(sq, wl.x, 12, 1024)
+    rows = P.sample_rows(wl.M, 40, seed=1)
+    x64 = wl.x[torch.from_numpy(rows)].double().numpy()
+    _check(aq[rows], asc[rows], x64, 12, 1024)
+
+
+@pytest.mark.parametrize("M", [1, 3, 33])
+def test_down_proj_ragged_m(cuda_ok, M):
+    import rotation_ptq_b200 as sq
+    wl = W.down_proj(M=M, with_weights=False, seed=77 + M)
+    aq, asc = _run(sq, wl.x, 12, 1024)
+    _check(aq, asc, wl.x.double().numpy(), 12, 1024)
+
+
+def test_quant_only_r1_folded_all_rows(cuda_ok):
+    import rotation_ptq_b200 as sq
+    wl = W.r1_folded(M=8192, Ns=(16,))[0]
+    aq, asc = _run(sq, wl.x, 1, 1)
+    _check(aq, asc, wl.x.double().numpy(), 1, 1)
+
+
+@pytest.mark.parametrize("ns,np2,K", [(1, 128, 256), (12, 16, 384), (12, 64, 768 * 2),
+                                      (1, 1024, 2048), (4, 8, 96), (1, 1, 160)])
+def test_generic_groups(cuda_ok, ns, np2, K):
+    import rotation_ptq_b200 as sq
+    rng = np.random.default_rng(ns * 1000 + np2)
+    x = torch.from_numpy(rng.standard_t(3, (37, K)).astype(np.float32))
+    aq, asc = _run(sq, x, ns, np2)
+    _check(aq, asc, x.double().numpy(), ns, np2)
+
+
+def test_clip_ratio_clamps(cuda_ok):
+    import rotation_ptq_b200 as sq
+    wl = W.tiny_linear(seed=5)
+    aq, asc = _run(sq, wl.x, 1, 256, clip=0.9)
+    codes = _check(aq, asc, wl.x.double().numpy(), 1, 256, clip=0.9)
+    assert (codes == -8).any() or (codes == 7).sum() > 16
+
+
+def test_zero_and_constant_rows(cuda_ok):
+    import rotation_ptq_b200 as sq
+    x = torch.zeros((4, 4096), dtype=torch.bfloat16)
+    x[1] = 3.0
+    x[2, 17] = -2.0
+    aq, asc = _run(sq, x, 1, 1)
+    _check(aq, asc, x.double().numpy(), 1, 1)
+    assert asc[0] == 1.0 and np.all(aq[0] == 0)
+
+
+def test_weights_quantization_matches_oracle_rows(cuda_ok):
+    # offline fold W H / sqrt(g) + per-channel RTN, done by the same kernel
+    import rotation_ptq_b200 as sq
+    rng = np.random.default_rng(42)
+    w = torch.from_numpy(rng.normal(0, 0.02, (64, 12288)).astype(np.float32))
+    wq, ws = sq.quantize_weights(w.cuda(), sq.paley_h12(), 1024)
+    ref_p, ref_s, ref_c = O.quantize_weights(w.double().numpy(), 12, 1024)
+    P.check_scales(ws.cpu().numpy(), ref_s)
+    _, _, _, ref_v = O.rotate_quant(w.double().numpy(), 12, 1024)
+    P.check_codes(O.unpack_int4(wq.cpu().numpy()), ref_c, ref_v)
+
+
+def test_strided_rows(cuda_ok):
+    import rotation_ptq_b200 as sq
+    rng = np.random.default_rng(3)
+    big = torch.from_numpy(rng.standard_normal((8, 4096 + 64)).astype(np.float32)).to(torch.bfloat16)
+    view = big.cuda()[:, :4096]
+    a_q, a_s = sq.rotate_quant(view, None, 1, 1.0)
+    _check(a_q.cpu().numpy(), a_s.cpu().numpy(), big[:, :4096].double().numpy(), 1, 1)

@@ -202,3 +202,20 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     """float64 values rounded to bf16 and returned as float64 (a dtype cast only)."""
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.bfloat16) \
         .to(torch.float64).numpy()
+
+
+def random_packed(seed: int, rows: int, K: int) -> np.ndarray:
+    """Uniform random bytes [rows, K/2] (GEMM test input).
+
+    Every byte is a valid pair of packed signed INT4 codes, so no packing
+    arithmetic is needed to produce operands; each side reads the bytes with
+    its own unpacking.
+    """
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 256, size=(rows, K // 2), dtype=np.int64).astype(np.uint8)
+
+
+def random_scales(seed: int, n: int) -> np.ndarray:
+    """Positive float32 scales spread over two decades (GEMM epilogue test input)."""
+    rng = np.random.default_rng(seed)
+    return (10.0 ** rng.uniform(-3, -1, n)).astype(np.float32)
