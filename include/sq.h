@@ -140,6 +140,34 @@ sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t
 size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ---------------------------------------------------------------------------
+ * sq_w4a4_linear_noalloc -- sq_w4a4_linear for callers that cannot allocate.
+ *
+ * The paper has no counterpart to this call; it is a deployment variant of
+ * the same GEMM.  Some callers may not allocate device memory at all: a
+ * plug-in that only receives buffers from its host framework, a runtime that
+ * forbids allocation once it has started, or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not allowed.
+ * sq_w4a4_linear needs a caller workspace for split-K at small M; this call
+ * instead takes that scratch from one static device array of 8 MiB + 64 KiB
+ * that every GPU loading the library holds until the process exits.  Same
+ * arguments (minus the workspace), shape rules and results as sq_w4a4_linear.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *     routine is called.
+ *   - A shape whose split-K scratch would exceed the array is rejected with
+ *     SQ_ERR_WORKSPACE before anything is enqueued (sq_last_error gives both
+ *     sizes).  Shapes that need no scratch always run.
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress, with that device current).  Make that first
+ *     call before any stream capture begins.
+ *   - All calls on a device share the one array; each clears the part it
+ *     uses on `stream` first.  Calls whose work overlaps on the GPU (other
+ *     streams or host threads) race on the array: order them.
+ * ------------------------------------------------------------------------- */
+sq_status sq_w4a4_linear_noalloc(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                                 const float* w_scale, int64_t M, int64_t N, int64_t K,
+                                 void* out, sq_out_kind kind, void* stream);
+
+/* ---------------------------------------------------------------------------
  * sq_kv_rotate_quant -- RoPE, head-wise Hadamard R3 on Q and K, and the
  * asymmetric 4-bit KV cache.
  *
