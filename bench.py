@@ -270,6 +270,49 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
                       % (rows, cols, n, t_rot + t_gemm), "full_step_s": full_s}
 
 
+PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
+                 "decode_gemm_m1", "decode_gemm_m16", "rotate_quant_r4", "kv_rotate_quant")
+
+
+def run_profile_case(case, steps, warmup):
+    """Launch one kernel of the path `warmup + steps` times (for ncu captures)."""
+    import torch
+    import rotation_ptq_b200 as sq
+    from workloads import synthetic as W
+    torch.cuda.set_device(0)
+    if case.startswith("down_proj_gemm") or case.startswith("decode_gemm"):
+        m = {"decode_gemm_m1": 1, "decode_gemm_m16": 16}.get(case, M)
+        a = torch.from_numpy(W.random_packed(11, m, K)).cuda()
+        w = torch.from_numpy(W.random_packed(12, N, K)).cuda()
+        sa = torch.from_numpy(W.random_scales(13, m)).cuda()
+        sw = torch.from_numpy(W.random_scales(14, N)).cuda()
+        out = torch.empty((m, N), dtype=torch.bfloat16, device="cuda")
+        sq.debug_set_gemm_path({"down_proj_gemm_1cta": 1, "down_proj_gemm_pair": 2}.get(case, 0))
+        fn = lambda: sq.w4a4_linear(a, sa, w, sw, out=out)  # noqa: E731
+    elif case == "rotate_quant_r4":
+        x = W.down_proj(M=M, K=K, N=N, with_weights=False).x.cuda()
+        hs = sq.paley_h12()
+        a_q = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        a_s = torch.empty((M,), dtype=torch.float32, device="cuda")
+        fn = lambda: sq.rotate_quant(x, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
+    elif case == "kv_rotate_quant":
+        kvw = W.kv_path()
+        q, k, v, pos = kvw.q.cuda(), kvw.k.cuda(), kvw.v.cuda(), kvw.pos.cuda()
+        cos, sin = sq.rope_tables(kvw.theta, kvw.max_pos, 128)
+        o = sq.kv_rotate_quant(q, k, v, pos, cos, sin)
+        fn = lambda: sq.kv_rotate_quant(q, k, v, pos, cos, sin, out=o)  # noqa: E731
+    else:
+        raise SystemExit("unknown case %s" % case)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup + steps):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    if sq.device_status() != 0:
+        raise SystemExit("device status set")
+    print("profile case %s: %d launches" % (case, warmup + steps))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -278,7 +321,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kv", action="store_true")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="launch one kernel of the path warmup+steps times and exit (for ncu)")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.steps, args.warmup)
+        return
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))

@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     SQ_OUT_BF16,
     SQ_OUT_I32,
     SqError,
+    debug_set_gemm_path,
     debug_set_spin_limit,
     device_status,
     kv_dequant,

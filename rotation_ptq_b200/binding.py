@@ -19,7 +19,7 @@ library_path = os.path.join(HERE, "libsq.so")
 if not os.path.exists(library_path):
     raise ImportError(
         "rotation_ptq_b200: CUDA library %s is missing; build it with "
-        "`python -m rotation_ptq_b200.build` (there is no CPU fallback)" % library_path)
+        "`python rotation_ptq_b200/build.py` (there is no CPU fallback)" % library_path)
 
 lib = ctypes.CDLL(library_path)
 
@@ -54,6 +54,8 @@ lib.sq_device_status.restype = _i32
 lib.sq_device_status.argtypes = [_vp]
 lib.sq_debug_set_spin_limit.restype = None
 lib.sq_debug_set_spin_limit.argtypes = [ctypes.c_uint32]
+lib.sq_debug_set_gemm_path.restype = None
+lib.sq_debug_set_gemm_path.argtypes = [ctypes.c_int]
 
 
 class SqError(RuntimeError):
@@ -243,3 +245,8 @@ def device_status(device=None) -> int:
 
 def debug_set_spin_limit(polls: int) -> None:
     lib.sq_debug_set_spin_limit(int(polls))
+
+
+def debug_set_gemm_path(path: int) -> None:
+    """0 = automatic, 1 = one-CTA tiles, 2 = CTA-pair tiles (large M)."""
+    lib.sq_debug_set_gemm_path(int(path))

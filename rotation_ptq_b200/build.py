@@ -1,7 +1,8 @@
 """Build the in-tree CUDA library ``libsq.so`` for sm_100a with nvcc.
 
-Usage: ``python -m rotation_ptq_b200.build [--verbose]``.  The library is
-written next to this file so that it travels with the source tree.
+Usage: ``python rotation_ptq_b200/build.py [--verbose] [--ptxas]`` (run it as a
+script: importing the package would first load the library being rebuilt).
+The library is written next to this file so that it travels with the tree.
 """
 from __future__ import annotations
 

@@ -189,34 +189,80 @@ __device__ __forceinline__ int xoff(int c) {
 }
 
 // One row of 12,288 channels, c = i*1024 + j, j = (j9..j0).
+// Rows are prefetched one ahead with a 1-D bulk async copy (24 KB) into a
+// two-slot shared-memory ring, so HBM latency overlaps the current row.
 // Phase A (threads 0..127, t = j0..j6): the 96 values of all 12 i and the
-//   top three j bits (jt = j7..j9) are loaded from global memory; H8 over jt
+//   top three j bits (jt = j7..j9) are read from the staged row; H8 over jt
 //   and H12 over i run in registers; the result goes to the exchange buffer.
 // Phase B (threads 0..191, u = (i, jt, j6)): 64 consecutive channels
 //   (j0..j5) come back from the buffer; H64 runs in registers and the j6
 //   stage pairs lanes u and u^1 through one shuffle.  Then the row's absmax
 //   (block reduction), the scale, and 64 codes = 32 bytes per thread.
 // The 1/sqrt(12288) normalisation is folded into the quantizer multiplier.
+// CLAMP is false when clip == 1: then |y / scale| <= 7 up to rounding, so the
+// codes already lie in [-7, 7].
 constexpr int H12_THREADS = 192;
+constexpr int H12_ROW_BYTES = 12288 * 2;
+constexpr int H12_SMEM = 12288 * 4 + 2 * H12_ROW_BYTES + 64;
 
-template <int MINB>
-__global__ void __launch_bounds__(H12_THREADS, MINB)
+// Two codes per byte from the low bytes of magic-rounded floats (the low
+// byte holds the code in two's complement): byte = lo nibble of a | lo
+// nibble of b << 4; four such bytes gathered into one word.
+__device__ __forceinline__ uint32_t pack8(const uint32_t* u) {
+  uint32_t b[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) b[k] = (u[2 * k] & 0x0Fu) | ((u[2 * k + 1] << 4) & 0xF0u);
+  const uint32_t lo = __byte_perm(b[0], b[1], 0x3340);
+  const uint32_t hi = __byte_perm(b[2], b[3], 0x3340);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+template <bool CLAMP>
+__global__ void __launch_bounds__(H12_THREADS, 2)
     rq_h12x1024_kernel(const uint16_t* __restrict__ x, int64_t ldx, int M, float norm,
-                       float clip, uint8_t* __restrict__ aq, float* __restrict__ ascale) {
-  extern __shared__ __align__(16) float X[];      // 12,288 floats (dynamic)
+                       float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
+                       float* __restrict__ ascale) {
+  extern __shared__ __align__(128) uint8_t rq_smem[];
+  float* X = reinterpret_cast<float*>(rq_smem);                        // 12,288 floats
+  uint16_t* stage = reinterpret_cast<uint16_t*>(rq_smem + 12288 * 4);  // 2 staged rows
+  uint64_t* bar = reinterpret_cast<uint64_t*>(rq_smem + 12288 * 4 + 2 * H12_ROW_BYTES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
   __shared__ float red[H12_THREADS / 32];
   const int tid = threadIdx.x;
-  for (int m = blockIdx.x; m < M; m += gridDim.x) {
-    const uint16_t* xr = x + static_cast<int64_t>(m) * ldx;
+
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    if (blockIdx.x < M) {
+      mbar_arrive_expect_tx(&bar[0], H12_ROW_BYTES);
+      bulk_g2s(stage, x + static_cast<int64_t>(blockIdx.x) * ldx, H12_ROW_BYTES, &bar[0]);
+    }
+  }
+  __syncthreads();
+  uint32_t iter = 0;
+  for (int m = blockIdx.x; m < M; m += gridDim.x, ++iter) {
+    const int slot = iter & 1;
+    if (tid == 0 && m + gridDim.x < M) {
+      // the other slot was read by phase A of the previous row, which every
+      // thread finished before the barrier after it
+      mbar_arrive_expect_tx(&bar[slot ^ 1], H12_ROW_BYTES);
+      bulk_g2s(stage + (slot ^ 1) * 12288, x + static_cast<int64_t>(m + gridDim.x) * ldx,
+               H12_ROW_BYTES, &bar[slot ^ 1]);
+    }
     if (tid < 128) {
+      if (!mbar_wait(&bar[slot], (iter >> 1) & 1, spin_limit)) *abort_flag = 1;
+      const uint16_t* xr = stage + slot * 12288;
       // z[i][q] = (value at jt = q, value at jt = q + 4)
       f2 z[12][4];
 #pragma unroll
       for (int i = 0; i < 12; ++i) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint32_t lo = __ldg(xr + i * 1024 + q * 128 + tid);
-          const uint32_t hi = __ldg(xr + i * 1024 + (q + 4) * 128 + tid);
+          const uint32_t lo = xr[i * 1024 + q * 128 + tid];
+          const uint32_t hi = xr[i * 1024 + (q + 4) * 128 + tid];
           z[i][q].x = __uint_as_float(lo << 16);
           z[i][q].y = __uint_as_float(hi << 16);
         }
@@ -270,6 +316,7 @@ __global__ void __launch_bounds__(H12_THREADS, MINB)
       }
     }
     __syncthreads();
+    if (*abort_flag) break;
     // Phase B: segment u = 64 consecutive channels starting at c0 = 64 u
     const int u = tid;
     f2 v[32];                                   // v[j] = (value j, value j + 32)
@@ -315,25 +362,31 @@ __global__ void __launch_bounds__(H12_THREADS, MINB)
     const float s = row_scale(amax * norm, clip);
     const float k = norm * __frcp_rn(s);         // y_unnormalised -> y / scale
     const f2 k2{k, k};
-    // codes: clamp to [-8, 7], then 1.5 * 2^23 + v rounds to the nearest
-    // integer (ties to even) and leaves it in the low mantissa bits
-    uint32_t w[8];
-#pragma unroll
-    for (int g = 0; g < 8; ++g) w[g] = 0;
+    const f2 magic{12582912.f, 12582912.f};      // 1.5 * 2^23: round to nearest even
+    uint32_t ux[32], uy[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       f2 c = mul2(v[j], k2);
-      c.x = fminf(fmaxf(c.x, -8.f), 7.f);
-      c.y = fminf(fmaxf(c.y, -8.f), 7.f);
-      c = add2(c, f2{12582912.f, 12582912.f});
-      const uint32_t nx = __float_as_uint(c.x) & 0xFu, ny = __float_as_uint(c.y) & 0xFu;
-      w[j >> 3] |= nx << (4 * (j & 7));           // channel j
-      w[4 + (j >> 3)] |= ny << (4 * (j & 7));     // channel j + 32
+      if (CLAMP) {
+        c.x = fminf(fmaxf(c.x, -8.f), 7.f);
+        c.y = fminf(fmaxf(c.y, -8.f), 7.f);
+      }
+      c = add2(c, magic);
+      ux[j] = __float_as_uint(c.x);              // channel j
+      uy[j] = __float_as_uint(c.y);              // channel j + 32
     }
     uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + u * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    dst[0] = make_uint4(pack8(ux), pack8(ux + 8), pack8(ux + 16), pack8(ux + 24));
+    dst[1] = make_uint4(pack8(uy), pack8(uy + 8), pack8(uy + 16), pack8(uy + 24));
     if (tid == 0) ascale[m] = s;
+  }
+  // every bulk copy issued must land before the CTA exits
+  if (tid == 0) {
+    const uint32_t n_issued = (M > static_cast<int>(blockIdx.x))
+        ? static_cast<uint32_t>((M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1)
+        : 0u;
+    for (uint32_t j = n_issued > 2 ? n_issued - 2 : 0u; j < n_issued; ++j)
+      mbar_wait(&bar[j & 1], (j >> 1) & 1, 0);
   }
 }
 
@@ -461,12 +514,13 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const int m = static_cast<int>(M), k = static_cast<int>(K);
   if (x_bf16 && n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small)) {
     const int grid = m < 2 * host::num_sms() ? m : 2 * host::num_sms();
-    constexpr int kSmem = 12288 * sizeof(float);
-    cudaError_t ea = cudaFuncSetAttribute(rq_h12x1024_kernel<2>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    const bool clamp = clip < 1.0f;
+    auto kfn = clamp ? rq_h12x1024_kernel<true> : rq_h12x1024_kernel<false>;
+    cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          H12_SMEM);
     if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
-    rq_h12x1024_kernel<2><<<grid, H12_THREADS, kSmem, stream>>>(
-        static_cast<const uint16_t*>(x), ld_x, m, norm, clip, a_q, a_scale);
+    kfn<<<grid, H12_THREADS, H12_SMEM, stream>>>(static_cast<const uint16_t*>(x), ld_x, m, norm,
+                                                 clip, host::spin_limit(), a_q, a_scale);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_h12x1024 launch", e);
   }

@@ -19,6 +19,7 @@ namespace host {
 
 static thread_local char t_err[512] = {0};
 static std::atomic<uint32_t> g_spin_limit{0};
+static std::atomic<int> g_gemm_path{0};
 
 void set_error(const char* fmt, ...) {
   va_list ap;
@@ -71,6 +72,8 @@ int num_sms() {
 
 uint32_t spin_limit() { return g_spin_limit.load(std::memory_order_relaxed); }
 
+int gemm_path() { return g_gemm_path.load(std::memory_order_relaxed); }
+
 }  // namespace host
 }  // namespace sq
 
@@ -108,6 +111,10 @@ int sq_version(void) { return (1 << 16) | 0; }
 
 void sq_debug_set_spin_limit(uint32_t polls) {
   sq::host::g_spin_limit.store(polls, std::memory_order_relaxed);
+}
+
+void sq_debug_set_gemm_path(int path) {
+  sq::host::g_gemm_path.store(path == 1 || path == 2 ? path : 0, std::memory_order_relaxed);
 }
 
 sq_status sq_device_status(void* stream) {
@@ -160,8 +167,8 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
     }
   }
   const int64_t g = static_cast<int64_t>(n_small) * n_pow2;
-  if (K % 32 != 0 || K < 32 || K > 65536 || K % g != 0) {
-    set_error("K=%lld must be a multiple of 32 in [32, 65536] and of the group %lld",
+  if (K % 32 != 0 || K < 32 || K > 32768 || K % g != 0) {
+    set_error("K=%lld must be a multiple of 32 in [32, 32768] and of the group %lld",
               (long long)K, (long long)g);
     return SQ_ERR_UNSUPPORTED_SHAPE;
   }

@@ -24,6 +24,8 @@ int current_device();
 int num_sms();
 // Poll limit for device waits set by sq_debug_set_spin_limit (0 = default).
 uint32_t spin_limit();
+// GEMM kernel selection set by sq_debug_set_gemm_path (0 = automatic).
+int gemm_path();
 
 }  // namespace host
 

@@ -40,6 +40,8 @@ constexpr int BM = 128;          // MMA M: TMEM lanes
 constexpr int BK = 128;          // int8 K elements per stage (one 128-byte swizzle row)
 constexpr int KP = BK / 2;       // packed bytes per row per stage
 constexpr int UMMA_K = 32;       // K per tcgen05.mma kind::i8
+constexpr int KM = 2;            // k-tiles per packed stage (one TMA box per operand)
+constexpr int PROW = KP * KM;    // packed bytes per row per packed stage (128: one swizzle span)
 constexpr int EPI_WARPS = 4;
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
@@ -67,8 +69,8 @@ struct Params {
 
 template <int BN, int PST, int UST>
 struct Layout {
-  static constexpr int PA = BM * KP;                 // packed A bytes per stage
-  static constexpr int PB = BN * KP;
+  static constexpr int PA = BM * PROW;               // packed A bytes per stage
+  static constexpr int PB = BN * PROW;
   static constexpr int PSTAGE = PA + PB;
   static constexpr int UA = BM * BK;                 // int8 A bytes per stage
   static constexpr int UB = BN * BK;
@@ -184,11 +186,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == TMA_WARP) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0;                           // packed stages issued
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units && !*abort_flag; u += gridDim.x) {
         const Unit w = decompose(p, u);
-        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+        for (int kt = w.kt0; kt < w.kt1; kt += KM, ++it) {
           const int ps = it % PST;
           const uint32_t ph = (it / PST) & 1;
           if (!mbar_wait(&pempty[ps], ph ^ 1, p.spin_limit)) {
@@ -210,49 +212,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= UNPACK_WARP0) {
     // ------------------------------------------------ unpack: INT4 -> INT8
-    constexpr int ITEMS = (BM + BN) * 4;                 // 16-byte packed chunks per stage
+    // A packed stage holds KM k-tiles: rows of 128 bytes, 16-byte chunks
+    // swizzled by the copy engine (chunk c of row r at c ^ (r % 8)).  Eight
+    // consecutive threads take eight consecutive rows, so both the swizzled
+    // reads and the swizzled int8 writes hit eight different bank groups.
+    constexpr int ROWS = BM + BN;
+    constexpr int ITEMS = ROWS * 4;                      // 16-byte chunks per k-tile
     constexpr int IPT = (ITEMS + NPT - 1) / NPT;
     const int t = threadIdx.x - UNPACK_WARP0 * 32;
     uint32_t src_off[IPT], dst_off0[IPT], dst_off1[IPT];
 #pragma unroll
     for (int i = 0; i < IPT; ++i) {
       const int idx = t + i * NPT;
-      const int row_all = idx >> 2, q = idx & 3;
-      // packed stage: rows of 64 bytes, A rows then B rows
-      src_off[i] = static_cast<uint32_t>(row_all * KP + q * 16);
+      const int q = idx / ROWS, row_all = idx % ROWS;
+      src_off[i] = static_cast<uint32_t>(row_all * PROW + ((q ^ (row_all & 7)) << 4));
       const bool is_a = row_all < BM;
       const int row = is_a ? row_all : row_all - BM;
       const uint32_t base = is_a ? 0u : static_cast<uint32_t>(L::UA);
       dst_off0[i] = base + sw128_off(row, 2 * q);
       dst_off1[i] = base + sw128_off(row, 2 * q + 1);
     }
-    uint32_t it = 0;
+    uint32_t it = 0, itp = 0;                    // k-tiles and packed stages consumed
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
       const Unit w = decompose(p, u);
-      for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
-        const int ps = it % PST, us = it % UST;
-        const uint32_t pph = (it / PST) & 1, uph = (it / UST) & 1;
-        if (!mbar_wait(&pfull[ps], pph, p.spin_limit) ||
-            !mbar_wait(&uempty[us], uph ^ 1, p.spin_limit) || *abort_flag) {
+      for (int kt = w.kt0; ok && kt < w.kt1; kt += KM, ++itp) {
+        const int ps = itp % PST;
+        const uint32_t pph = (itp / PST) & 1;
+        bool got = mbar_wait(&pfull[ps], pph, p.spin_limit);
+        got = __all_sync(0xffffffffu, got && !*abort_flag);
+        if (!got) {
           *abort_flag = 1;
           ok = false;
           break;
         }
         const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
-        const uint32_t udst = smem_base + L::U_OFF + us * L::USTAGE;
-#pragma unroll
-        for (int i = 0; i < IPT; ++i) {
-          if (t + i * NPT < ITEMS) {
-            const uint4 v = lds128(psrc + src_off[i]);
-            const uint32_t m = 0xF0F0F0F0u;
-            sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
-            sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+        const int nsub = min(KM, w.kt1 - kt);
+        for (int sub = 0; sub < nsub; ++sub, ++it) {
+          const int us = it % UST;
+          const uint32_t uph = (it / UST) & 1;
+          bool free_slot = mbar_wait(&uempty[us], uph ^ 1, p.spin_limit);
+          // the warp decides together: it arrives once per barrier below
+          free_slot = __all_sync(0xffffffffu, free_slot && !*abort_flag);
+          if (!free_slot) {
+            *abort_flag = 1;
+            ok = false;
+            break;
           }
+          const uint32_t udst = smem_base + L::U_OFF + us * L::USTAGE;
+          const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;   // chunk index + 4*sub
+#pragma unroll
+          for (int i = 0; i < IPT; ++i) {
+            if (t + i * NPT < ITEMS) {
+              const uint4 v = lds128(psrc + (src_off[i] ^ sub_x));
+              const uint32_t m = 0xF0F0F0F0u;
+              sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+              sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();                          // the warp's writes are ordered before
+          if (lane == 0) mbar_arrive_n(&ufull[us], 32);   // its one arrival
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&pempty[ps]);
-        mbar_arrive(&ufull[us]);
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive_n(&pempty[ps], 32);
       }
     }
   } else if (warp == MMA_WARP) {
@@ -385,7 +409,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&tempty[buf], 32);
 
       if (split) {
         // Last of the p.splits CTAs of this tile applies the epilogue.
@@ -438,6 +463,307 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------- CTA pairs
+//
+// Large M: a cluster of two CTAs computes one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads and widens its own 128
+// rows of A and its own 128 rows of B (half of N), so per SM the B bytes that
+// cross shared memory are halved against the one-CTA kernel.  The even CTA
+// issues the MMAs; both CTAs' unpack threads arrive on its ring barrier, its
+// commits arrive on the matching barriers of both CTAs, and each CTA drains
+// its own 128 accumulator rows from its own tensor memory.
+
+struct PairParams {
+  int rowsA, rowsB;        // M, N
+  int tilesM, tilesN;      // 256-wide tiles
+  int KT;
+  int units;
+  const float* a_scale;
+  const float* w_scale;
+  void* out;
+  int out_i32;
+  int M, N;
+  uint32_t spin_limit;
+};
+
+template <int PST, int UST>
+struct PairLayout {
+  static constexpr int HALF = 128;                    // rows of A and of B per CTA
+  static constexpr int PA = HALF * PROW;
+  static constexpr int PSTAGE = 2 * HALF * PROW;      // packed A + packed B (KM k-tiles)
+  static constexpr int UA = HALF * BK;
+  static constexpr int USTAGE = 2 * HALF * BK;        // int8 A + int8 B
+  static constexpr int U_OFF = 0;
+  static constexpr int P_OFF = UST * USTAGE;
+  static constexpr int BAR_OFF = P_OFF + PST * PSTAGE;
+  static constexpr int NBAR = 2 * PST + 2 * UST + 5;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = MISC_OFF + 32 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;          // two 256-column accumulators
+  static_assert(BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <int PST, int UST>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA,
+                          const __grid_constant__ CUtensorMap mapB, const PairParams p) {
+  using L = PairLayout<PST, UST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* pempty = pfull + PST;
+  uint64_t* ufull = pempty + PST;      // used on the even CTA: both CTAs arrive
+  uint64_t* uempty = ufull + UST;      // both CTAs: arrival from the pair commit
+  uint64_t* tfull = uempty + UST;      // both CTAs: arrival from the pair commit
+  uint64_t* tempty = tfull + 2;        // used on the even CTA: both CTAs' epilogues arrive
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair_id = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PST; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], NPT);
+    }
+    for (int s = 0; s < UST; ++s) {
+      mbar_init(&ufull[s], 2 * NPT);
+      mbar_init(&uempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * EPI_WARPS * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();                      // both CTAs' barriers and tensor memory are ready
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      uint32_t it = 0;                           // packed stages issued
+      bool ok = true;
+      for (int u = pair_id; ok && u < p.units && !*abort_flag; u += num_pairs) {
+        const int tm = u % p.tilesM, tn = u / p.tilesM;
+        for (int kt = 0; kt < p.KT; kt += KM, ++it) {
+          const int ps = it % PST;
+          const uint32_t ph = (it / PST) & 1;
+          if (!mbar_wait(&pempty[ps], ph ^ 1, p.spin_limit)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* dst = smem + L::P_OFF + ps * L::PSTAGE;
+          mbar_arrive_expect_tx(&pfull[ps], L::PSTAGE);
+          tma_load_2d(dst, &mapA, kt * KP, tm * 256 + rank * L::HALF, &pfull[ps]);
+          tma_load_2d(dst + L::PA, &mapB, kt * KP, tn * 256 + rank * L::HALF, &pfull[ps]);
+        }
+      }
+      for (uint32_t j = it > static_cast<uint32_t>(PST) ? it - PST : 0u; j < it; ++j)
+        mbar_wait(&pfull[j % PST], (j / PST) & 1, 0);
+    }
+  } else if (warp >= UNPACK_WARP0) {
+    constexpr int ROWS = 2 * L::HALF;
+    constexpr int ITEMS = ROWS * 4;
+    constexpr int IPT = ITEMS / NPT;
+    static_assert(ITEMS % NPT == 0, "items per thread");
+    const int t = threadIdx.x - UNPACK_WARP0 * 32;
+    uint32_t src_off[IPT], dst_off0[IPT], dst_off1[IPT];
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const int idx = t + i * NPT;
+      const int q = idx / ROWS, row_all = idx % ROWS;
+      src_off[i] = static_cast<uint32_t>(row_all * PROW + ((q ^ (row_all & 7)) << 4));
+      const bool is_a = row_all < L::HALF;
+      const int row = is_a ? row_all : row_all - L::HALF;
+      const uint32_t base = is_a ? 0u : static_cast<uint32_t>(L::UA);
+      dst_off0[i] = base + sw128_off(row, 2 * q);
+      dst_off1[i] = base + sw128_off(row, 2 * q + 1);
+    }
+    uint32_t ufull_leader[UST];
+#pragma unroll
+    for (int s = 0; s < UST; ++s) ufull_leader[s] = mapa_shared(smem_u32(&ufull[s]), 0);
+    uint32_t it = 0, itp = 0;
+    bool ok = true;
+    for (int u = pair_id; ok && u < p.units; u += num_pairs) {
+      for (int kt = 0; ok && kt < p.KT; kt += KM, ++itp) {
+        const int ps = itp % PST;
+        const uint32_t pph = (itp / PST) & 1;
+        bool got = mbar_wait(&pfull[ps], pph, p.spin_limit);
+        got = __all_sync(0xffffffffu, got && !*abort_flag);
+        if (!got) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
+        const int nsub = min(KM, p.KT - kt);
+        for (int sub = 0; sub < nsub; ++sub, ++it) {
+          const int us = it % UST;
+          const uint32_t uph = (it / UST) & 1;
+          bool free_slot = mbar_wait(&uempty[us], uph ^ 1, p.spin_limit);
+          free_slot = __all_sync(0xffffffffu, free_slot && !*abort_flag);
+          if (!free_slot) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t udst = smem_base + L::U_OFF + us * L::USTAGE;
+          const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;
+#pragma unroll
+          for (int i = 0; i < IPT; ++i) {
+            const uint4 v = lds128(psrc + (src_off[i] ^ sub_x));
+            const uint32_t m = 0xF0F0F0F0u;
+            sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+            sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed_n(ufull_leader[us], 32);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive_n(&pempty[ps], 32);
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t IDESC = idesc_i8(256, 256);
+      uint32_t it = 0, acc_it = 0;
+      for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
+        const int buf = acc_it & 1;
+        const uint32_t aph = (acc_it >> 1) & 1;
+        if (*abort_flag || !mbar_wait(&tempty[buf], aph ^ 1, p.spin_limit)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
+        bool ok = true;
+        for (int kt = 0; kt < p.KT; ++kt, ++it) {
+          const int us = it % UST;
+          const uint32_t uph = (it / UST) & 1;
+          if (!mbar_wait(&ufull[us], uph, p.spin_limit) || *abort_flag) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_base + L::U_OFF + us * L::USTAGE;
+          const uint32_t b_addr = a_addr + L::UA;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            mma_i8_pair(d_tmem, desc_sw128(a_addr + kk * UMMA_K),
+                        desc_sw128(b_addr + kk * UMMA_K), IDESC, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit_pair_mc(&uempty[us], 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&tfull[buf], 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int row = warp * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t tempty_leader[2];
+    tempty_leader[0] = mapa_shared(smem_u32(&tempty[0]), 0);
+    tempty_leader[1] = mapa_shared(smem_u32(&tempty[1]), 0);
+    uint32_t acc_it = 0;
+    for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
+      const int tm = u % p.tilesM, tn = u / p.tilesM;
+      const int buf = acc_it & 1;
+      const uint32_t aph = (acc_it >> 1) & 1;
+      if (threadIdx.x == 0) {
+        const bool ok = !*abort_flag && mbar_wait(&tfull[buf], aph, p.spin_limit);
+        if (!ok) *abort_flag = 1;
+        bcast[0] = ok ? 1 : 0;
+      }
+      named_bar_sync(1, EPI_WARPS * 32);
+      const bool ok = bcast[0] != 0;
+      named_bar_sync(1, EPI_WARPS * 32);
+      if (!ok) break;
+      tc_fence_after();
+      const int m = tm * 256 + static_cast<int>(rank) * L::HALF + row;
+      const bool m_valid = m < p.M;
+      const float sa = m_valid ? p.a_scale[m] : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(lane_addr + static_cast<uint32_t>(buf * 256 + c * 16), v);
+        tmem_ld_wait();
+        const int n0 = tn * 256 + c * 16;
+        if (!m_valid || n0 >= p.N) continue;
+        if (p.out_i32) {
+          int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
+                                              static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_int4(static_cast<int>(v[4 * j]) >> 8, static_cast<int>(v[4 * j + 1]) >> 8,
+                               static_cast<int>(v[4 * j + 2]) >> 8,
+                               static_cast<int>(v[4 * j + 3]) >> 8);
+        } else {
+          const float4* sw4 = reinterpret_cast<const float4*>(p.w_scale + n0);
+          uint32_t packed[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 s = __ldg(sw4 + j);
+            const float sj[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+              const int k = 4 * j + e;
+              const float f0 = static_cast<float>(static_cast<int>(v[k]) >> 8) * sa * sj[e];
+              const float f1 = static_cast<float>(static_cast<int>(v[k + 1]) >> 8) * sa * sj[e + 1];
+              __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+              packed[k / 2] = *reinterpret_cast<uint32_t*>(&h);
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                static_cast<int64_t>(m) * p.N + n0);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed_n(tempty_leader[buf], 32);
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP && rank == 0) {
+    tc_fence_after();
+    if (lane == 0) {
+      mma_commit_pair_mc(drain, 0x1);    // every pair MMA has finished with both CTAs
+      mbar_wait(drain, 0, 0);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  cluster_sync();                        // neither CTA leaves while the pair may touch it
+  tc_fence_after();
+  if (warp == MMA_WARP) tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+}
+
 // ------------------------------------------------------------------ host side
 
 static bool make_map(CUtensorMap* map, const uint8_t* base, int rows, int64_t K,
@@ -446,11 +772,11 @@ static bool make_map(CUtensorMap* map, const uint8_t* base, int rows, int64_t K,
   if (!encode) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(KP), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(PROW), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     host::set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -479,6 +805,54 @@ static sq_status launch(const Plan& plan, const uint8_t* opA, const uint8_t* opB
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return host::cuda_fail("w4a4_gemm launch", e);
   return SQ_OK;
+}
+
+
+template <int PST, int UST>
+static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, int64_t N,
+                             int64_t K, PairParams prm, int num_sms, cudaStream_t stream) {
+  using L = PairLayout<PST, UST>;
+  CUtensorMap mapA, mapB;
+  if (!make_map(&mapA, a_q, static_cast<int>(M), K, L::HALF) ||
+      !make_map(&mapB, w_q, static_cast<int>(N), K, L::HALF))
+    return SQ_ERR_CUDA;
+  auto kfn = w4a4_gemm_pair_kernel<PST, UST>;
+  static int max_clusters[64] = {0};
+  const int dev = host::current_device();
+  if (dev < 0) return SQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = L::BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_clusters[dev & 63] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(pair)", e);
+    int n = 0;
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    e = cudaOccupancyMaxActiveClusters(&n, kfn, &cfg);
+    if (e != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms / 2;
+    }
+    max_clusters[dev & 63] = n;
+  }
+  const int pairs = prm.units < max_clusters[dev & 63] ? prm.units : max_clusters[dev & 63];
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, mapA, mapB, prm);
+  if (e != cudaSuccess) return host::cuda_fail("w4a4_gemm_pair launch", e);
+  return SQ_OK;
+}
+
+static bool use_pair(int64_t M, int64_t N) {
+  if (M < 256 || N < 256) return false;
+  return host::gemm_path() != 1;
 }
 
 static int pick_bn_swap(int64_t M) {
@@ -513,6 +887,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
     }
   }
   pl.kps = (pl.KT + splits - 1) / splits;
+  pl.kps = (pl.kps + KM - 1) / KM * KM;            // splits start on a packed stage
   pl.splits = (pl.KT + pl.kps - 1) / pl.kps;
   pl.units = static_cast<int>(base * pl.splits);
   pl.grid = static_cast<int>(pl.units < num_sms ? pl.units : num_sms);
@@ -521,6 +896,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
 
 size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K < BK) return 0;
+  if (use_pair(M, N)) return 0;
   Plan pl = plan_gemm(M, N, K, true, num_sms);
   if (pl.splits <= 1) return 0;
   const size_t acc = static_cast<size_t>(M) * static_cast<size_t>(N) * 4;
@@ -532,6 +908,23 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
               int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
               size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
               const Plan* forced) {
+  if (!forced && use_pair(M, N)) {
+    PairParams pp{};
+    pp.rowsA = static_cast<int>(M);
+    pp.rowsB = static_cast<int>(N);
+    pp.tilesM = static_cast<int>((M + 255) / 256);
+    pp.tilesN = static_cast<int>((N + 255) / 256);
+    pp.KT = static_cast<int>(K / BK);
+    pp.units = pp.tilesM * pp.tilesN;
+    pp.a_scale = a_scale;
+    pp.w_scale = w_scale;
+    pp.out = out;
+    pp.out_i32 = out_i32;
+    pp.M = static_cast<int>(M);
+    pp.N = static_cast<int>(N);
+    pp.spin_limit = spin_limit;
+    return launch_pair<3, 3>(a_q, w_q, M, N, K, pp, num_sms, stream);
+  }
   Plan pl = forced ? *forced : plan_gemm(M, N, K, ws != nullptr, num_sms);
   Params prm{};
   prm.swap = pl.swap;
@@ -565,11 +958,11 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
   const uint8_t* opA = pl.swap ? w_q : a_q;
   const uint8_t* opB = pl.swap ? a_q : w_q;
   switch (pl.bn) {
-    case 16: return launch<16, 8, 3>(pl, opA, opB, K, prm, stream);
-    case 32: return launch<32, 8, 3>(pl, opA, opB, K, prm, stream);
-    case 64: return launch<64, 6, 3>(pl, opA, opB, K, prm, stream);
-    case 128: return launch<128, 4, 3>(pl, opA, opB, K, prm, stream);
-    case 256: return launch<256, 4, 2>(pl, opA, opB, K, prm, stream);
+    case 16: return launch<16, 6, 3>(pl, opA, opB, K, prm, stream);
+    case 32: return launch<32, 6, 3>(pl, opA, opB, K, prm, stream);
+    case 64: return launch<64, 4, 3>(pl, opA, opB, K, prm, stream);
+    case 128: return launch<128, 3, 3>(pl, opA, opB, K, prm, stream);
+    case 256: return launch<256, 2, 2>(pl, opA, opB, K, prm, stream);
     default: break;
   }
   host::set_error("no kernel for tile width %d", pl.bn);

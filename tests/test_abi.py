@@ -20,8 +20,12 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def sq():
-    from rotation_ptq_b200 import build
-    build.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_sq_build", os.path.join(ROOT, "rotation_ptq_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
     import rotation_ptq_b200 as m
     return m
 

@@ -139,3 +139,21 @@ def test_forced_timeout_reports_status_and_recovers(cuda_ok):
     assert sq.device_status() == 0
     ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("M,N,K", [(256, 4096, 12288), (300, 528, 1024), (1000, 768, 512),
+                                   (4096, 4096, 12288)])
+def test_large_m_kernels_agree(cuda_ok, path, M, N, K):
+    # the one-CTA and the CTA-pair kernels give bit-identical accumulators
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 500 + M)
+    sq.debug_set_gemm_path(path)
+    try:
+        acc = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True)
+        assert sq.device_status() == 0
+    finally:
+        sq.debug_set_gemm_path(0)
+    rows = P.sample_rows(M, 24, seed=path)
+    got = acc[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64)
+    assert np.array_equal(got, O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w)))

@@ -110,3 +110,25 @@ def test_strided_rows(cuda_ok):
     view = big.cuda()[:, :4096]
     a_q, a_s = sq.rotate_quant(view, None, 1, 1.0)
     _check(a_q.cpu().numpy(), a_s.cpu().numpy(), big[:, :4096].double().numpy(), 1, 1)
+
+
+def test_down_proj_clip_and_strided_rows(cuda_ok):
+    # the R4 kernel with clamping (clip < 1) and with padded rows (ld_x > K)
+    import rotation_ptq_b200 as sq
+    wl = W.down_proj(M=9, with_weights=False, seed=91)
+    aq, asc = _run(sq, wl.x, 12, 1024, clip=0.85)
+    codes = _check(aq, asc, wl.x.double().numpy(), 12, 1024, clip=0.85)
+    assert (codes == 7).any() and (codes == -8).any()
+    padded = torch.zeros((9, 12288 + 256), dtype=torch.bfloat16)
+    padded[:, :12288] = wl.x
+    a_q, a_s = sq.rotate_quant(padded.cuda()[:, :12288], sq.paley_h12(), 1024, 1.0)
+    _check(a_q.cpu().numpy(), a_s.cpu().numpy(), wl.x.double().numpy(), 12, 1024)
+
+
+def test_down_proj_more_rows_than_ctas(cuda_ok):
+    # exercises the two-slot row prefetch ring over many rows per CTA
+    import rotation_ptq_b200 as sq
+    wl = W.down_proj(M=1500, with_weights=False, seed=92)
+    aq, asc = _run(sq, wl.x, 12, 1024)
+    rows = P.sample_rows(wl.M, 30, seed=4)
+    _check(aq[rows], asc[rows], wl.x[torch.from_numpy(rows)].double().numpy(), 12, 1024)
