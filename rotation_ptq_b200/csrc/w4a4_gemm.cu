@@ -86,6 +86,7 @@ struct Layout {
   static_assert(USTAGE % 1024 == 0 && UA % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
                 "TMEM allocation must be a power of two in [32, 512]");
+  static_assert(BYTES <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -427,19 +428,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (last) {
           __threadfence();
           if (a_valid) {
-            for (int j = 0; j < BN; ++j) {
-              const int b = w.tb * BN + j;
-              if (b >= p.rowsB) break;
-              const int m = p.swap ? b : a_row;
-              const int n = p.swap ? a_row : b;
-              const int64_t o = static_cast<int64_t>(m) * p.N + n;
-              const int acc = __ldcg(p.ws_acc + o);
-              __stcg(p.ws_acc + o, 0);
-              if (p.out_i32) {
-                static_cast<int*>(p.out)[o] = acc;
-              } else {
-                const float f = static_cast<float>(acc) * __ldg(p.a_scale + m) * __ldg(p.w_scale + n);
-                static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(f);
+            // 16 independent loads in flight per chunk, then the stores
+            const float s_lane = p.swap ? __ldg(p.w_scale + a_row) : __ldg(p.a_scale + a_row);
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN; j0 += 16) {
+              int acc[16];
+              float sb[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int b = w.tb * BN + j0 + j;
+                const bool ok = b < p.rowsB;
+                const int m = p.swap ? b : a_row;
+                const int n = p.swap ? a_row : b;
+                const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                acc[j] = ok ? __ldcg(p.ws_acc + o) : 0;
+                sb[j] = ok ? __ldg((p.swap ? p.a_scale : p.w_scale) + b) : 0.f;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int b = w.tb * BN + j0 + j;
+                if (b < p.rowsB) {
+                  const int m = p.swap ? b : a_row;
+                  const int n = p.swap ? a_row : b;
+                  const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                  __stcg(p.ws_acc + o, 0);
+                  if (p.out_i32) {
+                    static_cast<int*>(p.out)[o] = acc[j];
+                  } else {
+                    // the pinned order: float(acc) * a_scale[m] * w_scale[n]
+                    const float sa = p.swap ? sb[j] : s_lane;
+                    const float sw = p.swap ? s_lane : sb[j];
+                    static_cast<__nv_bfloat16*>(p.out)[o] =
+                        __float2bfloat16_rn(static_cast<float>(acc[j]) * sa * sw);
+                  }
+                }
               }
             }
           }
@@ -923,7 +945,7 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
     pp.M = static_cast<int>(M);
     pp.N = static_cast<int>(N);
     pp.spin_limit = spin_limit;
-    return launch_pair<3, 3>(a_q, w_q, M, N, K, pp, num_sms, stream);
+    return launch_pair<3, 4>(a_q, w_q, M, N, K, pp, num_sms, stream);
   }
   Plan pl = forced ? *forced : plan_gemm(M, N, K, ws != nullptr, num_sms);
   Params prm{};
@@ -958,10 +980,10 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
   const uint8_t* opA = pl.swap ? w_q : a_q;
   const uint8_t* opB = pl.swap ? a_q : w_q;
   switch (pl.bn) {
-    case 16: return launch<16, 6, 3>(pl, opA, opB, K, prm, stream);
-    case 32: return launch<32, 6, 3>(pl, opA, opB, K, prm, stream);
-    case 64: return launch<64, 4, 3>(pl, opA, opB, K, prm, stream);
-    case 128: return launch<128, 3, 3>(pl, opA, opB, K, prm, stream);
+    case 16: return launch<16, 4, 8>(pl, opA, opB, K, prm, stream);
+    case 32: return launch<32, 4, 7>(pl, opA, opB, K, prm, stream);
+    case 64: return launch<64, 3, 6>(pl, opA, opB, K, prm, stream);
+    case 128: return launch<128, 3, 4>(pl, opA, opB, K, prm, stream);
     case 256: return launch<256, 2, 2>(pl, opA, opB, K, prm, stream);
     default: break;
   }
