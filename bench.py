@@ -25,7 +25,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -55,52 +54,57 @@ def load_peaks():
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and throttle reasons while the timed region runs.
+
+    NVML is polled from a background thread every 2 ms (nvidia-smi's own
+    loop is too coarse for a region of a few tens of milliseconds).
+    """
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
+        self.samples = []
+        self.result = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+    def _run(self):
+        import pynvml
+        h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            self._stop.wait(0.002)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._thread = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
-        time.sleep(0.3)
+            self._thread = None
         return self
 
     def __exit__(self, *a):
-        self.result = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        if self.proc is None:
+        if self._thread is None:
             return
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out = ""
-        rows = []
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
-            except ValueError:
-                continue
-        if not rows:
+        self._stop.set()
+        self._thread.join(timeout=2)
+        if not self.samples:
             return
-        sm = [r[0] for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v == "Active"})
-        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
-        self.result = {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
-                       "reasons": reasons, "samples": len(rows)}
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        self.result = {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.sm_max,
+                       "reasons": reasons, "samples": len(sm)}
 
 
 # --------------------------------------------------------------- our arm

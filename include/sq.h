@@ -232,8 +232,11 @@ void sq_debug_set_spin_limit(uint32_t polls);
 
 /* sq_debug_set_gemm_path -- test hook: which sq_w4a4_linear kernel large-M
  * shapes use.  0 = automatic (default), 1 = one-CTA 128-row tiles,
- * 2 = two-CTA 256-row tiles (M >= 256 and N >= 256 only; smaller shapes keep
- * their automatic kernel).  Results are identical; only speed differs.
+ * 2 = two-CTA 256-row tiles with both operands in shared memory (M >= 256
+ * and N >= 256 only; smaller shapes keep
+ * their automatic kernel), 3 = two-CTA tiles with the widened A operand in
+ * tensor memory (the automatic choice for those shapes).  Results are
+ * identical; only speed differs.
  * Applies to calls made afterwards from any thread. */
 void sq_debug_set_gemm_path(int path);
 

@@ -726,11 +726,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m = tm * 256 + static_cast<int>(rank) * L::HALF + row;
       const bool m_valid = m < p.M;
       const float sa = m_valid ? p.a_scale[m] : 0.f;
+      // four 16-column loads in flight per wait: 64 accumulator columns
 #pragma unroll 1
-      for (int c = 0; c < 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(lane_addr + static_cast<uint32_t>(buf * 256 + c * 16), v);
+      for (int c4 = 0; c4 < 16; c4 += 4) {
+        uint32_t vv[4][16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          tmem_ld16(lane_addr + static_cast<uint32_t>(buf * 256 + (c4 + g) * 16), vv[g]);
         tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+        const int c = c4 + g;
+        const uint32_t (&v)[16] = vv[g];
         const int n0 = tn * 256 + c * 16;
         if (!m_valid || n0 >= p.N) continue;
         if (p.out_i32) {
@@ -762,6 +769,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -782,6 +790,332 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   cluster_sync();                        // neither CTA leaves while the pair may touch it
+  tc_fence_after();
+  if (warp == MMA_WARP) tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+}
+
+// ----------------------------------------------- CTA pairs, A in tensor memory
+//
+// As the pair kernel above, but the widened A operand never goes back to
+// shared memory: four unpack warps (one per TMEM lane quadrant, one A row per
+// thread) write each k-tile's 128 int8 bytes per row straight into tensor
+// memory with tcgen05.st, and the MMAs read A from there
+// (tcgen05.mma.cta_group::2 with an A operand address in TMEM).  The other
+// four unpack warps widen this CTA's half of B into the shared-memory ring,
+// which, holding only B, can be twice as deep.  Tensor memory: one 256-column
+// int32 accumulator and eight 32-column A slots.
+
+template <int PST, int UST>
+struct PairTSLayout {
+  static constexpr int HALF = 128;
+  static constexpr int PA = HALF * PROW;              // packed A (KM k-tiles)
+  static constexpr int PSTAGE = 2 * HALF * PROW;      // packed A + packed B
+  static constexpr int UB = HALF * BK;                // int8 B per k-tile
+  static constexpr int U_OFF = 0;
+  static constexpr int P_OFF = UST * UB;
+  static constexpr int BAR_OFF = P_OFF + PST * PSTAGE;
+  static constexpr int NBAR = 2 * PST + 2 * UST + 3;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = MISC_OFF + 32 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t A_COL0 = 256;             // A slots follow the accumulator
+  static_assert(UST * 32 <= 256, "A slots must fit beside the accumulator");
+  static_assert(BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(P_OFF % 1024 == 0 && PSTAGE % 1024 == 0, "swizzle atoms need 1 KB alignment");
+};
+
+constexpr int A_WARP0 = UNPACK_WARP0;       // warps 6..9 widen A into tensor memory
+constexpr int B_WARP0 = UNPACK_WARP0 + 4;   // warps 10..13 widen B into shared memory
+
+template <int PST, int UST>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    w4a4_gemm_pair_ts_kernel(const __grid_constant__ CUtensorMap mapA,
+                             const __grid_constant__ CUtensorMap mapB, const PairParams p) {
+  using L = PairTSLayout<PST, UST>;
+  // int8 slots change hands in groups of KM k-tiles (one packed stage): one
+  // barrier wait and one tensor-core commit per group rather than per k-tile
+  constexpr int G = UST / KM;
+  static_assert(UST % KM == 0, "int8 slots come in whole groups");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* pempty = pfull + PST;
+  uint64_t* ufull = pempty + PST;      // on the even CTA: A and B of both CTAs arrive
+  uint64_t* uempty = ufull + UST;      // both CTAs: arrival from the pair commit
+  uint64_t* tfull = uempty + UST;      // both CTAs: accumulator ready
+  uint64_t* tempty = tfull + 1;        // on the even CTA: both CTAs' epilogues arrive
+  uint64_t* drain = tempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair_id = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PST; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], NPT);
+    }
+    for (int s = 0; s < G; ++s) {
+      mbar_init(&ufull[s], 2 * NPT);
+      mbar_init(&uempty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * EPI_WARPS * 32);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = pair_id; ok && u < p.units && !*abort_flag; u += num_pairs) {
+        const int tm = u % p.tilesM, tn = u / p.tilesM;
+        for (int kt = 0; kt < p.KT; kt += KM, ++it) {
+          const int ps = it % PST;
+          const uint32_t ph = (it / PST) & 1;
+          if (!mbar_wait(&pempty[ps], ph ^ 1, p.spin_limit)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* dst = smem + L::P_OFF + ps * L::PSTAGE;
+          mbar_arrive_expect_tx(&pfull[ps], L::PSTAGE);
+          tma_load_2d(dst, &mapA, kt * KP, tm * 256 + rank * L::HALF, &pfull[ps]);
+          tma_load_2d(dst + L::PA, &mapB, kt * KP, tn * 256 + rank * L::HALF, &pfull[ps]);
+        }
+      }
+      for (uint32_t j = it > static_cast<uint32_t>(PST) ? it - PST : 0u; j < it; ++j)
+        mbar_wait(&pfull[j % PST], (j / PST) & 1, 0);
+    }
+  } else if (warp >= A_WARP0) {
+    const bool is_a = warp < B_WARP0;
+    // A warps: thread = A row (its TMEM lane); B warps: 4 chunks of 16 bytes each
+    const int quad = warp & 3;
+    const int a_row = quad * 32 + lane;
+    const uint32_t a_src = static_cast<uint32_t>(a_row * PROW);
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + L::A_COL0;
+    const int tb = threadIdx.x - B_WARP0 * 32;                 // 0..127 for B warps
+    uint32_t b_src[4], b_dst0[4], b_dst1[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tb + i * 128;
+      const int q = idx >> 7, row = idx & 127;
+      b_src[i] = static_cast<uint32_t>(L::PA + row * PROW + ((q ^ (row & 7)) << 4));
+      b_dst0[i] = sw128_off(row, 2 * q);
+      b_dst1[i] = sw128_off(row, 2 * q + 1);
+    }
+    const uint32_t ufull_leader0 = mapa_shared(smem_u32(&ufull[0]), 0);
+    uint32_t itp = 0;
+    bool ok = true;
+    for (int u = pair_id; ok && u < p.units; u += num_pairs) {
+      for (int kt = 0; ok && kt < p.KT; kt += KM, ++itp) {
+        const int ps = itp % PST;
+        const uint32_t pph = (itp / PST) & 1;
+        bool got = mbar_wait(&pfull[ps], pph, p.spin_limit);
+        got = __all_sync(0xffffffffu, got && !*abort_flag);
+        if (!got) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
+        const int nsub = min(KM, p.KT - kt);
+        // one protocol round per packed stage: wait for its group of int8
+        // slots, widen every k-tile, one fence, one arrival
+        const int g = itp % G;
+        bool free_slots = mbar_wait(&uempty[g], ((itp / G) & 1) ^ 1, p.spin_limit);
+        free_slots = __all_sync(0xffffffffu, free_slots && !*abort_flag);
+        if (!free_slots) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t m = 0xF0F0F0F0u;
+        if (is_a) {
+#pragma unroll
+          for (int sub = 0; sub < KM; ++sub) {
+            if (sub < nsub) {
+              uint32_t w[32];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int c = (sub * 4 + q) ^ (a_row & 7);
+                const uint4 v = lds128(psrc + a_src + (c << 4));
+                w[8 * q + 0] = (v.x << 4) & m;
+                w[8 * q + 1] = v.x & m;
+                w[8 * q + 2] = (v.y << 4) & m;
+                w[8 * q + 3] = v.y & m;
+                w[8 * q + 4] = (v.z << 4) & m;
+                w[8 * q + 5] = v.z & m;
+                w[8 * q + 6] = (v.w << 4) & m;
+                w[8 * q + 7] = v.w & m;
+              }
+              tmem_st32(a_lane + static_cast<uint32_t>((g * KM + sub) * 32), w);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+        } else {
+#pragma unroll
+          for (int sub = 0; sub < KM; ++sub) {
+            if (sub < nsub) {
+              const uint32_t udst = smem_base + L::U_OFF + (g * KM + sub) * L::UB;
+              const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint4 v = lds128(psrc + (b_src[i] ^ sub_x));
+                sts128(udst + b_dst0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+                sts128(udst + b_dst1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster_relaxed_n(ufull_leader0 + g * 8, 32);
+          mbar_arrive_n(&pempty[ps], 32);
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t IDESC = idesc_i8(256, 256);
+      uint32_t ig = 0, acc_it = 0;
+      for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
+        if (*abort_flag || !mbar_wait(tempty, (acc_it & 1) ^ 1, p.spin_limit)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < p.KT; kt += KM, ++ig) {
+          const int g = ig % G;
+          if (!mbar_wait(&ufull[g], (ig / G) & 1, p.spin_limit) || *abort_flag) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nsub = min(KM, p.KT - kt);
+          for (int sub = 0; sub < nsub; ++sub) {
+            const int slot = g * KM + sub;
+            const uint32_t a_tmem = tmem_base + L::A_COL0 + static_cast<uint32_t>(slot * 32);
+            const uint32_t b_addr = smem_base + L::U_OFF + slot * L::UB;
+#pragma unroll
+            for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+              mma_i8_pair_ts(tmem_base, a_tmem + kk * (UMMA_K / 4),
+                             desc_sw128(b_addr + kk * UMMA_K), IDESC,
+                             (kt + sub > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit_pair_mc(&uempty[g], 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(tfull, 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int row = warp * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
+    uint32_t acc_it = 0;
+    for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
+      const int tm = u % p.tilesM, tn = u / p.tilesM;
+      if (threadIdx.x == 0) {
+        const bool ok = !*abort_flag && mbar_wait(tfull, acc_it & 1, p.spin_limit);
+        if (!ok) *abort_flag = 1;
+        bcast[0] = ok ? 1 : 0;
+      }
+      named_bar_sync(1, EPI_WARPS * 32);
+      const bool ok = bcast[0] != 0;
+      named_bar_sync(1, EPI_WARPS * 32);
+      if (!ok) break;
+      tc_fence_after();
+      const int m = tm * 256 + static_cast<int>(rank) * L::HALF + row;
+      const bool m_valid = m < p.M;
+      const float sa = m_valid ? p.a_scale[m] : 0.f;
+      // four 16-column loads in flight per wait: 64 accumulator columns
+#pragma unroll 1
+      for (int c4 = 0; c4 < 16; c4 += 4) {
+        uint32_t vv[4][16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          tmem_ld16(lane_addr + static_cast<uint32_t>((c4 + g) * 16), vv[g]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+        const int c = c4 + g;
+        const uint32_t (&v)[16] = vv[g];
+        const int n0 = tn * 256 + c * 16;
+        if (!m_valid || n0 >= p.N) continue;
+        if (p.out_i32) {
+          int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
+                                              static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_int4(static_cast<int>(v[4 * j]) >> 8, static_cast<int>(v[4 * j + 1]) >> 8,
+                               static_cast<int>(v[4 * j + 2]) >> 8,
+                               static_cast<int>(v[4 * j + 3]) >> 8);
+        } else {
+          const float4* sw4 = reinterpret_cast<const float4*>(p.w_scale + n0);
+          uint32_t packed[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 s = __ldg(sw4 + j);
+            const float sj[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+              const int k = 4 * j + e;
+              const float f0 = static_cast<float>(static_cast<int>(v[k]) >> 8) * sa * sj[e];
+              const float f1 = static_cast<float>(static_cast<int>(v[k + 1]) >> 8) * sa * sj[e + 1];
+              __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+              packed[k / 2] = *reinterpret_cast<uint32_t*>(&h);
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                static_cast<int64_t>(m) * p.N + n0);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed_n(tempty_leader, 32);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP && rank == 0) {
+    tc_fence_after();
+    if (lane == 0) {
+      mma_commit_pair_mc(drain, 0x1);
+      mbar_wait(drain, 0, 0);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  cluster_sync();
   tc_fence_after();
   if (warp == MMA_WARP) tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
 }
@@ -830,15 +1164,22 @@ static sq_status launch(const Plan& plan, const uint8_t* opA, const uint8_t* opB
 }
 
 
-template <int PST, int UST>
+template <bool TS, int PST, int UST>
 static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, int64_t N,
                              int64_t K, PairParams prm, int num_sms, cudaStream_t stream) {
-  using L = PairLayout<PST, UST>;
+  constexpr int BYTES = [] {
+    if constexpr (TS) return PairTSLayout<PST, UST>::BYTES;
+    else return PairLayout<PST, UST>::BYTES;
+  }();
+  constexpr int HALF = 128;
   CUtensorMap mapA, mapB;
-  if (!make_map(&mapA, a_q, static_cast<int>(M), K, L::HALF) ||
-      !make_map(&mapB, w_q, static_cast<int>(N), K, L::HALF))
+  if (!make_map(&mapA, a_q, static_cast<int>(M), K, HALF) ||
+      !make_map(&mapB, w_q, static_cast<int>(N), K, HALF))
     return SQ_ERR_CUDA;
-  auto kfn = w4a4_gemm_pair_kernel<PST, UST>;
+  auto kfn = [] {
+    if constexpr (TS) return w4a4_gemm_pair_ts_kernel<PST, UST>;
+    else return w4a4_gemm_pair_kernel<PST, UST>;
+  }();
   static int max_clusters[64] = {0};
   const int dev = host::current_device();
   if (dev < 0) return SQ_ERR_CUDA;
@@ -849,12 +1190,12 @@ static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, 
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = L::BYTES;
+  cfg.dynamicSmemBytes = BYTES;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_clusters[dev & 63] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, BYTES);
     if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(pair)", e);
     int n = 0;
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
@@ -945,7 +1286,8 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
     pp.M = static_cast<int>(M);
     pp.N = static_cast<int>(N);
     pp.spin_limit = spin_limit;
-    return launch_pair<3, 4>(a_q, w_q, M, N, K, pp, num_sms, stream);
+    if (host::gemm_path() == 2) return launch_pair<false, 3, 4>(a_q, w_q, M, N, K, pp, num_sms, stream);
+    return launch_pair<true, 3, 8>(a_q, w_q, M, N, K, pp, num_sms, stream);
   }
   Plan pl = forced ? *forced : plan_gemm(M, N, K, ws != nullptr, num_sms);
   Params prm{};

@@ -141,11 +141,11 @@ def test_forced_timeout_reports_status_and_recovers(cuda_ok):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
 
 
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 @pytest.mark.parametrize("M,N,K", [(256, 4096, 12288), (300, 528, 1024), (1000, 768, 512),
                                    (4096, 4096, 12288)])
 def test_large_m_kernels_agree(cuda_ok, path, M, N, K):
-    # the one-CTA and the CTA-pair kernels give bit-identical accumulators
+    # the one-CTA and both CTA-pair kernels give bit-identical accumulators
     import rotation_ptq_b200 as sq
     a, w, sa, sw = _operands(M, N, K, 500 + M)
     sq.debug_set_gemm_path(path)
