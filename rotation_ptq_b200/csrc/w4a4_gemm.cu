@@ -824,9 +824,6 @@ struct PairTSLayout {
   static_assert(P_OFF % 1024 == 0 && PSTAGE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
 
-constexpr int A_WARP0 = UNPACK_WARP0;       // warps 6..9 widen A into tensor memory
-constexpr int B_WARP0 = UNPACK_WARP0 + 4;   // warps 10..13 widen B into shared memory
-
 template <int PST, int UST>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_pair_ts_kernel(const __grid_constant__ CUtensorMap mapA,
@@ -905,22 +902,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (uint32_t j = it > static_cast<uint32_t>(PST) ? it - PST : 0u; j < it; ++j)
         mbar_wait(&pfull[j % PST], (j / PST) & 1, 0);
     }
-  } else if (warp >= A_WARP0) {
-    const bool is_a = warp < B_WARP0;
-    // A warps: thread = A row (its TMEM lane); B warps: 4 chunks of 16 bytes each
+  } else if (warp >= UNPACK_WARP0) {
+    // Every unpack warp widens half of A and half of B of each packed stage.
+    // A: the thread's row is its TMEM lane (quadrant = warp % 4) and the warp
+    // writes 16 of the 32 columns of each k-tile slot.  B: the thread's row,
+    // two of the four 16-byte chunks of each k-tile.
+    const int uw = warp - UNPACK_WARP0;                        // 0..7
+    const int half = uw >> 2;
     const int quad = warp & 3;
     const int a_row = quad * 32 + lane;
     const uint32_t a_src = static_cast<uint32_t>(a_row * PROW);
-    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + L::A_COL0;
-    const int tb = threadIdx.x - B_WARP0 * 32;                 // 0..127 for B warps
-    uint32_t b_src[4], b_dst0[4], b_dst1[4];
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + L::A_COL0 +
+                            static_cast<uint32_t>(16 * half);
+    const int b_row = (uw & 3) * 32 + lane;
+    uint32_t b_src[2], b_dst0[2], b_dst1[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = tb + i * 128;
-      const int q = idx >> 7, row = idx & 127;
-      b_src[i] = static_cast<uint32_t>(L::PA + row * PROW + ((q ^ (row & 7)) << 4));
-      b_dst0[i] = sw128_off(row, 2 * q);
-      b_dst1[i] = sw128_off(row, 2 * q + 1);
+    for (int i = 0; i < 2; ++i) {
+      const int q = 2 * half + i;
+      b_src[i] = static_cast<uint32_t>(L::PA + b_row * PROW + ((q ^ (b_row & 7)) << 4));
+      b_dst0[i] = sw128_off(b_row, 2 * q);
+      b_dst1[i] = sw128_off(b_row, 2 * q + 1);
     }
     const uint32_t ufull_leader0 = mapa_shared(smem_u32(&ufull[0]), 0);
     uint32_t itp = 0;
@@ -939,7 +940,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
         const int nsub = min(KM, p.KT - kt);
         // one protocol round per packed stage: wait for its group of int8
-        // slots, widen every k-tile, one fence, one arrival
+        // slots, widen every k-tile, fence, one arrival
         const int g = itp % G;
         bool free_slots = mbar_wait(&uempty[g], ((itp / G) & 1) ^ 1, p.spin_limit);
         free_slots = __all_sync(0xffffffffu, free_slots && !*abort_flag);
@@ -949,45 +950,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         const uint32_t m = 0xF0F0F0F0u;
-        if (is_a) {
 #pragma unroll
-          for (int sub = 0; sub < KM; ++sub) {
-            if (sub < nsub) {
-              uint32_t w[32];
+        for (int sub = 0; sub < KM; ++sub) {
+          if (sub < nsub) {
+            const int slot = g * KM + sub;
+            uint32_t w[16];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int c = (sub * 4 + q) ^ (a_row & 7);
-                const uint4 v = lds128(psrc + a_src + (c << 4));
-                w[8 * q + 0] = (v.x << 4) & m;
-                w[8 * q + 1] = v.x & m;
-                w[8 * q + 2] = (v.y << 4) & m;
-                w[8 * q + 3] = v.y & m;
-                w[8 * q + 4] = (v.z << 4) & m;
-                w[8 * q + 5] = v.z & m;
-                w[8 * q + 6] = (v.w << 4) & m;
-                w[8 * q + 7] = v.w & m;
-              }
-              tmem_st32(a_lane + static_cast<uint32_t>((g * KM + sub) * 32), w);
+            for (int j = 0; j < 2; ++j) {
+              const int c = (sub * 4 + 2 * half + j) ^ (a_row & 7);
+              const uint4 v = lds128(psrc + a_src + (c << 4));
+              w[8 * j + 0] = (v.x << 4) & m;
+              w[8 * j + 1] = v.x & m;
+              w[8 * j + 2] = (v.y << 4) & m;
+              w[8 * j + 3] = v.y & m;
+              w[8 * j + 4] = (v.z << 4) & m;
+              w[8 * j + 5] = v.z & m;
+              w[8 * j + 6] = (v.w << 4) & m;
+              w[8 * j + 7] = v.w & m;
+            }
+            tmem_st16(a_lane + static_cast<uint32_t>(slot * 32), w);
+            const uint32_t udst = smem_base + L::U_OFF + slot * L::UB;
+            const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint4 v = lds128(psrc + (b_src[i] ^ sub_x));
+              sts128(udst + b_dst0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+              sts128(udst + b_dst1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
             }
           }
-          tmem_st_wait();
-          tc_fence_before();
-        } else {
-#pragma unroll
-          for (int sub = 0; sub < KM; ++sub) {
-            if (sub < nsub) {
-              const uint32_t udst = smem_base + L::U_OFF + (g * KM + sub) * L::UB;
-              const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint4 v = lds128(psrc + (b_src[i] ^ sub_x));
-                sts128(udst + b_dst0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
-                sts128(udst + b_dst1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
-              }
-            }
-          }
-          fence_proxy_async_smem();
         }
+        tmem_st_wait();
+        tc_fence_before();
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive_cluster_relaxed_n(ufull_leader0 + g * 8, 32);
