@@ -115,13 +115,20 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import rotation_ptq_b200 as sq
+    from rotation_ptq_b200 import shard
     from workloads import synthetic as W
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    # one model (the canonical weights) on every rank; each rank serves its
+    # own M-token shard of the global batch (rank 0's is the 1-GPU workload)
     wl = W.down_proj(M=M, K=K, N=N)
     hs = sq.paley_h12()
-    x = wl.x.to(dev)
+    if rank == 0:
+        x = wl.x.to(dev)
+    else:
+        x = W.down_proj(M=M, K=K, N=N, seed=shard.shard_seed(W.SEED_BASE + 1, rank),
+                        with_weights=False).x.to(dev)
     w_q, w_s = sq.quantize_weights(wl.w.to(dev), hs, N_POW2)
     del wl
     a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
@@ -222,10 +229,7 @@ def run_ours(args, rank, world, local_rank):
         del q, k, v, kvo, kdq, vdq
 
     # max over ranks
-    vals = torch.tensor([ms_step, ms_rq, ms_gemm, ms_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_step, ms_rq, ms_gemm, ms_e2e = vals.tolist()
+    ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
                 clocks=clk.result, kv=kv_info)
 
@@ -372,12 +376,14 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample()
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
-    tops_step = OPS / (r["ms_step"] * 1e-3) / 1e12
+    from rotation_ptq_b200.shard import job_rate
+    # whole job: every rank's M tokens over the slowest rank's step time
+    tops_job = job_rate(world * OPS, r["ms_step"] * 1e-3) / 1e12
     tops_gemm = OPS / (r["ms_gemm"] * 1e-3) / 1e12
     gbs_rq = RQ_BYTES / (r["ms_rq"] * 1e-3) / 1e9
-    tops_e2e = OPS / (r["ms_e2e"] * 1e-3) / 1e12
+    tops_e2e_job = job_rate(world * OPS, r["ms_e2e"] * 1e-3) / 1e12
     line = {
-        "metric": METRIC, "value": world * tops_step, "unit": "TOPS", "n_gpus": world,
+        "metric": METRIC, "value": tops_job, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
         "data": "synthetic (seeded numpy; SwiGLU of Student-t(3) + 8 outlier channels, "
@@ -400,7 +406,7 @@ def main():
                                   "frac": gbs_rq / hbm, "traffic": None,
                                   "peak_source": peak_src + " copy bandwidth"},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
+        "e2e": {"value": tops_e2e_job, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
                 "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
         "clocks": r["clocks"],
