@@ -180,92 +180,149 @@ __host__ __device__ constexpr int paley12(int i, int j) {
   return i == j ? 1 : (i == 0 ? 1 : (j == 0 ? -1 : chi11((j - 1) - (i - 1))));
 }
 
-// Shared exchange buffer: 12,288 floats in segments of 64 (one phase-B
-// thread each); the 16-byte chunk index inside a segment is XORed with the
-// segment's low three bits so both phases access it without bank conflicts.
-__device__ __forceinline__ int xoff(int c) {
-  const int seg = c >> 6, w = c & 63;
-  return (seg << 6) + ((((w >> 2) ^ (seg & 7))) << 2) + (w & 3);
+// Exchange buffer: 12,288 floats in 192 segments of 64 channels, segment u
+// holding c = 64 u + k.  Inside a segment, channels k and k + 32 sit side by
+// side (position p = 2 (k mod 32) + k / 32), so a 16-byte read yields two
+// ready-made (k, k + 32) pairs; the 16-byte chunk index is XORed with u mod 8
+// so that both the phase-A scalar writes and the phase-B vector reads are free
+// of bank conflicts.
+__device__ __forceinline__ int xpos(int u, int k) {
+  const int p = 2 * (k & 31) + (k >> 5);
+  return (u << 6) + ((((p >> 2) ^ (u & 7))) << 2) + (p & 3);
 }
 
-// One row of 12,288 channels, c = i*1024 + j, j = (j9..j0).
-// Rows are prefetched one ahead with a 1-D bulk async copy (24 KB) into a
-// two-slot shared-memory ring, so HBM latency overlaps the current row.
-// Phase A (threads 0..127, t = j0..j6): the 96 values of all 12 i and the
-//   top three j bits (jt = j7..j9) are read from the staged row; H8 over jt
-//   and H12 over i run in registers; the result goes to the exchange buffer.
-// Phase B (threads 0..191, u = (i, jt, j6)): 64 consecutive channels
-//   (j0..j5) come back from the buffer; H64 runs in registers and the j6
-//   stage pairs lanes u and u^1 through one shuffle.  Then the row's absmax
-//   (block reduction), the scale, and 64 codes = 32 bytes per thread.
+// Barrier over `n` threads (named barrier `id`) returning whether any of
+// them passed `v`: one uniform verdict for the whole group.
+__device__ __forceinline__ bool bar_any(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// One persistent CTA per SM; rows m = blockIdx.x + r * gridDim.x.  Rows of
+// 12,288 channels, c = i * 1024 + j, j = (j9..j0), are staged by 1-D bulk
+// copies into a three-slot ring.  Two warp groups work on different rows at
+// once, handing rows over through a double-buffered exchange buffer:
+//
+// Phase A (warps 0-3): a thread owns j0..j6 (a fixed permutation of the
+//   thread index that keeps its exchange writes conflict-free) and the 96
+//   values of all 12 i and the top three j bits (jt = j7..j9).  H8 over jt and
+//   H12 over i run in registers; the result goes to the exchange buffer.
+// Phase B (warps 4-9): thread u owns segment u (64 consecutive channels):
+//   H64 in registers (five stages across register pairs, one inside them),
+//   the j6 stage with lane u ^ 1 by one shuffle per pair, the row absmax
+//   across the six warps, the scale, and 64 codes stored as 32 bytes.
+//
 // The 1/sqrt(12288) normalisation is folded into the quantizer multiplier.
 // CLAMP is false when clip == 1: then |y / scale| <= 7 up to rounding, so the
-// codes already lie in [-7, 7].
-constexpr int H12_THREADS = 192;
+// codes already lie in [-7, 7].  Every wait is bounded; a wait that runs out
+// records SQ_ERR_TIMEOUT, and each group leaves its loop on one shared
+// verdict (barrier.cta.red.or) so no named barrier is left half-arrived.
+constexpr int H12_A_WARPS = 4;
+constexpr int H12_B_WARPS = 6;
+constexpr int H12_THREADS = 32 * (H12_A_WARPS + H12_B_WARPS);
+constexpr int H12_STAGES = 3;
 constexpr int H12_ROW_BYTES = 12288 * 2;
-constexpr int H12_SMEM = 12288 * 4 + 2 * H12_ROW_BYTES + 64;
+constexpr int H12_X_BYTES = 12288 * 4;
+constexpr int H12_BAR_OFF = 2 * H12_X_BYTES + H12_STAGES * H12_ROW_BYTES;
+constexpr int H12_SMEM = H12_BAR_OFF + 8 * (H12_STAGES + 4) + 16 + 2 * H12_B_WARPS * 4;
+constexpr int H12_BAR_A = 1;   // named barrier of the phase-A group
+constexpr int H12_BAR_B = 2;   // named barrier of the phase-B group
 
-// Two codes per byte from the low bytes of magic-rounded floats (the low
-// byte holds the code in two's complement): byte = lo nibble of a | lo
-// nibble of b << 4; four such bytes gathered into one word.
+// Eight codes from the low nibbles of eight magic-rounded floats (the low
+// byte holds the code in two's complement): even codes to the low nibbles,
+// odd codes to the high nibbles of four bytes.
 __device__ __forceinline__ uint32_t pack8(const uint32_t* u) {
-  uint32_t b[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) b[k] = (u[2 * k] & 0x0Fu) | ((u[2 * k + 1] << 4) & 0xF0u);
-  const uint32_t lo = __byte_perm(b[0], b[1], 0x3340);
-  const uint32_t hi = __byte_perm(b[2], b[3], 0x3340);
-  return __byte_perm(lo, hi, 0x5410);
+  const uint32_t ev = __byte_perm(__byte_perm(u[0], u[2], 0x0040),
+                                  __byte_perm(u[4], u[6], 0x0040), 0x5410);
+  const uint32_t od = __byte_perm(__byte_perm(u[1], u[3], 0x0040),
+                                  __byte_perm(u[5], u[7], 0x0040), 0x5410);
+  return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
 }
 
 template <bool CLAMP>
-__global__ void __launch_bounds__(H12_THREADS, 2)
+__global__ void __launch_bounds__(H12_THREADS, 1)
     rq_h12x1024_kernel(const uint16_t* __restrict__ x, int64_t ldx, int M, float norm,
                        float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
                        float* __restrict__ ascale) {
   extern __shared__ __align__(128) uint8_t rq_smem[];
-  float* X = reinterpret_cast<float*>(rq_smem);                        // 12,288 floats
-  uint16_t* stage = reinterpret_cast<uint16_t*>(rq_smem + 12288 * 4);  // 2 staged rows
-  uint64_t* bar = reinterpret_cast<uint64_t*>(rq_smem + 12288 * 4 + 2 * H12_ROW_BYTES);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
-  __shared__ float red[H12_THREADS / 32];
+  float* X = reinterpret_cast<float*>(rq_smem);                             // 2 x 12,288
+  uint16_t* stage = reinterpret_cast<uint16_t*>(rq_smem + 2 * H12_X_BYTES);  // ring of rows
+  uint64_t* sfull = reinterpret_cast<uint64_t*>(rq_smem + H12_BAR_OFF);
+  uint64_t* xfull = sfull + H12_STAGES;       // phase A wrote exchange buffer b
+  uint64_t* xempty = xfull + 2;               // phase B read exchange buffer b
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(xempty + 2);
+  float* red = reinterpret_cast<float*>(xempty + 2) + 4;   // [2][H12_B_WARPS]
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nrows = M > static_cast<int>(blockIdx.x)
+                        ? (M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                        : 0;
+  auto row_ptr = [&](int r) {
+    return x + (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(r) * gridDim.x) * ldx;
+  };
 
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int s = 0; s < H12_STAGES; ++s) mbar_init(&sfull[s], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xfull[b], H12_A_WARPS);
+      mbar_init(&xempty[b], H12_B_WARPS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
-    if (blockIdx.x < M) {
-      mbar_arrive_expect_tx(&bar[0], H12_ROW_BYTES);
-      bulk_g2s(stage, x + static_cast<int64_t>(blockIdx.x) * ldx, H12_ROW_BYTES, &bar[0]);
+    for (int r = 0; r < H12_STAGES && r < nrows; ++r) {
+      mbar_arrive_expect_tx(&sfull[r], H12_ROW_BYTES);
+      bulk_g2s(stage + r * 12288, row_ptr(r), H12_ROW_BYTES, &sfull[r]);
     }
   }
   __syncthreads();
-  uint32_t iter = 0;
-  for (int m = blockIdx.x; m < M; m += gridDim.x, ++iter) {
-    const int slot = iter & 1;
-    if (tid == 0 && m + gridDim.x < M) {
-      // the other slot was read by phase A of the previous row, which every
-      // thread finished before the barrier after it
-      mbar_arrive_expect_tx(&bar[slot ^ 1], H12_ROW_BYTES);
-      bulk_g2s(stage + (slot ^ 1) * 12288, x + static_cast<int64_t>(m + gridDim.x) * ldx,
-               H12_ROW_BYTES, &bar[slot ^ 1]);
+
+  if (warp < H12_A_WARPS) {
+    // ------------------------------------------------------------ phase A
+    const int j = 64 * (warp >> 1) + 16 * (warp & 1) + (lane & 15) + 32 * (lane >> 4);
+    const int j6 = j >> 6, kk = j & 63;
+    const int p = 2 * (kk & 31) + (kk >> 5);
+    // exchange offset of (o, jt) = xpos(16 o + 2 jt + j6, kk): for jt and
+    // jt + 4 the segment differs by 8, so u mod 8 and the swizzle agree
+    int xo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int s = 2 * q + j6;
+      xo[q] = (s << 6) + ((((p >> 2) ^ s)) << 2) + (p & 3);
     }
-    if (tid < 128) {
-      if (!mbar_wait(&bar[slot], (iter >> 1) & 1, spin_limit)) *abort_flag = 1;
-      const uint16_t* xr = stage + slot * 12288;
+    int issued = nrows < H12_STAGES ? nrows : H12_STAGES;
+    int r = 0;
+    for (; r < nrows; ++r) {
+      const int s = r % H12_STAGES;
+      bool fail = !mbar_wait(&sfull[s], (r / H12_STAGES) & 1, spin_limit);
+      const uint16_t* xr = stage + s * 12288;
       // z[i][q] = (value at jt = q, value at jt = q + 4)
       f2 z[12][4];
 #pragma unroll
       for (int i = 0; i < 12; ++i) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint32_t lo = xr[i * 1024 + q * 128 + tid];
-          const uint32_t hi = xr[i * 1024 + (q + 4) * 128 + tid];
+          const uint32_t lo = xr[i * 1024 + q * 128 + j];
+          const uint32_t hi = xr[i * 1024 + (q + 4) * 128 + j];
           z[i][q].x = __uint_as_float(lo << 16);
           z[i][q].y = __uint_as_float(hi << 16);
         }
+      }
+      // every phase-A thread holds its values: the slot can be refilled
+      if (bar_any(H12_BAR_A, 32 * H12_A_WARPS, fail || *abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      if (tid == 0 && r + H12_STAGES < nrows) {
+        mbar_arrive_expect_tx(&sfull[s], H12_ROW_BYTES);
+        bulk_g2s(stage + s * 12288, row_ptr(r + H12_STAGES), H12_ROW_BYTES, &sfull[s]);
+        ++issued;
       }
       // H8 over jt: bits 0 and 1 of q as packed pairs, bit 2 inside the pair
 #pragma unroll
@@ -288,15 +345,22 @@ __global__ void __launch_bounds__(H12_THREADS, 2)
           z[i][q].y = a - b;
         }
       }
-      // H12 over i: y_o = sum_i H[i][o] z_i = T - 2 * (sum of z_i with H[i][o] = -1)
+      const int b = r & 1;
+      if (!mbar_wait(&xempty[b], ((r >> 1) & 1) ^ 1, spin_limit)) *abort_flag = 1;
+      float* Xb = X + b * 12288;
+      // H12 over i: column 0 of the Paley matrix is +1 then -1, so
+      // y_0 = z_0 - sum_{i>0} z_i; for o > 0, y_o = T - 2 (sum of the five
+      // z_i with H[i][o] = -1), T = sum of all z_i
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        f2 T = z[0][q];
+        f2 rest = z[1][q];
 #pragma unroll
-        for (int i = 1; i < 12; ++i) T = add2(T, z[i][q]);
+        for (int i = 2; i < 12; ++i) rest = add2(rest, z[i][q]);
+        const f2 T = add2(z[0][q], rest);
         f2 y[12];
+        y[0] = sub2(z[0][q], rest);
 #pragma unroll
-        for (int o = 0; o < 12; ++o) {
+        for (int o = 1; o < 12; ++o) {
           f2 neg = {0.f, 0.f};
           bool any = false;
 #pragma unroll
@@ -306,87 +370,102 @@ __global__ void __launch_bounds__(H12_THREADS, 2)
               any = true;
             }
           }
-          y[o] = any ? fma2(f2{-2.f, -2.f}, neg, T) : T;
+          y[o] = fma2(f2{-2.f, -2.f}, neg, T);
         }
 #pragma unroll
         for (int o = 0; o < 12; ++o) {
-          X[xoff(o * 1024 + q * 128 + tid)] = y[o].x;
-          X[xoff(o * 1024 + (q + 4) * 128 + tid)] = y[o].y;
+          Xb[o * 1024 + xo[q]] = y[o].x;
+          Xb[o * 1024 + 512 + xo[q]] = y[o].y;
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xfull[b]);
     }
-    __syncthreads();
-    if (*abort_flag) break;
-    // Phase B: segment u = 64 consecutive channels starting at c0 = 64 u
-    const int u = tid;
-    f2 v[32];                                   // v[j] = (value j, value j + 32)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&X[(u << 6) + ((k ^ (u & 7)) << 2)]);
-      const float4 b =
-          *reinterpret_cast<const float4*>(&X[(u << 6) + (((k + 8) ^ (u & 7)) << 2)]);
-      v[4 * k + 0] = f2{a.x, b.x};
-      v[4 * k + 1] = f2{a.y, b.y};
-      v[4 * k + 2] = f2{a.z, b.z};
-      v[4 * k + 3] = f2{a.w, b.w};
+    // a group that stopped early lets its bulk copies land before exit
+    if (tid == 0) {
+      for (int rr = r; rr < issued; ++rr)
+        mbar_wait(&sfull[rr % H12_STAGES], (rr / H12_STAGES) & 1, 0);
     }
+  } else {
+    // ------------------------------------------------------------ phase B
+    const int u = tid - 32 * H12_A_WARPS;
+    const int bw = warp - H12_A_WARPS;
+    const float sg = (u & 1) ? -1.f : 1.f;
+    const f2 s2{sg, sg};
+    for (int r = 0; r < nrows; ++r) {
+      const int b = r & 1;
+      const int m = static_cast<int>(blockIdx.x) + r * static_cast<int>(gridDim.x);
+      bool fail = !mbar_wait(&xfull[b], (r >> 1) & 1, spin_limit);
+      const float* Xb = X + b * 12288;
+      f2 v[32];                                   // v[j] = (value j, value j + 32)
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
+      for (int ch = 0; ch < 16; ++ch) {
+        const float4 a = *reinterpret_cast<const float4*>(&Xb[(u << 6) + ((ch ^ (u & 7)) << 2)]);
+        v[2 * ch] = f2{a.x, a.y};
+        v[2 * ch + 1] = f2{a.z, a.w};
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xempty[b]);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if ((j & h) == 0) {
-          const f2 a = v[j], b = v[j + h];
-          v[j] = add2(a, b);
-          v[j + h] = sub2(a, b);
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          if ((jj & h) == 0) {
+            const f2 a = v[jj], c = v[jj + h];
+            v[jj] = add2(a, c);
+            v[jj + h] = sub2(a, c);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {              // bit j5: inside each pair
-      const float a = v[j].x, b = v[j].y;
-      v[j] = f2{a + b, a - b};
-    }
-    {                                            // bit j6: lanes u and u ^ 1
-      const float sg = (u & 1) ? -1.f : 1.f;
-      const f2 s2{sg, sg};
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const f2 o{__shfl_xor_sync(0xffffffffu, v[j].x, 1), __shfl_xor_sync(0xffffffffu, v[j].y, 1)};
-        v[j] = fma2(s2, v[j], o);
+      for (int jj = 0; jj < 32; ++jj) {            // bit j5: inside each pair
+        const float a = v[jj].x, c = v[jj].y;
+        v[jj] = f2{a + c, a - c};
       }
-    }
-    float amax = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
-    amax = block_max<H12_THREADS>(amax, red);
-    const float s = row_scale(amax * norm, clip);
-    const float k = norm * __frcp_rn(s);         // y_unnormalised -> y / scale
-    const f2 k2{k, k};
-    const f2 magic{12582912.f, 12582912.f};      // 1.5 * 2^23: round to nearest even
-    uint32_t ux[32], uy[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      f2 c = mul2(v[j], k2);
-      if (CLAMP) {
-        c.x = fminf(fmaxf(c.x, -8.f), 7.f);
-        c.y = fminf(fmaxf(c.y, -8.f), 7.f);
+      for (int jj = 0; jj < 32; ++jj) {            // bit j6: lanes u and u ^ 1
+        const f2 o{__shfl_xor_sync(0xffffffffu, v[jj].x, 1),
+                   __shfl_xor_sync(0xffffffffu, v[jj].y, 1)};
+        v[jj] = fma2(s2, v[jj], o);
       }
-      c = add2(c, magic);
-      ux[j] = __float_as_uint(c.x);              // channel j
-      uy[j] = __float_as_uint(c.y);              // channel j + 32
+      float amax = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) amax = fmaxf(amax, fmaxf(fabsf(v[jj].x), fabsf(v[jj].y)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) red[(r & 1) * H12_B_WARPS + bw] = amax;
+      // one barrier per row: publishes the partial maxima and the verdict
+      if (bar_any(H12_BAR_B, 32 * H12_B_WARPS, fail || *abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      amax = red[(r & 1) * H12_B_WARPS];
+#pragma unroll
+      for (int w = 1; w < H12_B_WARPS; ++w) amax = fmaxf(amax, red[(r & 1) * H12_B_WARPS + w]);
+      const float sc = row_scale(amax * norm, clip);
+      const float k = norm * __frcp_rn(sc);         // y_unnormalised -> y / scale
+      const f2 k2{k, k};
+      const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: round to nearest even
+      uint32_t ux[32], uy[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        f2 c;
+        if (CLAMP) {
+          c = mul2(v[jj], k2);
+          c.x = fminf(fmaxf(c.x, -8.f), 7.f);
+          c.y = fminf(fmaxf(c.y, -8.f), 7.f);
+          c = add2(c, magic);
+        } else {
+          c = fma2(v[jj], k2, magic);
+        }
+        ux[jj] = __float_as_uint(c.x);              // channel jj
+        uy[jj] = __float_as_uint(c.y);              // channel jj + 32
+      }
+      uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + u * 32);
+      dst[0] = make_uint4(pack8(ux), pack8(ux + 8), pack8(ux + 16), pack8(ux + 24));
+      dst[1] = make_uint4(pack8(uy), pack8(uy + 8), pack8(uy + 16), pack8(uy + 24));
+      if (u == 0) ascale[m] = sc;
     }
-    uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + u * 32);
-    dst[0] = make_uint4(pack8(ux), pack8(ux + 8), pack8(ux + 16), pack8(ux + 24));
-    dst[1] = make_uint4(pack8(uy), pack8(uy + 8), pack8(uy + 16), pack8(uy + 24));
-    if (tid == 0) ascale[m] = s;
-  }
-  // every bulk copy issued must land before the CTA exits
-  if (tid == 0) {
-    const uint32_t n_issued = (M > static_cast<int>(blockIdx.x))
-        ? static_cast<uint32_t>((M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1)
-        : 0u;
-    for (uint32_t j = n_issued > 2 ? n_issued - 2 : 0u; j < n_issued; ++j)
-      mbar_wait(&bar[j & 1], (j >> 1) & 1, 0);
   }
 }
 
@@ -513,7 +592,7 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   const int m = static_cast<int>(M), k = static_cast<int>(K);
   if (x_bf16 && n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small)) {
-    const int grid = m < 2 * host::num_sms() ? m : 2 * host::num_sms();
+    const int grid = m < host::num_sms() ? m : host::num_sms();
     const bool clamp = clip < 1.0f;
     auto kfn = clamp ? rq_h12x1024_kernel<true> : rq_h12x1024_kernel<false>;
     cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,

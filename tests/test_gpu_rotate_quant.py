@@ -48,8 +48,9 @@ def test_down_proj_full_size_sampled_rows(cuda_ok):
     _check(aq[rows], asc[rows], x64, 12, 1024)
 
 
-@pytest.mark.parametrize("M", [1, 3, 33])
+@pytest.mark.parametrize("M", [1, 3, 33, 149, 300])
 def test_down_proj_ragged_m(cuda_ok, M):
+    # 149 and 300 rows: some CTAs of the persistent grid take one row more
     import rotation_ptq_b200 as sq
     wl = W.down_proj(M=M, with_weights=False, seed=77 + M)
     aq, asc = _run(sq, wl.x, 12, 1024)
@@ -126,9 +127,14 @@ def test_down_proj_clip_and_strided_rows(cuda_ok):
 
 
 def test_down_proj_more_rows_than_ctas(cuda_ok):
-    # exercises the two-slot row prefetch ring over many rows per CTA
+    # Ten or eleven rows per CTA: the row-staging ring and the double-buffered
+    # exchange wrap several times.  Every row of three CTAs is checked (rows
+    # c, c + grid, ... for the grid of one CTA per SM), plus a random sample.
     import rotation_ptq_b200 as sq
-    wl = W.down_proj(M=1500, with_weights=False, seed=92)
+    M = 1500
+    wl = W.down_proj(M=M, with_weights=False, seed=92)
     aq, asc = _run(sq, wl.x, 12, 1024)
-    rows = P.sample_rows(wl.M, 30, seed=4)
+    grid = min(M, torch.cuda.get_device_properties(0).multi_processor_count)
+    per_cta = [np.arange(c, M, grid) for c in (0, 1, grid - 1)]
+    rows = np.unique(np.concatenate(per_cta + [P.sample_rows(M, 12, seed=4)]))
     _check(aq[rows], asc[rows], wl.x[torch.from_numpy(rows)].double().numpy(), 12, 1024)
