@@ -180,17 +180,6 @@ __host__ __device__ constexpr int paley12(int i, int j) {
   return i == j ? 1 : (i == 0 ? 1 : (j == 0 ? -1 : chi11((j - 1) - (i - 1))));
 }
 
-// Exchange buffer: 12,288 floats in 192 segments of 64 channels, segment u
-// holding c = 64 u + k.  Inside a segment, channels k and k + 32 sit side by
-// side (position p = 2 (k mod 32) + k / 32), so a 16-byte read yields two
-// ready-made (k, k + 32) pairs; the 16-byte chunk index is XORed with u mod 8
-// so that both the phase-A scalar writes and the phase-B vector reads are free
-// of bank conflicts.
-__device__ __forceinline__ int xpos(int u, int k) {
-  const int p = 2 * (k & 31) + (k >> 5);
-  return (u << 6) + ((((p >> 2) ^ (u & 7))) << 2) + (p & 3);
-}
-
 // Barrier over `n` threads (named barrier `id`) returning whether any of
 // them passed `v`: one uniform verdict for the whole group.
 __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
@@ -204,36 +193,6 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
   return r != 0;
 }
 
-// One persistent CTA per SM; rows m = blockIdx.x + r * gridDim.x.  Rows of
-// 12,288 channels, c = i * 1024 + j, j = (j9..j0), are staged by 1-D bulk
-// copies into a three-slot ring.  Two warp groups work on different rows at
-// once, handing rows over through a double-buffered exchange buffer:
-//
-// Phase A (warps 0-3): a thread owns j0..j6 (a fixed permutation of the
-//   thread index that keeps its exchange writes conflict-free) and the 96
-//   values of all 12 i and the top three j bits (jt = j7..j9).  H8 over jt and
-//   H12 over i run in registers; the result goes to the exchange buffer.
-// Phase B (warps 4-9): thread u owns segment u (64 consecutive channels):
-//   H64 in registers (five stages across register pairs, one inside them),
-//   the j6 stage with lane u ^ 1 by one shuffle per pair, the row absmax
-//   across the six warps, the scale, and 64 codes stored as 32 bytes.
-//
-// The 1/sqrt(12288) normalisation is folded into the quantizer multiplier.
-// CLAMP is false when clip == 1: then |y / scale| <= 7 up to rounding, so the
-// codes already lie in [-7, 7].  Every wait is bounded; a wait that runs out
-// records SQ_ERR_TIMEOUT, and each group leaves its loop on one shared
-// verdict (barrier.cta.red.or) so no named barrier is left half-arrived.
-constexpr int H12_A_WARPS = 4;
-constexpr int H12_B_WARPS = 6;
-constexpr int H12_THREADS = 32 * (H12_A_WARPS + H12_B_WARPS);
-constexpr int H12_STAGES = 3;
-constexpr int H12_ROW_BYTES = 12288 * 2;
-constexpr int H12_X_BYTES = 12288 * 4;
-constexpr int H12_BAR_OFF = 2 * H12_X_BYTES + H12_STAGES * H12_ROW_BYTES;
-constexpr int H12_SMEM = H12_BAR_OFF + 8 * (H12_STAGES + 4) + 16 + 2 * H12_B_WARPS * 4;
-constexpr int H12_BAR_A = 1;   // named barrier of the phase-A group
-constexpr int H12_BAR_B = 2;   // named barrier of the phase-B group
-
 // Eight codes from the low nibbles of eight magic-rounded floats (the low
 // byte holds the code in two's complement): even codes to the low nibbles,
 // odd codes to the high nibbles of four bytes.
@@ -245,227 +204,249 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t* u) {
   return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
 }
 
+// R4 = H12 (x) H1024 with the Sylvester factor split as H8 (x) H128 (jt =
+// j7..j9 outer, jl = j0..j6 inner).  Write row m as X[kappa][jl], kappa =
+// 8 i + jt (96 rows of 128 contiguous channels), and mu = 8 o + jt' for the
+// output block.  Then
+//     D[mu][jl] = sum_kappa A[mu][kappa] X[kappa][jl],
+//     A[mu][kappa] = H12[i][o] * H8[jt][jt'],
+//     y[128 mu + l] = sum_jl D[mu][jl] H128[jl][l] / sqrt(12288).
+// D is a dense bf16 x bf16 contraction with +-1 weights: the tensor core
+// forms it exactly in products with f32 accumulation (the bf16 input is its
+// own operand, no rounding before the MMA).  The H128 factor, the absmax,
+// the quantizer and the packing run in registers on the TMEM rows: one
+// thread owns the 128 consecutive output channels of one mu.
+//
+// Roles (one persistent CTA per SM, rows m = blockIdx.x + r * gridDim.x):
+//   warp 3, lane 0: TMA producer, two 64-column boxes per row (128-byte
+//     swizzle) into a ring of TC_STAGES rows;
+//   warp 7, lane 0: MMA issuer, six K = 16 steps per row into one of
+//     TC_NBUF TMEM accumulators of 128 columns;
+//   warps 4g + {0,1,2}: row group g < TC_NBUF (TMEM lane quadrants 0..2 =
+//     mu 0..95), the groups taking rows in turn; warp 11 idles.
+// Every wait is bounded; a group leaves its loop on one shared verdict
+// (barrier.cta.red.or), and the MMA thread drains its MMAs before the TMEM
+// is freed.
+constexpr int TC_STAGES = 6;
+constexpr int TC_NBUF = 3;                         // TMEM accumulators = row groups
+constexpr int TC_THREADS = 32 * 4 * TC_NBUF;       // 384
+constexpr int TC_ROW_BYTES = 12288 * 2;
+constexpr int TC_BOX_BYTES = 96 * 128;             // one 64-column box of a row
+constexpr int TC_A_ATOM = 128 * 128;               // 128 rows x 64 bf16 (one K atom)
+constexpr int TC_A_BYTES = 2 * TC_A_ATOM;          // K = 96 padded to two atoms
+constexpr int TC_BAR_OFF = TC_A_BYTES + TC_STAGES * TC_ROW_BYTES;
+constexpr int TC_NBARS = 2 * TC_STAGES + 2 * TC_NBUF + 1;
+constexpr int TC_MISC_OFF = TC_BAR_OFF + 8 * TC_NBARS;
+constexpr int TC_SMEM = TC_MISC_OFF + 16 + 4 * TC_NBUF * 2 * 3 + 1024;
+constexpr uint32_t TC_TMEM_COLS = 512;            // 128 * TC_NBUF, rounded to a power of 2
+constexpr int TC_TMA_WARP = 3;
+constexpr int TC_MMA_WARP = 7;
+static_assert(TC_SMEM <= 227 * 1024, "shared memory budget");
+static_assert(TC_A_BYTES % 1024 == 0 && TC_ROW_BYTES % 1024 == 0 && TC_BOX_BYTES % 1024 == 0,
+              "swizzle atoms need 1 KB alignment");
+
 template <bool CLAMP>
-__global__ void __launch_bounds__(H12_THREADS, 1)
-    rq_h12x1024_kernel(const uint16_t* __restrict__ x, int64_t ldx, int M, float norm,
-                       float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
-                       float* __restrict__ ascale) {
-  extern __shared__ __align__(128) uint8_t rq_smem[];
-  float* X = reinterpret_cast<float*>(rq_smem);                             // 2 x 12,288
-  uint16_t* stage = reinterpret_cast<uint16_t*>(rq_smem + 2 * H12_X_BYTES);  // ring of rows
-  uint64_t* sfull = reinterpret_cast<uint64_t*>(rq_smem + H12_BAR_OFF);
-  uint64_t* xfull = sfull + H12_STAGES;       // phase A wrote exchange buffer b
-  uint64_t* xempty = xfull + 2;               // phase B read exchange buffer b
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(xempty + 2);
-  float* red = reinterpret_cast<float*>(xempty + 2) + 4;   // [2][H12_B_WARPS]
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    rq_h12x1024_tc_kernel(const __grid_constant__ CUtensorMap map_x, int M, float norm,
+                          float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
+                          float* __restrict__ ascale) {
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* Asm = smem;
+  uint8_t* stage = smem + TC_A_BYTES;
+  uint64_t* sfull = reinterpret_cast<uint64_t*>(smem + TC_BAR_OFF);
+  uint64_t* sempty = sfull + TC_STAGES;
+  uint64_t* dfull = sempty + TC_STAGES;
+  uint64_t* dempty = dfull + TC_NBUF;
+  uint64_t* drain = dempty + TC_NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + TC_MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + TC_MISC_OFF + 4);
+  float* red = reinterpret_cast<float*>(smem + TC_MISC_OFF + 16);   // [group][parity][3]
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int nrows = M > static_cast<int>(blockIdx.x)
                         ? (M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                         : 0;
-  auto row_ptr = [&](int r) {
-    return x + (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(r) * gridDim.x) * ldx;
-  };
 
-  if (tid == 0) {
-    for (int s = 0; s < H12_STAGES; ++s) mbar_init(&sfull[s], 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&xfull[b], H12_A_WARPS);
-      mbar_init(&xempty[b], H12_B_WARPS);
+  // The constant operand A (K-major, 128-byte swizzle): row mu, column kappa
+  // at atom kappa / 64, byte (mu / 8) * 1024 + (mu % 8) * 128 + 16-byte chunk
+  // ((2 (kappa % 64)) / 16) ^ (mu % 8).  Rows 96..127 and kappa >= 96 are 0.
+  for (int e = tid; e < 128 * 128; e += TC_THREADS) {
+    const int mu = e >> 7, kap = e & 127;
+    float val = 0.f;
+    if (mu < 96 && kap < 96) {
+      const int o = mu >> 3, jtp = mu & 7, i = kap >> 3, jt = kap & 7;
+      val = static_cast<float>(paley12(i, o) * ((__popc(jt & jtp) & 1) ? -1 : 1));
     }
+    const int a = kap >> 6, kb = 2 * (kap & 63);
+    const int byte = a * TC_A_ATOM + (mu >> 3) * 1024 + (mu & 7) * 128 +
+                     ((((kb >> 4) ^ (mu & 7))) << 4) + (kb & 15);
+    *reinterpret_cast<__nv_bfloat16*>(Asm + byte) = __float2bfloat16_rn(val);
+  }
+  if (tid == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int b = 0; b < TC_NBUF; ++b) {
+      mbar_init(&dfull[b], 1);
+      mbar_init(&dempty[b], 3);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    fence_proxy_async_smem();
-    for (int r = 0; r < H12_STAGES && r < nrows; ++r) {
-      mbar_arrive_expect_tx(&sfull[r], H12_ROW_BYTES);
-      bulk_g2s(stage + r * 12288, row_ptr(r), H12_ROW_BYTES, &sfull[r]);
-    }
   }
+  if (warp == TC_MMA_WARP) {
+    tmem_alloc(tmem_slot, TC_TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();          // A was written by generic stores
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < H12_A_WARPS) {
-    // ------------------------------------------------------------ phase A
-    const int j = 64 * (warp >> 1) + 16 * (warp & 1) + (lane & 15) + 32 * (lane >> 4);
-    const int j6 = j >> 6, kk = j & 63;
-    const int p = 2 * (kk & 31) + (kk >> 5);
-    // exchange offset of (o, jt) = xpos(16 o + 2 jt + j6, kk): for jt and
-    // jt + 4 the segment differs by 8, so u mod 8 and the swizzle agree
-    int xo[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int s = 2 * q + j6;
-      xo[q] = (s << 6) + ((((p >> 2) ^ s)) << 2) + (p & 3);
-    }
-    int issued = nrows < H12_STAGES ? nrows : H12_STAGES;
-    int r = 0;
-    for (; r < nrows; ++r) {
-      const int s = r % H12_STAGES;
-      bool fail = !mbar_wait(&sfull[s], (r / H12_STAGES) & 1, spin_limit);
-      const uint16_t* xr = stage + s * 12288;
-      // z[i][q] = (value at jt = q, value at jt = q + 4)
-      f2 z[12][4];
-#pragma unroll
-      for (int i = 0; i < 12; ++i) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t lo = xr[i * 1024 + q * 128 + j];
-          const uint32_t hi = xr[i * 1024 + (q + 4) * 128 + j];
-          z[i][q].x = __uint_as_float(lo << 16);
-          z[i][q].y = __uint_as_float(hi << 16);
+  if (warp == TC_TMA_WARP) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int r = 0; r < nrows; ++r) {
+        const int s = r % TC_STAGES;
+        if (!mbar_wait(&sempty[s], ((r / TC_STAGES) & 1) ^ 1, spin_limit) || *abort_flag) {
+          *abort_flag = 1;
+          break;
         }
-      }
-      // every phase-A thread holds its values: the slot can be refilled
-      if (bar_any(H12_BAR_A, 32 * H12_A_WARPS, fail || *abort_flag)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (tid == 0 && r + H12_STAGES < nrows) {
-        mbar_arrive_expect_tx(&sfull[s], H12_ROW_BYTES);
-        bulk_g2s(stage + s * 12288, row_ptr(r + H12_STAGES), H12_ROW_BYTES, &sfull[s]);
+        const int m = static_cast<int>(blockIdx.x) + r * static_cast<int>(gridDim.x);
+        uint8_t* dst = stage + s * TC_ROW_BYTES;
+        mbar_arrive_expect_tx(&sfull[s], TC_ROW_BYTES);
+        tma_load_3d(dst, &map_x, 0, 0, m, &sfull[s]);
+        tma_load_3d(dst + TC_BOX_BYTES, &map_x, 64, 0, m, &sfull[s]);
         ++issued;
       }
-      // H8 over jt: bits 0 and 1 of q as packed pairs, bit 2 inside the pair
-#pragma unroll
-      for (int i = 0; i < 12; ++i) {
-#pragma unroll
-        for (int h = 1; h < 4; h <<= 1) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if ((q & h) == 0) {
-              const f2 a = z[i][q], b = z[i][q + h];
-              z[i][q] = add2(a, b);
-              z[i][q + h] = sub2(a, b);
-            }
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = z[i][q].x, b = z[i][q].y;
-          z[i][q].x = a + b;
-          z[i][q].y = a - b;
-        }
-      }
-      const int b = r & 1;
-      if (!mbar_wait(&xempty[b], ((r >> 1) & 1) ^ 1, spin_limit)) *abort_flag = 1;
-      float* Xb = X + b * 12288;
-      // H12 over i: column 0 of the Paley matrix is +1 then -1, so
-      // y_0 = z_0 - sum_{i>0} z_i; for o > 0, y_o = T - 2 (sum of the five
-      // z_i with H[i][o] = -1), T = sum of all z_i
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        f2 rest = z[1][q];
-#pragma unroll
-        for (int i = 2; i < 12; ++i) rest = add2(rest, z[i][q]);
-        const f2 T = add2(z[0][q], rest);
-        f2 y[12];
-        y[0] = sub2(z[0][q], rest);
-#pragma unroll
-        for (int o = 1; o < 12; ++o) {
-          f2 neg = {0.f, 0.f};
-          bool any = false;
-#pragma unroll
-          for (int i = 0; i < 12; ++i) {
-            if (paley12(i, o) < 0) {
-              neg = any ? add2(neg, z[i][q]) : z[i][q];
-              any = true;
-            }
-          }
-          y[o] = fma2(f2{-2.f, -2.f}, neg, T);
-        }
-#pragma unroll
-        for (int o = 0; o < 12; ++o) {
-          Xb[o * 1024 + xo[q]] = y[o].x;
-          Xb[o * 1024 + 512 + xo[q]] = y[o].y;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&xfull[b]);
+      // the latest copy into each slot must land before the CTA exits
+      for (int rr = issued > TC_STAGES ? issued - TC_STAGES : 0; rr < issued; ++rr)
+        mbar_wait(&sfull[rr % TC_STAGES], (rr / TC_STAGES) & 1, 0);
     }
-    // a group that stopped early lets its bulk copies land before exit
-    if (tid == 0) {
-      for (int rr = r; rr < issued; ++rr)
-        mbar_wait(&sfull[rr % H12_STAGES], (rr / H12_STAGES) & 1, 0);
+  } else if (warp == TC_MMA_WARP) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, 128, false, true);
+      const uint32_t a0 = smem_u32(Asm);
+      for (int r = 0; r < nrows; ++r) {
+        const int s = r % TC_STAGES, d = r % TC_NBUF;
+        if (!mbar_wait(&sfull[s], (r / TC_STAGES) & 1, spin_limit) ||
+            !mbar_wait(&dempty[d], ((r / TC_NBUF) & 1) ^ 1, spin_limit) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t b0 = smem_u32(stage + s * TC_ROW_BYTES);
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+          // A: K step k of 16 columns = 32 bytes inside atom k / 4;
+          // B: rows 16 k.. of both boxes (8-row atoms 1024 B apart, boxes
+          // TC_BOX_BYTES apart along the 128 channels)
+          mma_bf16(tmem_base + static_cast<uint32_t>(d * 128),
+                   desc_sw128(a0 + (k >> 2) * TC_A_ATOM + (k & 3) * 32),
+                   desc_sw128_mn(b0 + k * 2048, TC_BOX_BYTES, 1024), IDESC, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&sempty[s]);
+        mma_commit(&dfull[d]);
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0, 0);
     }
-  } else {
-    // ------------------------------------------------------------ phase B
-    const int u = tid - 32 * H12_A_WARPS;
-    const int bw = warp - H12_A_WARPS;
-    const float sg = (u & 1) ? -1.f : 1.f;
-    const f2 s2{sg, sg};
-    for (int r = 0; r < nrows; ++r) {
-      const int b = r & 1;
+    __syncwarp();
+  } else if ((warp & 3) != 3) {
+    const int g = warp >> 2, q = warp & 3;
+    const int mu = 32 * q + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    float* gred = red + g * 2 * 3;
+    int it = 0;
+    for (int r = g; r < nrows; r += TC_NBUF, ++it) {
+      const int d = r % TC_NBUF;
       const int m = static_cast<int>(blockIdx.x) + r * static_cast<int>(gridDim.x);
-      bool fail = !mbar_wait(&xfull[b], (r >> 1) & 1, spin_limit);
-      const float* Xb = X + b * 12288;
-      f2 v[32];                                   // v[j] = (value j, value j + 32)
+      const bool fail = !mbar_wait(&dfull[d], (r / TC_NBUF) & 1, spin_limit);
+      tc_fence_after();
+      // w[p] = (column 2p, column 2p + 1) of this thread's TMEM lane
+      f2 w[64];
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const float4 a = *reinterpret_cast<const float4*>(&Xb[(u << 6) + ((ch ^ (u & 7)) << 2)]);
-        v[2 * ch] = f2{a.x, a.y};
-        v[2 * ch + 1] = f2{a.z, a.w};
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[32];
+        tmem_ld32(lane_addr + static_cast<uint32_t>(d * 128 + 32 * c), t);
+#pragma unroll
+        for (int p = 0; p < 16; ++p)
+          w[16 * c + p] = f2{__uint_as_float(t[2 * p]), __uint_as_float(t[2 * p + 1])};
       }
+      tmem_ld_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&xempty[b]);
+      if (lane == 0) mbar_arrive(&dempty[d]);
+      // H128 over jl: bit 0 inside each pair, bits 1..6 across pairs
 #pragma unroll
-      for (int h = 1; h < 32; h <<= 1) {
+      for (int p = 0; p < 64; ++p) {
+        const float a = w[p].x, b = w[p].y;
+        w[p] = f2{a + b, a - b};
+      }
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          if ((jj & h) == 0) {
-            const f2 a = v[jj], c = v[jj + h];
-            v[jj] = add2(a, c);
-            v[jj + h] = sub2(a, c);
+      for (int h = 1; h < 64; h <<= 1) {
+#pragma unroll
+        for (int p = 0; p < 64; ++p) {
+          if ((p & h) == 0) {
+            const f2 a = w[p], b = w[p + h];
+            w[p] = add2(a, b);
+            w[p + h] = sub2(a, b);
           }
         }
-      }
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {            // bit j5: inside each pair
-        const float a = v[jj].x, c = v[jj].y;
-        v[jj] = f2{a + c, a - c};
-      }
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {            // bit j6: lanes u and u ^ 1
-        const f2 o{__shfl_xor_sync(0xffffffffu, v[jj].x, 1),
-                   __shfl_xor_sync(0xffffffffu, v[jj].y, 1)};
-        v[jj] = fma2(s2, v[jj], o);
       }
       float amax = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) amax = fmaxf(amax, fmaxf(fabsf(v[jj].x), fabsf(v[jj].y)));
+      for (int p = 0; p < 64; ++p) amax = fmaxf(amax, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      if (lane == 0) red[(r & 1) * H12_B_WARPS + bw] = amax;
-      // one barrier per row: publishes the partial maxima and the verdict
-      if (bar_any(H12_BAR_B, 32 * H12_B_WARPS, fail || *abort_flag)) {
+      if (lane == 0) gred[(it & 1) * 3 + q] = amax;
+      // one barrier per row and group: partial maxima and the verdict
+      if (bar_any(1 + g, 96, fail || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
-      amax = red[(r & 1) * H12_B_WARPS];
-#pragma unroll
-      for (int w = 1; w < H12_B_WARPS; ++w) amax = fmaxf(amax, red[(r & 1) * H12_B_WARPS + w]);
+      amax = fmaxf(fmaxf(gred[(it & 1) * 3], gred[(it & 1) * 3 + 1]), gred[(it & 1) * 3 + 2]);
       const float sc = row_scale(amax * norm, clip);
-      const float k = norm * __frcp_rn(sc);         // y_unnormalised -> y / scale
-      const f2 k2{k, k};
-      const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: round to nearest even
-      uint32_t ux[32], uy[32];
+      const f2 k2{norm * __frcp_rn(sc), norm * __frcp_rn(sc)};   // y_unnormalised -> y / scale
+      const f2 magic{12582912.f, 12582912.f};                  // 1.5 * 2^23: nearest even
+      uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + mu * 64);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        f2 c;
-        if (CLAMP) {
-          c = mul2(v[jj], k2);
-          c.x = fminf(fmaxf(c.x, -8.f), 7.f);
-          c.y = fminf(fmaxf(c.y, -8.f), 7.f);
-          c = add2(c, magic);
-        } else {
-          c = fma2(v[jj], k2, magic);
+      for (int n4 = 0; n4 < 4; ++n4) {
+        uint32_t word[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          uint32_t u8[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            f2 c;
+            if (CLAMP) {
+              c = mul2(w[16 * n4 + 4 * n + e], k2);
+              c.x = fminf(fmaxf(c.x, -8.f), 7.f);
+              c.y = fminf(fmaxf(c.y, -8.f), 7.f);
+              c = add2(c, magic);
+            } else {
+              c = fma2(w[16 * n4 + 4 * n + e], k2, magic);
+            }
+            u8[2 * e] = __float_as_uint(c.x);
+            u8[2 * e + 1] = __float_as_uint(c.y);
+          }
+          word[n] = pack8(u8);
         }
-        ux[jj] = __float_as_uint(c.x);              // channel jj
-        uy[jj] = __float_as_uint(c.y);              // channel jj + 32
+        dst[n4] = make_uint4(word[0], word[1], word[2], word[3]);
       }
-      uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + u * 32);
-      dst[0] = make_uint4(pack8(ux), pack8(ux + 8), pack8(ux + 16), pack8(ux + 24));
-      dst[1] = make_uint4(pack8(uy), pack8(uy + 8), pack8(uy + 16), pack8(uy + 24));
-      if (u == 0) ascale[m] = sc;
+      if (mu == 0) ascale[m] = sc;
     }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == TC_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TC_TMEM_COLS);
   }
 }
 
@@ -592,14 +573,30 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   const int m = static_cast<int>(M), k = static_cast<int>(K);
   if (x_bf16 && n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small)) {
+    // row m as a [96][128] bf16 tile: dims (jl, kappa, m), boxes of 64 x 96
+    auto encode = host::tensor_map_encoder();
+    if (!encode) return SQ_ERR_CUDA;
+    CUtensorMap map;
+    cuuint64_t dims[3] = {128, 96, static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[3] = {64, 96, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) {
+      host::set_error("cuTensorMapEncodeTiled(rotate) failed (%d)", static_cast<int>(cr));
+      return SQ_ERR_CUDA;
+    }
     const int grid = m < host::num_sms() ? m : host::num_sms();
     const bool clamp = clip < 1.0f;
-    auto kfn = clamp ? rq_h12x1024_kernel<true> : rq_h12x1024_kernel<false>;
+    auto kfn = clamp ? rq_h12x1024_tc_kernel<true> : rq_h12x1024_tc_kernel<false>;
     cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          H12_SMEM);
+                                          TC_SMEM);
     if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
-    kfn<<<grid, H12_THREADS, H12_SMEM, stream>>>(static_cast<const uint16_t*>(x), ld_x, m, norm,
-                                                 clip, host::spin_limit(), a_q, a_scale);
+    kfn<<<grid, TC_THREADS, TC_SMEM, stream>>>(map, m, norm, clip, host::spin_limit(), a_q,
+                                               a_scale);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_h12x1024 launch", e);
   }
