@@ -127,6 +127,10 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
  *           and whose kernel finishes leaves it zero-filled again.  After a
  *           device timeout (SQ_ERR_TIMEOUT) zero it again.  Concurrent calls
  *           must not share one workspace.  With NULL, no split-K is used.
+ *           A workspace of sq_w4a4_tail_workspace_bytes(M, N, K) bytes or
+ *           more also lets large-M shapes split their last, partial wave of
+ *           256 x 256 tiles into K halves (same zero-fill contract); with
+ *           less, that wave runs whole.  Results are identical either way.
  * Shape rules: M >= 0 (0 is a no-op), N % 16 == 0, N >= 16, K % 128 == 0,
  * 128 <= K <= 65536 (so |acc| < 2^31).
  * ------------------------------------------------------------------------- */
@@ -138,6 +142,16 @@ sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t
 /* Bytes of split-K workspace sq_w4a4_linear may use for this shape (0 if the
  * shape never splits). */
 size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Optional workspace for large M (M >= 256, N >= 256): with at least this
+ * many bytes, sq_w4a4_linear splits the tiles of a last wave that would
+ * occupy at most half of the SM pairs into two K halves, so the wave takes
+ * about half a tile's time.  The halves add their exact int32 partial sums
+ * in the workspace (int32 [tiles][256][256] plus two counters per tile); the
+ * second half to finish applies the epilogue and re-zeroes what it used.
+ * 0 for shapes that never take the CTA-pair path.  No counterpart in the
+ * paper: it only schedules the same integer sums differently. */
+size_t sq_w4a4_tail_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ---------------------------------------------------------------------------
  * sq_w4a4_linear_noalloc -- sq_w4a4_linear for callers that cannot allocate.

@@ -30,6 +30,7 @@ from .binding import (  # noqa: F401
     rotate_quant,
     version,
     w4a4_linear,
+    w4a4_tail_workspace_bytes,
     w4a4_workspace_bytes,
 )
 from .hadamard import paley_h12  # noqa: F401

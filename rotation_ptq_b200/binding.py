@@ -43,6 +43,8 @@ lib.sq_w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, 
                                ctypes.c_size_t, _vp]
 lib.sq_w4a4_workspace_bytes.restype = ctypes.c_size_t
 lib.sq_w4a4_workspace_bytes.argtypes = [_i64, _i64, _i64]
+lib.sq_w4a4_tail_workspace_bytes.restype = ctypes.c_size_t
+lib.sq_w4a4_tail_workspace_bytes.argtypes = [_i64, _i64, _i64]
 lib.sq_kv_rotate_quant.restype = _i32
 lib.sq_kv_rotate_quant.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -152,6 +154,10 @@ def w4a4_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib.sq_w4a4_workspace_bytes(M, N, K))
 
 
+def w4a4_tail_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.sq_w4a4_tail_workspace_bytes(M, N, K))
+
+
 def w4a4_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
                 w_scale: torch.Tensor, out_int32: bool = False, out: torch.Tensor = None,
                 workspace: torch.Tensor = None, use_workspace: bool = True):
@@ -170,7 +176,7 @@ def w4a4_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
     stream = _stream(a_q)
     ws_ptr, ws_bytes = None, 0
     if use_workspace:
-        need = w4a4_workspace_bytes(M, N, K)
+        need = max(w4a4_workspace_bytes(M, N, K), w4a4_tail_workspace_bytes(M, N, K))
         if workspace is not None:
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
         elif need > 0:
@@ -248,5 +254,6 @@ def debug_set_spin_limit(polls: int) -> None:
 
 
 def debug_set_gemm_path(path: int) -> None:
-    """0 = automatic, 1 = one-CTA tiles, 2 = CTA-pair tiles (large M)."""
+    """0 = automatic, 1 = one-CTA tiles, 2 = CTA-pair tiles with both operands
+    widened in shared memory, 3 = CTA-pair tiles with A in tensor memory."""
     lib.sq_debug_set_gemm_path(int(path))

@@ -198,6 +198,12 @@ size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return sq::gemm::workspace_bytes(M, N, K, sq::host::num_sms());
 }
 
+size_t sq_w4a4_tail_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N < 16 || N % 16 || K < 128 || K % 128 || K > 65536) return 0;
+  if (sq::host::current_device() < 0) return 0;
+  return sq::gemm::tail_workspace_bytes(M, N, K, sq::host::num_sms());
+}
+
 sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
                          const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
                          sq_out_kind kind, void* workspace, size_t workspace_bytes,

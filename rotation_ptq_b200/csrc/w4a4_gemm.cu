@@ -499,7 +499,11 @@ struct PairParams {
   int rowsA, rowsB;        // M, N
   int tilesM, tilesN;      // 256-wide tiles
   int KT;
-  int units;
+  int units;               // work units: full_units whole tiles, then K halves
+  int full_units;          // tiles computed over all of K (== units: no split)
+  int kt_half;             // k-tile where the two halves of a split tile meet
+  int* ws_acc;             // [split tiles][256 cols][256 rows] int32 partial sums, zero at rest
+  unsigned* ws_cnt;        // [split tiles][ticket x2 | ready x2], zero at rest
   const float* a_scale;
   const float* w_scale;
   void* out;
@@ -507,6 +511,19 @@ struct PairParams {
   int M, N;
   uint32_t spin_limit;
 };
+
+// Work unit u of a CTA pair: a whole tile, or one K half of a tile of the
+// last, partial wave (split so that the wave's tiles spread over twice as
+// many pairs; the two halves add up through the int32 workspace).
+struct PairUnit {
+  int tile, kt0, kt1, part;   // part -1: whole tile; 0 / 1: K half
+};
+__device__ __forceinline__ PairUnit pair_unit(const PairParams& p, int u) {
+  if (u < p.full_units) return PairUnit{u, 0, p.KT, -1};
+  const int v = u - p.full_units;
+  const int tile = p.full_units + (v >> 1);
+  return (v & 1) ? PairUnit{tile, p.kt_half, p.KT, 1} : PairUnit{tile, 0, p.kt_half, 0};
+}
 
 template <int PST, int UST>
 struct PairLayout {
@@ -816,10 +833,12 @@ struct PairTSLayout {
   static constexpr int BAR_OFF = P_OFF + PST * PSTAGE;
   static constexpr int NBAR = 2 * PST + 2 * UST + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int BYTES = MISC_OFF + 32 + 1024;
+  static constexpr int WSC_OFF = (MISC_OFF + 32 + 15) & ~15;   // the tile's 256 w_scale values
+  static constexpr int BYTES = WSC_OFF + 256 * 4 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t A_COL0 = 256;             // A slots follow the accumulator
   static_assert(UST * 32 <= 256, "A slots must fit beside the accumulator");
+  static_assert(WSC_OFF % 16 == 0, "the scale buffer is read as float4");
   static_assert(BYTES <= 227 * 1024, "shared memory budget");
   static_assert(P_OFF % 1024 == 0 && PSTAGE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
@@ -846,6 +865,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+  float* wsc = reinterpret_cast<float*>(smem + L::WSC_OFF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -884,8 +904,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int u = pair_id; ok && u < p.units && !*abort_flag; u += num_pairs) {
-        const int tm = u % p.tilesM, tn = u / p.tilesM;
-        for (int kt = 0; kt < p.KT; kt += KM, ++it) {
+        const PairUnit un = pair_unit(p, u);
+        const int tm = un.tile % p.tilesM, tn = un.tile / p.tilesM;
+        for (int kt = un.kt0; kt < un.kt1; kt += KM, ++it) {
           const int ps = it % PST;
           const uint32_t ph = (it / PST) & 1;
           if (!mbar_wait(&pempty[ps], ph ^ 1, p.spin_limit)) {
@@ -927,7 +948,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t itp = 0;
     bool ok = true;
     for (int u = pair_id; ok && u < p.units; u += num_pairs) {
-      for (int kt = 0; ok && kt < p.KT; kt += KM, ++itp) {
+      const PairUnit un = pair_unit(p, u);
+      for (int kt = un.kt0; ok && kt < un.kt1; kt += KM, ++itp) {
         const int ps = itp % PST;
         const uint32_t pph = (itp / PST) & 1;
         bool got = mbar_wait(&pfull[ps], pph, p.spin_limit);
@@ -938,7 +960,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
-        const int nsub = min(KM, p.KT - kt);
+        const int nsub = min(KM, un.kt1 - kt);
         // one protocol round per packed stage: wait for its group of int8
         // slots, widen every k-tile, fence, one arrival
         const int g = itp % G;
@@ -994,13 +1016,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC = idesc_i8(256, 256);
       uint32_t ig = 0, acc_it = 0;
       for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
+        const PairUnit un = pair_unit(p, u);
         if (*abort_flag || !mbar_wait(tempty, (acc_it & 1) ^ 1, p.spin_limit)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
         bool ok = true;
-        for (int kt = 0; kt < p.KT; kt += KM, ++ig) {
+        for (int kt = un.kt0; kt < un.kt1; kt += KM, ++ig) {
           const int g = ig % G;
           if (!mbar_wait(&ufull[g], (ig / G) & 1, p.spin_limit) || *abort_flag) {
             *abort_flag = 1;
@@ -1008,7 +1031,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const int nsub = min(KM, p.KT - kt);
+          const int nsub = min(KM, un.kt1 - kt);
           for (int sub = 0; sub < nsub; ++sub) {
             const int slot = g * KM + sub;
             const uint32_t a_tmem = tmem_base + L::A_COL0 + static_cast<uint32_t>(slot * 32);
@@ -1017,7 +1040,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int kk = 0; kk < BK / UMMA_K; ++kk) {
               mma_i8_pair_ts(tmem_base, a_tmem + kk * (UMMA_K / 4),
                              desc_sw128(b_addr + kk * UMMA_K), IDESC,
-                             (kt + sub > 0 || kk > 0) ? 1u : 0u);
+                             (kt + sub > un.kt0 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit_pair_mc(&uempty[g], 0x3);
@@ -1031,15 +1054,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = warp * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
+    // 16 exact sums of row m, columns n0..n0+15 -> int32 or scaled bf16
+    auto emit16 = [&](int m, int n0, float sa, const int (&v)[16]) {
+      if (p.out_i32) {
+        int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
+                                            static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = make_int4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      } else {
+        const float4* sw4 = reinterpret_cast<const float4*>(wsc + (n0 & 255));
+        uint32_t packed[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 sw = sw4[j];
+          const float sj[4] = {sw.x, sw.y, sw.z, sw.w};
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int kk = 4 * j + e;
+            const float f0 = static_cast<float>(v[kk]) * sa * sj[e];
+            const float f1 = static_cast<float>(v[kk + 1]) * sa * sj[e + 1];
+            __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+            packed[kk / 2] = *reinterpret_cast<uint32_t*>(&h);
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                              static_cast<int64_t>(m) * p.N + n0);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      }
+    };
     uint32_t acc_it = 0;
     for (int u = pair_id; u < p.units; u += num_pairs, ++acc_it) {
-      const int tm = u % p.tilesM, tn = u / p.tilesM;
+      const PairUnit un = pair_unit(p, u);
+      const int tm = un.tile % p.tilesM, tn = un.tile / p.tilesM;
+      // this tile's weight scales, fetched while the mainloop runs
+      float2 wpre = make_float2(0.f, 0.f);
+      {
+        const int n = tn * 256 + 2 * static_cast<int>(threadIdx.x);
+        if (n < p.N) wpre = *reinterpret_cast<const float2*>(p.w_scale + n);
+      }
       if (threadIdx.x == 0) {
         const bool ok = !*abort_flag && mbar_wait(tfull, acc_it & 1, p.spin_limit);
         if (!ok) *abort_flag = 1;
         bcast[0] = ok ? 1 : 0;
       }
       named_bar_sync(1, EPI_WARPS * 32);
+      // every epilogue thread is past the previous tile: refill the scales
+      reinterpret_cast<float2*>(wsc)[threadIdx.x] = wpre;
       const bool ok = bcast[0] != 0;
       named_bar_sync(1, EPI_WARPS * 32);
       if (!ok) break;
@@ -1047,6 +1109,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m = tm * 256 + static_cast<int>(rank) * L::HALF + row;
       const bool m_valid = m < p.M;
       const float sa = m_valid ? p.a_scale[m] : 0.f;
+      // K half of a split tile: the first half to reach its epilogue stores
+      // its partial sums (column-major: a warp's 32 rows of one column are
+      // one 128-byte line) and raises `ready`; the second waits for `ready`
+      // (the first is already running, so the wait ends), adds, and emits.
+      int* wcol = nullptr;
+      unsigned* ticket = nullptr;
+      unsigned* ready = nullptr;
+      bool first = false;
+      if (un.part >= 0) {
+        const int t = un.tile - p.full_units;
+        wcol = p.ws_acc + static_cast<int64_t>(t) * 256 * 256 + static_cast<int>(rank) * L::HALF +
+               row;
+        ticket = p.ws_cnt + t * 4 + rank;
+        ready = p.ws_cnt + t * 4 + 2 + rank;
+        if (threadIdx.x == 0) {
+          const unsigned order = atomicAdd(ticket, 1u);
+          bool ok2 = true;
+          if (order == 1u) {
+            // bounded wait for the first half's partial sums
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t polls = 1;; ++polls) {
+              unsigned r;
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(r) : "l"(ready) : "memory");
+              if (r != 0u) break;
+              if ((p.spin_limit != 0 && polls >= p.spin_limit) ||
+                  ((polls & 255u) == 0 && globaltimer_ns() - t0 > kWaitNs)) {
+                record_status(SQ_ERR_TIMEOUT);
+                *abort_flag = 1;
+                ok2 = false;
+                break;
+              }
+            }
+          }
+          bcast[1] = order == 0u ? 1 : (ok2 ? 0 : 2);
+        }
+        named_bar_sync(1, EPI_WARPS * 32);
+        first = bcast[1] == 1;
+        if (bcast[1] == 2) wcol = nullptr;     // gave up: emit this half alone
+        named_bar_sync(1, EPI_WARPS * 32);
+      }
       // four 16-column loads in flight per wait: 64 accumulator columns
 #pragma unroll 1
       for (int c4 = 0; c4 < 16; c4 += 4) {
@@ -1055,46 +1157,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int g = 0; g < 4; ++g)
           tmem_ld16(lane_addr + static_cast<uint32_t>((c4 + g) * 16), vv[g]);
         tmem_ld_wait();
+        int v4[4][16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v4[g][j] = static_cast<int>(vv[g][j]) >> 8;
+        if (wcol != nullptr) {
+          int* wc = wcol + c4 * 16 * 256;
+          if (first) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) wc[(g * 16 + j) * 256] = v4[g][j];
+            continue;
+          }
+          // the batch's 64 partial sums are all loaded before any store
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v4[g][j] += __ldcg(wc + (g * 16 + j) * 256);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) wc[(g * 16 + j) * 256] = 0;
+        }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-        const int c = c4 + g;
-        const uint32_t (&v)[16] = vv[g];
-        const int n0 = tn * 256 + c * 16;
-        if (!m_valid || n0 >= p.N) continue;
-        if (p.out_i32) {
-          int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
-                                              static_cast<int64_t>(m) * p.N + n0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_int4(static_cast<int>(v[4 * j]) >> 8, static_cast<int>(v[4 * j + 1]) >> 8,
-                               static_cast<int>(v[4 * j + 2]) >> 8,
-                               static_cast<int>(v[4 * j + 3]) >> 8);
-        } else {
-          const float4* sw4 = reinterpret_cast<const float4*>(p.w_scale + n0);
-          uint32_t packed[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float4 s = __ldg(sw4 + j);
-            const float sj[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-              const int k = 4 * j + e;
-              const float f0 = static_cast<float>(static_cast<int>(v[k]) >> 8) * sa * sj[e];
-              const float f1 = static_cast<float>(static_cast<int>(v[k + 1]) >> 8) * sa * sj[e + 1];
-              __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
-              packed[k / 2] = *reinterpret_cast<uint32_t*>(&h);
-            }
-          }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                static_cast<int64_t>(m) * p.N + n0);
-          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        }
+          const int n0 = tn * 256 + (c4 + g) * 16;
+          if (!m_valid || n0 >= p.N) continue;
+          emit16(m, n0, sa, v4[g]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed_n(tempty_leader, 32);
+      if (un.part >= 0) {
+        if (first) {
+          // publish the partial sums, then raise `ready`
+          __threadfence();
+          named_bar_sync(1, EPI_WARPS * 32);
+          if (threadIdx.x == 0)
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ready), "r"(1u) : "memory");
+        } else if (threadIdx.x == 0) {
+          // both halves are done with this tile: rearm for the next call
+          *ticket = 0u;
+          *ready = 0u;
+        }
+      }
     }
   }
 
@@ -1158,9 +1267,19 @@ static sq_status launch(const Plan& plan, const uint8_t* opA, const uint8_t* opB
 }
 
 
+// Workspace of a split tail of `tail` tiles: int32 partial sums of 256 x 256
+// per tile, then two arrival counters per tile.
+static size_t tail_acc_bytes(int tail) {
+  return (static_cast<size_t>(tail) * 256 * 256 * 4 + 255) & ~static_cast<size_t>(255);
+}
+static size_t tail_ws_bytes(int tail) {
+  return tail_acc_bytes(tail) + ((static_cast<size_t>(tail) * 4 * 4 + 255) & ~static_cast<size_t>(255));
+}
+
 template <bool TS, int PST, int UST>
 static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, int64_t N,
-                             int64_t K, PairParams prm, int num_sms, cudaStream_t stream) {
+                             int64_t K, PairParams prm, int num_sms, cudaStream_t stream,
+                             void* ws, size_t ws_bytes) {
   constexpr int BYTES = [] {
     if constexpr (TS) return PairTSLayout<PST, UST>::BYTES;
     else return PairLayout<PST, UST>::BYTES;
@@ -1201,6 +1320,24 @@ static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, 
     max_clusters[dev & 63] = n;
   }
   const int pairs = prm.units < max_clusters[dev & 63] ? prm.units : max_clusters[dev & 63];
+  prm.full_units = prm.units;
+  if constexpr (TS) {
+    // A last wave that fills at most half of the pairs is split by K in two
+    // halves (when the caller's workspace holds the partial sums).  Halves
+    // shorter than 32 k-tiles do not repay the partial-sum round trip.
+    const int tiles = prm.units;
+    const int full = tiles / pairs * pairs;
+    const int tail = tiles - full;
+    const int kt_half = prm.KT / 2 / KM * KM;
+    if (ws != nullptr && tail > 0 && 2 * tail <= pairs && kt_half >= 32 && kt_half < prm.KT &&
+        ws_bytes >= tail_ws_bytes(tail)) {
+      prm.full_units = full;
+      prm.units = full + 2 * tail;
+      prm.kt_half = kt_half;
+      prm.ws_acc = static_cast<int*>(ws);
+      prm.ws_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + tail_acc_bytes(tail));
+    }
+  }
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, mapA, mapB, prm);
   if (e != cudaSuccess) return host::cuda_fail("w4a4_gemm_pair launch", e);
@@ -1251,6 +1388,14 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
   return pl;
 }
 
+size_t tail_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= 0 || N <= 0 || K < BK || !use_pair(M, N)) return 0;
+  // at most a quarter of the SMs' worth of tail tiles: half of the pairs
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t cap = num_sms / 4 > 0 ? num_sms / 4 : 1;
+  return tail_ws_bytes(static_cast<int>(tiles < cap ? tiles : cap));
+}
+
 size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K < BK) return 0;
   if (use_pair(M, N)) return 0;
@@ -1280,8 +1425,9 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
     pp.M = static_cast<int>(M);
     pp.N = static_cast<int>(N);
     pp.spin_limit = spin_limit;
-    if (host::gemm_path() == 2) return launch_pair<false, 3, 4>(a_q, w_q, M, N, K, pp, num_sms, stream);
-    return launch_pair<true, 3, 8>(a_q, w_q, M, N, K, pp, num_sms, stream);
+    if (host::gemm_path() == 2)
+      return launch_pair<false, 3, 4>(a_q, w_q, M, N, K, pp, num_sms, stream, nullptr, 0);
+    return launch_pair<true, 3, 8>(a_q, w_q, M, N, K, pp, num_sms, stream, ws, ws_bytes);
   }
   Plan pl = forced ? *forced : plan_gemm(M, N, K, ws != nullptr, num_sms);
   Params prm{};

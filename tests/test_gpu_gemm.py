@@ -157,3 +157,29 @@ def test_large_m_kernels_agree(cuda_ok, path, M, N, K):
     rows = P.sample_rows(M, 24, seed=path)
     got = acc[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64)
     assert np.array_equal(got, O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w)))
+
+
+@pytest.mark.parametrize("out_int32", [True, False])
+def test_split_tail_matches_whole_tiles(cuda_ok, out_int32):
+    # 80 tiles of 256 x 256 on 74 CTA pairs: the 6 tiles of the last wave run
+    # as 12 K halves summed in the workspace.  Same result as without a
+    # workspace (whole tiles), exact int32, workspace left zero.
+    import rotation_ptq_b200 as sq
+    M, N, K = 2560, 2048, 1024
+    a, w, sa, sw = _operands(M, N, K, 808)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    nbytes = sq.w4a4_tail_workspace_bytes(M, N, K)
+    assert nbytes >= 6 * 256 * 256 * 4
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    split = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=out_int32, workspace=ws)
+    split2 = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=out_int32, workspace=ws)
+    whole = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=out_int32, use_workspace=False)
+    torch.cuda.synchronize()
+    assert sq.device_status() == 0
+    assert int(ws.count_nonzero()) == 0
+    assert torch.equal(split, whole) and torch.equal(split2, whole)
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    if out_int32:
+        assert np.array_equal(split.cpu().numpy().astype(np.int64), ref)
+    else:
+        P.check_fro(split.float().cpu().numpy(), O.dequant(ref, sa, sw))
