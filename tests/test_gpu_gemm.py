@@ -162,10 +162,10 @@ def test_large_m_kernels_agree(cuda_ok, path, M, N, K):
 @pytest.mark.parametrize("out_int32", [True, False])
 def test_split_tail_matches_whole_tiles(cuda_ok, out_int32):
     # 80 tiles of 256 x 256 on 74 CTA pairs: the 6 tiles of the last wave run
-    # as 12 K halves summed in the workspace.  Same result as without a
-    # workspace (whole tiles), exact int32, workspace left zero.
+    # as 12 K halves (32 k-tiles each) summed in the workspace.  Same result
+    # as without a workspace (whole tiles), exact int32, workspace left zero.
     import rotation_ptq_b200 as sq
-    M, N, K = 2560, 2048, 1024
+    M, N, K = 2560, 2048, 8192
     a, w, sa, sw = _operands(M, N, K, 808)
     da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
     nbytes = sq.w4a4_tail_workspace_bytes(M, N, K)
