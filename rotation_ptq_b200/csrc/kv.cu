@@ -6,12 +6,23 @@
 // path is folded offline, so V is only quantized.  SpinQuant abstract: the KV
 // cache is 4-bit.
 //
-// Thread layout (rotate/quant): one CTA handles one token; each head vector
-// of 128 values is owned by 4 consecutive lanes.  For Q and K the lane with
-// sub-index s holds elements s*16 + t and 64 + s*16 + t (t < 16), so each
-// RoPE pair (i, i + 64) sits in one thread, five of the seven butterfly bits
-// (j0..j3 and j6) are in-thread, and the remaining two (j4, j5 = s) take one
-// shuffle each.  V lanes hold 32 consecutive values.
+// Thread layout (rotate/quant): a CTA takes two tokens per iteration; each
+// head vector of 128 values is owned by 2 adjacent lanes.  Items are ordered
+// [Q of token 0 | Q of token 1 | K of both | V of both], so with 8 | hq and
+// 8 | hkv no warp mixes item kinds.  For Q and K the lane with sub-index s
+// holds elements s*32 + t and 64 + s*32 + t (t < 32) as float pairs: each
+// RoPE pair (i, i + 64) sits in one pair, the butterfly bits j0..j4 run
+// across the thread's pairs (f32x2), j6 inside each pair, and j5 = s takes
+// one shuffle with the partner lane.  V lanes hold 64 consecutive values.
+//
+// Quantization follows the pinned asymmetric rule, with one division per
+// group for the scale and the zero point.  V codes use the exactly rounded
+// quotient x / scale (raw bf16 inputs meet exact .5 ties often); K codes are
+// clamp(rint(x * k + zero), 0, 15) with k = norm / scale in float32, K being
+// rotated without the 1/sqrt(128) factor (its float32 rotation already
+// differs from the exact one in the last bits, so the codes can differ from
+// the oracle's only at a rounding tie); K's scale and zero point come from
+// the normalised extremes.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -22,11 +33,13 @@ namespace sq {
 namespace kv {
 
 constexpr int D = 128;
+constexpr float kNorm = 0.08838834764831845f;   // 1/sqrt(128)
 
-__device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* v) {
+// 32 bf16 (64 bytes, 16-byte aligned) -> 32 floats.
+__device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, float* v) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < 4; ++h) {
     const uint4 w = __ldcs(q + h);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -37,41 +50,26 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* v) {
   }
 }
 
+__device__ __forceinline__ uint32_t bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ void store16_bf16(__nv_bfloat16* p, const float* v) {
   uint32_t w[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-    w[e] = *reinterpret_cast<uint32_t*>(&h);
-  }
+  for (int e = 0; e < 8; ++e) w[e] = bf16x2(v[2 * e], v[2 * e + 1]);
   uint4* q = reinterpret_cast<uint4*>(p);
   q[0] = make_uint4(w[0], w[1], w[2], w[3]);
   q[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// In-thread Walsh-Hadamard butterflies over 16 values (natural order).
-__device__ __forceinline__ void fwht16(float* v) {
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
-      }
-    }
-  }
-}
-
-// Asymmetric 4-bit parameters over a 128-value group held by 4 lanes.
-// `gmask` names the 4 lanes of the group; all of them call this together.
-__device__ __forceinline__ void asym_params(float lo, float hi, unsigned gmask, float& scale,
-                                            float& zero) {
-  lo = fminf(lo, __shfl_xor_sync(gmask, lo, 1));
-  lo = fminf(lo, __shfl_xor_sync(gmask, lo, 2));
-  hi = fmaxf(hi, __shfl_xor_sync(gmask, hi, 1));
-  hi = fmaxf(hi, __shfl_xor_sync(gmask, hi, 2));
+// Asymmetric parameters of a group from its (normalised) extremes, with the
+// group's other lane: scale = (max' - min') / 15, zero = rint(-min' / scale).
+__device__ __forceinline__ void asym_params2(float lo, float hi, unsigned pmask, float& scale,
+                                             float& zero) {
+  lo = fminf(lo, __shfl_xor_sync(pmask, lo, 1));
+  hi = fmaxf(hi, __shfl_xor_sync(pmask, hi, 1));
   lo = fminf(lo, 0.f);
   hi = fmaxf(hi, 0.f);
   scale = __fdiv_rn(hi - lo, 15.0f);
@@ -79,19 +77,45 @@ __device__ __forceinline__ void asym_params(float lo, float hi, unsigned gmask, 
   zero = fminf(fmaxf(rintf(__fdiv_rn(-lo, scale)), 0.f), 15.f);
 }
 
-__device__ __forceinline__ uint32_t ucode(float x, float scale, float zero) {
-  const float c = fminf(fmaxf(rintf(__fdiv_rn(x, scale)) + zero, 0.f), 15.f);
-  return static_cast<uint32_t>(c);
+// 8 unsigned codes clamp(rint(x k + zero), 0, 15) packed into one word (even
+// element in the low nibble); x given as 4 float pairs.  For operands whose
+// quotient by the scale must round exactly as float32 division does (raw
+// bf16 values meet exact .5 ties often), see ucodes8_div.
+__device__ __forceinline__ uint32_t ucodes8(const f2* x, f2 k2, f2 z2) {
+  const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
+  uint32_t u[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f2 c = fma2(x[e], k2, z2);
+    c.x = fminf(fmaxf(c.x, 0.f), 15.f);
+    c.y = fminf(fmaxf(c.y, 0.f), 15.f);
+    c = add2(c, magic);
+    u[2 * e] = __float_as_uint(c.x);
+    u[2 * e + 1] = __float_as_uint(c.y);
+  }
+  return pack8(u);
 }
 
-// Pack 16 unsigned codes (even element in the low nibble) into 8 bytes.
-__device__ __forceinline__ uint2 pack16(const float* v, float scale, float zero) {
-  uint32_t w0 = 0, w1 = 0;
+// As ucodes8 with the quotient x / scale rounded exactly like IEEE float32
+// division: q = x r, e = x - q s, q' = q + e r with r = RN(1 / s), the
+// one-step fma correction of Markstein ("IA-64 and Elementary Functions",
+// 2000), which yields the correctly rounded quotient when r is the correctly
+// rounded reciprocal.  Then rint(q') + zero, clamped to [0, 15].
+__device__ __forceinline__ uint32_t ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2 z2) {
+  const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
+  const float lo = 12582912.f, hi = 12582912.f + 15.f;
+  uint32_t u[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) w0 |= ucode(v[e], scale, zero) << (4 * e);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) w1 |= ucode(v[8 + e], scale, zero) << (4 * e);
-  return make_uint2(w0, w1);
+  for (int e = 0; e < 4; ++e) {
+    const f2 q = mul2(x[e], r2);
+    const f2 er = fma2(q, s2neg, x[e]);
+    f2 c = add2(add2(fma2(er, r2, q), magic), z2);   // magic + rint(q') + zero, exact
+    c.x = fminf(fmaxf(c.x, lo), hi);
+    c.y = fminf(fmaxf(c.y, lo), hi);
+    u[2 * e] = __float_as_uint(c.x);
+    u[2 * e + 1] = __float_as_uint(c.y);
+  }
+  return pack8(u);
 }
 
 template <bool ROPE>
@@ -102,115 +126,163 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
     const float* __restrict__ rsin, int max_pos, __nv_bfloat16* __restrict__ q_out,
     uint8_t* __restrict__ k_cache, float* __restrict__ k_scale, uint8_t* __restrict__ k_zero,
     uint8_t* __restrict__ v_cache, float* __restrict__ v_scale, uint8_t* __restrict__ v_zero) {
-  const int nvec = hq + 2 * hkv;                 // head vectors per token
-  const int lanes = nvec * 4;
-  const float norm = 0.08838834764831845f;       // 1/sqrt(128)
-  for (int t = blockIdx.x; t < T; t += gridDim.x) {
-    int p = 0;
-    if (ROPE) {
-      p = pos[t];
-      if (p < 0 || p >= max_pos) {
-        if (threadIdx.x == 0) record_status(SQ_ERR_INVALID_ARG);
+  const int nq = 4 * hq, nk = 4 * hkv;           // lanes per token pair
+  const int items = nq + 2 * nk;
+  const int lane = threadIdx.x & 31;
+  const unsigned pmask = 0x3u << (lane & 30);    // this vector's 2 lanes
+  for (int t0 = 2 * blockIdx.x; t0 < T; t0 += 2 * gridDim.x) {
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      int kind, tok, head, s;
+      if (it < nq) {
+        kind = 0;
+        tok = t0 + it / (2 * hq);
+        head = (it % (2 * hq)) >> 1;
+      } else {
+        const int j = it < nq + nk ? it - nq : it - nq - nk;
+        kind = it < nq + nk ? 1 : 2;
+        tok = t0 + j / (2 * hkv);
+        head = (j % (2 * hkv)) >> 1;
+      }
+      s = it & 1;
+      if (tok >= T) continue;                    // both lanes of a vector leave together
+      if (kind == 2) {
+        // V: 64 consecutive values, asymmetric 4-bit
+        const int64_t g = static_cast<int64_t>(tok) * hkv + head;
+        float x[64];
+        load32_bf16(v + g * D + s * 64, x);
+        load32_bf16(v + g * D + s * 64 + 32, x + 32);
+        float mn = x[0], mx = x[0];
+#pragma unroll
+        for (int i = 1; i < 64; ++i) {
+          mn = fminf(mn, x[i]);
+          mx = fmaxf(mx, x[i]);
+        }
+        float scale, zero;
+        asym_params2(mn, mx, pmask, scale, zero);
+        const float rs = __frcp_rn(scale);
+        const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
+        uint32_t w[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          const f2 xs[4] = {f2{x[8 * n], x[8 * n + 1]}, f2{x[8 * n + 2], x[8 * n + 3]},
+                            f2{x[8 * n + 4], x[8 * n + 5]}, f2{x[8 * n + 6], x[8 * n + 7]}};
+          w[n] = ucodes8_div(xs, r2, sn2, z2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(v_cache + g * (D / 2) + s * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (s == 0) {
+          v_scale[g] = scale;
+          v_zero[g] = static_cast<uint8_t>(zero);
+        }
         continue;
       }
-    }
-    for (int lt = threadIdx.x; lt < ((lanes + 31) & ~31); lt += blockDim.x) {
-      const int vec = lt >> 2, s = lt & 3;
-      const bool active = vec < nvec;
-      const bool is_v = vec >= hq + hkv;
-      if (!active) continue;                 // whole groups of 4 lanes leave together
-      const unsigned gmask = 0xFu << (threadIdx.x & 28);   // this vector's 4 lanes
-      if (!is_v) {
-        const bool is_q = vec < hq;
-        const int head = is_q ? vec : vec - hq;
-        const __nv_bfloat16* src =
-            is_q ? q + (static_cast<int64_t>(t) * hq + head) * D
-                 : k + (static_cast<int64_t>(t) * hkv + head) * D;
-        float lo[16], hi[16];
-        load16_bf16(src + s * 16, lo);
-        load16_bf16(src + 64 + s * 16, hi);
+      int p = 0;
+      if (ROPE) {
+        p = pos[tok];
+        if (p < 0 || p >= max_pos) {
+          if (s == 0) record_status(SQ_ERR_INVALID_ARG);
+          continue;
+        }
+      }
+      const bool is_q = kind == 0;
+      const __nv_bfloat16* src = is_q ? q + (static_cast<int64_t>(tok) * hq + head) * D
+                                      : k + (static_cast<int64_t>(tok) * hkv + head) * D;
+      // w[t] = (element s*32 + t, element 64 + s*32 + t)
+      f2 w[32];
+      {
+        float lo[32], hi[32];
+        load32_bf16(src + s * 32, lo);
+        load32_bf16(src + 64 + s * 32, hi);
         if (ROPE) {
-          const float4* c4 = reinterpret_cast<const float4*>(rcos + static_cast<int64_t>(p) * 64 + s * 16);
-          const float4* s4 = reinterpret_cast<const float4*>(rsin + static_cast<int64_t>(p) * 64 + s * 16);
+          const float4* c4 = reinterpret_cast<const float4*>(rcos + static_cast<int64_t>(p) * 64 + s * 32);
+          const float4* s4 = reinterpret_cast<const float4*>(rsin + static_cast<int64_t>(p) * 64 + s * 32);
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
+          for (int qd = 0; qd < 8; ++qd) {
             const float4 c = __ldg(c4 + qd), sn = __ldg(s4 + qd);
             const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {sn.x, sn.y, sn.z, sn.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int i = qd * 4 + e;
               const float a = lo[i], b = hi[i];
-              lo[i] = a * cc[e] - b * ss[e];
-              hi[i] = b * cc[e] + a * ss[e];
+              w[i] = f2{a * cc[e] - b * ss[e], b * cc[e] + a * ss[e]};
             }
           }
-        }
-        fwht16(lo);
-        fwht16(hi);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {          // bit j6: the two halves
-          const float a = lo[i], b = hi[i];
-          lo[i] = a + b;
-          hi[i] = a - b;
-        }
-#pragma unroll
-        for (int mask = 1; mask <= 2; mask <<= 1) {   // bits j4, j5 across lanes
-          const bool upper = (s & mask) != 0;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float o1 = __shfl_xor_sync(gmask, lo[i], mask);
-            const float o2 = __shfl_xor_sync(gmask, hi[i], mask);
-            lo[i] = upper ? o1 - lo[i] : lo[i] + o1;
-            hi[i] = upper ? o2 - hi[i] : hi[i] + o2;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          lo[i] *= norm;
-          hi[i] *= norm;
-        }
-        if (is_q) {
-          __nv_bfloat16* dst = q_out + (static_cast<int64_t>(t) * hq + head) * D;
-          store16_bf16(dst + s * 16, lo);
-          store16_bf16(dst + 64 + s * 16, hi);
         } else {
-          float mn = lo[0], mx = lo[0];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            mn = fminf(mn, fminf(lo[i], hi[i]));
-            mx = fmaxf(mx, fmaxf(lo[i], hi[i]));
+          for (int i = 0; i < 32; ++i) w[i] = f2{lo[i], hi[i]};
+        }
+      }
+      // H128: bits j0..j4 across pairs, j6 inside pairs, j5 with the partner
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & h) == 0) {
+            const f2 a = w[i], b = w[i + h];
+            w[i] = add2(a, b);
+            w[i + h] = sub2(a, b);
           }
-          float scale, zero;
-          asym_params(mn, mx, gmask, scale, zero);
-          const int64_t g = static_cast<int64_t>(t) * hkv + head;
-          uint8_t* dst = k_cache + g * (D / 2);
-          *reinterpret_cast<uint2*>(dst + s * 8) = pack16(lo, scale, zero);
-          *reinterpret_cast<uint2*>(dst + 32 + s * 8) = pack16(hi, scale, zero);
-          if (s == 0) {
-            k_scale[g] = scale;
-            k_zero[g] = static_cast<uint8_t>(zero);
-          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = f2{w[i].x + w[i].y, w[i].x - w[i].y};
+      {
+        const float sg = s ? -1.f : 1.f;
+        const f2 s2{sg, sg};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const f2 o{__shfl_xor_sync(pmask, w[i].x, 1), __shfl_xor_sync(pmask, w[i].y, 1)};
+          w[i] = fma2(s2, w[i], o);
+        }
+      }
+      if (is_q) {
+        const f2 n2{kNorm, kNorm};
+        __nv_bfloat16* dst = q_out + (static_cast<int64_t>(tok) * hq + head) * D;
+        uint32_t lo_w[16], hi_w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const f2 a = mul2(w[i], n2), b = mul2(w[i + 1], n2);
+          lo_w[i / 2] = bf16x2(a.x, b.x);
+          hi_w[i / 2] = bf16x2(a.y, b.y);
+        }
+        uint4* dl = reinterpret_cast<uint4*>(dst + s * 32);
+        uint4* dh = reinterpret_cast<uint4*>(dst + 64 + s * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __stcs(dl + j, make_uint4(lo_w[4 * j], lo_w[4 * j + 1], lo_w[4 * j + 2], lo_w[4 * j + 3]));
+          __stcs(dh + j, make_uint4(hi_w[4 * j], hi_w[4 * j + 1], hi_w[4 * j + 2], hi_w[4 * j + 3]));
         }
       } else {
-        const int head = vec - hq - hkv;
-        const int64_t g = static_cast<int64_t>(t) * hkv + head;
-        float x[32];
-        load16_bf16(v + g * D + s * 32, x);
-        load16_bf16(v + g * D + s * 32 + 16, x + 16);
-        float mn = x[0], mx = x[0];
+        // K: extremes of the unnormalised values; scale and zero from the
+        // normalised ones
+        float mn = w[0].x, mx = w[0].x;
 #pragma unroll
-        for (int i = 1; i < 32; ++i) {
-          mn = fminf(mn, x[i]);
-          mx = fmaxf(mx, x[i]);
+        for (int i = 0; i < 32; ++i) {
+          mn = fminf(mn, fminf(w[i].x, w[i].y));
+          mx = fmaxf(mx, fmaxf(w[i].x, w[i].y));
         }
         float scale, zero;
-        asym_params(mn, mx, gmask, scale, zero);
-        uint8_t* dst = v_cache + g * (D / 2) + s * 16;
-        const uint2 a = pack16(x, scale, zero), b = pack16(x + 16, scale, zero);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(a.x, a.y, b.x, b.y);
+        asym_params2(mn * kNorm, mx * kNorm, pmask, scale, zero);
+        const float kq = kNorm * __frcp_rn(scale);
+        const f2 k2{kq, kq}, z2{zero, zero};
+        uint32_t wl[4], wh[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          const f2 xl[4] = {f2{w[8 * n].x, w[8 * n + 1].x}, f2{w[8 * n + 2].x, w[8 * n + 3].x},
+                            f2{w[8 * n + 4].x, w[8 * n + 5].x}, f2{w[8 * n + 6].x, w[8 * n + 7].x}};
+          const f2 xh[4] = {f2{w[8 * n].y, w[8 * n + 1].y}, f2{w[8 * n + 2].y, w[8 * n + 3].y},
+                            f2{w[8 * n + 4].y, w[8 * n + 5].y}, f2{w[8 * n + 6].y, w[8 * n + 7].y}};
+          wl[n] = ucodes8(xl, k2, z2);
+          wh[n] = ucodes8(xh, k2, z2);
+        }
+        const int64_t g = static_cast<int64_t>(tok) * hkv + head;
+        uint8_t* dst = k_cache + g * (D / 2);
+        *reinterpret_cast<uint4*>(dst + s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        *reinterpret_cast<uint4*>(dst + 32 + s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
         if (s == 0) {
-          v_scale[g] = scale;
-          v_zero[g] = static_cast<uint8_t>(zero);
+          k_scale[g] = scale;
+          k_zero[g] = static_cast<uint8_t>(zero);
         }
       }
     }
@@ -260,10 +332,11 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
                            int max_pos, void* q_out, uint8_t* k_cache, float* k_scale,
                            uint8_t* k_zero, uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
                            cudaStream_t stream) {
-  const int lanes = (hq + 2 * hkv) * 4;
-  const int threads = lanes >= 256 ? 256 : ((lanes + 31) & ~31);
+  const int items = 4 * hq + 8 * hkv;            // lanes per pair of tokens
+  const int threads = items >= 256 ? 256 : ((items + 31) & ~31);
+  const int64_t pairs = (T + 1) / 2;
   const int64_t cap = static_cast<int64_t>(host::num_sms()) * 8;
-  const int grid = static_cast<int>(T < cap ? T : cap);
+  const int grid = static_cast<int>(pairs < cap ? pairs : cap);
   auto qp = static_cast<const __nv_bfloat16*>(q);
   auto kp = static_cast<const __nv_bfloat16*>(k);
   auto vp = static_cast<const __nv_bfloat16*>(v);
