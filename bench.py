@@ -38,6 +38,11 @@ OPS = 2.0 * M * N * K
 RQ_BYTES = M * (2 * K + K // 2 + 4)
 KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
+# DRAM bytes (read + write) per launch from one ncu capture of the current
+# kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
+# set to None whenever the kernel changes until it is captured again.
+GEMM_TRAFFIC = 50515968 + 11369984
+RQ_TRAFFIC = 100705792 + 6795520
 WORKLOAD = "down_proj_M4096_K12288_N4096_R4_H12xH1024"
 
 
@@ -399,11 +404,11 @@ def main():
             "kv_path": r["kv"],
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
-                     "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": None,
-                     "kernel": "w4a4_gemm_kernel",
+                     "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,
+                     "kernel": "w4a4_gemm_pair_ts_kernel",
                      "peak_source": "%s bf16 %.1f TFLOP/s x 2 (nominal int8/bf16)" % (peak_src, bf16)},
         "roofline_rotate_quant": {"bound": "hbm", "achieved": gbs_rq, "peak": hbm, "unit": "GB/s",
-                                  "frac": gbs_rq / hbm, "traffic": None,
+                                  "frac": gbs_rq / hbm, "traffic": RQ_TRAFFIC,
                                   "peak_source": peak_src + " copy bandwidth"},
         "cpu_baseline": cpu,
         "e2e": {"value": tops_e2e_job, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
