@@ -326,6 +326,62 @@ def run_profile_case(case, steps, warmup):
     print("profile case %s: %d launches" % (case, warmup + steps))
 
 
+SWEEP_M = (1, 4, 16, 64, 256, 1024, 4096, 16384)
+SWEEP_SHAPES = (("down_proj", 12288, 4096), ("gate_up", 4096, 24576))
+
+
+def run_sweep(steps, warmup):
+    """The decode-to-prefill M sweep of the W4A4 GEMM (one JSON line per point).
+
+    Operands are seeded random packed codes of the configuration's shapes;
+    each point is timed with CUDA events over `steps` launches after `warmup`,
+    the L2 flushed (256 MB write) before each.  Bytes are the algorithmic
+    operand + output bytes (packed weights N*K/2, packed activations M*K/2,
+    scales 4(M+N), bf16 output 2MN); the roofline is the slower of the
+    measured-HBM and int8-tensor times.
+    """
+    import torch
+    import rotation_ptq_b200 as sq
+    from workloads import synthetic as W
+    hbm, bf16, _, peak_src = load_peaks()
+    int8_peak = 2.0 * bf16
+    torch.cuda.set_device(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for name, K, N in SWEEP_SHAPES:
+        w = torch.from_numpy(W.random_packed(21, N, K)).cuda()
+        sw = torch.from_numpy(W.random_scales(22, N)).cuda()
+        for m in SWEEP_M:
+            a = torch.from_numpy(W.random_packed(23 + m, m, K)).cuda()
+            sa = torch.from_numpy(W.random_scales(24 + m, m)).cuda()
+            out = torch.empty((m, N), dtype=torch.bfloat16, device="cuda")
+            for _ in range(warmup):
+                sq.w4a4_linear(a, sa, w, sw, out=out)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                sq.w4a4_linear(a, sa, w, sw, out=out)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) * 1e-3)
+            if sq.device_status() != 0:
+                raise SystemExit("device status set")
+            t = statistics.median(times)
+            ops = 2.0 * m * N * K
+            nbytes = N * K // 2 + m * K // 2 + 4 * (m + N) + 2 * m * N
+            t_roof = max(nbytes / (hbm * 1e9), ops / (int8_peak * 1e12))
+            print(json.dumps({
+                "sweep": name, "M": m, "K": K, "N": N, "us": t * 1e6,
+                "TOPS": ops / t / 1e12, "GB/s": nbytes / t / 1e9,
+                "bound": "hbm" if nbytes / (hbm * 1e9) >= ops / (int8_peak * 1e12) else "tensor",
+                "roofline_us": t_roof * 1e6, "frac": t_roof / t,
+                "peaks": "%s HBM %.1f GB/s, int8 %.0f TOPS" % (peak_src, hbm, int8_peak)}),
+                flush=True)
+            del a, sa, out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,11 +390,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kv", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the GEMM over the decode-to-prefill M sweep and exit")
     ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
                     help="launch one kernel of the path warmup+steps times and exit (for ncu)")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args.profile_case, args.steps, args.warmup)
+        return
+    if args.sweep:
+        run_sweep(min(args.steps, 20), max(args.warmup, 3))
         return
     args.warmup = max(args.warmup, 3)
 

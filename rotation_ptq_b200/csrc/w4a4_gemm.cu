@@ -62,7 +62,7 @@ struct Params {
   const float* w_scale;    // [N]
   void* out;               // [M][N] bf16 or int32
   int out_i32;
-  int* ws_acc;             // [M][N] int32 (split-K only; zero on entry and exit)
+  int* ws_acc;             // M*N int32 at [b * rowsA + a_row] (split-K only; zero on entry and exit)
   unsigned* ws_cnt;        // [tilesA * tilesB] (split-K only; zero on entry and exit)
   uint32_t spin_limit;
 };
@@ -356,9 +356,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // thread = token m, columns = channels n0..n0+15 (N % 16 == 0: all valid)
           const int m = a_row, n0 = b0;
           if (split) {
-            int* dst = p.ws_acc + static_cast<int64_t>(m) * p.N + n0;
+            // workspace index b * rowsA + a_row: a warp's 32 rows of one column
+            // are one 128-byte line
+            int* dst = p.ws_acc + static_cast<int64_t>(n0) * p.rowsA + m;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) atomicAdd(dst + j, static_cast<int>(v[j]) >> 8);
+            for (int j = 0; j < 16; ++j) atomicAdd(dst + static_cast<int64_t>(j) * p.rowsA,
+                                                   static_cast<int>(v[j]) >> 8);
           } else if (p.out_i32) {
             int4* dst = reinterpret_cast<int4*>(static_cast<int*>(p.out) +
                                                 static_cast<int64_t>(m) * p.N + n0);
@@ -399,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int acc = static_cast<int>(v[j]) >> 8;
             const int64_t o = static_cast<int64_t>(m) * p.N + n;
             if (split) {
-              atomicAdd(p.ws_acc + o, acc);
+              atomicAdd(p.ws_acc + o, acc);        // = b * rowsA + a_row (rowsA = N)
             } else if (p.out_i32) {
               static_cast<int*>(p.out)[o] = acc;
             } else {
@@ -438,10 +441,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int j = 0; j < 16; ++j) {
                 const int b = w.tb * BN + j0 + j;
                 const bool ok = b < p.rowsB;
-                const int m = p.swap ? b : a_row;
-                const int n = p.swap ? a_row : b;
-                const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                acc[j] = ok ? __ldcg(p.ws_acc + o) : 0;
+                const int64_t ow = static_cast<int64_t>(b) * p.rowsA + a_row;
+                acc[j] = ok ? __ldcg(p.ws_acc + ow) : 0;
                 sb[j] = ok ? __ldg((p.swap ? p.a_scale : p.w_scale) + b) : 0.f;
               }
 #pragma unroll
@@ -451,7 +452,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const int m = p.swap ? b : a_row;
                   const int n = p.swap ? a_row : b;
                   const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                  __stcg(p.ws_acc + o, 0);
+                  __stcg(p.ws_acc + static_cast<int64_t>(b) * p.rowsA + a_row, 0);
                   if (p.out_i32) {
                     static_cast<int*>(p.out)[o] = acc[j];
                   } else {
@@ -499,11 +500,12 @@ struct PairParams {
   int rowsA, rowsB;        // M, N
   int tilesM, tilesN;      // 256-wide tiles
   int KT;
-  int units;               // work units: full_units whole tiles, then K halves
+  int units;               // work units: full_units whole tiles, then K parts
   int full_units;          // tiles computed over all of K (== units: no split)
-  int kt_half;             // k-tile where the two halves of a split tile meet
-  int* ws_acc;             // [split tiles][256 cols][256 rows] int32 partial sums, zero at rest
-  unsigned* ws_cnt;        // [split tiles][ticket x2 | ready x2], zero at rest
+  int parts;               // K parts of each split tile (2..4)
+  int kchunk;              // k-tiles per part (a multiple of KM; the last part is shorter)
+  int* ws_acc;             // [split tiles][parts-1 slots][256 cols][256 rows] int32, zero at rest
+  unsigned* ws_cnt;        // [split tiles][ticket x2 | done x2], zero at rest
   const float* a_scale;
   const float* w_scale;
   void* out;
@@ -512,17 +514,19 @@ struct PairParams {
   uint32_t spin_limit;
 };
 
-// Work unit u of a CTA pair: a whole tile, or one K half of a tile of the
-// last, partial wave (split so that the wave's tiles spread over twice as
-// many pairs; the two halves add up through the int32 workspace).
+// Work unit u of a CTA pair: a whole tile, or one K part of a tile of the
+// last, partial wave (split so that the wave's tiles spread over more pairs;
+// the parts add up through the int32 workspace).
 struct PairUnit {
-  int tile, kt0, kt1, part;   // part -1: whole tile; 0 / 1: K half
+  int tile, kt0, kt1, part;   // part -1: whole tile; 0 .. parts-1: K part
 };
 __device__ __forceinline__ PairUnit pair_unit(const PairParams& p, int u) {
   if (u < p.full_units) return PairUnit{u, 0, p.KT, -1};
   const int v = u - p.full_units;
-  const int tile = p.full_units + (v >> 1);
-  return (v & 1) ? PairUnit{tile, p.kt_half, p.KT, 1} : PairUnit{tile, 0, p.kt_half, 0};
+  const int part = v % p.parts;
+  const int kt0 = part * p.kchunk;
+  const int kt1 = part == p.parts - 1 ? p.KT : kt0 + p.kchunk;
+  return PairUnit{p.full_units + v / p.parts, kt0, kt1, part};
 }
 
 template <int PST, int UST>
@@ -1109,30 +1113,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m = tm * 256 + static_cast<int>(rank) * L::HALF + row;
       const bool m_valid = m < p.M;
       const float sa = m_valid ? p.a_scale[m] : 0.f;
-      // K half of a split tile: the first half to reach its epilogue stores
-      // its partial sums (column-major: a warp's 32 rows of one column are
-      // one 128-byte line) and raises `ready`; the second waits for `ready`
-      // (the first is already running, so the wait ends), adds, and emits.
+      // K part of a split tile.  Parts take tickets in the order they reach
+      // their epilogue; every ticket but the last stores its partial sums in
+      // a slot of its own (column-major: a warp's 32 rows of one column are
+      // one 128-byte line) and counts itself done; the last ticket waits until
+      // the others are done (they are already in their epilogues, so the wait
+      // ends), adds every slot to its own sums, emits the tile and re-zeroes.
       int* wcol = nullptr;
       unsigned* ticket = nullptr;
-      unsigned* ready = nullptr;
-      bool first = false;
+      unsigned* done = nullptr;
+      bool last = true;
+      int nslot = 0;
       if (un.part >= 0) {
         const int t = un.tile - p.full_units;
-        wcol = p.ws_acc + static_cast<int64_t>(t) * 256 * 256 + static_cast<int>(rank) * L::HALF +
-               row;
+        nslot = p.parts - 1;
+        wcol = p.ws_acc + static_cast<int64_t>(t) * nslot * 256 * 256 +
+               static_cast<int>(rank) * L::HALF + row;
         ticket = p.ws_cnt + t * 4 + rank;
-        ready = p.ws_cnt + t * 4 + 2 + rank;
+        done = p.ws_cnt + t * 4 + 2 + rank;
         if (threadIdx.x == 0) {
-          const unsigned order = atomicAdd(ticket, 1u);
+          const unsigned o = atomicAdd(ticket, 1u);
           bool ok2 = true;
-          if (order == 1u) {
-            // bounded wait for the first half's partial sums
+          if (o == static_cast<unsigned>(nslot)) {
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t polls = 1;; ++polls) {
               unsigned r;
-              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(r) : "l"(ready) : "memory");
-              if (r != 0u) break;
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(r) : "l"(done) : "memory");
+              if (r >= static_cast<unsigned>(nslot)) break;
               if ((p.spin_limit != 0 && polls >= p.spin_limit) ||
                   ((polls & 255u) == 0 && globaltimer_ns() - t0 > kWaitNs)) {
                 record_status(SQ_ERR_TIMEOUT);
@@ -1142,12 +1149,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
           }
-          bcast[1] = order == 0u ? 1 : (ok2 ? 0 : 2);
+          bcast[1] = ok2 ? static_cast<int>(o) : -1;
         }
         named_bar_sync(1, EPI_WARPS * 32);
-        first = bcast[1] == 1;
-        if (bcast[1] == 2) wcol = nullptr;     // gave up: emit this half alone
+        const int got = bcast[1];
         named_bar_sync(1, EPI_WARPS * 32);
+        if (got < 0) {
+          wcol = nullptr;                      // gave up: emit this part alone
+        } else if (got < nslot) {
+          last = false;
+          wcol += static_cast<int64_t>(got) * 256 * 256;   // this ticket's slot
+        }
       }
       // four 16-column loads in flight per wait: 64 accumulator columns
 #pragma unroll 1
@@ -1164,22 +1176,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 16; ++j) v4[g][j] = static_cast<int>(vv[g][j]) >> 8;
         if (wcol != nullptr) {
           int* wc = wcol + c4 * 16 * 256;
-          if (first) {
+          if (!last) {
 #pragma unroll
             for (int g = 0; g < 4; ++g)
 #pragma unroll
               for (int j = 0; j < 16; ++j) wc[(g * 16 + j) * 256] = v4[g][j];
             continue;
           }
-          // the batch's 64 partial sums are all loaded before any store
+          // every slot's 64 sums of the batch are loaded before any store
+#pragma unroll 1
+          for (int sl = 0; sl < nslot; ++sl) {
+            const int* ws_sl = wc + static_cast<int64_t>(sl) * 256 * 256;
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
+            for (int g = 0; g < 4; ++g)
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v4[g][j] += __ldcg(wc + (g * 16 + j) * 256);
+              for (int j = 0; j < 16; ++j) v4[g][j] += __ldcg(ws_sl + (g * 16 + j) * 256);
+          }
+#pragma unroll 1
+          for (int sl = 0; sl < nslot; ++sl) {
+            int* ws_sl = wc + static_cast<int64_t>(sl) * 256 * 256;
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
+            for (int g = 0; g < 4; ++g)
 #pragma unroll
-            for (int j = 0; j < 16; ++j) wc[(g * 16 + j) * 256] = 0;
+              for (int j = 0; j < 16; ++j) ws_sl[(g * 16 + j) * 256] = 0;
+          }
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -1191,17 +1211,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed_n(tempty_leader, 32);
-      if (un.part >= 0) {
-        if (first) {
-          // publish the partial sums, then raise `ready`
+      if (un.part >= 0 && wcol != nullptr) {
+        if (!last) {
+          // publish the partial sums, then count this part done
           __threadfence();
           named_bar_sync(1, EPI_WARPS * 32);
-          if (threadIdx.x == 0)
-            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ready), "r"(1u) : "memory");
+          if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(done) : "memory");
         } else if (threadIdx.x == 0) {
-          // both halves are done with this tile: rearm for the next call
+          // every part is done with this tile: rearm for the next call
           *ticket = 0u;
-          *ready = 0u;
+          *done = 0u;
         }
       }
     }
@@ -1267,13 +1286,15 @@ static sq_status launch(const Plan& plan, const uint8_t* opA, const uint8_t* opB
 }
 
 
-// Workspace of a split tail of `tail` tiles: int32 partial sums of 256 x 256
-// per tile, then two arrival counters per tile.
-static size_t tail_acc_bytes(int tail) {
-  return (static_cast<size_t>(tail) * 256 * 256 * 4 + 255) & ~static_cast<size_t>(255);
+// Workspace of a split wave of `tail` tiles in `parts` K parts: parts - 1
+// int32 slots of 256 x 256 per tile, then four counters per tile.
+static size_t tail_acc_bytes(int tail, int parts) {
+  return (static_cast<size_t>(tail) * (parts - 1) * 256 * 256 * 4 + 255) &
+         ~static_cast<size_t>(255);
 }
-static size_t tail_ws_bytes(int tail) {
-  return tail_acc_bytes(tail) + ((static_cast<size_t>(tail) * 4 * 4 + 255) & ~static_cast<size_t>(255));
+static size_t tail_ws_bytes(int tail, int parts) {
+  return tail_acc_bytes(tail, parts) +
+         ((static_cast<size_t>(tail) * 4 * 4 + 255) & ~static_cast<size_t>(255));
 }
 
 template <bool TS, int PST, int UST>
@@ -1319,25 +1340,43 @@ static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, 
     }
     max_clusters[dev & 63] = n;
   }
-  const int pairs = prm.units < max_clusters[dev & 63] ? prm.units : max_clusters[dev & 63];
+  const int cap_pairs = max_clusters[dev & 63];   // pairs that can be resident at once
   prm.full_units = prm.units;
   if constexpr (TS) {
-    // A last wave that fills at most half of the pairs is split by K in two
-    // halves (when the caller's workspace holds the partial sums).  Halves
-    // shorter than 32 k-tiles do not repay the partial-sum round trip.
+    // The tiles of a last wave that fills at most half of the pairs (all the
+    // tiles, when there are fewer than pairs) are split by K into `parts`
+    // parts, when the caller's workspace holds the partial sums.  The number
+    // of parts minimises the modelled time: the longest part's k-tiles at
+    // ~0.4 us each plus ~10 us per extra part (the slot stores, the wait and
+    // the summing epilogue, as measured on the down_proj shapes).
     const int tiles = prm.units;
+    const int pairs = cap_pairs;
     const int full = tiles / pairs * pairs;
     const int tail = tiles - full;
-    const int kt_half = prm.KT / 2 / KM * KM;
-    if (ws != nullptr && tail > 0 && 2 * tail <= pairs && kt_half >= 32 && kt_half < prm.KT &&
-        ws_bytes >= tail_ws_bytes(tail)) {
+    int best_parts = 1, best_chunk = prm.KT;
+    double best_t = 0.4 * prm.KT;
+    for (int parts = 2; parts <= 4 && tail > 0 && tail * parts <= pairs; ++parts) {
+      const int per = (prm.KT + parts - 1) / parts;
+      const int chunk = (per + KM - 1) / KM * KM;
+      if (chunk < 16 || chunk * (parts - 1) >= prm.KT) continue;
+      const double t = 0.4 * chunk + 10.0 * (parts - 1);
+      if (t < best_t) {
+        best_t = t;
+        best_parts = parts;
+        best_chunk = chunk;
+      }
+    }
+    if (ws != nullptr && best_parts > 1 && ws_bytes >= tail_ws_bytes(tail, best_parts)) {
       prm.full_units = full;
-      prm.units = full + 2 * tail;
-      prm.kt_half = kt_half;
+      prm.units = full + best_parts * tail;
+      prm.parts = best_parts;
+      prm.kchunk = best_chunk;
       prm.ws_acc = static_cast<int*>(ws);
-      prm.ws_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + tail_acc_bytes(tail));
+      prm.ws_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
+                                               tail_acc_bytes(tail, best_parts));
     }
   }
+  const int pairs = prm.units < cap_pairs ? prm.units : cap_pairs;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, mapA, mapB, prm);
   if (e != cudaSuccess) return host::cuda_fail("w4a4_gemm_pair launch", e);
@@ -1345,7 +1384,7 @@ static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, 
 }
 
 static bool use_pair(int64_t M, int64_t N) {
-  if (M < 256 || N < 256) return false;
+  if (M <= 128 || N < 256) return false;
   return host::gemm_path() != 1;
 }
 
@@ -1390,10 +1429,18 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
 
 size_t tail_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K < BK || !use_pair(M, N)) return 0;
-  // at most a quarter of the SMs' worth of tail tiles: half of the pairs
+  // the largest split any wave of these tiles can take: `parts` parts of at
+  // most pairs / parts tiles (pairs <= num_sms / 2)
   const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
-  const int64_t cap = num_sms / 4 > 0 ? num_sms / 4 : 1;
-  return tail_ws_bytes(static_cast<int>(tiles < cap ? tiles : cap));
+  const int64_t pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
+  size_t best = 0;
+  for (int parts = 2; parts <= 4; ++parts) {
+    const int64_t tail = tiles < pairs / parts ? tiles : pairs / parts;
+    if (tail < 1) continue;
+    const size_t b = tail_ws_bytes(static_cast<int>(tail), parts);
+    if (b > best) best = b;
+  }
+  return best;
 }
 
 size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {

@@ -183,3 +183,27 @@ def test_split_tail_matches_whole_tiles(cuda_ok, out_int32):
         assert np.array_equal(split.cpu().numpy().astype(np.int64), ref)
     else:
         P.check_fro(split.float().cpu().numpy(), O.dequant(ref, sa, sw))
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 4096, 12288), (256, 4096, 12288), (512, 4096, 6144)])
+def test_few_tile_k_split_matches_whole_tiles(cuda_ok, M, N, K):
+    # Fewer 256 x 256 tiles than CTA pairs: every tile runs as 2-3 K parts
+    # chained through the workspace (M = 200 also takes the pair kernel with
+    # a ragged tile).  Identical to whole tiles, exact on sampled rows,
+    # workspace left zero.
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 900 + M)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    nbytes = max(sq.w4a4_workspace_bytes(M, N, K), sq.w4a4_tail_workspace_bytes(M, N, K))
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    split = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True, workspace=ws)
+    whole = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True, use_workspace=False)
+    bf = sq.w4a4_linear(da, dsa, dw, dsw, workspace=ws)
+    torch.cuda.synchronize()
+    assert sq.device_status() == 0
+    assert int(ws.count_nonzero()) == 0
+    assert torch.equal(split, whole)
+    rows = P.sample_rows(M, 24, seed=M)
+    ref = O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w))
+    assert np.array_equal(split[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64), ref)
+    P.check_fro(bf[torch.from_numpy(rows).cuda()].float().cpu().numpy(), O.dequant(ref, sa[rows], sw))
