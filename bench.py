@@ -335,7 +335,9 @@ def run_sweep(steps, warmup):
 
     Operands are seeded random packed codes of the configuration's shapes;
     each point is timed with CUDA events over `steps` launches after `warmup`,
-    the L2 flushed (256 MB write) before each.  Bytes are the algorithmic
+    the L2 flushed (256 MB write) before each and the device kept busy (a
+    ~0.1 ms device sleep) while the host prepares the launch, so that the
+    events bracket the kernel alone.  Bytes are the algorithmic
     operand + output bytes (packed weights N*K/2, packed activations M*K/2,
     scales 4(M+N), bf16 output 2MN); the roofline is the slower of the
     measured-HBM and int8-tensor times.
@@ -360,6 +362,9 @@ def run_sweep(steps, warmup):
             times = []
             for _ in range(steps):
                 flush.zero_()
+                # keep the device busy while the host prepares the launch, so
+                # that the events bracket the kernel and not host overhead
+                torch.cuda._sleep(200000)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
                 sq.w4a4_linear(a, sa, w, sw, out=out)

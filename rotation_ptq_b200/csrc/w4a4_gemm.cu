@@ -139,6 +139,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                      const __grid_constant__ CUtensorMap mapB, const Params p) {
   using L = Layout<BN, PST, UST>;
+  // int8 slots change hands in groups of GK k-tiles: one packed stage when the
+  // ring holds at least two such groups, else one k-tile (so that unpack and
+  // MMA still overlap)
+  constexpr int GK = UST >= 2 * KM ? KM : 1;
+  constexpr int G = UST / GK;
+  static_assert(UST % GK == 0, "int8 slots come in whole groups");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -161,7 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&pfull[s], 1);
       mbar_init(&pempty[s], NPT);
     }
-    for (int s = 0; s < UST; ++s) {
+    for (int s = 0; s < G; ++s) {
       mbar_init(&ufull[s], NPT);
       mbar_init(&uempty[s], 1);
     }
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       dst_off0[i] = base + sw128_off(row, 2 * q);
       dst_off1[i] = base + sw128_off(row, 2 * q + 1);
     }
-    uint32_t it = 0, itp = 0;                    // k-tiles and packed stages consumed
+    uint32_t ig = 0, itp = 0;                    // slot groups and packed stages consumed
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
       const Unit w = decompose(p, u);
@@ -249,10 +255,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint32_t psrc = smem_base + L::P_OFF + ps * L::PSTAGE;
         const int nsub = min(KM, w.kt1 - kt);
-        for (int sub = 0; sub < nsub; ++sub, ++it) {
-          const int us = it % UST;
-          const uint32_t uph = (it / UST) & 1;
-          bool free_slot = mbar_wait(&uempty[us], uph ^ 1, p.spin_limit);
+        for (int sub0 = 0; sub0 < nsub; sub0 += GK, ++ig) {
+          const int gsz = min(GK, nsub - sub0);
+          const int g = ig % G;
+          bool free_slot = mbar_wait(&uempty[g], ((ig / G) & 1) ^ 1, p.spin_limit);
           // the warp decides together: it arrives once per barrier below
           free_slot = __all_sync(0xffffffffu, free_slot && !*abort_flag);
           if (!free_slot) {
@@ -260,20 +266,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const uint32_t udst = smem_base + L::U_OFF + us * L::USTAGE;
-          const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;   // chunk index + 4*sub
+          for (int j = 0; j < gsz; ++j) {
+            const int sub = sub0 + j;
+            const uint32_t udst = smem_base + L::U_OFF + (g * GK + j) * L::USTAGE;
+            const uint32_t sub_x = static_cast<uint32_t>(sub) << 6;   // chunk index + 4*sub
 #pragma unroll
-          for (int i = 0; i < IPT; ++i) {
-            if (t + i * NPT < ITEMS) {
-              const uint4 v = lds128(psrc + (src_off[i] ^ sub_x));
-              const uint32_t m = 0xF0F0F0F0u;
-              sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
-              sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+            for (int i = 0; i < IPT; ++i) {
+              if (t + i * NPT < ITEMS) {
+                const uint4 v = lds128(psrc + (src_off[i] ^ sub_x));
+                const uint32_t m = 0xF0F0F0F0u;
+                sts128(udst + dst_off0[i], (v.x << 4) & m, v.x & m, (v.y << 4) & m, v.y & m);
+                sts128(udst + dst_off1[i], (v.z << 4) & m, v.z & m, (v.w << 4) & m, v.w & m);
+              }
             }
           }
           fence_proxy_async_smem();
           __syncwarp();                          // the warp's writes are ordered before
-          if (lane == 0) mbar_arrive_n(&ufull[us], 32);   // its one arrival
+          if (lane == 0) mbar_arrive_n(&ufull[g], 32);    // its one arrival
         }
         if (!ok) break;
         __syncwarp();
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_i8(BM, BN);
-      uint32_t it = 0, acc_it = 0;
+      uint32_t ig = 0, acc_it = 0;
       for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++acc_it) {
         const Unit w = decompose(p, u);
         const int buf = acc_it & 1;
@@ -296,23 +305,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
         bool ok = true;
-        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
-          const int us = it % UST;
-          const uint32_t uph = (it / UST) & 1;
-          if (!mbar_wait(&ufull[us], uph, p.spin_limit) || *abort_flag) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_base + L::U_OFF + us * L::USTAGE;
-          const uint32_t b_addr = a_addr + L::UA;
+        // the same groups as the unpack warps: GK k-tiles inside each packed stage
+        for (int kt = w.kt0; ok && kt < w.kt1; kt += KM) {
+          const int nsub = min(KM, w.kt1 - kt);
+          for (int sub0 = 0; sub0 < nsub; sub0 += GK, ++ig) {
+            const int gsz = min(GK, nsub - sub0);
+            const int g = ig % G;
+            if (!mbar_wait(&ufull[g], (ig / G) & 1, p.spin_limit) || *abort_flag) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int j = 0; j < gsz; ++j) {
+              const uint32_t a_addr = smem_base + L::U_OFF + (g * GK + j) * L::USTAGE;
+              const uint32_t b_addr = a_addr + L::UA;
+              const int ktile = kt + sub0 + j;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            mma_i8(d_tmem, desc_sw128(a_addr + kk * UMMA_K), desc_sw128(b_addr + kk * UMMA_K),
-                   IDESC, (kt > w.kt0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                mma_i8(d_tmem, desc_sw128(a_addr + kk * UMMA_K),
+                       desc_sw128(b_addr + kk * UMMA_K), IDESC,
+                       (ktile > w.kt0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit(&uempty[g]);
           }
-          mma_commit(&uempty[us]);
         }
         if (!ok) break;
         mma_commit(&tfull[buf]);
@@ -1404,23 +1421,26 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool have_ws, int num_sms) {
   pl.tilesB = static_cast<int>((rowsB + pl.bn - 1) / pl.bn);
   pl.KT = static_cast<int>(K / BK);
   const int64_t base = static_cast<int64_t>(pl.tilesA) * pl.tilesB;
-  int splits = 1;
+  // Split K to minimise the modelled time of the busiest CTA: its units'
+  // k-tiles at ~0.25 us each plus ~2 us per unit (pipeline fill, epilogue),
+  // with the k-tiles per split rounded to whole packed stages.
+  int kps_best = pl.KT;
   if (have_ws && base < 2 * num_sms) {
-    // choose the split that best fills whole waves, with >= 4 k-tiles each
-    double best = -1.0;
+    double best = 1e30;
     for (int s = 1; s <= 16 && s <= pl.KT / 4; ++s) {
-      const int64_t units = base * s;
-      const int64_t waves = (units + num_sms - 1) / num_sms;
-      double eff = static_cast<double>(units) / static_cast<double>(waves * num_sms);
-      eff -= 0.01 * (s - 1);                       // mild preference for fewer splits
-      if (eff > best + 1e-9) {
-        best = eff;
-        splits = s;
+      int kps = (pl.KT + s - 1) / s;
+      kps = (kps + KM - 1) / KM * KM;              // splits start on a packed stage
+      const int64_t splits = (pl.KT + kps - 1) / kps;
+      const int64_t units = base * splits;
+      const int64_t per_cta = (units + num_sms - 1) / num_sms;
+      const double t = 0.25 * static_cast<double>(per_cta * kps) + 2.0 * static_cast<double>(per_cta);
+      if (t < best - 1e-9) {
+        best = t;
+        kps_best = kps;
       }
     }
   }
-  pl.kps = (pl.KT + splits - 1) / splits;
-  pl.kps = (pl.kps + KM - 1) / KM * KM;            // splits start on a packed stage
+  pl.kps = kps_best;
   pl.splits = (pl.KT + pl.kps - 1) / pl.kps;
   pl.units = static_cast<int>(base * pl.splits);
   pl.grid = static_cast<int>(pl.units < num_sms ? pl.units : num_sms);
@@ -1457,6 +1477,9 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
               int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
               size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
               const Plan* forced) {
+  if (!forced && host::gemm_path() == 0 && gemv::eligible(M, K))
+    return gemv::run(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32, num_sms, spin_limit,
+                     stream);
   if (!forced && use_pair(M, N)) {
     PairParams pp{};
     pp.rowsA = static_cast<int>(M);
@@ -1510,7 +1533,7 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
   const uint8_t* opB = pl.swap ? a_q : w_q;
   switch (pl.bn) {
     case 16: return launch<16, 4, 8>(pl, opA, opB, K, prm, stream);
-    case 32: return launch<32, 4, 7>(pl, opA, opB, K, prm, stream);
+    case 32: return launch<32, 4, 6>(pl, opA, opB, K, prm, stream);
     case 64: return launch<64, 3, 6>(pl, opA, opB, K, prm, stream);
     case 128: return launch<128, 3, 4>(pl, opA, opB, K, prm, stream);
     case 256: return launch<256, 2, 2>(pl, opA, opB, K, prm, stream);

@@ -207,3 +207,26 @@ def test_few_tile_k_split_matches_whole_tiles(cuda_ok, M, N, K):
     ref = O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w))
     assert np.array_equal(split[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64), ref)
     P.check_fro(bf[torch.from_numpy(rows).cuda()].float().cpu().numpy(), O.dequant(ref, sa[rows], sw))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 272, 12288), (2, 4096, 4096), (3, 1040, 12288),
+                                   (7, 4096, 12288), (8, 24576, 4096)])
+def test_decode_gemv_matches_tensor_path(cuda_ok, M, N, K):
+    # M <= 8 runs on the CUDA-core GEMV (dp4a); the one-CTA tensor-core
+    # kernel (forced with debug path 1) must give identical int32 and bf16
+    # results, and the int32 sums equal the oracle's exactly.
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 1200 + M)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    gi = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+    gb = sq.w4a4_linear(da, dsa, dw, dsw)
+    sq.debug_set_gemm_path(1)
+    try:
+        ti = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+        tb = sq.w4a4_linear(da, dsa, dw, dsw)
+    finally:
+        sq.debug_set_gemm_path(0)
+    assert sq.device_status() == 0
+    assert torch.equal(gi, ti) and torch.equal(gb, tb)
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    assert np.array_equal(gi.cpu().numpy().astype(np.int64), ref)
