@@ -42,7 +42,7 @@ def needs_build() -> bool:
 def build(verbose: bool = False, ptxas_verbose: bool = False, force: bool = False) -> str:
     if not force and not needs_build():
         return LIB
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-shared",
+    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O2", "-I" + os.path.join(ROOT, "include"), "-I" + CSRC,
            "--expt-relaxed-constexpr", "-o", LIB + ".tmp", *sources()]
     if ptxas_verbose:

@@ -145,6 +145,19 @@ __host__ __device__ constexpr int paley12(int i, int j) {
   return i == j ? 1 : (i == 0 ? 1 : (j == 0 ? -1 : chi11((j - 1) - (i - 1))));
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max over the warp of |v|
+__device__ __forceinline__ float warp_max_abs(float v) {
+  float r;
+  asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // Barrier over `n` threads (named barrier `id`) returning whether any of
 // them passed `v`: one uniform verdict for the whole group.
 __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
@@ -223,20 +236,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         ? (M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                         : 0;
 
-  // The constant operand A (K-major, 128-byte swizzle): row mu, column kappa
-  // at atom kappa / 64, byte (mu / 8) * 1024 + (mu % 8) * 128 + 16-byte chunk
-  // ((2 (kappa % 64)) / 16) ^ (mu % 8).  Rows 96..127 and kappa >= 96 are 0.
-  for (int e = tid; e < 128 * 128; e += TC_THREADS) {
-    const int mu = e >> 7, kap = e & 127;
-    float val = 0.f;
-    if (mu < 96 && kap < 96) {
-      const int o = mu >> 3, jtp = mu & 7, i = kap >> 3, jt = kap & 7;
-      val = static_cast<float>(paley12(i, o) * ((__popc(jt & jtp) & 1) ? -1 : 1));
+  // The constant operand A (K-major, 128-byte swizzle) in 16-byte chunks:
+  // chunk c (kappa 8c .. 8c + 7, i.e. i = c, jt = 0..7) of row mu sits in
+  // atom c / 8 at (mu / 8) * 1024 + (mu % 8) * 128 + 16 * ((c % 8) ^ (mu %
+  // 8)) and holds eight bf16 +-1 values H12[c][o] * H8[jt][jt'] (mu = 8 o +
+  // jt').  Rows 96..127 and kappa >= 96 (c >= 12) are 0.
+  for (int e = tid; e < 128 * 16; e += TC_THREADS) {
+    const int mu = e >> 4, c = e & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (mu < 96 && c < 12) {
+      const int o = mu >> 3, jtp = mu & 7;
+      const uint32_t neg = paley12(c, o) < 0 ? 0x80008000u : 0u;
+      uint32_t wd[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t lo = (__popc((2 * h) & jtp) & 1) ? 0xBF80u : 0x3F80u;
+        const uint32_t hi = (__popc((2 * h + 1) & jtp) & 1) ? 0xBF80u : 0x3F80u;
+        wd[h] = (lo | (hi << 16)) ^ neg;
+      }
+      v = make_uint4(wd[0], wd[1], wd[2], wd[3]);
     }
-    const int a = kap >> 6, kb = 2 * (kap & 63);
-    const int byte = a * TC_A_ATOM + (mu >> 3) * 1024 + (mu & 7) * 128 +
-                     ((((kb >> 4) ^ (mu & 7))) << 4) + (kb & 15);
-    *reinterpret_cast<__nv_bfloat16*>(Asm + byte) = __float2bfloat16_rn(val);
+    const int byte = (c >> 3) * TC_A_ATOM + (mu >> 3) * 1024 + (mu & 7) * 128 +
+                     (((c & 7) ^ (mu & 7)) << 4);
+    *reinterpret_cast<uint4*>(Asm + byte) = v;
   }
   if (tid == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
@@ -352,11 +374,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       }
-      float amax = 0.f;
+      // four independent max chains, then one warp reduction
+      float mx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int p = 0; p < 64; ++p) amax = fmaxf(amax, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int p = 0; p < 64; ++p) mx[p & 3] = fmax3(mx[p & 3], fabsf(w[p].x), fabsf(w[p].y));
+      float amax = warp_max_abs(fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]));
       if (lane == 0) gred[(it & 1) * 3 + q] = amax;
       // one barrier per row and group: partial maxima and the verdict
       if (bar_any(1 + g, 96, fail || *abort_flag)) {

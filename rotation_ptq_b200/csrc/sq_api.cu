@@ -13,9 +13,20 @@
 
 namespace sq {
 
-__device__ unsigned int g_status = 0;
-
 namespace host {
+
+// Status-word readers of the translation units (constant-initialised, so
+// they are ready before any unit's load-time registration runs).
+constexpr int kMaxUnits = 16;
+static std::mutex g_units_mu;
+static status_io g_units[kMaxUnits] = {};
+static int g_nunits = 0;
+
+bool register_status_word(status_io io) {
+  std::lock_guard<std::mutex> lock(g_units_mu);
+  if (g_nunits < kMaxUnits) g_units[g_nunits++] = io;
+  return true;
+}
 
 static thread_local char t_err[512] = {0};
 static std::atomic<uint32_t> g_spin_limit{0};
@@ -121,15 +132,21 @@ sq_status sq_device_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return sq::host::cuda_fail("cudaStreamSynchronize", e);
-  unsigned int v = 0;
-  e = cudaMemcpyFromSymbol(&v, sq::g_status, sizeof(v));
-  if (e != cudaSuccess) return sq::host::cuda_fail("read device status", e);
-  if (v != 0) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(sq::g_status, &zero, sizeof(zero));
-    if (e != cudaSuccess) return sq::host::cuda_fail("clear device status", e);
-    set_error("device reported %s", sq_status_string(static_cast<sq_status>(v)));
-    return static_cast<sq_status>(v);
+  unsigned int first = 0;
+  std::lock_guard<std::mutex> lock(sq::host::g_units_mu);
+  for (int i = 0; i < sq::host::g_nunits; ++i) {
+    unsigned int v = 0;
+    e = sq::host::g_units[i](&v, false);
+    if (e != cudaSuccess) return sq::host::cuda_fail("read device status", e);
+    if (v != 0) {
+      if (first == 0) first = v;
+      e = sq::host::g_units[i](nullptr, true);
+      if (e != cudaSuccess) return sq::host::cuda_fail("clear device status", e);
+    }
+  }
+  if (first != 0) {
+    set_error("device reported %s", sq_status_string(static_cast<sq_status>(first)));
+    return static_cast<sq_status>(first);
   }
   return SQ_OK;
 }

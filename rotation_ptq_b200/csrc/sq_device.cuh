@@ -10,9 +10,26 @@
 
 namespace sq {
 
-// Device status word: the first failing kernel records its sq_status here.
-// Read and cleared by sq_device_status().
-extern __device__ unsigned int g_status;
+// Device status word of this translation unit: the first failing kernel of
+// the unit records its sq_status here.  The library is compiled whole-program
+// (no relocatable device code, which would also disable setmaxnreg), so each
+// unit has its own word; every unit registers a reader at load time and
+// sq_device_status() reads and clears them all.
+static __device__ unsigned int g_status = 0;
+
+namespace host {
+using status_io = cudaError_t (*)(unsigned int* value, bool clear);
+bool register_status_word(status_io io);
+}  // namespace host
+
+static cudaError_t unit_status_io(unsigned int* value, bool clear) {
+  if (clear) {
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+  }
+  return cudaMemcpyFromSymbol(value, g_status, sizeof(*value));
+}
+[[maybe_unused]] static const bool g_status_registered = host::register_status_word(&unit_status_io);
 
 __device__ __forceinline__ void record_status(unsigned int s) {
   atomicCAS(&g_status, 0u, s);
