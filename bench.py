@@ -41,8 +41,8 @@ METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
 # set to None whenever the kernel changes until it is captured again.
-GEMM_TRAFFIC = 50515968 + 11369984
-RQ_TRAFFIC = 100705792 + 6795520
+GEMM_TRAFFIC = 50544896 + 12481280
+RQ_TRAFFIC = 100713984 + 5578496
 WORKLOAD = "down_proj_M4096_K12288_N4096_R4_H12xH1024"
 
 
