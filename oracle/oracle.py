@@ -28,6 +28,8 @@ Readings of points the pages leave open (each listed in the design doc):
     integer zero point; the range is widened to include 0.
   * RoPE: half-split ("rotate_half") convention, host tables in float64 rounded
     to float32, theta 1e6.
+  * SwiGLU ahead of R4: h = bf16(silu(gate) * up), the product at full
+    precision rounded once to bf16; the gate half first in [gate | up].
 
 Parity pins: every function below is checked in tests/test_oracle_pins.py
 against closed forms, brute force or invariants that do not reuse it.
@@ -193,6 +195,47 @@ def quantize_weights(w: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0
     wr = rotate(w, n_small, n_pow2)
     codes, scale, _ = quant_sym_int4(wr, clip)
     return pack_int4(codes), scale, codes
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU ahead of down_proj.  "SpinQuant, Reproduced", Q5 places R4 on the
+# input of down_proj, which in the Qwen3-8B MLP of the same section is the
+# SwiGLU product silu(gate) * up of the gate and up projections.  Reading (the
+# pages give no precision for this step): the product is formed at full
+# precision and rounded once to bf16, the dtype of the down_proj input, and
+# the gate half comes first in the fused gate_up output ([gate | up]).
+# ---------------------------------------------------------------------------
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """silu(x) = x / (1 + exp(-x)) = x * sigmoid(x), float64."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest bf16 value (8 significant bits), ties to even.
+
+    x = m * 2^e with 0.5 <= |m| < 1; m * 2^8 is rounded to an integer with
+    round-half-to-even and scaled back.  Normal range only (the values here
+    are far from bf16's overflow and subnormal limits).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def swiglu_bf16(gate_up: np.ndarray, K: int) -> np.ndarray:
+    """h = bf16(silu(gate) * up) from gate_up [M, >= 2K]: gate = columns [0, K), up = [K, 2K)."""
+    gu = np.asarray(gate_up, dtype=np.float64)
+    return round_bf16(silu(gu[:, :K]) * gu[:, K:2 * K])
+
+
+def swiglu_rotate_quant(gate_up: np.ndarray, K: int, n_small: int, n_pow2: int,
+                        clip: float = 1.0):
+    """SwiGLU product, then the online rotation and per-token INT4 (rotate_quant)."""
+    return rotate_quant(swiglu_bf16(gate_up, K), n_small, n_pow2, clip)
 
 
 # ---------------------------------------------------------------------------

@@ -101,9 +101,41 @@ def _sylvester_walsh_order(n):
     return H[np.argsort(changes, kind="stable")]
 
 
+def _silu_wrong_sign(x):
+    x = np.asarray(x, np.float64)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(x))
+
+
+def _round_bf16_truncate(x):
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.trunc(m * 256.0) / 256.0, e)
+
+
+def _round_bf16_half_away(x):
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.sign(m) * np.floor(np.abs(m) * 256.0 + 0.5) / 256.0, e)
+
+
+def _round_to_f32(x):
+    return np.asarray(x, np.float64).astype(np.float32).astype(np.float64)
+
+
+def _swiglu_halves_swapped(gate_up, K):
+    gu = np.asarray(gate_up, np.float64)
+    return O.round_bf16(O.silu(gu[:, K:2 * K]) * gu[:, :K])
+
+
+def _swiglu_no_up(gate_up, K):
+    gu = np.asarray(gate_up, np.float64)
+    return O.round_bf16(O.silu(gu[:, :K]))
+
+
 _orig = {name: getattr(O, name) for name in
          ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
-          "quant_asym_uint4", "dequant", "sylvester"]}
+          "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16"]}
 
 MUTATIONS = {
     "paley_transposed": ("paley1", _transposed_paley),
@@ -117,6 +149,12 @@ MUTATIONS = {
     "asym_zero_point_sign": ("quant_asym_uint4", _asym_zero_sign),
     "dequant_scales_swapped": ("dequant", _dequant_swapped),
     "sylvester_walsh_order": ("sylvester", _sylvester_walsh_order),
+    "silu_wrong_sign": ("silu", _silu_wrong_sign),
+    "bf16_truncates": ("round_bf16", _round_bf16_truncate),
+    "bf16_ties_away_from_zero": ("round_bf16", _round_bf16_half_away),
+    "bf16_is_float32": ("round_bf16", _round_to_f32),
+    "swiglu_halves_swapped": ("swiglu_bf16", _swiglu_halves_swapped),
+    "swiglu_drops_up": ("swiglu_bf16", _swiglu_no_up),
 }
 
 PIN_TESTS = [
@@ -139,6 +177,11 @@ PIN_TESTS = [
     P.test_headwise_hadamard_matches_butterfly,
     P.test_asym_quant_bounds_and_zero_point,
     P.test_asym_quant_constant_and_zero_rows,
+    P.test_round_bf16_matches_bit_rule_and_ties,
+    P.test_round_bf16_is_nearest_of_two_neighbours,
+    P.test_silu_identities,
+    P.test_swiglu_layout_and_special_values,
+    P.test_swiglu_rotate_quant_bruteforce,
 ]
 
 

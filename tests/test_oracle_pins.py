@@ -444,8 +444,106 @@ def test_kv_rotate_quant_composition():
 
 
 # --------------------------------------------------------------------------
+# SwiGLU ahead of down_proj (fused SwiGLU + R4)
+# --------------------------------------------------------------------------
+
+def _bf16_rne_bits(x32):
+    """bf16 round-to-nearest-even of float32 values by the integer rule on
+    their bits: add 0x7FFF plus the lowest kept bit, then truncate."""
+    b = np.asarray(x32, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
+def test_round_bf16_matches_bit_rule_and_ties():
+    rng = np.random.default_rng(71)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    assert np.array_equal(O.round_bf16(x.astype(np.float64)), _bf16_rne_bits(x))
+    # exact bf16 values are fixed points
+    exact = (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+    assert np.array_equal(O.round_bf16(exact), exact)
+    # ties go to the even neighbour; just past a tie goes to the nearer one
+    one = 1.0
+    assert O.round_bf16(np.array([one + 2.0 ** -8]))[0] == 1.0
+    assert O.round_bf16(np.array([one + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+    assert O.round_bf16(np.array([one + 2.0 ** -8 + 2.0 ** -30]))[0] == 1.0 + 2.0 ** -7
+    assert O.round_bf16(np.array([-(one + 2.0 ** -8)]))[0] == -1.0
+    assert O.round_bf16(np.array([0.0]))[0] == 0.0
+
+
+def test_round_bf16_is_nearest_of_two_neighbours():
+    rng = np.random.default_rng(72)
+    x = rng.standard_normal(2000) * 1e3
+    r = O.round_bf16(x)
+    for xi, ri in zip(x, r):
+        m, e = math.frexp(xi)
+        lo = math.ldexp(math.floor(m * 256) / 256, e)
+        hi = math.ldexp(math.ceil(m * 256) / 256, e)
+        assert ri in (lo, hi)
+        assert abs(ri - xi) <= min(abs(lo - xi), abs(hi - xi))
+
+
+def test_silu_identities():
+    x = np.linspace(-30, 30, 2001)
+    s = O.silu(x)
+    # silu(x) - silu(-x) = x (sigmoid(x) + sigmoid(-x) = 1)
+    assert np.allclose(s - O.silu(-x), x, rtol=0, atol=1e-12)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    # silu(x) = x * sigmoid(x): sigmoid from its tanh form for x >= 0 and as
+    # e^x / (1 + e^x) for x < 0 (both free of cancellation there)
+    pos, neg = x >= 0, x < 0
+    assert np.allclose(s[pos], x[pos] * 0.5 * (1.0 + np.tanh(0.5 * x[pos])), rtol=1e-13, atol=0)
+    en = np.exp(x[neg])
+    assert np.allclose(s[neg], x[neg] * en / (1.0 + en), rtol=1e-13, atol=0)
+    # tails: silu(40) = 40 to double precision; silu(-800) = -0
+    assert O.silu(np.array([40.0]))[0] == 40.0
+    assert O.silu(np.array([-800.0]))[0] == 0.0
+
+
+def test_swiglu_layout_and_special_values():
+    K = 4
+    g = np.array([[0.0, 10.0, -3.0, 2.0]])
+    u = np.array([[5.0, 2.0, 0.0, 1.5]])
+    h = O.swiglu_bf16(np.concatenate([g, u], axis=1), K)
+    want = [0.0, O.round_bf16(np.array([10.0 / (1 + math.exp(-10.0)) * 2.0]))[0], 0.0,
+            O.round_bf16(np.array([2.0 / (1 + math.exp(-2.0)) * 1.5]))[0]]
+    assert np.array_equal(h[0], np.array(want))
+    # the gate half is the first one: swapping the halves changes the result
+    assert not np.array_equal(O.swiglu_bf16(np.concatenate([u, g], axis=1), K), h)
+    # extra columns beyond 2K are ignored (row stride > 2K)
+    pad = np.concatenate([g, u, np.full((1, 3), 7.0)], axis=1)
+    assert np.array_equal(O.swiglu_bf16(pad, K), h)
+
+
+def test_swiglu_rotate_quant_bruteforce():
+    # K = 4, no small factor, H4: y = h H4 / 2, then the INT4 rule by hand
+    K = 4
+    gu = np.array([[1.0, -2.0, 0.5, 3.0, 2.0, 1.0, -4.0, 0.25]])
+    h = [O.round_bf16(np.array([gu[0, k] / (1 + math.exp(-gu[0, k])) * gu[0, K + k]]))[0]
+         for k in range(K)]
+    H4 = [[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]]
+    y = [sum(h[i] * H4[i][j] for i in range(4)) / 2 for j in range(4)]
+    scale = np.float32(np.float32(max(abs(v) for v in y)) / np.float32(7.0))
+    codes = [int(np.clip(np.rint(np.float32(np.float32(v) / scale)), -8, 7)) for v in y]
+    packed, sc, c, _ = O.swiglu_rotate_quant(gu, K, 1, 4)
+    assert sc[0] == scale and list(c[0]) == codes
+
+
+# --------------------------------------------------------------------------
 # Workload generators (shapes and distributions only)
 # --------------------------------------------------------------------------
+
+def test_gate_up_workload_layout():
+    gu = W.gate_up_out(M=64, K=1024, seed=5)
+    assert gu.shape == (64, 2048) and gu.dtype.is_floating_point
+    x = gu.float().numpy()
+    assert np.array_equal(x, W.gate_up_out(M=64, K=1024, seed=5).float().numpy())
+    big = np.abs(x[:, 1024:]).max(axis=0)
+    assert (big > 100).sum() >= 8                   # the x100 up channels
+    assert np.abs(x[:, :1024]).max() < 100          # none in the gate half
+    h = O.swiglu_bf16(x, 1024)
+    assert (np.abs(h).max(axis=0) > 50).sum() >= 8  # they reach the SwiGLU product
+
 
 def test_workload_shapes_and_determinism():
     a = W.tiny_linear()

@@ -115,6 +115,23 @@ def swiglu_acts(rng: np.random.Generator, M: int, K: int, n_out: int = 8,
     return h
 
 
+def gate_up_out(M: int = 4096, K: int = MLP, seed: int = SEED_BASE + 6, n_out: int = 8,
+                factor: float = 100.0) -> torch.Tensor:
+    """The gate_up GEMM output as bf16 [M, 2K] = [gate | up], feeding SwiGLU + R4.
+
+    gate, up ~ Student-t(3); ``n_out`` up channels scaled by ``factor`` so the
+    SwiGLU product carries the outlier channels of ``swiglu_acts``.
+    """
+    rng = np.random.default_rng(seed)
+    out = np.empty((M, 2 * K))
+    out[:, :K] = rng.standard_t(3.0, (M, K))
+    up = rng.standard_t(3.0, (M, K))
+    _outliers(rng, up, n_out, factor)
+    out[:, K:] = up
+    del up
+    return _bf16(out)
+
+
 def down_proj(M: int = 4096, K: int = MLP, N: int = HIDDEN, seed: int = SEED_BASE + 1,
               with_weights: bool = True) -> LinearWorkload:
     """Online-R4 ``down_proj`` at Qwen3-8B shape: bf16 SwiGLU acts, H12 x H1024 rotation."""
