@@ -36,6 +36,8 @@ N_SMALL, N_POW2 = 12, 1024
 OPS = 2.0 * M * N * K
 # algorithmic bytes of sq_rotate_quant per row: bf16 in, packed INT4 out, f32 scale
 RQ_BYTES = M * (2 * K + K // 2 + 4)
+# ... of sq_swiglu_rotate_quant: bf16 gate and up in, packed INT4 out, f32 scale
+SWIGLU_BYTES = M * (2 * 2 * K + K // 2 + 4)
 KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
@@ -233,10 +235,31 @@ def run_ours(args, rank, world, local_rank):
                    "dequant_us": md * 1e3, "dequant_gbs": kv_rb_bytes / (md * 1e-3) / 1e9}
         del q, k, v, kvo, kdq, vdq
 
+    # fused SwiGLU + R4 rotate + quant on the gate_up output of the same
+    # tokens (the step before down_proj), timed alone for the record
+    sw_info = None
+    if not args.no_kv:
+        gu = W.gate_up_out(M=M, K=K).to(dev)
+        sq.swiglu_rotate_quant(gu, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+        torch.cuda.synchronize()
+        tsw = []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            sq.swiglu_rotate_quant(gu, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)
+            e1.record(stream)
+            tsw.append((e0, e1))
+        torch.cuda.synchronize()
+        msw = ms(tsw)
+        sw_info = {"workload": "gate_up_out_M%d_K%d_swiglu_R4" % (M, K), "us": msw * 1e3,
+                   "GB/s": SWIGLU_BYTES / (msw * 1e-3) / 1e9, "bytes": SWIGLU_BYTES}
+        del gu
+
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
-                clocks=clk.result, kv=kv_info)
+                clocks=clk.result, kv=kv_info, swiglu=sw_info)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -284,7 +307,8 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
 
 
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
-                 "decode_gemm_m1", "decode_gemm_m16", "rotate_quant_r4", "kv_rotate_quant")
+                 "decode_gemm_m1", "decode_gemm_m16", "rotate_quant_r4", "kv_rotate_quant",
+                 "swiglu_rotate_quant_r4")
 
 
 def run_profile_case(case, steps, warmup):
@@ -308,6 +332,12 @@ def run_profile_case(case, steps, warmup):
         a_q = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
         a_s = torch.empty((M,), dtype=torch.float32, device="cuda")
         fn = lambda: sq.rotate_quant(x, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
+    elif case == "swiglu_rotate_quant_r4":
+        gu = W.gate_up_out(M=M, K=K).cuda()
+        hs = sq.paley_h12()
+        a_q = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        a_s = torch.empty((M,), dtype=torch.float32, device="cuda")
+        fn = lambda: sq.swiglu_rotate_quant(gu, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
     elif case == "kv_rotate_quant":
         kvw = W.kv_path()
         q, k, v, pos = kvw.q.cuda(), kvw.k.cuda(), kvw.v.cuda(), kvw.pos.cuda()
@@ -468,6 +498,8 @@ def main():
             "w4a4_gemm": {"us": r["ms_gemm"] * 1e3, "TOPS": tops_gemm,
                           "frac_of_int8_peak": tops_gemm * 1e12 / (int8_peak * 1e12)},
             "kv_path": r["kv"],
+            "swiglu_rotate_quant": (dict(r["swiglu"], frac_of_hbm=r["swiglu"]["GB/s"] / hbm)
+                                    if r["swiglu"] else None),
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,

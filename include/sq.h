@@ -106,6 +106,36 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
                           float clip_ratio, uint8_t* a_q, float* a_scale, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * sq_swiglu_rotate_quant -- SwiGLU product, then the online rotation and
+ * per-token INT4 of sq_rotate_quant, in one pass.
+ *
+ * Source: "SpinQuant, Reproduced", Q5: R4 is applied online to the input of
+ * down_proj, which in the Qwen3-8B MLP of the same section is the SwiGLU
+ * product of the gate and up projections; fusing the two steps keeps that
+ * product out of memory.  Reading (the pages give no precision for it): the
+ * product is rounded once to bf16, the dtype of the down_proj input.
+ *
+ * For every row m and channel k < K:
+ *     g = gate_up[m][k],  u = gate_up[m][K + k]              (gate half first)
+ *     h[m][k] = bf16_round_nearest_even(silu(g) * u),  silu(g) = g / (1 + e^-g)
+ * evaluated in float32; then exactly sq_rotate_quant on x = h (bf16).  h is
+ * never written to memory.
+ *
+ * gate_up   device, bf16 [M][ld] (ld >= 2K, ld * 2 a multiple of 16 bytes),
+ *           16-byte aligned; read only.
+ * had_small, n_small, n_pow2, clip_ratio, a_q, a_scale: as sq_rotate_quant
+ *           (a_q [M][K/2] packed codes, a_scale [M] float32, both written).
+ * Shape rules and errors as sq_rotate_quant, with ld >= 2K; M == 0 is a
+ * no-op.  The SwiGLU is evaluated with hardware exponential and reciprocal
+ * approximations (a few float32 ulps), so h can differ from a correctly
+ * rounded product in its last bf16 bit where the product lies next to a
+ * rounding midpoint.
+ * ------------------------------------------------------------------------- */
+sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int64_t ld,
+                                 const int8_t* had_small, int n_small, int n_pow2,
+                                 float clip_ratio, uint8_t* a_q, float* a_scale, void* stream);
+
+/* ---------------------------------------------------------------------------
  * sq_w4a4_linear -- INT4 x INT4 GEMM with the per-token x per-channel dequant
  * fused into its epilogue.
  *

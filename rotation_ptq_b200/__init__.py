@@ -7,7 +7,7 @@ device.  There is no CPU fallback: if the library is missing, importing this
 package raises.
 
 Entry points (same names as the C ABI without the ``sq_`` prefix):
-  rotate_quant, w4a4_linear, w4a4_workspace_bytes, kv_rotate_quant,
+  rotate_quant, swiglu_rotate_quant, w4a4_linear, w4a4_workspace_bytes, kv_rotate_quant,
   kv_dequant, rope_tables, device_status, debug_set_spin_limit.
 """
 from __future__ import annotations
@@ -28,6 +28,7 @@ from .binding import (  # noqa: F401
     quantize_weights,
     rope_tables,
     rotate_quant,
+    swiglu_rotate_quant,
     version,
     w4a4_linear,
     w4a4_tail_workspace_bytes,

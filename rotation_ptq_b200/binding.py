@@ -38,6 +38,8 @@ lib.sq_last_error.argtypes = []
 lib.sq_version.restype = _i32
 lib.sq_rotate_quant.restype = _i32
 lib.sq_rotate_quant.argtypes = [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
+lib.sq_swiglu_rotate_quant.restype = _i32
+lib.sq_swiglu_rotate_quant.argtypes = [_vp, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
 lib.sq_w4a4_linear.restype = _i32
 lib.sq_w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp,
                                ctypes.c_size_t, _vp]
@@ -123,6 +125,44 @@ def rotate_quant(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float =
     st = lib.sq_rotate_quant(x.data_ptr(), dt, M, K, x.stride(0), hs_ptr, n_small, n_pow2,
                              float(clip), a_q.data_ptr(), a_scale.data_ptr(), _stream(x))
     _check(st, "sq_rotate_quant")
+    return a_q, a_scale
+
+
+def _small_hadamard(had_small):
+    if had_small is None:
+        return None, 1, None
+    hs = np.ascontiguousarray(np.asarray(had_small, dtype=np.int8))
+    n_small = hs.shape[0]
+    if hs.shape != (n_small, n_small):
+        raise ValueError("had_small must be square")
+    return hs, n_small, hs.ctypes.data
+
+
+def swiglu_rotate_quant(gate_up: torch.Tensor, had_small=None, n_pow2: int = 1,
+                        clip: float = 1.0, a_q: torch.Tensor = None,
+                        a_scale: torch.Tensor = None):
+    """SwiGLU of [gate | up] + online rotation + per-token INT4 (``sq_swiglu_rotate_quant``).
+
+    gate_up: CUDA bf16 [M, >= 2K] with unit stride along the columns; K is
+    half its width (gate = columns [0, K), up = [K, 2K)).  Returns
+    (a_q uint8 [M, K/2], a_scale f32 [M]).
+    """
+    _need_cuda(gate_up)
+    if gate_up.dim() != 2 or gate_up.stride(1) != 1 or gate_up.dtype != torch.bfloat16:
+        raise ValueError("gate_up must be a 2-D bf16 tensor with unit stride along columns")
+    M, W2 = gate_up.shape
+    if W2 % 2:
+        raise ValueError("gate_up width must be even ([gate | up])")
+    K = W2 // 2
+    hs, n_small, hs_ptr = _small_hadamard(had_small)
+    if a_q is None:
+        a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=gate_up.device)
+    if a_scale is None:
+        a_scale = torch.empty((M,), dtype=torch.float32, device=gate_up.device)
+    st = lib.sq_swiglu_rotate_quant(gate_up.data_ptr(), M, K, gate_up.stride(0), hs_ptr,
+                                    n_small, n_pow2, float(clip), a_q.data_ptr(),
+                                    a_scale.data_ptr(), _stream(gate_up))
+    _check(st, "sq_swiglu_rotate_quant")
     return a_q, a_scale
 
 

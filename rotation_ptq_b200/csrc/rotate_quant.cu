@@ -72,7 +72,14 @@ __device__ __forceinline__ float row_scale(float absmax, float clip) {
 // contiguous blocks of n_pow2 channels, then each thread applies the small
 // Hadamard to the n_small values (i * n_pow2 + j, i < n_small) of one
 // (group, j), then the row is normalised, reduced and quantized.
-template <typename T>
+// h = bf16(silu(g) * u), silu(g) = g / (1 + e^-g), in float32.
+__device__ __forceinline__ float swiglu_bf16(float g, float u) {
+  return __bfloat162float(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u));
+}
+
+// With SWIGLU the row is the SwiGLU product of x[m][0, K) (gate) and
+// x[m][K, 2K) (up), rounded to bf16 as it is staged.
+template <typename T, bool SWIGLU>
 __global__ void __launch_bounds__(256) rq_generic_kernel(const T* __restrict__ x, int64_t ldx,
                                                           int M, int K, SmallH hs, int ns, int np,
                                                           float norm, float clip,
@@ -83,7 +90,8 @@ __global__ void __launch_bounds__(256) rq_generic_kernel(const T* __restrict__ x
   const int G = ns * np;
   for (int m = blockIdx.x; m < M; m += gridDim.x) {
     const T* xr = x + static_cast<int64_t>(m) * ldx;
-    for (int i = threadIdx.x; i < K; i += blockDim.x) buf[i] = to_f<T>(xr[i]);
+    for (int i = threadIdx.x; i < K; i += blockDim.x)
+      buf[i] = SWIGLU ? swiglu_bf16(to_f<T>(xr[i]), to_f<T>(xr[K + i])) : to_f<T>(xr[i]);
     __syncthreads();
     for (int h = 1; h < np; h <<= 1) {
       for (int p = threadIdx.x; p < K / 2; p += blockDim.x) {
@@ -194,42 +202,107 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
 // Every wait is bounded; a group leaves its loop on one shared verdict
 // (barrier.cta.red.or), and the MMA thread drains its MMAs before the TMEM
 // is freed.
-constexpr int TC_STAGES = 6;
+//
+// With SWIGLU the input is the gate_up output [gate | up] and the row is
+// h = bf16(silu(gate) * up): a stage holds the gate row and the up row as
+// two identically swizzled copies, and h is formed element by element in
+// place of the gate row (the operation is elementwise, so the swizzle does
+// not matter).  A row is 1,536 chunks of 16 bytes: warp 11, which otherwise
+// idles, takes chunks [0, 672), and each of the three warps of the group
+// that will rotate the row three rows later takes 288 more (they form them
+// before waiting for their current row's accumulator, so the MMA of row
+// r + 3 overlaps their work on row r).  The split evens out the instructions
+// per SM sub-partition: the group's warps also run the butterflies.  The MMA
+// waits for all four parts instead of the TMA.
 constexpr int TC_NBUF = 3;                         // TMEM accumulators = row groups
 constexpr int TC_THREADS = 32 * 4 * TC_NBUF;       // 384
 constexpr int TC_ROW_BYTES = 12288 * 2;
 constexpr int TC_BOX_BYTES = 96 * 128;             // one 64-column box of a row
 constexpr int TC_A_ATOM = 128 * 128;               // 128 rows x 64 bf16 (one K atom)
 constexpr int TC_A_BYTES = 2 * TC_A_ATOM;          // K = 96 padded to two atoms
-constexpr int TC_BAR_OFF = TC_A_BYTES + TC_STAGES * TC_ROW_BYTES;
-constexpr int TC_NBARS = 2 * TC_STAGES + 2 * TC_NBUF + 1;
-constexpr int TC_MISC_OFF = TC_BAR_OFF + 8 * TC_NBARS;
-constexpr int TC_SMEM = TC_MISC_OFF + 16 + 4 * TC_NBUF * 2 * 3 + 1024;
 constexpr uint32_t TC_TMEM_COLS = 512;            // 128 * TC_NBUF, rounded to a power of 2
 constexpr int TC_TMA_WARP = 3;
 constexpr int TC_MMA_WARP = 7;
-static_assert(TC_SMEM <= 227 * 1024, "shared memory budget");
+constexpr int TC_AUX_WARP = 11;
+#ifndef SQ_TC_AUX_CHUNKS
+#define SQ_TC_AUX_CHUNKS 288
+#endif
+constexpr int TC_AUX_CHUNKS = SQ_TC_AUX_CHUNKS;     // SwiGLU chunks of warp 11 per row
+constexpr int TC_GROUP_CHUNKS = (TC_ROW_BYTES / 16 - TC_AUX_CHUNKS) / 3;   // ... of each group warp
+static_assert(TC_AUX_CHUNKS + 3 * TC_GROUP_CHUNKS == TC_ROW_BYTES / 16,
+              "the SwiGLU split covers the row");
+
+// Shared-memory plan: the constant operand, then STAGES row slots, then the
+// barriers (slot full, slot free, h ready; accumulator full / read; drain).
+template <bool SWIGLU>
+struct TcCfg {
+  static constexpr int STAGES = SWIGLU ? 4 : 6;
+  static constexpr int SLOT = (SWIGLU ? 2 : 1) * TC_ROW_BYTES;
+  static constexpr int BAR_OFF = TC_A_BYTES + STAGES * SLOT;
+  static constexpr int NBARS = 3 * STAGES + 2 * TC_NBUF + 1;
+  static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
+  static constexpr int SMEM = MISC_OFF + 16 + 4 * TC_NBUF * 2 * 3 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
 static_assert(TC_A_BYTES % 1024 == 0 && TC_ROW_BYTES % 1024 == 0 && TC_BOX_BYTES % 1024 == 0,
               "swizzle atoms need 1 KB alignment");
 
-template <bool CLAMP>
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));   // PTX: at most 1 ulp
+  return r;
+}
+
+// Chunks [c0, c1) of a row's SwiGLU product, in place: lane l takes 16-byte
+// chunks c0 + l, c0 + l + 32, ... (8 bf16 of gate and of up each);
+// h = bf16(g * u * (1 / (1 + e^-g))) = bf16(silu(g) * u) in float32, the
+// multiplies and adds on float pairs.
+__device__ __forceinline__ void swiglu_chunks(uint8_t* slot, int c0, int c1, int lane) {
+  uint8_t* gbase = slot;
+  const uint8_t* ubase = gbase + TC_ROW_BYTES;
+  const f2 one{1.0f, 1.0f};
+#pragma unroll 4
+  for (int c = c0 + lane; c < c1; c += 32) {
+    const uint4 g4 = *reinterpret_cast<const uint4*>(gbase + 16 * c);
+    const uint4 u4 = *reinterpret_cast<const uint4*>(ubase + 16 * c);
+    const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w}, uw[4] = {u4.x, u4.y, u4.z, u4.w};
+    uint32_t hw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const f2 g{__uint_as_float(gw[e] << 16), __uint_as_float(gw[e] & 0xFFFF0000u)};
+      const f2 u{__uint_as_float(uw[e] << 16), __uint_as_float(uw[e] & 0xFFFF0000u)};
+      const f2 d = add2(one, f2{__expf(-g.x), __expf(-g.y)});
+      const f2 h = mul2(mul2(g, u), f2{rcp_approx(d.x), rcp_approx(d.y)});
+      __nv_bfloat162 hb = __floats2bfloat162_rn(h.x, h.y);
+      hw[e] = *reinterpret_cast<uint32_t*>(&hb);
+    }
+    *reinterpret_cast<uint4*>(gbase + 16 * c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  }
+  fence_proxy_async_smem();          // h is read by the tensor core (async proxy)
+}
+
+template <bool CLAMP, bool SWIGLU>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    rq_h12x1024_tc_kernel(const __grid_constant__ CUtensorMap map_x, int M, float norm,
+    rq_h12x1024_tc_kernel(const __grid_constant__ CUtensorMap map_x,
+                          const __grid_constant__ CUtensorMap map_u, int M, float norm,
                           float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
                           float* __restrict__ ascale) {
+  using C = TcCfg<SWIGLU>;
+  constexpr int TC_STAGES = C::STAGES;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* Asm = smem;
   uint8_t* stage = smem + TC_A_BYTES;
-  uint64_t* sfull = reinterpret_cast<uint64_t*>(smem + TC_BAR_OFF);
+  uint64_t* sfull = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* sempty = sfull + TC_STAGES;
-  uint64_t* dfull = sempty + TC_STAGES;
+  uint64_t* hready = sempty + TC_STAGES;
+  uint64_t* dfull = hready + TC_STAGES;
   uint64_t* dempty = dfull + TC_NBUF;
   uint64_t* drain = dempty + TC_NBUF;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + TC_MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + TC_MISC_OFF + 4);
-  float* red = reinterpret_cast<float*>(smem + TC_MISC_OFF + 16);   // [group][parity][3]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  float* red = reinterpret_cast<float*>(smem + C::MISC_OFF + 16);   // [group][parity][3]
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int nrows = M > static_cast<int>(blockIdx.x)
@@ -264,6 +337,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int s = 0; s < TC_STAGES; ++s) {
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 1);
+      mbar_init(&hready[s], 4);
     }
     for (int b = 0; b < TC_NBUF; ++b) {
       mbar_init(&dfull[b], 1);
@@ -293,10 +367,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           break;
         }
         const int m = static_cast<int>(blockIdx.x) + r * static_cast<int>(gridDim.x);
-        uint8_t* dst = stage + s * TC_ROW_BYTES;
-        mbar_arrive_expect_tx(&sfull[s], TC_ROW_BYTES);
+        uint8_t* dst = stage + s * C::SLOT;
+        mbar_arrive_expect_tx(&sfull[s], C::SLOT);
         tma_load_3d(dst, &map_x, 0, 0, m, &sfull[s]);
         tma_load_3d(dst + TC_BOX_BYTES, &map_x, 64, 0, m, &sfull[s]);
+        if (SWIGLU) {
+          tma_load_3d(dst + TC_ROW_BYTES, &map_u, 0, 0, m, &sfull[s]);
+          tma_load_3d(dst + TC_ROW_BYTES + TC_BOX_BYTES, &map_u, 64, 0, m, &sfull[s]);
+        }
         ++issued;
       }
       // the latest copy into each slot must land before the CTA exits
@@ -309,13 +387,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t a0 = smem_u32(Asm);
       for (int r = 0; r < nrows; ++r) {
         const int s = r % TC_STAGES, d = r % TC_NBUF;
-        if (!mbar_wait(&sfull[s], (r / TC_STAGES) & 1, spin_limit) ||
+        if (!mbar_wait(SWIGLU ? &hready[s] : &sfull[s], (r / TC_STAGES) & 1, spin_limit) ||
             !mbar_wait(&dempty[d], ((r / TC_NBUF) & 1) ^ 1, spin_limit) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t b0 = smem_u32(stage + s * TC_ROW_BYTES);
+        const uint32_t b0 = smem_u32(stage + s * C::SLOT);
 #pragma unroll
         for (int k = 0; k < 6; ++k) {
           // A: K step k of 16 columns = 32 bytes inside atom k / 4;
@@ -332,16 +410,43 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_wait(drain, 0, 0);
     }
     __syncwarp();
+  } else if (SWIGLU && warp == TC_AUX_WARP) {
+    // the first TC_AUX_CHUNKS chunks of every row's SwiGLU product, in order
+    for (int r = 0; r < nrows; ++r) {
+      const int s = r % TC_STAGES;
+      if (!mbar_wait(&sfull[s], (r / TC_STAGES) & 1, spin_limit) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      swiglu_chunks(stage + s * C::SLOT, 0, TC_AUX_CHUNKS, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hready[s]);
+    }
   } else if ((warp & 3) != 3) {
     const int g = warp >> 2, q = warp & 3;
     const int mu = 32 * q + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
     float* gred = red + g * 2 * 3;
+    // this warp's part of row rr's SwiGLU product (rows g, g + 3, ... of
+    // this group)
+    auto swiglu_row = [&](int rr) -> bool {
+      const int s = rr % TC_STAGES;
+      if (!mbar_wait(&sfull[s], (rr / TC_STAGES) & 1, spin_limit)) return false;
+      const int c0 = TC_AUX_CHUNKS + q * TC_GROUP_CHUNKS;
+      swiglu_chunks(stage + s * C::SLOT, c0, c0 + TC_GROUP_CHUNKS, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hready[s]);
+      return true;
+    };
+    bool sw_ok = true;
+    if (SWIGLU && g < nrows) sw_ok = swiglu_row(g);
     int it = 0;
     for (int r = g; r < nrows; r += TC_NBUF, ++it) {
+      // the next row of this group first: its MMA then overlaps this row
+      if (SWIGLU && sw_ok && r + TC_NBUF < nrows) sw_ok = swiglu_row(r + TC_NBUF);
       const int d = r % TC_NBUF;
       const int m = static_cast<int>(blockIdx.x) + r * static_cast<int>(gridDim.x);
-      const bool fail = !mbar_wait(&dfull[d], (r / TC_NBUF) & 1, spin_limit);
+      const bool fail = !sw_ok || !mbar_wait(&dfull[d], (r / TC_NBUF) & 1, spin_limit);
       tc_fence_after();
       // w[p] = (column 2p, column 2p + 1) of this thread's TMEM lane
       f2 w[64];
@@ -482,12 +587,12 @@ __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, i
 
 // -------------------------------------------------------------- host launch
 
-template <typename T>
+template <typename T, bool SWIGLU = false>
 static sq_status launch_generic(const T* x, int64_t ldx, int M, int K, const SmallH& hs, int ns,
                                 int np, float norm, float clip, uint8_t* aq, float* as,
                                 cudaStream_t st) {
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
-  auto kfn = rq_generic_kernel<T>;
+  auto kfn = rq_generic_kernel<T, SWIGLU>;
   // opt in to the largest row the API admits (K <= 32768 floats = 128 KB)
   cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         32768 * static_cast<int>(sizeof(float)));
@@ -540,6 +645,55 @@ bool quant_fast_shape(int64_t K) {
   }
 }
 
+// Row m of a bf16 [.][ld] array as a [96][128] tile: dims (jl, kappa, m),
+// boxes of 64 x 96, 128-byte swizzle.
+static sq_status r4_map(CUtensorMap* map, const void* base, int64_t M, int64_t ld) {
+  auto encode = host::tensor_map_encoder();
+  if (!encode) return SQ_ERR_CUDA;
+  cuuint64_t dims[3] = {128, 96, static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[3] = {64, 96, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    host::set_error("cuTensorMapEncodeTiled(rotate) failed (%d)", static_cast<int>(cr));
+    return SQ_ERR_CUDA;
+  }
+  return SQ_OK;
+}
+
+template <bool SWIGLU>
+static sq_status launch_r4(const void* x, const void* u, int64_t M, int64_t ld, float norm,
+                           float clip, uint8_t* a_q, float* a_scale, cudaStream_t stream) {
+  CUtensorMap map_x, map_u;
+  sq_status st = r4_map(&map_x, x, M, ld);
+  if (st != SQ_OK) return st;
+  if (SWIGLU) {
+    st = r4_map(&map_u, u, M, ld);
+    if (st != SQ_OK) return st;
+  } else {
+    map_u = map_x;
+  }
+  const int m = static_cast<int>(M);
+  const int grid = m < host::num_sms() ? m : host::num_sms();
+  auto kfn = clip < 1.0f ? rq_h12x1024_tc_kernel<true, SWIGLU>
+                         : rq_h12x1024_tc_kernel<false, SWIGLU>;
+  constexpr int smem = TcCfg<SWIGLU>::SMEM;
+  cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
+  kfn<<<grid, TC_THREADS, smem, stream>>>(map_x, map_u, m, norm, clip, host::spin_limit(), a_q,
+                                          a_scale);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_h12x1024 launch", e);
+}
+
+static bool is_r4(int n_small, int n_pow2, int64_t K, const int8_t* had_small) {
+  return n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small);
+}
+
 sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
               const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
               float* a_scale, cudaStream_t stream) {
@@ -548,34 +702,8 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const int G = n_small * n_pow2;
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   const int m = static_cast<int>(M), k = static_cast<int>(K);
-  if (x_bf16 && n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small)) {
-    // row m as a [96][128] bf16 tile: dims (jl, kappa, m), boxes of 64 x 96
-    auto encode = host::tensor_map_encoder();
-    if (!encode) return SQ_ERR_CUDA;
-    CUtensorMap map;
-    cuuint64_t dims[3] = {128, 96, static_cast<cuuint64_t>(M)};
-    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
-    cuuint32_t box[3] = {64, 96, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) {
-      host::set_error("cuTensorMapEncodeTiled(rotate) failed (%d)", static_cast<int>(cr));
-      return SQ_ERR_CUDA;
-    }
-    const int grid = m < host::num_sms() ? m : host::num_sms();
-    const bool clamp = clip < 1.0f;
-    auto kfn = clamp ? rq_h12x1024_tc_kernel<true> : rq_h12x1024_tc_kernel<false>;
-    cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          TC_SMEM);
-    if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
-    kfn<<<grid, TC_THREADS, TC_SMEM, stream>>>(map, m, norm, clip, host::spin_limit(), a_q,
-                                               a_scale);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_h12x1024 launch", e);
-  }
+  if (x_bf16 && is_r4(n_small, n_pow2, K, had_small))
+    return launch_r4<false>(x, nullptr, M, ld_x, norm, clip, a_q, a_scale, stream);
   if (G == 1 && quant_fast_shape(K)) {
     return x_bf16 ? launch_quant(static_cast<const __nv_bfloat16*>(x), ld_x, m, k, clip, a_q,
                                  a_scale, stream)
@@ -586,6 +714,21 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
                                  n_pow2, norm, clip, a_q, a_scale, stream)
                 : launch_generic(static_cast<const float*>(x), ld_x, m, k, hs, n_small, n_pow2,
                                  norm, clip, a_q, a_scale, stream);
+}
+
+sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,
+                     const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
+                     float* a_scale, cudaStream_t stream) {
+  SmallH hs{};
+  for (int i = 0; i < n_small * n_small; ++i) hs.h[i] = n_small > 1 ? had_small[i] : 1;
+  const int G = n_small * n_pow2;
+  const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
+  auto gu = static_cast<const __nv_bfloat16*>(gate_up);
+  if (is_r4(n_small, n_pow2, K, had_small))
+    return launch_r4<true>(gu, gu + K, M, ld, norm, clip, a_q, a_scale, stream);
+  return launch_generic<__nv_bfloat16, true>(gu, ld, static_cast<int>(M), static_cast<int>(K),
+                                             hs, n_small, n_pow2, norm, clip, a_q, a_scale,
+                                             stream);
 }
 
 }  // namespace rq

@@ -151,15 +151,16 @@ sq_status sq_device_status(void* stream) {
   return SQ_OK;
 }
 
-sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
-                          int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
-                          float clip_ratio, uint8_t* a_q, float* a_scale, void* stream) {
-  if (x_dtype != SQ_IN_F32 && x_dtype != SQ_IN_BF16) {
-    set_error("x_dtype %d is not SQ_IN_F32 or SQ_IN_BF16", static_cast<int>(x_dtype));
-    return SQ_ERR_INVALID_ARG;
-  }
-  if (M < 0 || K < 0 || ld_x < K) {
-    set_error("bad sizes M=%lld K=%lld ld_x=%lld", (long long)M, (long long)K, (long long)ld_x);
+// Checks shared by sq_rotate_quant and sq_swiglu_rotate_quant: the rotation
+// and quantizer arguments, then sizes, pointers and alignment of an input of
+// `in_cols` columns (row stride ld elements of esz bytes).
+static sq_status check_rotate_args(const void* x, int64_t M, int64_t K, int64_t in_cols,
+                                   int64_t ld, int64_t esz, const int8_t* had_small,
+                                   int n_small, int n_pow2, float clip_ratio, const void* a_q,
+                                   const void* a_scale) {
+  if (M < 0 || K < 0 || ld < in_cols) {
+    set_error("bad sizes M=%lld K=%lld ld=%lld (need ld >= %lld)", (long long)M, (long long)K,
+              (long long)ld, (long long)in_cols);
     return SQ_ERR_INVALID_ARG;
   }
   if (!(clip_ratio > 0.f && clip_ratio <= 1.f)) {
@@ -198,15 +199,36 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
     set_error("null pointer argument");
     return SQ_ERR_INVALID_ARG;
   }
-  const int64_t esz = x_dtype == SQ_IN_BF16 ? 2 : 4;
-  if (!aligned16(x) || !aligned16(a_q) || !aligned16(a_scale) || (ld_x * esz) % 16 != 0) {
-    set_error("x, a_q and a_scale must be 16-byte aligned and ld_x*elem a multiple of 16");
+  if (!aligned16(x) || !aligned16(a_q) || !aligned16(a_scale) || (ld * esz) % 16 != 0) {
+    set_error("inputs, a_q and a_scale must be 16-byte aligned and ld*elem a multiple of 16");
     return SQ_ERR_MISALIGNED;
   }
-  sq_status st = precheck_device();
-  if (st != SQ_OK) return st;
+  return precheck_device();
+}
+
+sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
+                          float clip_ratio, uint8_t* a_q, float* a_scale, void* stream) {
+  if (x_dtype != SQ_IN_F32 && x_dtype != SQ_IN_BF16) {
+    set_error("x_dtype %d is not SQ_IN_F32 or SQ_IN_BF16", static_cast<int>(x_dtype));
+    return SQ_ERR_INVALID_ARG;
+  }
+  const int64_t esz = x_dtype == SQ_IN_BF16 ? 2 : 4;
+  sq_status st = check_rotate_args(x, M, K, K, ld_x, esz, had_small, n_small, n_pow2,
+                                   clip_ratio, a_q, a_scale);
+  if (st != SQ_OK || M == 0) return st;
   return sq::rq::run(x, x_dtype == SQ_IN_BF16, M, K, ld_x, had_small, n_small, n_pow2,
                      clip_ratio, a_q, a_scale, static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int64_t ld,
+                                 const int8_t* had_small, int n_small, int n_pow2,
+                                 float clip_ratio, uint8_t* a_q, float* a_scale, void* stream) {
+  sq_status st = check_rotate_args(gate_up, M, K, 2 * K, ld, 2, had_small, n_small, n_pow2,
+                                   clip_ratio, a_q, a_scale);
+  if (st != SQ_OK || M == 0) return st;
+  return sq::rq::run_swiglu(gate_up, M, K, ld, had_small, n_small, n_pow2, clip_ratio, a_q,
+                            a_scale, static_cast<cudaStream_t>(stream));
 }
 
 size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {

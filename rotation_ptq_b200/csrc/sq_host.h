@@ -63,6 +63,11 @@ namespace rq {
 sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
               const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
               float* a_scale, cudaStream_t stream);
+// SwiGLU of gate_up[m][0, K) and gate_up[m][K, 2K) (bf16, row stride ld),
+// rounded to bf16, then as run().
+sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,
+                     const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
+                     float* a_scale, cudaStream_t stream);
 }  // namespace rq
 
 namespace kv {

@@ -32,7 +32,8 @@ def sq():
 
 def test_header_declares_the_hot_path_calls():
     names = declared_functions()
-    for n in ["sq_rotate_quant", "sq_w4a4_linear", "sq_kv_rotate_quant", "sq_kv_dequant",
+    for n in ["sq_rotate_quant", "sq_swiglu_rotate_quant", "sq_w4a4_linear",
+              "sq_kv_rotate_quant", "sq_kv_dequant",
               "sq_status_string", "sq_w4a4_workspace_bytes", "sq_device_status"]:
         assert n in names
 
@@ -62,6 +63,15 @@ def test_validation_happens_before_any_launch(sq):
     assert lib.sq_rotate_quant(None, 1, 4, 12288, 12288, hs.ctypes.data, 12, 1024, 1.0,
                                None, None, None) == 1
     assert b"not +-1" in lib.sq_last_error()
+    # fused SwiGLU: the row must hold both halves (ld >= 2K); same K and clip rules
+    assert lib.sq_swiglu_rotate_quant(None, 4, 256, 300, None, 1, 256, 1.0, None, None,
+                                      None) == 1
+    assert lib.sq_swiglu_rotate_quant(None, 4, 256, 512, None, 1, 256, 0.0, None, None,
+                                      None) == 1
+    assert lib.sq_swiglu_rotate_quant(None, 4, 100, 200, None, 1, 4, 1.0, None, None,
+                                      None) == 2
+    assert lib.sq_swiglu_rotate_quant(None, 0, 256, 512, None, 1, 256, 1.0, None, None,
+                                      None) == 0
     # GEMM shape rules: N % 16, K % 128
     assert lib.sq_w4a4_linear(None, None, None, None, 4, 24, 256, None, 0, None, 0, None) == 2
     assert lib.sq_w4a4_linear(None, None, None, None, 4, 32, 200, None, 0, None, 0, None) == 2
