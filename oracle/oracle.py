@@ -30,6 +30,9 @@ Readings of points the pages leave open (each listed in the design doc):
     to float32, theta 1e6.
   * SwiGLU ahead of R4: h = bf16(silu(gate) * up), the product at full
     precision rounded once to bf16; the gate half first in [gate | up].
+  * Decode attention over the 4-bit caches: query head h reads KV head
+    h // (hq / hkv); softmax(q k^T / sqrt(d)) v over the first lengths[b]
+    cache rows b * S_max + s of sequence b.
 
 Parity pins: every function below is checked in tests/test_oracle_pins.py
 against closed forms, brute force or invariants that do not reuse it.
@@ -353,6 +356,45 @@ def kv_rotate_quant(q, k, v, pos, cos, sin):
 def kv_dequant(cache: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
     """Read-back of a packed asymmetric cache to float64 values."""
     return dequant_asym(unpack_int4(cache, signed=False), scale, zero)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention over the 4-bit caches.  "SpinQuant, Reproduced", Q5: R3 is a
+# head-wise Hadamard applied to Q and K after RoPE; being orthonormal it leaves
+# every query-key product unchanged, (q H)(k H)^T = q k^T, so attention can read
+# the rotated 4-bit K cache directly.  SpinQuant abstract: the KV cache is
+# 4-bit.  Reading (the pages give no attention kernel): one decode step with
+# grouped-query heads, query head h reading KV head h // (hq / hkv), and
+# softmax(q k^T / sqrt(d)) v over the first lengths[b] cached tokens of
+# sequence b (cache row b * S_max + s), in float64.
+# ---------------------------------------------------------------------------
+
+
+def decode_attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray,
+                     lengths: np.ndarray, S_max: int) -> np.ndarray:
+    """q [B, hq, d]; k_hat, v_hat [B * S_max, hkv, d]; lengths [B] -> o [B, hq, d]."""
+    q = np.asarray(q, np.float64)
+    B, hq, d = q.shape
+    hkv = k_hat.shape[1]
+    group = hq // hkv
+    o = np.zeros((B, hq, d))
+    for b in range(B):
+        n = int(lengths[b])
+        rows = slice(b * S_max, b * S_max + n)
+        for h in range(hq):
+            K = np.asarray(k_hat[rows, h // group], np.float64)
+            V = np.asarray(v_hat[rows, h // group], np.float64)
+            s = K @ q[b, h] / math.sqrt(d)
+            p = np.exp(s - s.max())
+            o[b, h] = (p / p.sum()) @ V
+    return o
+
+
+def kv4_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
+                         lengths, S_max: int) -> np.ndarray:
+    """decode_attention over the read-back (code - zero) * scale of both caches."""
+    return decode_attention(q, kv_dequant(k_cache, k_scale, k_zero),
+                            kv_dequant(v_cache, v_scale, v_zero), lengths, S_max)
 
 
 # ---------------------------------------------------------------------------

@@ -133,9 +133,38 @@ def _swiglu_no_up(gate_up, K):
     return O.round_bf16(O.silu(gu[:, :K]))
 
 
+def _attn_gqa_modulo(q, k_hat, v_hat, lengths, S_max):
+    q = np.asarray(q, np.float64)
+    B, hq, d = q.shape
+    hkv = k_hat.shape[1]
+    o = np.zeros((B, hq, d))
+    for b in range(B):
+        rows = slice(b * S_max, b * S_max + int(lengths[b]))
+        for h in range(hq):
+            s = k_hat[rows, h % hkv] @ q[b, h] / math.sqrt(d)
+            p = np.exp(s - s.max())
+            o[b, h] = (p / p.sum()) @ v_hat[rows, h % hkv]
+    return o
+
+
+def _attn_no_sqrt_d(q, k_hat, v_hat, lengths, S_max):
+    return _orig["decode_attention"](np.asarray(q, np.float64) * math.sqrt(q.shape[2]),
+                                     k_hat, v_hat, lengths, S_max)
+
+
+def _attn_one_extra_row(q, k_hat, v_hat, lengths, S_max):
+    return _orig["decode_attention"](q, k_hat, v_hat, np.minimum(np.asarray(lengths) + 1, S_max),
+                                     S_max)
+
+
+def _attn_k_for_v(q, k_hat, v_hat, lengths, S_max):
+    return _orig["decode_attention"](q, k_hat, k_hat, lengths, S_max)
+
+
 _orig = {name: getattr(O, name) for name in
          ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
-          "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16"]}
+          "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16",
+          "decode_attention"]}
 
 MUTATIONS = {
     "paley_transposed": ("paley1", _transposed_paley),
@@ -155,6 +184,10 @@ MUTATIONS = {
     "bf16_is_float32": ("round_bf16", _round_to_f32),
     "swiglu_halves_swapped": ("swiglu_bf16", _swiglu_halves_swapped),
     "swiglu_drops_up": ("swiglu_bf16", _swiglu_no_up),
+    "attention_gqa_modulo": ("decode_attention", _attn_gqa_modulo),
+    "attention_missing_sqrt_d": ("decode_attention", _attn_no_sqrt_d),
+    "attention_reads_one_row_too_many": ("decode_attention", _attn_one_extra_row),
+    "attention_k_used_as_v": ("decode_attention", _attn_k_for_v),
 }
 
 PIN_TESTS = [
@@ -182,6 +215,11 @@ PIN_TESTS = [
     P.test_silu_identities,
     P.test_swiglu_layout_and_special_values,
     P.test_swiglu_rotate_quant_bruteforce,
+    P.test_decode_attention_bruteforce,
+    P.test_decode_attention_closed_forms,
+    P.test_decode_attention_gqa_mapping,
+    P.test_decode_attention_rotation_invariance,
+    P.test_kv4_decode_attention_reads_the_caches,
 ]
 
 

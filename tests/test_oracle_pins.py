@@ -530,6 +530,87 @@ def test_swiglu_rotate_quant_bruteforce():
 
 
 # --------------------------------------------------------------------------
+# Decode attention over the 4-bit caches
+# --------------------------------------------------------------------------
+
+def _attn_inputs(seed, B=2, hq=4, hkv=2, d=8, S_max=5, lengths=(5, 3)):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, hq, d))
+    k = rng.standard_normal((B * S_max, hkv, d))
+    v = rng.standard_normal((B * S_max, hkv, d))
+    return q, k, v, np.array(lengths), S_max
+
+
+def test_decode_attention_bruteforce():
+    q, k, v, lengths, S = _attn_inputs(81)
+    o = O.decode_attention(q, k, v, lengths, S)
+    B, hq, d = q.shape
+    group = hq // k.shape[1]
+    for b in range(B):
+        for h in range(hq):
+            kv = h // group
+            rows = [b * S + s for s in range(int(lengths[b]))]
+            sc = [sum(q[b, h, i] * k[r, kv, i] for i in range(d)) / math.sqrt(d) for r in rows]
+            w = [math.exp(x) for x in sc]
+            tot = sum(w)
+            want = [sum(w[j] * v[r, kv, i] for j, r in enumerate(rows)) / tot for i in range(d)]
+            assert np.allclose(o[b, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_attention_closed_forms():
+    q, k, v, lengths, S = _attn_inputs(82)
+    # q = 0: uniform weights, the mean of the first lengths[b] rows
+    o = O.decode_attention(np.zeros_like(q), k, v, lengths, S)
+    assert np.allclose(o[0, 0], v[0:5, 0].mean(axis=0)) and np.allclose(o[1, 3], v[5:8, 1].mean(axis=0))
+    # one cached token: the output is its value row
+    o1 = O.decode_attention(q, k, v, np.array([1, 1]), S)
+    assert np.allclose(o1[1, 2], v[5, 1])
+    # two tokens: weight of the first = 1 / (1 + exp((s2 - s1) / sqrt(d)))
+    d = q.shape[2]
+    kk = np.zeros_like(k); vv = np.zeros_like(v)
+    kk[0, 0, 0], kk[1, 0, 0] = 2.0, -1.0
+    vv[0, 0, :], vv[1, 0, :] = 1.0, 0.0
+    qq = np.zeros_like(q); qq[0, 0, 0] = 3.0
+    o2 = O.decode_attention(qq, kk, vv, np.array([2, 1]), S)
+    assert np.isclose(o2[0, 0, 0], 1.0 / (1.0 + math.exp((-3.0 - 6.0) / math.sqrt(d))), rtol=1e-14)
+
+
+def test_decode_attention_gqa_mapping():
+    q, k, v, lengths, S = _attn_inputs(83, hq=4, hkv=2)
+    v = np.zeros_like(v)
+    v[:, 0, :], v[:, 1, :] = 1.0, 2.0
+    o = O.decode_attention(q, k, v, lengths, S)
+    # heads 0, 1 read KV head 0; heads 2, 3 read KV head 1
+    assert np.allclose(o[:, :2], 1.0) and np.allclose(o[:, 2:], 2.0)
+
+
+def test_decode_attention_rotation_invariance():
+    # R3 on both q and k (orthonormal H_d / sqrt(d)) leaves the output unchanged
+    q, k, v, lengths, S = _attn_inputs(84, d=8)
+    H = O.sylvester(8) / math.sqrt(8)
+    o = O.decode_attention(q, k, v, lengths, S)
+    o_rot = O.decode_attention(q @ H, k @ H, v, lengths, S)
+    assert np.allclose(o, o_rot, rtol=1e-12, atol=1e-12)
+
+
+def test_kv4_decode_attention_reads_the_caches():
+    # d = 2: one byte per cache row; row codes (3, 5), zero 1, scale 0.5 -> (1, 2)
+    kc = np.array([[[0x53]], [[0x21]]], np.uint8)          # [2 rows, 1 head, 1 byte]
+    ks = np.array([[0.5], [1.0]], np.float32)
+    kz = np.array([[1], [0]], np.uint8)
+    vc = np.array([[[0x10]], [[0x02]]], np.uint8)          # codes (0, 1) and (2, 0)
+    vs = np.array([[2.0], [0.25]], np.float32)
+    vz = np.array([[0], [2]], np.uint8)
+    q = np.array([[[1.0, 0.0]]])
+    o = O.kv4_decode_attention(q, kc, ks, kz, vc, vs, vz, np.array([2]), 2)
+    k_hat = np.array([[1.0, 2.0], [1.0, 2.0]])             # row 1: codes (1, 2), zero 0
+    v_hat = np.array([[0.0, 2.0], [0.0, -0.5]])            # row 1: (2 - 2, 0 - 2) * 0.25
+    sc = k_hat @ q[0, 0] / math.sqrt(2)
+    w = np.exp(sc - sc.max()); w /= w.sum()
+    assert np.allclose(o[0, 0], w @ v_hat, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
 # Workload generators (shapes and distributions only)
 # --------------------------------------------------------------------------
 

@@ -236,3 +236,46 @@ def random_scales(seed: int, n: int) -> np.ndarray:
     """Positive float32 scales spread over two decades (GEMM epilogue test input)."""
     rng = np.random.default_rng(seed)
     return (10.0 ** rng.uniform(-3, -1, n)).astype(np.float32)
+
+
+@dataclasses.dataclass
+class DecodeWorkload:
+    """One decode step over 4-bit caches: rotated queries, packed caches, lengths."""
+    name: str
+    q: torch.Tensor            # bf16 [B, hq, d]
+    k_cache: torch.Tensor      # uint8 [B * S_max, hkv, d / 2]
+    k_scale: torch.Tensor      # f32 [B * S_max, hkv]
+    k_zero: torch.Tensor       # uint8 [B * S_max, hkv]
+    v_cache: torch.Tensor
+    v_scale: torch.Tensor
+    v_zero: torch.Tensor
+    lengths: torch.Tensor      # int32 [B]
+    S_max: int
+
+
+def kv4_decode(B: int = 16, S_max: int = 4096, hq: int = N_HEADS, hkv: int = N_KV_HEADS,
+               d: int = 128, seed: int = SEED_BASE + 7, ragged: bool = False) -> DecodeWorkload:
+    """Decode step of the KV configuration (B 16 x S 4096, 32 / 8 heads, d 128).
+
+    Codes are uniform 4-bit values; scales and zero points take the range that
+    quantizing unit-variance head vectors gives (scale ~ 0.3..0.5, zero ~ 5..10);
+    queries ~ N(0, 1).  With ``ragged`` the lengths vary from 1 to S_max.
+    """
+    rng = np.random.default_rng(seed)
+    T = B * S_max
+    q = rng.standard_normal((B, hq, d))
+    kc = rng.integers(0, 256, (T, hkv, d // 2), dtype=np.uint8)
+    vc = rng.integers(0, 256, (T, hkv, d // 2), dtype=np.uint8)
+    ks = (0.3 + 0.2 * rng.random((T, hkv))).astype(np.float32)
+    vs = (0.3 + 0.2 * rng.random((T, hkv))).astype(np.float32)
+    kz = rng.integers(5, 11, (T, hkv)).astype(np.uint8)
+    vz = rng.integers(5, 11, (T, hkv)).astype(np.uint8)
+    if ragged:
+        lengths = rng.integers(1, S_max + 1, B)
+        lengths[0], lengths[-1] = S_max, 1
+    else:
+        lengths = np.full(B, S_max)
+    t = torch.from_numpy
+    return DecodeWorkload("kv4_decode_B%d_S%d_hq%d_hkv%d" % (B, S_max, hq, hkv), _bf16(q),
+                          t(kc), t(ks), t(kz), t(vc), t(vs), t(vz),
+                          t(lengths.astype(np.int32)), S_max)
