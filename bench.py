@@ -39,6 +39,9 @@ RQ_BYTES = M * (2 * K + K // 2 + 4)
 # ... of sq_swiglu_rotate_quant: bf16 gate and up in, packed INT4 out, f32 scale
 SWIGLU_BYTES = M * (2 * 2 * K + K // 2 + 4)
 KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
+# ... of one decode step of sq_kv4_decode_attention (B 16 x S 4096): both
+# caches with their scales and zeros, bf16 queries in and outputs out
+DECODE_BYTES = 2 * KV_T * KV_HKV * (64 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
@@ -256,10 +259,33 @@ def run_ours(args, rank, world, local_rank):
                    "GB/s": SWIGLU_BYTES / (msw * 1e-3) / 1e9, "bytes": SWIGLU_BYTES}
         del gu
 
+    # one decode step of attention over 4-bit caches of the KV configuration
+    dec_info = None
+    if not args.no_kv:
+        dw = W.kv4_decode()
+        dq, dkc, dks, dkz = dw.q.to(dev), dw.k_cache.to(dev), dw.k_scale.to(dev), dw.k_zero.to(dev)
+        dvc, dvs, dvz, dln = dw.v_cache.to(dev), dw.v_scale.to(dev), dw.v_zero.to(dev), dw.lengths.to(dev)
+        dout = sq.kv4_decode_attention(dq, dkc, dks, dkz, dvc, dvs, dvz, dln, dw.S_max)
+        torch.cuda.synchronize()
+        tde = []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            sq.kv4_decode_attention(dq, dkc, dks, dkz, dvc, dvs, dvz, dln, dw.S_max, out=dout)
+            e1.record(stream)
+            tde.append((e0, e1))
+        torch.cuda.synchronize()
+        mde = ms(tde)
+        dec_bytes = DECODE_BYTES
+        dec_info = {"workload": dw.name, "us": mde * 1e3,
+                    "GB/s": dec_bytes / (mde * 1e-3) / 1e9, "bytes": dec_bytes}
+        del dq, dkc, dks, dkz, dvc, dvs, dvz, dln, dout
+
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
-                clocks=clk.result, kv=kv_info, swiglu=sw_info)
+                clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -308,7 +334,7 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
 
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
                  "decode_gemm_m1", "decode_gemm_m16", "rotate_quant_r4", "kv_rotate_quant",
-                 "swiglu_rotate_quant_r4")
+                 "swiglu_rotate_quant_r4", "kv4_decode")
 
 
 def run_profile_case(case, steps, warmup):
@@ -338,6 +364,12 @@ def run_profile_case(case, steps, warmup):
         a_q = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
         a_s = torch.empty((M,), dtype=torch.float32, device="cuda")
         fn = lambda: sq.swiglu_rotate_quant(gu, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
+    elif case == "kv4_decode":
+        dw = W.kv4_decode()
+        t = [x.cuda() for x in (dw.q, dw.k_cache, dw.k_scale, dw.k_zero, dw.v_cache, dw.v_scale,
+                                dw.v_zero, dw.lengths)]
+        o = sq.kv4_decode_attention(*t, dw.S_max)
+        fn = lambda: sq.kv4_decode_attention(*t, dw.S_max, out=o)  # noqa: E731
     elif case == "kv_rotate_quant":
         kvw = W.kv_path()
         q, k, v, pos = kvw.q.cuda(), kvw.k.cuda(), kvw.v.cuda(), kvw.pos.cuda()
@@ -500,6 +532,8 @@ def main():
             "kv_path": r["kv"],
             "swiglu_rotate_quant": (dict(r["swiglu"], frac_of_hbm=r["swiglu"]["GB/s"] / hbm)
                                     if r["swiglu"] else None),
+            "kv4_decode_attention": (dict(r["decode"], frac_of_hbm=r["decode"]["GB/s"] / hbm)
+                                     if r["decode"] else None),
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,

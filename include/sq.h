@@ -284,6 +284,44 @@ void sq_debug_set_spin_limit(uint32_t polls);
  * Applies to calls made afterwards from any thread. */
 void sq_debug_set_gemm_path(int path);
 
+/* ---------------------------------------------------------------------------
+ * sq_kv4_decode_attention -- one decode step of attention over the 4-bit
+ * caches written by sq_kv_rotate_quant.
+ *
+ * Source: "SpinQuant, Reproduced", Q5 (R3 is a head-wise Hadamard on Q and K
+ * after RoPE; being orthonormal it leaves q . k unchanged, so attention reads
+ * the rotated K cache directly) and the SpinQuant abstract (4-bit KV cache).
+ *
+ * For sequence b < B and query head h < hq (KV head kh = h / 4):
+ *     o[b][h] = sum_s p_s v_hat[r][kh],  p = softmax_s(q[b][h] . k_hat[r][kh] / sqrt(128))
+ * over s < lengths[b], cache row r = b * S_max + s, x_hat = (code - zero) *
+ * scale; float32 arithmetic, output rounded to bf16.
+ *
+ * q          device bf16 [B][hq][128]: the step's rotated queries (the q_out of
+ *            sq_kv_rotate_quant for the new tokens), 16-byte aligned.
+ * k_cache, v_cache  device uint8 [B * S_max][hkv][64] (packed unsigned codes,
+ *            even element in the low nibble), 16-byte aligned.
+ * k_scale, v_scale  device float32 [B * S_max][hkv];  k_zero, v_zero  device
+ *            uint8 [B * S_max][hkv].
+ * lengths    device int32 [B], 1 <= lengths[b] <= S_max.  A length outside
+ *            that range is reported through sq_device_status() as
+ *            SQ_ERR_INVALID_ARG and gives a zero output row; nothing outside
+ *            the caches is read.
+ * out        device bf16 [B][hq][128] (written).
+ * workspace  optional device scratch of sq_kv4_decode_workspace_bytes() bytes,
+ *            zero on first use and left zero on return (one call at a time per
+ *            workspace).  With less (or NULL) the sequence is not split across
+ *            CTAs: same result, fewer CTAs.
+ * Shape rules: d == 128, hq == 4 * hkv, hkv <= 64; B == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+size_t sq_kv4_decode_workspace_bytes(int64_t B, int64_t S_max, int hq, int hkv);
+sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
+                                  const uint8_t* k_zero, const uint8_t* v_cache,
+                                  const float* v_scale, const uint8_t* v_zero,
+                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
+                                  int hkv, int d, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,7 +8,8 @@ package raises.
 
 Entry points (same names as the C ABI without the ``sq_`` prefix):
   rotate_quant, swiglu_rotate_quant, w4a4_linear, w4a4_workspace_bytes, kv_rotate_quant,
-  kv_dequant, rope_tables, device_status, debug_set_spin_limit.
+  kv_dequant, kv4_decode_attention, kv4_decode_workspace_bytes, rope_tables,
+  device_status, debug_set_spin_limit.
 """
 from __future__ import annotations
 
@@ -21,6 +22,8 @@ from .binding import (  # noqa: F401
     debug_set_gemm_path,
     debug_set_spin_limit,
     device_status,
+    kv4_decode_attention,
+    kv4_decode_workspace_bytes,
     kv_dequant,
     kv_rotate_quant,
     lib,

@@ -43,6 +43,11 @@ lib.sq_swiglu_rotate_quant.argtypes = [_vp, _i64, _i64, _i64, _vp, _i32, _i32, _
 lib.sq_w4a4_linear.restype = _i32
 lib.sq_w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp,
                                ctypes.c_size_t, _vp]
+lib.sq_kv4_decode_workspace_bytes.restype = ctypes.c_size_t
+lib.sq_kv4_decode_workspace_bytes.argtypes = [_i64, _i64, _i32, _i32]
+lib.sq_kv4_decode_attention.restype = _i32
+lib.sq_kv4_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32,
+                                        _i32, _i32, _vp, _vp, ctypes.c_size_t, _vp]
 lib.sq_w4a4_workspace_bytes.restype = ctypes.c_size_t
 lib.sq_w4a4_workspace_bytes.argtypes = [_i64, _i64, _i64]
 lib.sq_w4a4_tail_workspace_bytes.restype = ctypes.c_size_t
@@ -226,6 +231,45 @@ def w4a4_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
                             w_scale.data_ptr(), M, N, K, out.data_ptr(),
                             SQ_OUT_I32 if out_int32 else SQ_OUT_BF16, ws_ptr, ws_bytes, stream)
     _check(st, "sq_w4a4_linear")
+    return out
+
+
+def kv4_decode_workspace_bytes(B: int, S_max: int, hq: int, hkv: int) -> int:
+    """Scratch bytes that let sq_kv4_decode_attention split sequences across CTAs."""
+    return int(lib.sq_kv4_decode_workspace_bytes(B, S_max, hq, hkv))
+
+
+def kv4_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.Tensor,
+                         k_zero: torch.Tensor, v_cache: torch.Tensor, v_scale: torch.Tensor,
+                         v_zero: torch.Tensor, lengths: torch.Tensor, S_max: int,
+                         out: torch.Tensor = None, workspace: torch.Tensor = None):
+    """One decode step of attention over the 4-bit caches (``sq_kv4_decode_attention``).
+
+    q: bf16 [B, hq, 128]; caches uint8 [B * S_max, hkv, 64]; scales f32 and
+    zeros uint8 [B * S_max, hkv]; lengths int32 [B].  Returns bf16 [B, hq, 128].
+    Without ``workspace`` a cached zero-filled buffer of the stream is used.
+    """
+    _need_cuda(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths)
+    B, hq, d = q.shape
+    hkv = k_scale.shape[1]
+    for t, dt in ((q, torch.bfloat16), (k_cache, torch.uint8), (v_cache, torch.uint8),
+                  (k_scale, torch.float32), (v_scale, torch.float32), (k_zero, torch.uint8),
+                  (v_zero, torch.uint8), (lengths, torch.int32)):
+        if t.dtype != dt or not t.is_contiguous():
+            raise ValueError("decode attention inputs must be contiguous with the documented dtypes")
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=q.device)
+    stream = _stream(q)
+    need = kv4_decode_workspace_bytes(B, S_max, hq, hkv)
+    if workspace is None and need > 0:
+        workspace = _workspace(q.device, stream, need)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sq_kv4_decode_attention(q.data_ptr(), k_cache.data_ptr(), k_scale.data_ptr(),
+                                     k_zero.data_ptr(), v_cache.data_ptr(), v_scale.data_ptr(),
+                                     v_zero.data_ptr(), lengths.data_ptr(), B, S_max, hq, hkv, d,
+                                     out.data_ptr(), ws_ptr, ws_bytes, stream)
+    _check(st, "sq_kv4_decode_attention")
     return out
 
 

@@ -231,6 +231,46 @@ sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int6
                             a_scale, static_cast<cudaStream_t>(stream));
 }
 
+size_t sq_kv4_decode_workspace_bytes(int64_t B, int64_t S_max, int hq, int hkv) {
+  if (B <= 0 || S_max < 1 || hkv < 1 || hq != 4 * hkv) return 0;
+  if (sq::host::current_device() < 0) return 0;
+  return sq::kvd::workspace_bytes(B, S_max, hkv, sq::host::num_sms());
+}
+
+sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
+                                  const uint8_t* k_zero, const uint8_t* v_cache,
+                                  const float* v_scale, const uint8_t* v_zero,
+                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
+                                  int hkv, int d, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (B < 0 || S_max < 1 || hq < 1 || hkv < 1) {
+    set_error("bad sizes B=%lld S_max=%lld hq=%d hkv=%d", (long long)B, (long long)S_max, hq,
+              hkv);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (d != 128 || hq != 4 * hkv || hkv > 64 || B * hkv > (1LL << 24) ||
+      B * S_max > 0x7fffffffLL) {
+    set_error("unsupported shape d=%d hq=%d hkv=%d (need d == 128, hq == 4 * hkv)", d, hq, hkv);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (B == 0) return SQ_OK;
+  if (!q || !k_cache || !k_scale || !k_zero || !v_cache || !v_scale || !v_zero || !lengths ||
+      !out) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (workspace && !aligned16(workspace))) {
+    set_error("q, the caches, out and the workspace must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::kvd::run(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, B, S_max,
+                      hq, hkv, out, workspace, workspace ? workspace_bytes : 0,
+                      sq::host::num_sms(), static_cast<cudaStream_t>(stream));
+}
+
 size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N < 16 || N % 16 || K < 128 || K % 128 || K > 65536) return 0;
   if (sq::host::current_device() < 0) return 0;

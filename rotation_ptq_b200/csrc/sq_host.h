@@ -70,6 +70,17 @@ sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,
                      float* a_scale, cudaStream_t stream);
 }  // namespace rq
 
+namespace kvd {
+// Split count of the decode-attention kernel and the workspace it needs (0
+// when it runs unsplit).
+int choose_splits(int64_t B, int64_t S_max, int hkv, int num_sms);
+size_t workspace_bytes(int64_t B, int64_t S_max, int hkv, int num_sms);
+sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const uint8_t* k_zero,
+              const uint8_t* v_cache, const float* v_scale, const uint8_t* v_zero,
+              const int32_t* lengths, int64_t B, int64_t S_max, int hq, int hkv, void* out,
+              void* workspace, size_t workspace_bytes, int num_sms, cudaStream_t stream);
+}  // namespace kvd
+
 namespace kv {
 sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
                            int hkv, const int32_t* pos, const float* cos, const float* sin,

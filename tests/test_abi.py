@@ -33,6 +33,7 @@ def sq():
 def test_header_declares_the_hot_path_calls():
     names = declared_functions()
     for n in ["sq_rotate_quant", "sq_swiglu_rotate_quant", "sq_w4a4_linear",
+              "sq_kv4_decode_attention", "sq_kv4_decode_workspace_bytes",
               "sq_kv_rotate_quant", "sq_kv_dequant",
               "sq_status_string", "sq_w4a4_workspace_bytes", "sq_device_status"]:
         assert n in names
@@ -85,6 +86,12 @@ def test_validation_happens_before_any_launch(sq):
                                   None, None, None, None, None, None, None, None) == 2
     assert lib.sq_kv_dequant(None, None, None, 4, 8, 64, None, None) == 2
     assert lib.sq_rope_tables(0.5, 16, 128, None, None, None) == 1
+    # decode attention: d == 128 and hq == 4 * hkv; B == 0 is a no-op
+    args = [None] * 8
+    assert lib.sq_kv4_decode_attention(*args, 2, 16, 32, 8, 64, None, None, 0, None) == 2
+    assert lib.sq_kv4_decode_attention(*args, 2, 16, 16, 8, 128, None, None, 0, None) == 2
+    assert lib.sq_kv4_decode_attention(*args, 2, 0, 32, 8, 128, None, None, 0, None) == 1
+    assert lib.sq_kv4_decode_attention(*args, 0, 16, 32, 8, 128, None, None, 0, None) == 0
 
 
 def test_product_paley_matches_oracle():
