@@ -1,4 +1,4 @@
-// Decode attention over the asymmetric 4-bit KV caches, sm_100a CUDA cores.
+// Decode attention over the asymmetric 4-bit KV caches, sm_100a tensor cores.
 //
 // "SpinQuant, Reproduced", Q5: R3, the head-wise Hadamard on Q and K after
 // RoPE, is orthonormal, so q' k'^T = q k^T and a decode step can attend over
@@ -8,21 +8,32 @@
 //     r = b * S_max + s, s < lengths[b],  x_hat = (code - zero) * scale.
 // With the zero points factored out, q . k_hat = scale_k (q . code - zero_k
 // sum(q)) and sum_s p v_hat = sum_s p scale_v code - sum_s p scale_v zero_v,
-// so the inner loops multiply raw codes.
+// so both products multiply raw codes.
 //
 // Work split: one CTA per (b, kh, split), a split being a contiguous range of
-// the sequence's tokens; its 8 warps take batches of 8 tokens in turn.  In a
-// warp, half-warp j = lane / 16 takes token 2i + j of step i (4 steps per
-// batch) and lane e = lane % 16 owns dims 8e .. 8e + 7 of the 4 query heads:
-// its 8 codes of a token are one 32-bit word of the token's 64-byte row (the
-// 16 lanes of a half read the row in one coalesced 64-byte access).  The
-// 16 partial dot products of a half (4 tokens x 4 heads) are reduce-scattered
-// over its 16 lanes (15 shuffles), leaving lane e the score of token e / 4,
-// head e % 4; an online softmax in the exp2 domain follows, and the weights
-// go through shared memory to the value accumulators.  Warps combine in
-// shared memory; splits combine through the caller's workspace, the last CTA
-// of a (b, kh) reading all splits in split order (deterministic).
+// the sequence's tokens, taken in tiles of 128.  Both products run on the
+// tensor cores (tcgen05.mma kind::f16, f32 accumulation) with the 4-bit codes
+// as exact operands: a code c read as an f16 bit pattern is the subnormal
+// c * 2^-24, so eight packed codes become a 16-byte f16 operand chunk with two
+// masks and four byte permutes, and the products are exact.
+//   scores:  D_S[t][h] = sum_d code_k[t][d] q[h][d]   (M = 128 tokens, N = 16:
+//            the 4 heads and 12 zero rows, K = 128 dims; A = the tile's K codes,
+//            K-major, B = the queries as f16, exact for bf16 queries in f16's
+//            normal range)
+//   values:  D_O[d][n] = sum_t code_v[t][d] w[n][t]   (M = 128 dims, N = 32,
+//            K = 128 tokens; A = the V codes in the same rows, read MN-major;
+//            B = the weights p * scale_v split into an f16 high part (rows
+//            0..3) and the f16 remainder (rows 16..19), so they are not rounded)
+// Thread t of the CTA's 128 loads and widens token row t of a tile and owns
+// its scores; after the second product it owns output dim t.  The softmax is
+// online in the exp2 domain (tile maxima from redux.sync and 4 warps); the
+// output accumulates in registers, rescaled per tile.  V is widened into the
+// buffer of K once the score product has completed, so a CTA holds one 32 KB
+// code tile.  Warp 0 lane 0 issues the MMAs; every wait is bounded.  Splits
+// combine through the caller's workspace, the last CTA of a (b, kh) reading
+// all splits in split order (deterministic).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "sq_device.cuh"
@@ -33,10 +44,28 @@ namespace kvd {
 
 constexpr int D = 128;
 constexpr int G = 4;                       // query heads per KV head
-constexpr int WARPS = 8;
-constexpr int THREADS = 32 * WARPS;
+constexpr int TILE = 128;                  // tokens per tile (MMA rows)
+constexpr int THREADS = 128;
 constexpr int PART = D + 2;                // partial of one (split, head): m, l, o[128]
 constexpr float kLog2eOverSqrtD = 1.4426950408889634f / 11.313708498984761f;
+constexpr float kTwo24 = 16777216.0f;      // codes are read as c * 2^-24
+
+constexpr int A_ATOM = TILE * 128;         // [128 rows][64 f16], 128-byte swizzle
+constexpr int A_BYTES = 2 * A_ATOM;        // one code tile: K, then V
+constexpr int BQ_ATOM = 16 * 128;
+constexpr int BQ_BYTES = 2 * BQ_ATOM;      // queries [16][128]
+constexpr int BP_ATOM = 32 * 128;
+constexpr int BP_BYTES = 2 * BP_ATOM;      // weights [32][128 tokens]
+constexpr int OFF_BQ = A_BYTES;
+constexpr int OFF_BP = OFF_BQ + BQ_BYTES;
+constexpr int OFF_BAR = OFF_BP + BP_BYTES;
+constexpr int OFF_MISC = OFF_BAR + 16;
+constexpr int SMEM = OFF_MISC + 16 + 4 * 4 * 4 + 4 * 8 * 4 + 1024;
+constexpr uint32_t TMEM_COLS = 64;         // scores at column 0, outputs at 32
+constexpr uint32_t IDESC_QK = idesc_f16(128, 16, false, false);
+constexpr uint32_t IDESC_PV = idesc_f16(128, 32, true, false);
+static_assert(A_BYTES % 1024 == 0 && OFF_BQ % 1024 == 0 && OFF_BP % 1024 == 0,
+              "swizzle atoms need 1 KB alignment");
 
 struct Params {
   const __nv_bfloat16* q;
@@ -48,280 +77,337 @@ struct Params {
   const uint8_t* vz;
   const int32_t* lengths;
   int S_max, hkv, nsplit;
+  uint32_t spin_limit;
   __nv_bfloat16* out;
   unsigned* count;                         // [B * hkv] arrival counters (workspace start)
   float* part;                             // [B * hkv][nsplit][G][PART] after them (nsplit > 1)
 };
 
-// code (0..15) as float: the exponent of 2^23 with the code in the low mantissa bits
-__device__ __forceinline__ float code_f(uint32_t w, int e) {
-  return __uint_as_float(0x4B000000u | ((w >> (4 * e)) & 0xFu)) - 8388608.0f;
+// Byte offset of 16-byte chunk c (elements 8c .. 8c + 7) of row r in a
+// [rows][128] f16 tile kept as two 64-element atoms of atom_bytes each.
+__device__ __forceinline__ int sw_off(int r, int c, int atom_bytes) {
+  return (c >> 3) * atom_bytes + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
-// a[i] for a lane-dependent i without indexing memory
-__device__ __forceinline__ float pick4(const float (&a)[4], int i) {
-  return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
 }
 
-__global__ void __launch_bounds__(THREADS) kv4_decode_kernel(Params P) {
-  __shared__ float wo[WARPS][G][D];        // per-warp unnormalised outputs
-  __shared__ float wm[WARPS][G], wl[WARPS][G];
-  __shared__ __align__(16) float pbuf[WARPS][2][16];   // a half's 16 weights (read as float4)
-  __shared__ int last_flag;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, e = lane & 15;
+// The 8 codes of a packed word (element 2j in the low nibble of byte j) as
+// the f16 bit patterns 0..15: even codes in the bytes of lo, odd codes in the
+// bytes of hi; each pair takes one byte permute whose sign-replicating
+// selector nibbles (bit 3 set, source byte < 0x80) write the zero bytes.
+__device__ __forceinline__ uint4 codes_f16(uint32_t w) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  return make_uint4(prmt(lo, hi, 0xC480u), prmt(lo, hi, 0xD591u), prmt(lo, hi, 0xE6A2u),
+                    prmt(lo, hi, 0xF7B3u));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+struct Row {
+  uint4 k[4], v[4];
+  float sk, zk, sv, zv;
+};
+
+__global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
+  extern __shared__ uint8_t kvd_smem_raw[];
+  uint8_t* smem = kvd_smem_raw + ((1024u - (smem_u32(kvd_smem_raw) & 1023u)) & 1023u);
+  uint8_t* At = smem;
+  uint8_t* Bq = smem + OFF_BQ;
+  uint8_t* Bp = smem + OFF_BP;
+  uint64_t* done = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* drain = done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  float* red = reinterpret_cast<float*>(smem + OFF_MISC + 16);          // [warp][head]
+  float* red2 = red + 16;                                                // [warp][8]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bkh = blockIdx.x / P.nsplit, split = blockIdx.x - bkh * P.nsplit;
   const int b = bkh / P.hkv, kh = bkh - b * P.hkv;
   int len = __ldg(P.lengths + b);
   if (len < 1 || len > P.S_max) {
-    if (threadIdx.x == 0 && split == 0) record_status(SQ_ERR_INVALID_ARG);
+    if (tid == 0 && split == 0) record_status(SQ_ERR_INVALID_ARG);
     len = 0;                               // no token read; the output row becomes 0
   }
   const int per = (len + P.nsplit - 1) / P.nsplit;
   const int t0 = split * per, t1 = min(len, t0 + per);
-
-  // this lane's query slice: dims 8e..8e+7 of heads kh*G + h, as float pairs
-  f2 q[G][4];
-  float qsum[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(
-        P.q + (static_cast<int64_t>(b) * (P.hkv * G) + kh * G + h) * D + 8 * e));
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      q[h][k] = f2{__uint_as_float(ws[k] << 16), __uint_as_float(ws[k] & 0xFFFF0000u)};
-      s += q[h][k].x + q[h][k].y;
-    }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    qsum[h] = s;                           // sum over all 128 dims
-  }
-
-  const int hl = e & 3, tl = e >> 2;       // (head, token) of this lane's score
-  float m[G], lsum = 0.f, zsum = 0.f;      // running max per head; this lane's l, zero term
-  f2 acc[G][4];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[h][k] = f2{0.f, 0.f};
-  }
+  const int ntiles = t1 > t0 ? (t1 - t0 + TILE - 1) / TILE : 0;
   const int64_t row_stride = static_cast<int64_t>(P.hkv) * (D / 2);
   const int64_t row0 = static_cast<int64_t>(b) * P.S_max;
 
-  // all loads of a batch (8 tokens): the lane's K and V code words of its
-  // half's 4 tokens, and the scales and zeros of its score token
-  struct Batch {
-    uint32_t kw[4], vw[4];
-    float sk, zk, sv, zv;
-  };
-  auto load = [&](int base, Batch& bt) {
+  auto load_row = [&](int tok, Row& r) {
+    if (tok < t1) {
+      const int64_t off = (row0 + tok) * row_stride + kh * (D / 2);
+      const uint4* kp = reinterpret_cast<const uint4*>(P.kc + off);
+      const uint4* vp = reinterpret_cast<const uint4*>(P.vc + off);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = base + 2 * i + half;
-      bt.kw[i] = 0;
-      bt.vw[i] = 0;
-      if (t < t1) {
-        const int64_t off = (row0 + t) * row_stride + kh * (D / 2);
-        bt.kw[i] = __ldg(reinterpret_cast<const uint32_t*>(P.kc + off) + e);
-        bt.vw[i] = __ldg(reinterpret_cast<const uint32_t*>(P.vc + off) + e);
+      for (int i = 0; i < 4; ++i) {
+        r.k[i] = __ldg(kp + i);
+        r.v[i] = __ldg(vp + i);
       }
-    }
-    const int t = base + 2 * tl + half;
-    bt.sk = bt.zk = bt.sv = bt.zv = 0.f;
-    if (t < t1) {
-      const int64_t g = (row0 + t) * P.hkv + kh;
-      bt.sk = __ldg(P.ks + g);
-      bt.zk = static_cast<float>(__ldg(P.kz + g));
-      bt.sv = __ldg(P.vs + g);
-      bt.zv = static_cast<float>(__ldg(P.vz + g));
+      const int64_t g = (row0 + tok) * P.hkv + kh;
+      r.sk = __ldg(P.ks + g);
+      r.zk = static_cast<float>(__ldg(P.kz + g));
+      r.sv = __ldg(P.vs + g);
+      r.zv = static_cast<float>(__ldg(P.vz + g));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r.k[i] = r.v[i] = make_uint4(0u, 0u, 0u, 0u);
+      r.sk = r.zk = r.sv = r.zv = 0.f;
     }
   };
-  Batch cur;
-  int tb = t0 + 8 * warp;                  // first token of this warp's batch
-  if (tb < t1) load(tb, cur);
-  for (; tb < t1; tb += 8 * WARPS) {
-    // the next batch's loads go out before this batch is computed
-    Batch nxt;
-    if (tb + 8 * WARPS < t1) load(tb + 8 * WARPS, nxt);
-    // scores: 4 tokens x 4 heads of partial dots over this lane's 8 dims
-    float part[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f2 c[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) c[k] = f2{code_f(cur.kw[i], 2 * k), code_f(cur.kw[i], 2 * k + 1)};
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        f2 s = mul2(q[h][0], c[0]);
-#pragma unroll
-        for (int k = 1; k < 4; ++k) s = fma2(q[h][k], c[k], s);
-        part[4 * i + h] = s.x + s.y;
-      }
-    }
-    // reduce-scatter over the 16 lanes of the half: lane e keeps entry e
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) {
-      const bool up = (e & o) != 0;
-#pragma unroll
-      for (int k = 0; k < o; ++k) {
-        const float send = up ? part[k] : part[k + o];
-        const float keep = up ? part[k + o] : part[k];
-        part[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    const bool valid = tb + 2 * tl + half < t1;
-    const float score =
-        valid ? cur.sk * (part[0] - cur.zk * pick4(qsum, hl)) * kLog2eOverSqrtD : -INFINITY;
-    // online softmax: the batch maximum of each head, in every lane
-    float mx = score;
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    float alpha[G];
-    bool rescale = false;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mb = __shfl_sync(0xffffffffu, mx, h);
-      const float mn = fmaxf(m[h], mb);
-      alpha[h] = mn == m[h] ? 1.0f : exp2f(m[h] - mn);
-      rescale |= alpha[h] != 1.0f;
-      m[h] = mn;
-    }
-    const float a_l = pick4(alpha, hl);
-    const float p = valid ? exp2f(score - pick4(m, hl)) : 0.f;
-    lsum = lsum * a_l + p;
-    const float pv = p * cur.sv;           // weight times the value scale
-    zsum = zsum * a_l + pv * cur.zv;
-    pbuf[warp][half][e] = pv;
-    __syncwarp();
-    if (rescale) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const f2 a2{alpha[h], alpha[h]};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[h][k] = mul2(acc[h][k], a2);
-      }
-    }
-    // values: acc[h][dims] += pv(t, h) * code_v(t, dims) over the half's 4 tokens
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 pw = *reinterpret_cast<const float4*>(&pbuf[warp][half][4 * i]);
-      const float ph[G] = {pw.x, pw.y, pw.z, pw.w};
-      f2 c[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) c[k] = f2{code_f(cur.vw[i], 2 * k), code_f(cur.vw[i], 2 * k + 1)};
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const f2 p2{ph[h], ph[h]};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[h][k] = fma2(p2, c[k], acc[h][k]);
-      }
-    }
-    __syncwarp();
-    cur = nxt;
-  }
+  // the first tile's rows go out before the setup below
+  Row cur;
+  if (ntiles > 0) load_row(t0 + tid, cur);
 
-  // warp totals: l and the zero term per head, accumulators of both halves
+  // queries as f16 (rows 0..3 of Bq; rows 4..15 zero), their sums per head,
+  // and the weight tile's zero rows
+  float qsum[G];
+  for (int k = tid; k < 16 * 16; k += THREADS) {
+    const int r = k >> 4, c = k & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < G) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(
+          P.q + (static_cast<int64_t>(b) * (P.hkv * G) + kh * G + r) * D + 8 * c));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      uint32_t hw[4];
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
+      for (int e = 0; e < 4; ++e) {
+        __half2 h2 = __floats2half2_rn(__uint_as_float(ws[e] << 16),
+                                       __uint_as_float(ws[e] & 0xFFFF0000u));
+        hw[e] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      v = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+    *reinterpret_cast<uint4*>(Bq + sw_off(r, c, BQ_ATOM)) = v;
   }
-  float lw[G], zw[G];
+  for (int k = tid; k < BP_BYTES / 16; k += THREADS)
+    reinterpret_cast<uint4*>(Bp)[k] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    lw[h] = __shfl_sync(0xffffffffu, lsum, h);
-    zw[h] = __shfl_sync(0xffffffffu, zsum, h);
+    // the exact sum of the bf16 queries (tid < 128 covers all dims)
+    const float qv = __bfloat162float(
+        P.q[(static_cast<int64_t>(b) * (P.hkv * G) + kh * G + h) * D + tid]);
+    float s = qv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red2[warp * 8 + h] = s;
   }
+  if (tid == 0) {
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 #pragma unroll
   for (int h = 0; h < G; ++h)
+    qsum[h] = red2[h] + red2[8 + h] + red2[16 + h] + red2[24 + h];
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
+
+  auto store_codes = [&](const uint4 (&w)[4]) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      acc[h][k].x += __shfl_xor_sync(0xffffffffu, acc[h][k].x, 16);
-      acc[h][k].y += __shfl_xor_sync(0xffffffffu, acc[h][k].y, 16);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4*>(At + sw_off(tid, 4 * i + e, A_ATOM)) = codes_f16(ws[e]);
     }
-  if (half == 0) {
+  };
+
+  float m[G], lsum[G], zsum[G], o[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = -INFINITY;
+    lsum[h] = zsum[h] = o[h] = 0.f;
+  }
+  bool ok = true;
+  const uint32_t a_addr = smem_u32(At), bq_addr = smem_u32(Bq), bp_addr = smem_u32(Bp);
+  for (int it = 0; it < ntiles && ok; ++it) {
+    const int tok = t0 + it * TILE + tid;
+    const bool valid = tok < t1;
+    Row nxt;
+    if (it + 1 < ntiles) load_row(tok + TILE, nxt);
+    // scores: K codes of the tile, then the product with the queries
+    store_codes(cur.k);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16(tmem_base, desc_sw128(a_addr + (k >> 2) * A_ATOM + (k & 3) * 32),
+                 desc_sw128(bq_addr + (k >> 2) * BQ_ATOM + (k & 3) * 32), IDESC_QK,
+                 k > 0 ? 1u : 0u);
+      mma_commit(done);
+    }
+    ok = mbar_wait(done, 0, P.spin_limit);
+    tc_fence_after();
+    uint32_t s16[16];
+    tmem_ld16(lane_addr, s16);
+    tmem_ld_wait();
+    // the tile buffer is free again: V codes
+    store_codes(cur.v);
+    float sc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      sc[h] = valid ? cur.sk * (__uint_as_float(s16[h]) * kTwo24 - cur.zk * qsum[h]) *
+                          kLog2eOverSqrtD
+                    : -INFINITY;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        wo[warp][h][8 * e + 2 * k] = acc[h][k].x - zw[h];
-        wo[warp][h][8 * e + 2 * k + 1] = acc[h][k].y - zw[h];
-      }
+      const float mx = warp_max(sc[h]);
+      if (lane == 0) red[warp * 4 + h] = mx;
     }
+    __syncthreads();
+    float alpha[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mt = fmaxf(fmaxf(red[h], red[4 + h]), fmaxf(red[8 + h], red[12 + h]));
+      const float mn = fmaxf(m[h], mt);
+      alpha[h] = mn == m[h] ? 1.0f : exp2f(m[h] - mn);
+      m[h] = mn;
+      const float p = valid ? exp2f(sc[h] - mn) : 0.f;
+      lsum[h] = lsum[h] * alpha[h] + p;
+      // weight times the value scale as an f16 pair hi + lo
+      const float pv = p * cur.sv;
+      const __half hi = __float2half_rn(pv);
+      const __half lo = __float2half_rn(pv - __half2float(hi));
+      zsum[h] = zsum[h] * alpha[h] + (__half2float(hi) + __half2float(lo)) * cur.zv;
+      const int byte = (tid & 7) * 2;
+      *reinterpret_cast<__half*>(Bp + sw_off(h, tid >> 3, BP_ATOM) + byte) = hi;
+      *reinterpret_cast<__half*>(Bp + sw_off(16 + h, tid >> 3, BP_ATOM) + byte) = lo;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16(tmem_base + 32, desc_sw128_mn(a_addr + k * 2048, A_ATOM, 1024),
+                 desc_sw128(bp_addr + (k >> 2) * BP_ATOM + (k & 3) * 32), IDESC_PV,
+                 k > 0 ? 1u : 0u);
+      mma_commit(done);
+    }
+    ok = mbar_wait(done, 1, P.spin_limit) && ok;
+    tc_fence_after();
+    uint32_t o32[32];
+    tmem_ld32(lane_addr + 32, o32);
+    tmem_ld_wait();
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      o[h] = o[h] * alpha[h] +
+             (__uint_as_float(o32[h]) + __uint_as_float(o32[16 + h])) * kTwo24;
+    tc_fence_before();
+    cur = nxt;
+    ok = __syncthreads_and(ok) != 0;       // leave together if a wait gave up
   }
-  if (lane < G) {
-    wm[warp][lane] = m[lane];
-    wl[warp][lane] = lw[lane];
+
+  // totals over the CTA's threads: l and the zero term per head
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float l = lsum[h], z = zsum[h];
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, s);
+      z += __shfl_xor_sync(0xffffffffu, z, s);
+    }
+    if (lane == 0) {
+      red2[warp * 8 + h] = l;
+      red2[warp * 8 + 4 + h] = z;
+    }
   }
   __syncthreads();
-
-  // combine the warps: thread -> (head, two dims)
-  const int h = threadIdx.x >> 6, d0 = 2 * (threadIdx.x & 63);
-  float M = -INFINITY;
+  float L[G], Z[G];
 #pragma unroll
-  for (int w = 0; w < WARPS; ++w) M = fmaxf(M, wm[w][h]);
-  float L = 0.f, o0 = 0.f, o1 = 0.f;
-  if (M != -INFINITY) {
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) {
-      const float f = wm[w][h] == -INFINITY ? 0.f : exp2f(wm[w][h] - M);
-      L += wl[w][h] * f;
-      o0 += wo[w][h][d0] * f;
-      o1 += wo[w][h][d0 + 1] * f;
-    }
+  for (int h = 0; h < G; ++h) {
+    L[h] = red2[h] + red2[8 + h] + red2[16 + h] + red2[24 + h];
+    Z[h] = red2[4 + h] + red2[12 + h] + red2[20 + h] + red2[28 + h];
   }
-  __nv_bfloat16* dst =
-      P.out + (static_cast<int64_t>(b) * (P.hkv * G) + kh * G + h) * D + d0;
+  if (tid == 0) {                          // no MMA may still write the TMEM freed here
+    mma_commit(drain);
+    mbar_wait(drain, 0, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+
+  const int d = tid;
+  __nv_bfloat16* dst = P.out + (static_cast<int64_t>(b) * (P.hkv * G) + kh * G) * D + d;
   if (P.nsplit == 1) {
-    const float inv = L > 0.f ? 1.0f / L : 0.f;
-    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(o0 * inv, o1 * inv);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float inv = L[h] > 0.f ? 1.0f / L[h] : 0.f;
+      dst[h * D] = __float2bfloat16_rn((o[h] - Z[h]) * inv);
+    }
     return;
   }
-  float* mine = P.part + ((static_cast<int64_t>(bkh) * P.nsplit + split) * G + h) * PART;
-  if (d0 == 0) {
-    mine[0] = M;
-    mine[1] = L;
+  float* mine = P.part + (static_cast<int64_t>(bkh) * P.nsplit + split) * G * PART;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    if (d == 0) {
+      mine[h * PART] = m[h];
+      mine[h * PART + 1] = L[h];
+    }
+    mine[h * PART + 2 + d] = o[h] - Z[h];
   }
-  mine[2 + d0] = o0;
-  mine[3 + d0] = o1;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last_flag = atomicAdd(P.count + bkh, 1u) == static_cast<unsigned>(P.nsplit - 1);
+  __shared__ int last_flag;
+  if (tid == 0) last_flag = atomicAdd(P.count + bkh, 1u) == static_cast<unsigned>(P.nsplit - 1);
   __syncthreads();
   if (!last_flag) return;
   __threadfence();
   // the last CTA of (b, kh): all splits in split order
-  const float* base = P.part + (static_cast<int64_t>(bkh) * P.nsplit * G + h) * PART;
-  float Ms = -INFINITY;
-  for (int s = 0; s < P.nsplit; ++s) Ms = fmaxf(Ms, __ldcg(base + s * G * PART));
-  float Ls = 0.f, a0 = 0.f, a1 = 0.f;
-  if (Ms != -INFINITY) {
-    for (int s = 0; s < P.nsplit; ++s) {
-      const float* ps = base + s * G * PART;
-      const float ms = __ldcg(ps);
-      const float f = ms == -INFINITY ? 0.f : exp2f(ms - Ms);
-      Ls += __ldcg(ps + 1) * f;
-      a0 += __ldcg(ps + 2 + d0) * f;
-      a1 += __ldcg(ps + 3 + d0) * f;
+  const float* all = P.part + static_cast<int64_t>(bkh) * P.nsplit * G * PART;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float Ms = -INFINITY;
+    for (int s = 0; s < P.nsplit; ++s) Ms = fmaxf(Ms, __ldcg(all + (s * G + h) * PART));
+    float Ls = 0.f, acc = 0.f;
+    if (Ms != -INFINITY) {
+      for (int s = 0; s < P.nsplit; ++s) {
+        const float* ps = all + (s * G + h) * PART;
+        const float ms = __ldcg(ps);
+        const float f = ms == -INFINITY ? 0.f : exp2f(ms - Ms);
+        Ls += __ldcg(ps + 1) * f;
+        acc += __ldcg(ps + 2 + d) * f;
+      }
     }
+    dst[h * D] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
   }
-  const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
-  *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(a0 * inv, a1 * inv);
   // leave the workspace as it was found: counter and partials back to zero
   __syncthreads();
-  float* all = P.part + static_cast<int64_t>(bkh) * P.nsplit * G * PART;
-  for (int i = threadIdx.x; i < P.nsplit * G * PART; i += THREADS) all[i] = 0.f;
-  if (threadIdx.x == 0) P.count[bkh] = 0;
+  float* wall = P.part + static_cast<int64_t>(bkh) * P.nsplit * G * PART;
+  for (int i = tid; i < P.nsplit * G * PART; i += THREADS) wall[i] = 0.f;
+  if (tid == 0) P.count[bkh] = 0;
 }
 
 int choose_splits(int64_t B, int64_t S_max, int hkv, int num_sms) {
   const int64_t units = B * hkv;
-  int64_t s = (2 * static_cast<int64_t>(num_sms) + units - 1) / units;
-  const int64_t cap = (S_max + 255) / 256;           // at least 256 tokens per split
+  // as many splits as keep the grid within one wave of 4 CTAs per SM (the
+  // shared memory of a CTA allows 4), each at least two tiles long
+  int64_t s = 4 * static_cast<int64_t>(num_sms) / units;
+  const int64_t cap = (S_max + 2 * TILE - 1) / (2 * TILE);
   if (s > cap) s = cap;
   if (s < 1) s = 1;
   return static_cast<int>(s);
@@ -365,8 +451,12 @@ sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const
     P.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + count_bytes(B, hkv));
   }
   (void)hq;
+  P.spin_limit = host::spin_limit();
   const int64_t grid = B * hkv * ns;
-  kv4_decode_kernel<<<static_cast<unsigned>(grid), THREADS, 0, stream>>>(P);
+  cudaError_t ea = cudaFuncSetAttribute(kv4_decode_tc_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(kv4_decode)", ea);
+  kv4_decode_tc_kernel<<<static_cast<unsigned>(grid), THREADS, SMEM, stream>>>(P);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("kv4_decode launch", e);
 }
