@@ -30,6 +30,8 @@ Readings of points the pages leave open (each listed in the design doc):
     to float32, theta 1e6.
   * SwiGLU ahead of R4: h = bf16(silu(gate) * up), the product at full
     precision rounded once to bf16; the gate half first in [gate | up].
+  * W4A8: the activation quantizer on the 8-bit grid, scale = clip*absmax/127,
+    codes clamp(rint(y/scale), -128, 127).
   * Decode attention over the 4-bit caches: query head h reads KV head
     h // (hq / hkv); softmax(q k^T / sqrt(d)) v over the first lengths[b]
     cache rows b * S_max + s of sequence b.
@@ -250,12 +252,12 @@ def gemm_int(a_codes: np.ndarray, w_codes: np.ndarray) -> np.ndarray:
     """acc[m, n] = sum_k a[m, k] * w[n, k], exact, returned as int64.
 
     Uses a float64 BLAS matmul on integer-valued matrices: every partial sum is
-    an integer below 2^53 in magnitude (|a|,|w| <= 8, K < 2^40), so the result
-    is exact whatever order the library sums in.
+    an integer below 2^53 in magnitude (|a| <= 128, |w| <= 8, K < 2^43), so the
+    result is exact whatever order the library sums in.
     """
     a = np.asarray(a_codes, dtype=np.float64)
     w = np.asarray(w_codes, dtype=np.float64)
-    assert a.shape[1] == w.shape[1] and a.shape[1] * 64 < 2 ** 53
+    assert a.shape[1] == w.shape[1] and a.shape[1] * 128 * 8 < 2 ** 53
     return (a @ w.T).astype(np.int64)
 
 
@@ -268,6 +270,42 @@ def dequant(acc: np.ndarray, a_scale: np.ndarray, w_scale: np.ndarray) -> np.nda
 def w4a4_linear(a_packed, a_scale, w_packed, w_scale):
     """Packed-code W4A4 linear: returns (int64 acc, float64 dequantized output)."""
     acc = gemm_int(unpack_int4(a_packed), unpack_int4(w_packed))
+    return acc, dequant(acc, a_scale, w_scale)
+
+
+# ---------------------------------------------------------------------------
+# W4A8 ("SpinQuant, Reproduced", Q7: the evaluated settings include W4A8KV8,
+# 8-bit activations with 4-bit weights).  Reading (the pages give the setting,
+# not the quantizer): the activation quantizer of W4A4 on the 8-bit grid,
+# per token, scale = clip * absmax / 127, codes clamp(rint(y / scale), -128,
+# 127), one signed byte per code.
+# ---------------------------------------------------------------------------
+
+
+def quant_sym_int8(y: np.ndarray, clip: float = 1.0):
+    """Per-row symmetric INT8 round-to-nearest (decisions in float32).
+
+    scale = clip * max_k |y_k| / 127 (1 for an all-zero row); v = y / scale;
+    code = clamp(round_half_even(v), -128, 127).  Returns (codes int8, scale f32, v f32).
+    """
+    y = np.asarray(y, dtype=F32)
+    assert np.all(np.isfinite(y))
+    absmax = np.max(np.abs(y), axis=1)
+    scale = (F32(clip) * absmax) / F32(127.0)
+    scale = np.where(scale == 0, F32(1.0), scale).astype(F32)
+    v = (y / scale[:, None]).astype(F32)
+    codes = np.clip(np.rint(v), -128, 127).astype(np.int8)
+    return codes, scale, v
+
+
+def rotate_quant8(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
+    """Online rotation, then per-token INT8: returns (codes int8 [M, K], scale f32 [M], v f32)."""
+    return quant_sym_int8(rotate(x, n_small, n_pow2), clip)
+
+
+def w4a8_linear(a_codes, a_scale, w_packed, w_scale):
+    """INT8 activation codes x packed INT4 weights: (int64 acc, float64 dequantized output)."""
+    acc = gemm_int(np.asarray(a_codes, np.int64), unpack_int4(w_packed))
     return acc, dequant(acc, a_scale, w_scale)
 
 

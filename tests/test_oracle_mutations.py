@@ -161,10 +161,28 @@ def _attn_k_for_v(q, k_hat, v_hat, lengths, S_max):
     return _orig["decode_attention"](q, k_hat, k_hat, lengths, S_max)
 
 
+def _quant8_div128(y, clip=1.0):
+    y = np.asarray(y, F32)
+    s = (F32(clip) * np.max(np.abs(y), axis=1)) / F32(128.0)
+    s = np.where(s == 0, F32(1), s).astype(F32)
+    v = (y / s[:, None]).astype(F32)
+    return np.clip(np.rint(v), -128, 127).astype(np.int8), s, v
+
+
+def _quant8_symmetric_clamp(y, clip=1.0):
+    q, s, v = _orig["quant_sym_int8"](y, clip)
+    return np.clip(np.rint(v), -127, 127).astype(np.int8), s, v
+
+
+def _quant8_round_half_up(y, clip=1.0):
+    q, s, v = _orig["quant_sym_int8"](y, clip)
+    return np.clip(np.floor(v + F32(0.5)), -128, 127).astype(np.int8), s, v
+
+
 _orig = {name: getattr(O, name) for name in
          ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
           "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16",
-          "decode_attention"]}
+          "decode_attention", "quant_sym_int8"]}
 
 MUTATIONS = {
     "paley_transposed": ("paley1", _transposed_paley),
@@ -188,6 +206,9 @@ MUTATIONS = {
     "attention_missing_sqrt_d": ("decode_attention", _attn_no_sqrt_d),
     "attention_reads_one_row_too_many": ("decode_attention", _attn_one_extra_row),
     "attention_k_used_as_v": ("decode_attention", _attn_k_for_v),
+    "quant8_divisor_128": ("quant_sym_int8", _quant8_div128),
+    "quant8_clamps_at_minus_127": ("quant_sym_int8", _quant8_symmetric_clamp),
+    "quant8_round_half_up": ("quant_sym_int8", _quant8_round_half_up),
 }
 
 PIN_TESTS = [
@@ -220,6 +241,10 @@ PIN_TESTS = [
     P.test_decode_attention_gqa_mapping,
     P.test_decode_attention_rotation_invariance,
     P.test_kv4_decode_attention_reads_the_caches,
+    P.test_quant8_bruteforce_nearest_grid_point,
+    P.test_quant8_divisor_bound_and_special_rows,
+    P.test_w4a8_linear_bruteforce,
+    P.test_rotate_quant8_is_rotation_then_quant8,
 ]
 
 

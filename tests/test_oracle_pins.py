@@ -444,6 +444,74 @@ def test_kv_rotate_quant_composition():
 
 
 # --------------------------------------------------------------------------
+# W4A8: the 8-bit activation quantizer and the INT8 x INT4 linear
+# --------------------------------------------------------------------------
+
+def test_quant8_bruteforce_nearest_grid_point():
+    rng = np.random.default_rng(91)
+    for trial in range(200):
+        y = (rng.standard_normal(8) * rng.uniform(0.01, 10)).astype(np.float32)
+        q, s, v = O.quant_sym_int8(y[None, :])
+        sf = np.float32(s[0])
+        for k in range(8):
+            vk = np.float64(np.float32(y[k] / sf))
+            cands = np.arange(-128, 128)
+            d = np.abs(cands - vk)
+            best = cands[d == d.min()]
+            pick = best[best % 2 == 0][0] if len(best) > 1 else best[0]
+            assert q[0, k] == pick
+
+
+def test_quant8_divisor_bound_and_special_rows():
+    y = np.array([[1.0, -127.0, 2.5, 0.5]], dtype=np.float32)
+    q, s, _ = O.quant_sym_int8(y)
+    # divisor 127: the largest magnitude lands on -127; 2.5 -> 2 and 0.5 -> 0 (ties to even)
+    assert s[0] == np.float32(1.0) and list(q[0]) == [1, -127, 2, 0]
+    c = np.full((1, 16), 3.0, dtype=np.float32)
+    q, s, _ = O.quant_sym_int8(c)
+    assert np.all(q == 127) and np.isclose(s[0], 3.0 / 127)
+    q, s, _ = O.quant_sym_int8(np.zeros((1, 16), np.float32))
+    assert np.all(q == 0) and s[0] == 1.0
+    rng = np.random.default_rng(92)
+    y = (rng.standard_t(3, (50, 256)) * 3).astype(np.float32)
+    q, s, _ = O.quant_sym_int8(y)
+    assert np.all(np.abs(y - q.astype(np.float64) * s[:, None]) <= s[:, None] / 2 * (1 + 1e-6))
+    # clip < 1 saturates at the ends of the signed byte
+    q, s, _ = O.quant_sym_int8(np.array([[127.0, -127.0, 60.0, 0.0]], np.float32), clip=0.5)
+    assert s[0] == np.float32(0.5) and list(q[0]) == [127, -128, 120, 0]
+
+
+def test_w4a8_linear_bruteforce():
+    rng = np.random.default_rng(93)
+    a = rng.integers(-128, 128, (3, 16)).astype(np.int8)
+    wc = rng.integers(-8, 8, (4, 16)).astype(np.int8)
+    sa = rng.uniform(0.5, 2, 3).astype(np.float32)
+    sw = rng.uniform(0.5, 2, 4).astype(np.float32)
+    acc, out = O.w4a8_linear(a, sa, O.pack_int4(wc), sw)
+    for m in range(3):
+        for n in range(4):
+            want = sum(int(a[m, k]) * int(wc[n, k]) for k in range(16))
+            assert acc[m, n] == want
+            assert out[m, n] == want * float(sa[m]) * float(sw[n])
+    # extreme codes stay exact: 127 * 7 and -128 * -8 over a long K
+    K = 4096
+    acc, _ = O.w4a8_linear(np.full((1, K), -128, np.int8), np.ones(1, np.float32),
+                           O.pack_int4(np.full((1, K), -8, np.int8)), np.ones(1, np.float32))
+    assert acc[0, 0] == 1024 * K
+
+
+def test_rotate_quant8_is_rotation_then_quant8():
+    # K = 4, H4: y = x H4 / 2, then the 8-bit rule by hand
+    x = np.array([[1.0, -2.0, 0.5, 3.0]])
+    H4 = [[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]]
+    y = [sum(x[0, i] * H4[i][j] for i in range(4)) / 2 for j in range(4)]
+    scale = np.float32(np.float32(max(abs(v) for v in y)) / np.float32(127.0))
+    codes = [int(np.clip(np.rint(np.float32(np.float32(v) / scale)), -128, 127)) for v in y]
+    q, s, _ = O.rotate_quant8(x, 1, 4)
+    assert s[0] == scale and list(q[0]) == codes
+
+
+# --------------------------------------------------------------------------
 # SwiGLU ahead of down_proj (fused SwiGLU + R4)
 # --------------------------------------------------------------------------
 
