@@ -36,6 +36,8 @@ N_SMALL, N_POW2 = 12, 1024
 OPS = 2.0 * M * N * K
 # algorithmic bytes of sq_rotate_quant per row: bf16 in, packed INT4 out, f32 scale
 RQ_BYTES = M * (2 * K + K // 2 + 4)
+# ... of sq_rotate_quant8: bf16 in, one byte per code out, f32 scale
+RQ8_BYTES = M * (2 * K + K + 4)
 # ... of sq_swiglu_rotate_quant: bf16 gate and up in, packed INT4 out, f32 scale
 SWIGLU_BYTES = M * (2 * 2 * K + K // 2 + 4)
 KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
@@ -259,6 +261,34 @@ def run_ours(args, rank, world, local_rank):
                    "GB/s": SWIGLU_BYTES / (msw * 1e-3) / 1e9, "bytes": SWIGLU_BYTES}
         del gu
 
+    # W4A8 on the same down_proj step: 8-bit rotate+quant, INT8 x INT4 GEMM
+    a8_info = None
+    if not args.no_kv:
+        a8 = torch.empty((M, K), dtype=torch.int8, device=dev)
+        out8 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        sq.rotate_quant8(x_dev, hs, N_POW2, 1.0, a_q=a8, a_scale=a_s)
+        sq.w4a8_linear(a8, a_s, w_q, w_s, out=out8)
+        torch.cuda.synchronize()
+        tq8, tg8 = [], []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            sq.rotate_quant8(x_dev, hs, N_POW2, 1.0, a_q=a8, a_scale=a_s)
+            e1.record(stream)
+            sq.w4a8_linear(a8, a_s, w_q, w_s, out=out8)
+            e2.record(stream)
+            tq8.append((e0, e1))
+            tg8.append((e1, e2))
+        torch.cuda.synchronize()
+        mq8, mg8 = ms(tq8), ms(tg8)
+        a8_info = {"workload": WORKLOAD.replace("down_proj", "down_proj_W4A8"),
+                   "rotate_quant8_us": mq8 * 1e3,
+                   "rotate_quant8_GB/s": RQ8_BYTES / (mq8 * 1e-3) / 1e9,
+                   "gemm_us": mg8 * 1e3, "gemm_TOPS": OPS / (mg8 * 1e-3) / 1e12,
+                   "step_us": (mq8 + mg8) * 1e3}
+        del a8, out8
+
     # one decode step of attention over 4-bit caches of the KV configuration
     dec_info = None
     if not args.no_kv:
@@ -285,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
-                clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info)
+                clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info, a8=a8_info)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -534,6 +564,9 @@ def main():
                                     if r["swiglu"] else None),
             "kv4_decode_attention": (dict(r["decode"], frac_of_hbm=r["decode"]["GB/s"] / hbm)
                                      if r["decode"] else None),
+            "w4a8": (dict(r["a8"], rotate_quant8_frac_of_hbm=r["a8"]["rotate_quant8_GB/s"] / hbm,
+                          gemm_frac_of_int8_peak=r["a8"]["gemm_TOPS"] / int8_peak)
+                     if r["a8"] else None),
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,

@@ -106,6 +106,25 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
                           float clip_ratio, uint8_t* a_q, float* a_scale, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * sq_rotate_quant8 -- online Hadamard rotation + per-token symmetric INT8, the
+ * activation side of W4A8.
+ *
+ * Source: "SpinQuant, Reproduced", Q7 (the evaluated settings include W4A8KV8:
+ * 8-bit activations with 4-bit weights) and Q5 (where R4 sits).  Reading: the
+ * quantizer of sq_rotate_quant on the 8-bit grid.
+ *
+ * Same rotation and arguments as sq_rotate_quant, then per row
+ *     scale[m] = clip_ratio * max_k |y[m][k]| / 127     (1.0 for an all-zero row)
+ *     code[m][k] = clamp(round_half_even(y[m][k] / scale[m]), -128, 127)
+ * a_q       device, [M][K] signed bytes (written), 16-byte aligned.
+ * a_scale   device, [M] float32 (written).
+ * Shape rules and errors as sq_rotate_quant.
+ * ------------------------------------------------------------------------- */
+sq_status sq_rotate_quant8(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
+                           int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
+                           float clip_ratio, int8_t* a_q, float* a_scale, void* stream);
+
+/* ---------------------------------------------------------------------------
  * sq_swiglu_rotate_quant -- SwiGLU product, then the online rotation and
  * per-token INT4 of sq_rotate_quant, in one pass.
  *
@@ -210,6 +229,25 @@ size_t sq_w4a4_tail_workspace_bytes(int64_t M, int64_t N, int64_t K);
 sq_status sq_w4a4_linear_noalloc(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
                                  const float* w_scale, int64_t M, int64_t N, int64_t K,
                                  void* out, sq_out_kind kind, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * sq_w4a8_linear -- INT8 activations x INT4 weights (W4A8) with the same
+ * fused per-token x per-channel dequant as sq_w4a4_linear.
+ *
+ * Source: "SpinQuant, Reproduced", Q7 (W4A8KV8 among the evaluated settings).
+ *     acc[m][n] = sum_k a[m][k] * w[n][k]   (exact int32; |a| <= 128, |w| <= 8)
+ *     out[m][n] = bf16(float(acc) * a_scale[m] * w_scale[n])   or acc itself.
+ * a_q       device, [M][K] signed bytes (as sq_rotate_quant8 writes them).
+ * a_scale, w_q, w_scale, out, kind, workspace: as sq_w4a4_linear (the
+ *           workspace is optional here: it only lets a partial last wave of
+ *           large-M tiles split by K; size it with
+ *           sq_w4a4_tail_workspace_bytes).
+ * Shape rules and errors as sq_w4a4_linear.
+ * ------------------------------------------------------------------------- */
+sq_status sq_w4a8_linear(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                         const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
+                         sq_out_kind kind, void* workspace, size_t workspace_bytes,
+                         void* stream);
 
 /* ---------------------------------------------------------------------------
  * sq_kv_rotate_quant -- RoPE, head-wise Hadamard R3 on Q and K, and the

@@ -7,7 +7,8 @@ device.  There is no CPU fallback: if the library is missing, importing this
 package raises.
 
 Entry points (same names as the C ABI without the ``sq_`` prefix):
-  rotate_quant, swiglu_rotate_quant, w4a4_linear, w4a4_workspace_bytes, kv_rotate_quant,
+  rotate_quant, rotate_quant8, swiglu_rotate_quant, w4a4_linear, w4a8_linear,
+  w4a4_workspace_bytes, kv_rotate_quant,
   kv_dequant, kv4_decode_attention, kv4_decode_workspace_bytes, rope_tables,
   device_status, debug_set_spin_limit.
 """
@@ -31,10 +32,12 @@ from .binding import (  # noqa: F401
     quantize_weights,
     rope_tables,
     rotate_quant,
+    rotate_quant8,
     swiglu_rotate_quant,
     version,
     w4a4_linear,
     w4a4_tail_workspace_bytes,
     w4a4_workspace_bytes,
+    w4a8_linear,
 )
 from .hadamard import paley_h12  # noqa: F401

@@ -38,6 +38,11 @@ lib.sq_last_error.argtypes = []
 lib.sq_version.restype = _i32
 lib.sq_rotate_quant.restype = _i32
 lib.sq_rotate_quant.argtypes = [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
+lib.sq_w4a8_linear.restype = _i32
+lib.sq_w4a8_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp,
+                               ctypes.c_size_t, _vp]
+lib.sq_rotate_quant8.restype = _i32
+lib.sq_rotate_quant8.argtypes = [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
 lib.sq_swiglu_rotate_quant.restype = _i32
 lib.sq_swiglu_rotate_quant.argtypes = [_vp, _i64, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
 lib.sq_w4a4_linear.restype = _i32
@@ -141,6 +146,33 @@ def _small_hadamard(had_small):
     if hs.shape != (n_small, n_small):
         raise ValueError("had_small must be square")
     return hs, n_small, hs.ctypes.data
+
+
+def rotate_quant8(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float = 1.0,
+                  a_q: torch.Tensor = None, a_scale: torch.Tensor = None):
+    """Online rotation + per-token INT8 (``sq_rotate_quant8``, the A side of W4A8).
+
+    x: CUDA [M, K] bf16 or float32.  Returns (a_q int8 [M, K], a_scale f32 [M]).
+    """
+    _need_cuda(x)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit stride along K")
+    if x.dtype == torch.bfloat16:
+        dt = SQ_IN_BF16
+    elif x.dtype == torch.float32:
+        dt = SQ_IN_F32
+    else:
+        raise ValueError("x must be bf16 or float32")
+    M, K = x.shape
+    hs, n_small, hs_ptr = _small_hadamard(had_small)
+    if a_q is None:
+        a_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if a_scale is None:
+        a_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    st = lib.sq_rotate_quant8(x.data_ptr(), dt, M, K, x.stride(0), hs_ptr, n_small, n_pow2,
+                              float(clip), a_q.data_ptr(), a_scale.data_ptr(), _stream(x))
+    _check(st, "sq_rotate_quant8")
+    return a_q, a_scale
 
 
 def swiglu_rotate_quant(gate_up: torch.Tensor, had_small=None, n_pow2: int = 1,
@@ -270,6 +302,37 @@ def kv4_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.
                                      v_zero.data_ptr(), lengths.data_ptr(), B, S_max, hq, hkv, d,
                                      out.data_ptr(), ws_ptr, ws_bytes, stream)
     _check(st, "sq_kv4_decode_attention")
+    return out
+
+
+def w4a8_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
+                w_scale: torch.Tensor, out: torch.Tensor = None, out_i32: bool = False,
+                workspace: torch.Tensor = None):
+    """INT8 activations x packed INT4 weights (``sq_w4a8_linear``).
+
+    a_q: int8 [M, K] (from rotate_quant8); w_q: uint8 [N, K/2].  Returns bf16
+    (or, with out_i32, the exact int32 sums) [M, N].
+    """
+    _need_cuda(a_q, a_scale, w_q, w_scale)
+    if a_q.dtype != torch.int8 or w_q.dtype != torch.uint8:
+        raise ValueError("a_q must be int8 [M, K] and w_q uint8 [N, K/2]")
+    M, K = a_q.shape
+    N = w_q.shape[0]
+    if w_q.shape[1] * 2 != K:
+        raise ValueError("w_q must be [N, K/2]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if out_i32 else torch.bfloat16,
+                          device=a_q.device)
+    stream = _stream(a_q)
+    if workspace is None:
+        need = w4a4_tail_workspace_bytes(M, N, K)
+        workspace = _workspace(a_q.device, stream, need) if need > 0 else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sq_w4a8_linear(a_q.data_ptr(), a_scale.data_ptr(), w_q.data_ptr(),
+                            w_scale.data_ptr(), M, N, K, out.data_ptr(),
+                            SQ_OUT_I32 if out_i32 else SQ_OUT_BF16, ws_ptr, ws_bytes, stream)
+    _check(st, "sq_w4a8_linear")
     return out
 
 

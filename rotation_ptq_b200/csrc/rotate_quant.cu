@@ -65,6 +65,18 @@ __device__ __forceinline__ float row_scale(float absmax, float clip) {
   return s == 0.f ? 1.0f : s;
 }
 
+// INT8 (W4A8): signed byte code and the scale clip * absmax / 127.
+__device__ __forceinline__ uint32_t code_of8(float y, float scale) {
+  float v = __fdiv_rn(y, scale);
+  v = fminf(fmaxf(rintf(v), -128.f), 127.f);
+  return static_cast<uint32_t>(static_cast<int>(v)) & 0xFFu;
+}
+
+__device__ __forceinline__ float row_scale8(float absmax, float clip) {
+  float s = __fdiv_rn(clip * absmax, 127.0f);
+  return s == 0.f ? 1.0f : s;
+}
+
 // ------------------------------------------------------------------ generic
 
 // One CTA per row (grid-stride).  The row is staged in shared memory as
@@ -78,8 +90,9 @@ __device__ __forceinline__ float swiglu_bf16(float g, float u) {
 }
 
 // With SWIGLU the row is the SwiGLU product of x[m][0, K) (gate) and
-// x[m][K, 2K) (up), rounded to bf16 as it is staged.
-template <typename T, bool SWIGLU>
+// x[m][K, 2K) (up), rounded to bf16 as it is staged.  BITS 8 writes one
+// signed byte per code (W4A8) instead of packed nibbles.
+template <typename T, bool SWIGLU, int BITS = 4>
 __global__ void __launch_bounds__(256) rq_generic_kernel(const T* __restrict__ x, int64_t ldx,
                                                           int M, int K, SmallH hs, int ns, int np,
                                                           float norm, float clip,
@@ -124,12 +137,17 @@ __global__ void __launch_bounds__(256) rq_generic_kernel(const T* __restrict__ x
       amax = fmaxf(amax, fabsf(y));
     }
     amax = block_max<256>(amax, red);
-    const float s = row_scale(amax, clip);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(aq + static_cast<int64_t>(m) * (K / 2));
-    for (int w = threadIdx.x; w < K / 8; w += blockDim.x) {
+    const float s = BITS == 8 ? row_scale8(amax, clip) : row_scale(amax, clip);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(aq + static_cast<int64_t>(m) * (K * BITS / 8));
+    for (int w = threadIdx.x; w < K * BITS / 32; w += blockDim.x) {
       uint32_t word = 0;
+      if (BITS == 8) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) word |= code_of(buf[w * 8 + e], s) << (4 * e);
+        for (int e = 0; e < 4; ++e) word |= code_of8(buf[w * 4 + e], s) << (8 * e);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) word |= code_of(buf[w * 8 + e], s) << (4 * e);
+      }
       dst[w] = word;
     }
     if (threadIdx.x == 0) ascale[m] = s;
@@ -281,7 +299,7 @@ __device__ __forceinline__ void swiglu_chunks(uint8_t* slot, int c0, int c1, int
   fence_proxy_async_smem();          // h is read by the tensor core (async proxy)
 }
 
-template <bool CLAMP, bool SWIGLU>
+template <bool CLAMP, bool SWIGLU, bool A8>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     rq_h12x1024_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                           const __grid_constant__ CUtensorMap map_u, int M, float norm,
@@ -491,9 +509,38 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       amax = fmaxf(fmaxf(gred[(it & 1) * 3], gred[(it & 1) * 3 + 1]), gred[(it & 1) * 3 + 2]);
-      const float sc = row_scale(amax * norm, clip);
+      const float sc = A8 ? row_scale8(amax * norm, clip) : row_scale(amax * norm, clip);
       const f2 k2{norm * __frcp_rn(sc), norm * __frcp_rn(sc)};   // y_unnormalised -> y / scale
       const f2 magic{12582912.f, 12582912.f};                  // 1.5 * 2^23: nearest even
+      if (A8) {
+        // one signed byte per code: 128 bytes for this thread's 128 channels
+        uint4* dst8 = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 12288 + mu * 128);
+#pragma unroll
+        for (int n4 = 0; n4 < 8; ++n4) {
+          uint32_t word[4];
+#pragma unroll
+          for (int nn = 0; nn < 4; ++nn) {
+            f2 c[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const f2 wv = w[8 * n4 + 2 * nn + e];
+              if (CLAMP) {
+                c[e] = mul2(wv, k2);
+                c[e].x = fminf(fmaxf(c[e].x, -128.f), 127.f);
+                c[e].y = fminf(fmaxf(c[e].y, -128.f), 127.f);
+                c[e] = add2(c[e], magic);
+              } else {
+                c[e] = fma2(wv, k2, magic);
+              }
+            }
+            word[nn] = pack4b(__float_as_uint(c[0].x), __float_as_uint(c[0].y),
+                              __float_as_uint(c[1].x), __float_as_uint(c[1].y));
+          }
+          dst8[n4] = make_uint4(word[0], word[1], word[2], word[3]);
+        }
+        if (mu == 0) ascale[m] = sc;
+        continue;
+      }
       uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * 6144 + mu * 64);
 #pragma unroll
       for (int n4 = 0; n4 < 4; ++n4) {
@@ -587,12 +634,12 @@ __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, i
 
 // -------------------------------------------------------------- host launch
 
-template <typename T, bool SWIGLU = false>
+template <typename T, bool SWIGLU = false, int BITS = 4>
 static sq_status launch_generic(const T* x, int64_t ldx, int M, int K, const SmallH& hs, int ns,
                                 int np, float norm, float clip, uint8_t* aq, float* as,
                                 cudaStream_t st) {
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
-  auto kfn = rq_generic_kernel<T, SWIGLU>;
+  auto kfn = rq_generic_kernel<T, SWIGLU, BITS>;
   // opt in to the largest row the API admits (K <= 32768 floats = 128 KB)
   cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         32768 * static_cast<int>(sizeof(float)));
@@ -665,7 +712,7 @@ static sq_status r4_map(CUtensorMap* map, const void* base, int64_t M, int64_t l
   return SQ_OK;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool A8 = false>
 static sq_status launch_r4(const void* x, const void* u, int64_t M, int64_t ld, float norm,
                            float clip, uint8_t* a_q, float* a_scale, cudaStream_t stream) {
   CUtensorMap map_x, map_u;
@@ -679,8 +726,8 @@ static sq_status launch_r4(const void* x, const void* u, int64_t M, int64_t ld, 
   }
   const int m = static_cast<int>(M);
   const int grid = m < host::num_sms() ? m : host::num_sms();
-  auto kfn = clip < 1.0f ? rq_h12x1024_tc_kernel<true, SWIGLU>
-                         : rq_h12x1024_tc_kernel<false, SWIGLU>;
+  auto kfn = clip < 1.0f ? rq_h12x1024_tc_kernel<true, SWIGLU, A8>
+                         : rq_h12x1024_tc_kernel<false, SWIGLU, A8>;
   constexpr int smem = TcCfg<SWIGLU>::SMEM;
   cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
@@ -714,6 +761,25 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
                                  n_pow2, norm, clip, a_q, a_scale, stream)
                 : launch_generic(static_cast<const float*>(x), ld_x, m, k, hs, n_small, n_pow2,
                                  norm, clip, a_q, a_scale, stream);
+}
+
+sq_status run8(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
+               const int8_t* had_small, int n_small, int n_pow2, float clip, int8_t* a_q,
+               float* a_scale, cudaStream_t stream) {
+  SmallH hs{};
+  for (int i = 0; i < n_small * n_small; ++i) hs.h[i] = n_small > 1 ? had_small[i] : 1;
+  const int G = n_small * n_pow2;
+  const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
+  const int m = static_cast<int>(M), k = static_cast<int>(K);
+  uint8_t* q8 = reinterpret_cast<uint8_t*>(a_q);
+  if (x_bf16 && is_r4(n_small, n_pow2, K, had_small))
+    return launch_r4<false, true>(x, nullptr, M, ld_x, norm, clip, q8, a_scale, stream);
+  return x_bf16 ? launch_generic<__nv_bfloat16, false, 8>(static_cast<const __nv_bfloat16*>(x),
+                                                          ld_x, m, k, hs, n_small, n_pow2, norm,
+                                                          clip, q8, a_scale, stream)
+                : launch_generic<float, false, 8>(static_cast<const float*>(x), ld_x, m, k, hs,
+                                                  n_small, n_pow2, norm, clip, q8, a_scale,
+                                                  stream);
 }
 
 sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,

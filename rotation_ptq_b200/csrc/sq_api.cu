@@ -221,6 +221,21 @@ sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t
                      clip_ratio, a_q, a_scale, static_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_rotate_quant8(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
+                           int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,
+                           float clip_ratio, int8_t* a_q, float* a_scale, void* stream) {
+  if (x_dtype != SQ_IN_F32 && x_dtype != SQ_IN_BF16) {
+    set_error("x_dtype %d is not SQ_IN_F32 or SQ_IN_BF16", static_cast<int>(x_dtype));
+    return SQ_ERR_INVALID_ARG;
+  }
+  const int64_t esz = x_dtype == SQ_IN_BF16 ? 2 : 4;
+  sq_status st = check_rotate_args(x, M, K, K, ld_x, esz, had_small, n_small, n_pow2,
+                                   clip_ratio, a_q, a_scale);
+  if (st != SQ_OK || M == 0) return st;
+  return sq::rq::run8(x, x_dtype == SQ_IN_BF16, M, K, ld_x, had_small, n_small, n_pow2,
+                      clip_ratio, a_q, a_scale, static_cast<cudaStream_t>(stream));
+}
+
 sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int64_t ld,
                                  const int8_t* had_small, int n_small, int n_pow2,
                                  float clip_ratio, uint8_t* a_q, float* a_scale, void* stream) {
@@ -316,6 +331,41 @@ sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t
   return sq::gemm::run(a_q, a_scale, w_q, w_scale, M, N, K, out, kind == SQ_OUT_I32, workspace,
                        workspace_bytes, static_cast<cudaStream_t>(stream),
                        sq::host::spin_limit(), sq::host::num_sms(), nullptr);
+}
+
+sq_status sq_w4a8_linear(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                         const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
+                         sq_out_kind kind, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (kind != SQ_OUT_BF16 && kind != SQ_OUT_I32) {
+    set_error("kind %d is not SQ_OUT_BF16 or SQ_OUT_I32", static_cast<int>(kind));
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (M < 0 || N < 0 || K < 0) {
+    set_error("negative size");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (N < 16 || N % 16 != 0 || K < 128 || K % 128 != 0 || K > 65536 || M > 0x7fffffff ||
+      N > 0x7fffffff) {
+    set_error("shape M=%lld N=%lld K=%lld: need N %% 16 == 0, K %% 128 == 0, 128 <= K <= 65536",
+              (long long)M, (long long)N, (long long)K);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (M == 0) return SQ_OK;
+  if (!a_q || !a_scale || !w_q || !w_scale || !out) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(a_q) || !aligned16(a_scale) || !aligned16(w_q) || !aligned16(w_scale) ||
+      !aligned16(out) || (workspace && !aligned16(workspace))) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::gemm::run_a8(a_q, a_scale, w_q, w_scale, M, N, K, out, kind == SQ_OUT_I32,
+                          workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
+                          sq::host::spin_limit(), sq::host::num_sms());
 }
 
 sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,

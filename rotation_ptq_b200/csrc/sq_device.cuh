@@ -477,6 +477,12 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t* u) {
   return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
 }
 
+// Low bytes of four words (magic-rounded floats holding signed 8-bit codes)
+// packed into one word, first word in the low byte.
+__device__ __forceinline__ uint32_t pack4b(uint32_t u0, uint32_t u1, uint32_t u2, uint32_t u3) {
+  return __byte_perm(__byte_perm(u0, u1, 0x0040), __byte_perm(u2, u3, 0x0040), 0x5410);
+}
+
 // ------------------------------------------------------------- named bars
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

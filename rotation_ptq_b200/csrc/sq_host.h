@@ -49,6 +49,10 @@ bool eligible(int64_t M, int64_t K);
 sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
               int64_t M, int64_t N, int64_t K, void* out, int out_i32, int num_sms,
               uint32_t spin_limit, cudaStream_t stream);
+// The same with byte activations [M][K] (W4A8).
+sq_status run_a8(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                 const float* w_scale, int64_t M, int64_t N, int64_t K, void* out, int out_i32,
+                 int num_sms, cudaStream_t stream);
 }  // namespace gemv
 
 namespace gemm {
@@ -56,13 +60,21 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
               int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
               size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
               const Plan* forced);
-
+// W4A8: byte activations [M][K] x packed INT4 weights.
+sq_status run_a8(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                 const float* w_scale, int64_t M, int64_t N, int64_t K, void* out, int out_i32,
+                 void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit,
+                 int num_sms);
 }  // namespace gemm
 
 namespace rq {
 sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
               const int8_t* had_small, int n_small, int n_pow2, float clip, uint8_t* a_q,
               float* a_scale, cudaStream_t stream);
+// As run() with one signed byte per code (W4A8): a_q is [M][K].
+sq_status run8(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
+               const int8_t* had_small, int n_small, int n_pow2, float clip, int8_t* a_q,
+               float* a_scale, cudaStream_t stream);
 // SwiGLU of gate_up[m][0, K) and gate_up[m][K, 2K) (bf16, row stride ld),
 // rounded to bf16, then as run().
 sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,

@@ -834,11 +834,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // which, holding only B, can be twice as deep.  Tensor memory: one 256-column
 // int32 accumulator and eight 32-column A slots.
 
-template <int PST, int UST>
+// A8: the A operand arrives as signed bytes (W4A8): KM k-tiles of 128 bytes
+// per row in the stage (one TMA box each) instead of packed nibbles.
+template <int PST, int UST, bool A8 = false>
 struct PairTSLayout {
   static constexpr int HALF = 128;
-  static constexpr int PA = HALF * PROW;              // packed A (KM k-tiles)
-  static constexpr int PSTAGE = 2 * HALF * PROW;      // packed A + packed B
+  static constexpr int PA = HALF * PROW * (A8 ? 2 : 1);   // A of KM k-tiles
+  static constexpr int PSTAGE = PA + HALF * PROW;      // A + packed B
   static constexpr int UB = HALF * BK;                // int8 B per k-tile
   static constexpr int U_OFF = 0;
   static constexpr int P_OFF = UST * UB;
@@ -855,11 +857,14 @@ struct PairTSLayout {
   static_assert(P_OFF % 1024 == 0 && PSTAGE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
 
-template <int PST, int UST>
+template <int PST, int UST, bool A8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_pair_ts_kernel(const __grid_constant__ CUtensorMap mapA,
                              const __grid_constant__ CUtensorMap mapB, const PairParams p) {
-  using L = PairTSLayout<PST, UST>;
+  using L = PairTSLayout<PST, UST, A8>;
+  // every product is 256 x the true one (both operands widened x16), or 16 x
+  // with byte activations
+  constexpr int ACC_SHIFT = A8 ? 4 : 8;
   // int8 slots change hands in groups of KM k-tiles (one packed stage): one
   // barrier wait and one tensor-core commit per group rather than per k-tile
   constexpr int G = UST / KM;
@@ -928,7 +933,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t* dst = smem + L::P_OFF + ps * L::PSTAGE;
           mbar_arrive_expect_tx(&pfull[ps], L::PSTAGE);
-          tma_load_2d(dst, &mapA, kt * KP, tm * 256 + rank * L::HALF, &pfull[ps]);
+          if (A8) {
+#pragma unroll
+            for (int sub = 0; sub < KM; ++sub)
+              tma_load_2d(dst + sub * L::HALF * BK, &mapA, (kt + sub) * BK,
+                          tm * 256 + rank * L::HALF, &pfull[ps]);
+          } else {
+            tma_load_2d(dst, &mapA, kt * KP, tm * 256 + rank * L::HALF, &pfull[ps]);
+          }
           tma_load_2d(dst + L::PA, &mapB, kt * KP, tn * 256 + rank * L::HALF, &pfull[ps]);
         }
       }
@@ -989,18 +1001,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (sub < nsub) {
             const int slot = g * KM + sub;
             uint32_t w[16];
+            if (A8) {
+              // byte codes: each group of 8 goes in as its even codes, then
+              // its odd codes, the K order of the widened weights
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int c = (sub * 4 + 2 * half + j) ^ (a_row & 7);
-              const uint4 v = lds128(psrc + a_src + (c << 4));
-              w[8 * j + 0] = (v.x << 4) & m;
-              w[8 * j + 1] = v.x & m;
-              w[8 * j + 2] = (v.y << 4) & m;
-              w[8 * j + 3] = v.y & m;
-              w[8 * j + 4] = (v.z << 4) & m;
-              w[8 * j + 5] = v.z & m;
-              w[8 * j + 6] = (v.w << 4) & m;
-              w[8 * j + 7] = v.w & m;
+              for (int j = 0; j < 2; ++j) {
+                const uint32_t row_base = psrc + sub * L::HALF * BK + a_row * BK;
+                const uint4 v0 = lds128(row_base + (((4 * half + 2 * j) ^ (a_row & 7)) << 4));
+                const uint4 v1 = lds128(row_base + (((4 * half + 2 * j + 1) ^ (a_row & 7)) << 4));
+                const uint32_t b8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  w[8 * j + 2 * i] = __byte_perm(b8[2 * i], b8[2 * i + 1], 0x6420);
+                  w[8 * j + 2 * i + 1] = __byte_perm(b8[2 * i], b8[2 * i + 1], 0x7531);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const int c = (sub * 4 + 2 * half + j) ^ (a_row & 7);
+                const uint4 v = lds128(psrc + a_src + (c << 4));
+                w[8 * j + 0] = (v.x << 4) & m;
+                w[8 * j + 1] = v.x & m;
+                w[8 * j + 2] = (v.y << 4) & m;
+                w[8 * j + 3] = v.y & m;
+                w[8 * j + 4] = (v.z << 4) & m;
+                w[8 * j + 5] = v.z & m;
+                w[8 * j + 6] = (v.w << 4) & m;
+                w[8 * j + 7] = v.w & m;
+              }
             }
             tmem_st16(a_lane + static_cast<uint32_t>(slot * 32), w);
             const uint32_t udst = smem_base + L::U_OFF + slot * L::UB;
@@ -1181,7 +1210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int g = 0; g < 4; ++g)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v4[g][j] = static_cast<int>(vv[g][j]) >> 8;
+          for (int j = 0; j < 16; ++j) v4[g][j] = static_cast<int>(vv[g][j]) >> ACC_SHIFT;
         if (wcol != nullptr) {
           int* wc = wcol + c4 * 16 * 256;
           if (!last) {
@@ -1252,12 +1281,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ------------------------------------------------------------------ host side
 
+// Rows of `row_bytes` (K / 2 packed nibbles by default, or K signed bytes),
+// boxes of 128 bytes x box_rows, 128-byte swizzle.
 static bool make_map(CUtensorMap* map, const uint8_t* base, int rows, int64_t K,
-                     int box_rows) {
+                     int box_rows, int64_t row_bytes = -1) {
   auto encode = host::tensor_map_encoder();
   if (!encode) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  if (row_bytes < 0) row_bytes = K / 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(PROW), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
@@ -1305,21 +1337,22 @@ static size_t tail_ws_bytes(int tail, int parts) {
          ((static_cast<size_t>(tail) * 4 * 4 + 255) & ~static_cast<size_t>(255));
 }
 
-template <bool TS, int PST, int UST>
+template <bool TS, int PST, int UST, bool A8 = false>
 static sq_status launch_pair(const uint8_t* a_q, const uint8_t* w_q, int64_t M, int64_t N,
                              int64_t K, PairParams prm, int num_sms, cudaStream_t stream,
                              void* ws, size_t ws_bytes) {
+  static_assert(TS || !A8, "byte activations use the tensor-memory kernel");
   constexpr int BYTES = [] {
-    if constexpr (TS) return PairTSLayout<PST, UST>::BYTES;
+    if constexpr (TS) return PairTSLayout<PST, UST, A8>::BYTES;
     else return PairLayout<PST, UST>::BYTES;
   }();
   constexpr int HALF = 128;
   CUtensorMap mapA, mapB;
-  if (!make_map(&mapA, a_q, static_cast<int>(M), K, HALF) ||
+  if (!make_map(&mapA, a_q, static_cast<int>(M), K, HALF, A8 ? K : -1) ||
       !make_map(&mapB, w_q, static_cast<int>(N), K, HALF))
     return SQ_ERR_CUDA;
   auto kfn = [] {
-    if constexpr (TS) return w4a4_gemm_pair_ts_kernel<PST, UST>;
+    if constexpr (TS) return w4a4_gemm_pair_ts_kernel<PST, UST, A8>;
     else return w4a4_gemm_pair_kernel<PST, UST>;
   }();
   static int max_clusters[64] = {0};
@@ -1462,6 +1495,33 @@ size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   const size_t acc = static_cast<size_t>(M) * static_cast<size_t>(N) * 4;
   const size_t cnt = static_cast<size_t>(pl.tilesA) * pl.tilesB * 4;
   return ((acc + 255) & ~static_cast<size_t>(255)) + ((cnt + 255) & ~static_cast<size_t>(255));
+}
+
+// W4A8: byte activations.  Decode sizes run on the GEMV, everything else on
+// the CTA-pair kernel with A in tensor memory (its epilogue masks ragged M
+// and N, so it serves every shape, if not at its best below M = 256).
+sq_status run_a8(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                 const float* w_scale, int64_t M, int64_t N, int64_t K, void* out, int out_i32,
+                 void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit,
+                 int num_sms) {
+  if (gemv::eligible(M, K))
+    return gemv::run_a8(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32, num_sms, stream);
+  PairParams pp{};
+  pp.rowsA = static_cast<int>(M);
+  pp.rowsB = static_cast<int>(N);
+  pp.tilesM = static_cast<int>((M + 255) / 256);
+  pp.tilesN = static_cast<int>((N + 255) / 256);
+  pp.KT = static_cast<int>(K / BK);
+  pp.units = pp.tilesM * pp.tilesN;
+  pp.a_scale = a_scale;
+  pp.w_scale = w_scale;
+  pp.out = out;
+  pp.out_i32 = out_i32;
+  pp.M = static_cast<int>(M);
+  pp.N = static_cast<int>(N);
+  pp.spin_limit = spin_limit;
+  return launch_pair<true, 3, 4, true>(reinterpret_cast<const uint8_t*>(a_q), w_q, M, N, K, pp,
+                                       num_sms, stream, ws, ws_bytes);
 }
 
 sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,

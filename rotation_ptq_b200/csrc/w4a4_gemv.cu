@@ -40,7 +40,10 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // NW: warps per CTA.  CPL: 16-byte weight chunks per lane per row and pass (a
 // pass covers 32 * CPL chunks of each row).  R: rows a warp works on at once,
 // so that short rows still keep R * CPL loads per lane in flight.
-template <int MT, int NW, int CPL, int R>
+// A8: the activations are signed bytes [M][K] (W4A8); each group of 8 goes
+// into the even-code and odd-code words as its even and odd bytes, the
+// products are then 16 x the true ones.
+template <int MT, int NW, int CPL, int R, bool A8 = false>
 __global__ void __launch_bounds__(NW * 32) w4a4_gemv_kernel(
     const uint8_t* __restrict__ a_q, const float* __restrict__ a_scale,
     const uint8_t* __restrict__ w_q, const float* __restrict__ w_scale, int M, int N, int K,
@@ -71,6 +74,24 @@ __global__ void __launch_bounds__(NW * 32) w4a4_gemv_kernel(
 
   for (int i = threadIdx.x; i < MT * nchunk; i += blockDim.x) {
     const int m = i / nchunk, c = i - m * nchunk;
+    if (A8) {
+      uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+      if (m < M) {
+        const uint4* src = reinterpret_cast<const uint4*>(a_q + static_cast<int64_t>(m) * K) + 2 * c;
+        v0 = __ldg(src);
+        v1 = __ldg(src + 1);
+      }
+      const uint32_t b8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint32_t ev[4], od[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        ev[g] = __byte_perm(b8[2 * g], b8[2 * g + 1], 0x6420);
+        od[g] = __byte_perm(b8[2 * g], b8[2 * g + 1], 0x7531);
+      }
+      a_words[(2 * m) * nchunk + c] = make_uint4(ev[0], ev[1], ev[2], ev[3]);
+      a_words[(2 * m + 1) * nchunk + c] = make_uint4(od[0], od[1], od[2], od[3]);
+      continue;
+    }
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (m < M) v = __ldg(reinterpret_cast<const uint4*>(a_q + static_cast<int64_t>(m) * (K / 2)) + c);
     a_words[(2 * m) * nchunk + c] =
@@ -138,7 +159,7 @@ __global__ void __launch_bounds__(NW * 32) w4a4_gemv_kernel(
       for (int m = 0; m < MT; ++m) {
         const int n = n0 + r;
         if (lane == r * MT + m && m < M && n < N) {
-          const int sum = acc[r][m] >> 8;        // exact: every product is 256 x the true one
+          const int sum = acc[r][m] >> (A8 ? 4 : 8);   // exact: products are 256 (16) x the true ones
           const int64_t o = static_cast<int64_t>(m) * N + n;
           if (out_i32) {
             static_cast<int*>(out)[o] = sum;
@@ -159,12 +180,12 @@ bool eligible(int64_t M, int64_t K) {
   return mt * K <= MAX_SMEM;                   // widened codes: MT * K bytes
 }
 
-template <int MT, int NW, int CPL, int R>
+template <int MT, int NW, int CPL, int R, bool A8>
 static sq_status launch(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
                         const float* w_scale, int M, int N, int K, void* out, int out_i32,
                         int num_sms, cudaStream_t stream) {
   static_assert(R * MT <= 32, "one lane per output");
-  auto kfn = w4a4_gemv_kernel<MT, NW, CPL, R>;
+  auto kfn = w4a4_gemv_kernel<MT, NW, CPL, R, A8>;
   const int smem = MT * K;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(gemv)", e);
@@ -182,14 +203,16 @@ static sq_status launch(const uint8_t* a_q, const float* a_scale, const uint8_t*
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("w4a4_gemv launch", e);
 }
 
-sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
-              int64_t M, int64_t N, int64_t K, void* out, int out_i32, int num_sms,
-              uint32_t /*spin_limit: the GEMV has no waits*/, cudaStream_t stream) {
+template <bool A8>
+static sq_status run_t(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                       const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
+                       int out_i32, int num_sms, cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   // rows of at most 4 chunks per lane (K <= 4096) go several to a warp
   const bool short_rows = K <= 4096;
 #define SQ_GEMV(MT, NW, CPL, R) \
-  return launch<MT, NW, CPL, R>(a_q, a_scale, w_q, w_scale, m, n, k, out, out_i32, num_sms, stream)
+  return launch<MT, NW, CPL, R, A8>(a_q, a_scale, w_q, w_scale, m, n, k, out, out_i32, num_sms, \
+                                    stream)
   if (M <= 1) {
     if (short_rows) SQ_GEMV(1, 8, 4, 3);
     SQ_GEMV(1, 16, 12, 1);
@@ -205,6 +228,19 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
   if (short_rows) SQ_GEMV(8, 8, 4, 1);
   SQ_GEMV(8, 8, 8, 1);
 #undef SQ_GEMV
+}
+
+sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
+              int64_t M, int64_t N, int64_t K, void* out, int out_i32, int num_sms,
+              uint32_t /*spin_limit: the GEMV has no waits*/, cudaStream_t stream) {
+  return run_t<false>(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32, num_sms, stream);
+}
+
+sq_status run_a8(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
+                 const float* w_scale, int64_t M, int64_t N, int64_t K, void* out, int out_i32,
+                 int num_sms, cudaStream_t stream) {
+  return run_t<true>(reinterpret_cast<const uint8_t*>(a_q), a_scale, w_q, w_scale, M, N, K, out,
+                     out_i32, num_sms, stream);
 }
 
 }  // namespace gemv

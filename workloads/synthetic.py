@@ -232,6 +232,11 @@ def random_packed(seed: int, rows: int, K: int) -> np.ndarray:
     return rng.integers(0, 256, size=(rows, K // 2), dtype=np.int64).astype(np.uint8)
 
 
+def random_int8(seed: int, rows: int, K: int) -> np.ndarray:
+    """Uniform signed byte codes [rows, K] (8-bit activations for the W4A8 GEMM)."""
+    return np.random.default_rng(seed).integers(-128, 128, (rows, K)).astype(np.int8)
+
+
 def random_scales(seed: int, n: int) -> np.ndarray:
     """Positive float32 scales spread over two decades (GEMM epilogue test input)."""
     rng = np.random.default_rng(seed)
