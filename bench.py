@@ -363,7 +363,8 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
 
 
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
-                 "decode_gemm_m1", "decode_gemm_m16", "rotate_quant_r4", "kv_rotate_quant",
+                 "decode_gemm_m1", "decode_gemm_m16", "decode_gemm_m64", "rotate_quant_r4",
+                 "kv_rotate_quant",
                  "swiglu_rotate_quant_r4", "kv4_decode")
 
 
@@ -374,7 +375,7 @@ def run_profile_case(case, steps, warmup):
     from workloads import synthetic as W
     torch.cuda.set_device(0)
     if case.startswith("down_proj_gemm") or case.startswith("decode_gemm"):
-        m = {"decode_gemm_m1": 1, "decode_gemm_m16": 16}.get(case, M)
+        m = {"decode_gemm_m1": 1, "decode_gemm_m16": 16, "decode_gemm_m64": 64}.get(case, M)
         a = torch.from_numpy(W.random_packed(11, m, K)).cuda()
         w = torch.from_numpy(W.random_packed(12, N, K)).cuda()
         sa = torch.from_numpy(W.random_scales(13, m)).cuda()

@@ -391,6 +391,46 @@ def kv_rotate_quant(q, k, v, pos, cos, sin):
                 v_cache=pack_int4(vc), v_codes=vc, v_scale=vs, v_zero=vz, v_v=vv_)
 
 
+def quant_asym_uint8(x: np.ndarray):
+    """Asymmetric 8-bit quantizer over the last axis (the KV8 of W4A8KV8,
+    "SpinQuant, Reproduced", Q7), decisions in float32.
+
+    The 4-bit rule on the 8-bit grid: lo = min(min x, 0), hi = max(max x, 0);
+    scale = (hi - lo) / 255 (1 if 0); zero = clamp(rint(-lo / scale), 0, 255);
+    code = clamp(rint(x / scale) + zero, 0, 255).
+    Returns (codes uint8 [..., d], scale f32 [...], zero uint8 [...], v f32 = x/scale).
+    """
+    x = np.asarray(x, dtype=F32)
+    lo = np.minimum(np.min(x, axis=-1), F32(0))
+    hi = np.maximum(np.max(x, axis=-1), F32(0))
+    scale = ((hi - lo) / F32(255.0)).astype(F32)
+    scale = np.where(scale == 0, F32(1.0), scale).astype(F32)
+    zero = np.clip(np.rint((-lo) / scale), 0, 255).astype(F32)
+    v = (x / scale[..., None]).astype(F32)
+    codes = np.clip(np.rint(v) + zero[..., None], 0, 255).astype(np.uint8)
+    return codes, scale, zero.astype(np.uint8), v
+
+
+def kv_rotate_quant8(q, k, v, pos, cos, sin):
+    """kv_rotate_quant with 8-bit caches: one byte per code, [T, h, d]."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    if cos is not None:
+        q = rope(q, pos, cos, sin)
+        k = rope(k, pos, cos, sin)
+    q_rot = headwise_hadamard(q).astype(F32)
+    k_rot = headwise_hadamard(k).astype(F32)
+    kc, ks, kz, kv_ = quant_asym_uint8(k_rot)
+    vc, vs, vz, vv_ = quant_asym_uint8(np.asarray(v, F32))
+    return dict(q_rot=q_rot, k_rot=k_rot, k_cache=kc, k_codes=kc, k_scale=ks, k_zero=kz,
+                k_v=kv_, v_cache=vc, v_codes=vc, v_scale=vs, v_zero=vz, v_v=vv_)
+
+
+def kv8_dequant(cache: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
+    """Read-back of an 8-bit asymmetric cache to float64 values."""
+    return dequant_asym(np.asarray(cache), scale, zero)
+
+
 def kv_dequant(cache: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
     """Read-back of a packed asymmetric cache to float64 values."""
     return dequant_asym(unpack_int4(cache, signed=False), scale, zero)

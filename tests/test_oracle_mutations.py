@@ -179,10 +179,26 @@ def _quant8_round_half_up(y, clip=1.0):
     return np.clip(np.floor(v + F32(0.5)), -128, 127).astype(np.int8), s, v
 
 
+def _asym8_div256(x):
+    x = np.asarray(x, F32)
+    lo = np.minimum(np.min(x, -1), F32(0))
+    hi = np.maximum(np.max(x, -1), F32(0))
+    s = ((hi - lo) / F32(256)).astype(F32)
+    s = np.where(s == 0, F32(1), s).astype(F32)
+    z = np.clip(np.rint(-lo / s), 0, 255).astype(F32)
+    vv = (x / s[..., None]).astype(F32)
+    return np.clip(np.rint(vv) + z[..., None], 0, 255).astype(np.uint8), s, z.astype(np.uint8), vv
+
+
+def _asym8_clamp_15(x):
+    c, s, z, vv = _orig["quant_asym_uint8"](x)
+    return np.minimum(c, 15).astype(np.uint8), s, z, vv
+
+
 _orig = {name: getattr(O, name) for name in
          ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
           "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16",
-          "decode_attention", "quant_sym_int8"]}
+          "decode_attention", "quant_sym_int8", "quant_asym_uint8"]}
 
 MUTATIONS = {
     "paley_transposed": ("paley1", _transposed_paley),
@@ -209,6 +225,8 @@ MUTATIONS = {
     "quant8_divisor_128": ("quant_sym_int8", _quant8_div128),
     "quant8_clamps_at_minus_127": ("quant_sym_int8", _quant8_symmetric_clamp),
     "quant8_round_half_up": ("quant_sym_int8", _quant8_round_half_up),
+    "asym8_divisor_256": ("quant_asym_uint8", _asym8_div256),
+    "asym8_4bit_clamp": ("quant_asym_uint8", _asym8_clamp_15),
 }
 
 PIN_TESTS = [
@@ -245,6 +263,8 @@ PIN_TESTS = [
     P.test_quant8_divisor_bound_and_special_rows,
     P.test_w4a8_linear_bruteforce,
     P.test_rotate_quant8_is_rotation_then_quant8,
+    P.test_asym8_bruteforce_and_bounds,
+    P.test_asym8_constant_and_zero_rows,
 ]
 
 

@@ -512,6 +512,56 @@ def test_rotate_quant8_is_rotation_then_quant8():
 
 
 # --------------------------------------------------------------------------
+# KV8: the 8-bit asymmetric cache
+# --------------------------------------------------------------------------
+
+def test_asym8_bruteforce_and_bounds():
+    rng = np.random.default_rng(101)
+    x = (rng.standard_normal((40, 128)) * rng.uniform(0.1, 5, (40, 1))).astype(np.float32)
+    x[3] = np.abs(x[3])                          # all positive: lo = 0, zero = 0
+    x[4] = -np.abs(x[4])                         # all negative: hi = 0, zero = 255
+    codes, s, z, v = O.quant_asym_uint8(x)
+    lo = np.minimum(x.min(-1), 0)
+    hi = np.maximum(x.max(-1), 0)
+    assert np.allclose(s, (hi - lo) / 255, rtol=1e-6)
+    assert z[3] == 0 and z[4] == 255
+    xh = O.kv8_dequant(codes, s, z)
+    inner = (codes > 0) & (codes < 255)
+    rows = np.nonzero(inner)[0]
+    assert np.all(np.abs(x - xh)[inner] <= s[rows] / 2 * (1 + 1e-5) + 1e-12)
+    assert np.all(np.abs(x - xh) <= s[:, None] * (1 + 1e-5))
+    # each code is the nearest grid point rint(x / s) + z (ties to even), clamped
+    for r in range(6):
+        for k in range(0, 128, 17):
+            want = min(max(int(np.rint(np.float32(x[r, k] / s[r]))) + int(z[r]), 0), 255)
+            assert codes[r, k] == want
+
+
+def test_asym8_constant_and_zero_rows():
+    c = np.full((1, 8), 2.0, np.float32)
+    codes, s, z, _ = O.quant_asym_uint8(c)
+    assert np.isclose(s[0], 2.0 / 255) and z[0] == 0 and np.all(codes == 255)
+    codes, s, z, _ = O.quant_asym_uint8(np.zeros((1, 8), np.float32))
+    assert s[0] == 1.0 and z[0] == 0 and np.all(codes == 0)
+
+
+def test_kv8_composition_uses_rope_and_r3():
+    rng = np.random.default_rng(102)
+    T, hq, hkv, d = 3, 2, 1, 128
+    q = rng.standard_normal((T, hq, d)); k = rng.standard_normal((T, hkv, d))
+    v = rng.standard_normal((T, hkv, d)).astype(np.float32)
+    pos = np.array([0, 5, 9]); cos, sin = O.rope_tables(1e6, 16, d)
+    r8 = O.kv_rotate_quant8(q, k, v, pos, cos, sin)
+    r4 = O.kv_rotate_quant(q, k, v, pos, cos, sin)
+    # the same rotated K and Q as the 4-bit path; only the grid differs
+    assert np.array_equal(r8["k_rot"], r4["k_rot"]) and np.array_equal(r8["q_rot"], r4["q_rot"])
+    kh8 = O.kv8_dequant(r8["k_cache"], r8["k_scale"], r8["k_zero"])
+    kh4 = O.kv_dequant(r4["k_cache"], r4["k_scale"], r4["k_zero"])
+    e8, e4 = np.abs(kh8 - r8["k_rot"]).max(), np.abs(kh4 - r4["k_rot"]).max()
+    assert e8 < e4 / 8                           # 17x finer grid
+
+
+# --------------------------------------------------------------------------
 # SwiGLU ahead of down_proj (fused SwiGLU + R4)
 # --------------------------------------------------------------------------
 
