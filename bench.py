@@ -44,6 +44,8 @@ KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
 # ... of one decode step of sq_kv4_decode_attention (B 16 x S 4096): both
 # caches with their scales and zeros, bf16 queries in and outputs out
 DECODE_BYTES = 2 * KV_T * KV_HKV * (64 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
+# ... of sq_kv8_decode_attention: one byte per code
+DECODE8_BYTES = 2 * KV_T * KV_HKV * (128 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
@@ -238,7 +240,31 @@ def run_ours(args, rank, world, local_rank):
         kv_info = {"workload": "kv_T65536_hq32_hkv8_d128", "rotate_quant_us": mq * 1e3,
                    "rotate_quant_gbs": kv_fwd_bytes / (mq * 1e-3) / 1e9,
                    "dequant_us": md * 1e3, "dequant_gbs": kv_rb_bytes / (md * 1e-3) / 1e9}
-        del q, k, v, kvo, kdq, vdq
+        # the same tokens into 8-bit caches (W4A8KV8) and their read-back
+        kvo8 = sq.kv_rotate_quant8(q, k, v, pos, cos, sin)
+        sq.kv8_dequant(kvo8["k_cache"], kvo8["k_scale"], kvo8["k_zero"], out=kdq)
+        torch.cuda.synchronize()
+        tq, td = [], []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            sq.kv_rotate_quant8(q, k, v, pos, cos, sin, out=kvo8)
+            e1.record(stream)
+            sq.kv8_dequant(kvo8["k_cache"], kvo8["k_scale"], kvo8["k_zero"], out=kdq)
+            sq.kv8_dequant(kvo8["v_cache"], kvo8["v_scale"], kvo8["v_zero"], out=vdq)
+            e2.record(stream)
+            tq.append((e0, e1))
+            td.append((e1, e2))
+        torch.cuda.synchronize()
+        kv8_fwd_bytes = KV_T * (2 * (KV_HQ * d * 2) + 2 * (KV_HKV * d * 2) + 2 * KV_HKV * (d + 5))
+        kv8_rb_bytes = 2 * KV_T * KV_HKV * ((d + 5) + d * 2)
+        mq, md = ms(tq), ms(td)
+        kv_info["kv8"] = {"rotate_quant8_us": mq * 1e3,
+                          "rotate_quant8_gbs": kv8_fwd_bytes / (mq * 1e-3) / 1e9,
+                          "dequant8_us": md * 1e3,
+                          "dequant8_gbs": kv8_rb_bytes / (md * 1e-3) / 1e9}
+        del q, k, v, kvo, kdq, vdq, kvo8
 
     # fused SwiGLU + R4 rotate + quant on the gate_up output of the same
     # tokens (the step before down_proj), timed alone for the record
@@ -311,6 +337,26 @@ def run_ours(args, rank, world, local_rank):
         dec_info = {"workload": dw.name, "us": mde * 1e3,
                     "GB/s": dec_bytes / (mde * 1e-3) / 1e9, "bytes": dec_bytes}
         del dq, dkc, dks, dkz, dvc, dvs, dvz, dln, dout
+        # the same step over 8-bit caches
+        dw = W.kv8_decode()
+        t8 = [x.to(dev) for x in (dw.q, dw.k_cache, dw.k_scale, dw.k_zero, dw.v_cache,
+                                  dw.v_scale, dw.v_zero, dw.lengths)]
+        dout = sq.kv8_decode_attention(*t8, dw.S_max)
+        torch.cuda.synchronize()
+        tde = []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            sq.kv8_decode_attention(*t8, dw.S_max, out=dout)
+            e1.record(stream)
+            tde.append((e0, e1))
+        torch.cuda.synchronize()
+        mde = ms(tde)
+        dec_info["kv8"] = {"workload": dw.name, "us": mde * 1e3,
+                           "GB/s": DECODE8_BYTES / (mde * 1e-3) / 1e9, "bytes": DECODE8_BYTES,
+                           "frac_of_hbm": DECODE8_BYTES / (mde * 1e-3) / 1e9 / load_peaks()[0]}
+        del t8, dout
 
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
@@ -365,7 +411,7 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
                  "decode_gemm_m1", "decode_gemm_m16", "decode_gemm_m64", "rotate_quant_r4",
                  "kv_rotate_quant",
-                 "swiglu_rotate_quant_r4", "kv4_decode")
+                 "swiglu_rotate_quant_r4", "kv4_decode", "kv8_decode", "kv_rotate_quant8")
 
 
 def run_profile_case(case, steps, warmup):
@@ -401,6 +447,18 @@ def run_profile_case(case, steps, warmup):
                                 dw.v_zero, dw.lengths)]
         o = sq.kv4_decode_attention(*t, dw.S_max)
         fn = lambda: sq.kv4_decode_attention(*t, dw.S_max, out=o)  # noqa: E731
+    elif case == "kv8_decode":
+        dw = W.kv8_decode()
+        t = [x.cuda() for x in (dw.q, dw.k_cache, dw.k_scale, dw.k_zero, dw.v_cache, dw.v_scale,
+                                dw.v_zero, dw.lengths)]
+        o = sq.kv8_decode_attention(*t, dw.S_max)
+        fn = lambda: sq.kv8_decode_attention(*t, dw.S_max, out=o)  # noqa: E731
+    elif case == "kv_rotate_quant8":
+        kw = W.kv_path()
+        q, k, v, pos = kw.q.cuda(), kw.k.cuda(), kw.v.cuda(), kw.pos.cuda()
+        cos, sin = sq.rope_tables(kw.theta, kw.max_pos, 128)
+        o = sq.kv_rotate_quant8(q, k, v, pos, cos, sin)
+        fn = lambda: sq.kv_rotate_quant8(q, k, v, pos, cos, sin, out=o)  # noqa: E731
     elif case == "kv_rotate_quant":
         kvw = W.kv_path()
         q, k, v, pos = kvw.q.cuda(), kvw.k.cuda(), kvw.v.cuda(), kvw.pos.cuda()

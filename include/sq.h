@@ -293,6 +293,25 @@ sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_
 sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
                         int64_t T, int h, int d, void* out_bf16, void* stream);
 
+/* sq_kv_rotate_quant8 -- sq_kv_rotate_quant with the 8-bit asymmetric KV
+ * cache of the W4A8KV8 setting ("SpinQuant, Reproduced", Q7): the same
+ * RoPE, R3 and q_out; the caches use the same rule on the grid 0..255:
+ *     scale = (hi - lo) / 255 (1 if 0), zero = clamp(rint(-lo / scale), 0, 255),
+ *     code = clamp(rint(x / scale) + zero, 0, 255).
+ * k_cache, v_cache  device, [T][hkv][d] uint8, one code per byte.
+ * All other arguments, shape rules and errors as sq_kv_rotate_quant. */
+sq_status sq_kv_rotate_quant8(const void* q, const void* k, const void* v, int64_t T, int hq,
+                              int hkv, int d, const int32_t* pos, const float* rope_cos,
+                              const float* rope_sin, int max_pos, void* q_out,
+                              uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                              uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                              void* stream);
+
+/* sq_kv8_dequant -- sq_kv_dequant for an 8-bit cache [T][h][d] (one code per
+ * byte).  Arguments, shape rules and errors as sq_kv_dequant. */
+sq_status sq_kv8_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                         int64_t T, int h, int d, void* out_bf16, void* stream);
+
 /* sq_rope_tables -- the cos/sin tables the KV call reads:
  *     angle(p, i) = p * theta^(-2i/d),  cos[p][i] = float(cos(angle)),
  *     sin[p][i] = float(sin(angle)),  evaluated in double precision on the
@@ -354,6 +373,20 @@ void sq_debug_set_gemm_path(int path);
  * ------------------------------------------------------------------------- */
 size_t sq_kv4_decode_workspace_bytes(int64_t B, int64_t S_max, int hq, int hkv);
 sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
+                                  const uint8_t* k_zero, const uint8_t* v_cache,
+                                  const float* v_scale, const uint8_t* v_zero,
+                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
+                                  int hkv, int d, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* sq_kv8_decode_attention -- sq_kv4_decode_attention over the 8-bit caches
+ * of sq_kv_rotate_quant8 ("SpinQuant, Reproduced", Q7: W4A8KV8).
+ * k_cache, v_cache  device uint8 [B * S_max][hkv][128], one code per byte,
+ *            16-byte aligned.  The workspace is sized by
+ *            sq_kv4_decode_workspace_bytes() (the split plan does not depend
+ *            on the code width).  All other arguments, the formula, shape
+ *            rules and errors as sq_kv4_decode_attention. */
+sq_status sq_kv8_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
                                   const uint8_t* k_zero, const uint8_t* v_cache,
                                   const float* v_scale, const uint8_t* v_zero,
                                   const int32_t* lengths, int64_t B, int64_t S_max, int hq,

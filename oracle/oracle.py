@@ -475,6 +475,13 @@ def kv4_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
                             kv_dequant(v_cache, v_scale, v_zero), lengths, S_max)
 
 
+def kv8_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
+                         lengths, S_max: int) -> np.ndarray:
+    """decode_attention over the 8-bit caches' read-back (W4A8KV8)."""
+    return decode_attention(q, kv8_dequant(k_cache, k_scale, k_zero),
+                            kv8_dequant(v_cache, v_scale, v_zero), lengths, S_max)
+
+
 # ---------------------------------------------------------------------------
 # Statistics ("SpinQuant, Reproduced", Q3: kurtosis across channels within a
 # token, averaged over tokens; 3 is a Gaussian).

@@ -10,6 +10,7 @@ Entry points (same names as the C ABI without the ``sq_`` prefix):
   rotate_quant, rotate_quant8, swiglu_rotate_quant, w4a4_linear, w4a8_linear,
   w4a4_workspace_bytes, kv_rotate_quant,
   kv_dequant, kv4_decode_attention, kv4_decode_workspace_bytes, rope_tables,
+  kv_rotate_quant8, kv8_dequant, kv8_decode_attention,
   device_status, debug_set_spin_limit.
 """
 from __future__ import annotations
@@ -25,8 +26,11 @@ from .binding import (  # noqa: F401
     device_status,
     kv4_decode_attention,
     kv4_decode_workspace_bytes,
+    kv8_decode_attention,
+    kv8_dequant,
     kv_dequant,
     kv_rotate_quant,
+    kv_rotate_quant8,
     lib,
     library_path,
     quantize_weights,

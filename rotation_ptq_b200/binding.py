@@ -50,18 +50,21 @@ lib.sq_w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, 
                                ctypes.c_size_t, _vp]
 lib.sq_kv4_decode_workspace_bytes.restype = ctypes.c_size_t
 lib.sq_kv4_decode_workspace_bytes.argtypes = [_i64, _i64, _i32, _i32]
-lib.sq_kv4_decode_attention.restype = _i32
-lib.sq_kv4_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32,
-                                        _i32, _i32, _vp, _vp, ctypes.c_size_t, _vp]
+for _f in (lib.sq_kv4_decode_attention, lib.sq_kv8_decode_attention):
+    _f.restype = _i32
+    _f.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp,
+                   ctypes.c_size_t, _vp]
 lib.sq_w4a4_workspace_bytes.restype = ctypes.c_size_t
 lib.sq_w4a4_workspace_bytes.argtypes = [_i64, _i64, _i64]
 lib.sq_w4a4_tail_workspace_bytes.restype = ctypes.c_size_t
 lib.sq_w4a4_tail_workspace_bytes.argtypes = [_i64, _i64, _i64]
-lib.sq_kv_rotate_quant.restype = _i32
-lib.sq_kv_rotate_quant.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32,
-                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
-lib.sq_kv_dequant.restype = _i32
-lib.sq_kv_dequant.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]
+for _f in (lib.sq_kv_rotate_quant, lib.sq_kv_rotate_quant8):
+    _f.restype = _i32
+    _f.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
+                   _vp, _vp, _vp, _vp]
+for _f in (lib.sq_kv_dequant, lib.sq_kv8_dequant):
+    _f.restype = _i32
+    _f.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]
 lib.sq_rope_tables.restype = _i32
 lib.sq_rope_tables.argtypes = [ctypes.c_double, _i32, _i32, _vp, _vp, _vp]
 lib.sq_device_status.restype = _i32
@@ -281,6 +284,22 @@ def kv4_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.
     zeros uint8 [B * S_max, hkv]; lengths int32 [B].  Returns bf16 [B, hq, 128].
     Without ``workspace`` a cached zero-filled buffer of the stream is used.
     """
+    return _kv_decode(lib.sq_kv4_decode_attention, "sq_kv4_decode_attention", q, k_cache,
+                      k_scale, k_zero, v_cache, v_scale, v_zero, lengths, S_max, out, workspace)
+
+
+def kv8_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.Tensor,
+                         k_zero: torch.Tensor, v_cache: torch.Tensor, v_scale: torch.Tensor,
+                         v_zero: torch.Tensor, lengths: torch.Tensor, S_max: int,
+                         out: torch.Tensor = None, workspace: torch.Tensor = None):
+    """kv4_decode_attention over 8-bit caches uint8 [B * S_max, hkv, 128]
+    (``sq_kv8_decode_attention``)."""
+    return _kv_decode(lib.sq_kv8_decode_attention, "sq_kv8_decode_attention", q, k_cache,
+                      k_scale, k_zero, v_cache, v_scale, v_zero, lengths, S_max, out, workspace)
+
+
+def _kv_decode(fn, name, q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, S_max,
+               out, workspace):
     _need_cuda(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths)
     B, hq, d = q.shape
     hkv = k_scale.shape[1]
@@ -297,11 +316,10 @@ def kv4_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.
         workspace = _workspace(q.device, stream, need)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib.sq_kv4_decode_attention(q.data_ptr(), k_cache.data_ptr(), k_scale.data_ptr(),
-                                     k_zero.data_ptr(), v_cache.data_ptr(), v_scale.data_ptr(),
-                                     v_zero.data_ptr(), lengths.data_ptr(), B, S_max, hq, hkv, d,
-                                     out.data_ptr(), ws_ptr, ws_bytes, stream)
-    _check(st, "sq_kv4_decode_attention")
+    st = fn(q.data_ptr(), k_cache.data_ptr(), k_scale.data_ptr(), k_zero.data_ptr(),
+            v_cache.data_ptr(), v_scale.data_ptr(), v_zero.data_ptr(), lengths.data_ptr(), B, S_max,
+            hq, hkv, d, out.data_ptr(), ws_ptr, ws_bytes, stream)
+    _check(st, name)
     return out
 
 
@@ -354,6 +372,18 @@ def kv_rotate_quant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torc
     q [T, hq, 128], k/v [T, hkv, 128] bf16; pos [T] int32.  Returns a dict with
     q_out, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero.
     """
+    return _kv_rotate_quant(lib.sq_kv_rotate_quant, "sq_kv_rotate_quant", 2, q, k, v, pos, cos,
+                            sin, out)
+
+
+def kv_rotate_quant8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+                     cos: torch.Tensor = None, sin: torch.Tensor = None, out=None):
+    """kv_rotate_quant with 8-bit caches [T, hkv, 128] (``sq_kv_rotate_quant8``)."""
+    return _kv_rotate_quant(lib.sq_kv_rotate_quant8, "sq_kv_rotate_quant8", 1, q, k, v, pos, cos,
+                            sin, out)
+
+
+def _kv_rotate_quant(fn, name, per_byte, q, k, v, pos, cos, sin, out):
     _need_cuda(q, k, v, pos, cos, sin)
     T, hq, d = q.shape
     hkv = k.shape[1]
@@ -361,20 +391,18 @@ def kv_rotate_quant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torc
     if out is None:
         out = dict(
             q_out=torch.empty_like(q),
-            k_cache=torch.empty((T, hkv, d // 2), dtype=torch.uint8, device=dev),
+            k_cache=torch.empty((T, hkv, d // per_byte), dtype=torch.uint8, device=dev),
             k_scale=torch.empty((T, hkv), dtype=torch.float32, device=dev),
             k_zero=torch.empty((T, hkv), dtype=torch.uint8, device=dev),
-            v_cache=torch.empty((T, hkv, d // 2), dtype=torch.uint8, device=dev),
+            v_cache=torch.empty((T, hkv, d // per_byte), dtype=torch.uint8, device=dev),
             v_scale=torch.empty((T, hkv), dtype=torch.float32, device=dev),
             v_zero=torch.empty((T, hkv), dtype=torch.uint8, device=dev))
     max_pos = cos.shape[0] if cos is not None else 0
-    st = lib.sq_kv_rotate_quant(q.data_ptr(), k.data_ptr(), v.data_ptr(), T, hq, hkv, d,
-                                pos.data_ptr(), _ptr(cos), _ptr(sin), max_pos,
-                                out["q_out"].data_ptr(), out["k_cache"].data_ptr(),
-                                out["k_scale"].data_ptr(), out["k_zero"].data_ptr(),
-                                out["v_cache"].data_ptr(), out["v_scale"].data_ptr(),
-                                out["v_zero"].data_ptr(), _stream(q))
-    _check(st, "sq_kv_rotate_quant")
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), T, hq, hkv, d, pos.data_ptr(), _ptr(cos),
+            _ptr(sin), max_pos, out["q_out"].data_ptr(), out["k_cache"].data_ptr(),
+            out["k_scale"].data_ptr(), out["k_zero"].data_ptr(), out["v_cache"].data_ptr(),
+            out["v_scale"].data_ptr(), out["v_zero"].data_ptr(), _stream(q))
+    _check(st, name)
     return out
 
 
@@ -387,6 +415,18 @@ def kv_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out
     st = lib.sq_kv_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, 2 * dh,
                            out.data_ptr(), _stream(cache))
     _check(st, "sq_kv_dequant")
+    return out
+
+
+def kv8_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out=None):
+    """8-bit asymmetric cache [T, h, 128] -> bf16 [T, h, 128] (``sq_kv8_dequant``)."""
+    _need_cuda(cache, scale, zero)
+    T, h, d = cache.shape
+    if out is None:
+        out = torch.empty((T, h, d), dtype=torch.bfloat16, device=cache.device)
+    st = lib.sq_kv8_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, d,
+                            out.data_ptr(), _stream(cache))
+    _check(st, "sq_kv8_dequant")
     return out
 
 

@@ -1,10 +1,13 @@
 // R3 KV path, sm_100a: RoPE, head-wise Hadamard on Q and K, asymmetric
-// 4-bit K/V cache, and the cache read-back.
+// 4-bit (or 8-bit) K/V cache, and the cache read-back.
 //
 // "SpinQuant, Reproduced", Q5: R3 is a head-wise Hadamard in the KV path that
 // sits after RoPE, so it cannot be folded and runs online; R2 on the value
 // path is folded offline, so V is only quantized.  SpinQuant abstract: the KV
-// cache is 4-bit.
+// cache is 4-bit; "SpinQuant, Reproduced", Q7: the W4A8KV8 setting keeps it at
+// 8 bits, the same asymmetric rule on the grid 0..255.  Caches are [T][h][64]
+// bytes of packed nibbles (element 2j in the low nibble of byte j) at 4 bits,
+// [T][h][128] bytes at 8.
 //
 // Thread layout (rotate/quant): a CTA takes two tokens per iteration; each
 // head vector of 128 values is owned by 2 adjacent lanes.  Items are ordered
@@ -18,7 +21,7 @@
 // Quantization follows the pinned asymmetric rule, with one division per
 // group for the scale and the zero point.  V codes use the exactly rounded
 // quotient x / scale (raw bf16 inputs meet exact .5 ties often); K codes are
-// clamp(rint(x * k + zero), 0, 15) with k = norm / scale in float32, K being
+// clamp(rint(x * k + zero), 0, top) with k = norm / scale in float32, K being
 // rotated without the 1/sqrt(128) factor (its float32 rotation already
 // differs from the exact one in the last bits, so the codes can differ from
 // the oracle's only at a rounding tie); K's scale and zero point come from
@@ -65,45 +68,63 @@ __device__ __forceinline__ void store16_bf16(__nv_bfloat16* p, const float* v) {
 }
 
 // Asymmetric parameters of a group from its (normalised) extremes, with the
-// group's other lane: scale = (max' - min') / 15, zero = rint(-min' / scale).
+// group's other lane: scale = (max' - min') / (2^BITS - 1),
+// zero = rint(-min' / scale).
+template <int BITS>
 __device__ __forceinline__ void asym_params2(float lo, float hi, unsigned pmask, float& scale,
                                              float& zero) {
+  const float top = static_cast<float>((1 << BITS) - 1);
   lo = fminf(lo, __shfl_xor_sync(pmask, lo, 1));
   hi = fmaxf(hi, __shfl_xor_sync(pmask, hi, 1));
   lo = fminf(lo, 0.f);
   hi = fmaxf(hi, 0.f);
-  scale = __fdiv_rn(hi - lo, 15.0f);
+  scale = __fdiv_rn(hi - lo, top);
   if (scale == 0.f) scale = 1.0f;
-  zero = fminf(fmaxf(rintf(__fdiv_rn(-lo, scale)), 0.f), 15.f);
+  zero = fminf(fmaxf(rintf(__fdiv_rn(-lo, scale)), 0.f), top);
 }
 
-// 8 unsigned codes clamp(rint(x k + zero), 0, 15) packed into one word (even
-// element in the low nibble); x given as 4 float pairs.  For operands whose
-// quotient by the scale must round exactly as float32 division does (raw
-// bf16 values meet exact .5 ties often), see ucodes8_div.
-__device__ __forceinline__ uint32_t ucodes8(const f2* x, f2 k2, f2 z2) {
+// Magic-rounded codes (low mantissa bits hold the code) of 8 elements into
+// BITS / 4 words: nibbles at 4 bits, bytes at 8, first element lowest.
+template <int BITS>
+__device__ __forceinline__ void pack_codes(const uint32_t (&u)[8], uint32_t* out) {
+  if (BITS == 4) {
+    out[0] = pack8(u);
+  } else {
+    out[0] = pack4b(u[0], u[1], u[2], u[3]);
+    out[1] = pack4b(u[4], u[5], u[6], u[7]);
+  }
+}
+
+// 8 unsigned codes clamp(rint(x k + zero), 0, 2^BITS - 1), packed; x given
+// as 4 float pairs.  For operands whose quotient by the scale must round
+// exactly as float32 division does (raw bf16 values meet exact .5 ties
+// often), see ucodes8_div.
+template <int BITS>
+__device__ __forceinline__ void ucodes8(const f2* x, f2 k2, f2 z2, uint32_t* out) {
   const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
+  const float top = static_cast<float>((1 << BITS) - 1);
   uint32_t u[8];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     f2 c = fma2(x[e], k2, z2);
-    c.x = fminf(fmaxf(c.x, 0.f), 15.f);
-    c.y = fminf(fmaxf(c.y, 0.f), 15.f);
+    c.x = fminf(fmaxf(c.x, 0.f), top);
+    c.y = fminf(fmaxf(c.y, 0.f), top);
     c = add2(c, magic);
     u[2 * e] = __float_as_uint(c.x);
     u[2 * e + 1] = __float_as_uint(c.y);
   }
-  return pack8(u);
+  pack_codes<BITS>(u, out);
 }
 
 // As ucodes8 with the quotient x / scale rounded exactly like IEEE float32
 // division: q = x r, e = x - q s, q' = q + e r with r = RN(1 / s), the
 // one-step fma correction of Markstein ("IA-64 and Elementary Functions",
 // 2000), which yields the correctly rounded quotient when r is the correctly
-// rounded reciprocal.  Then rint(q') + zero, clamped to [0, 15].
-__device__ __forceinline__ uint32_t ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2 z2) {
+// rounded reciprocal.  Then rint(q') + zero, clamped to [0, 2^BITS - 1].
+template <int BITS>
+__device__ __forceinline__ void ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2 z2, uint32_t* out) {
   const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
-  const float lo = 12582912.f, hi = 12582912.f + 15.f;
+  const float lo = 12582912.f, hi = 12582912.f + static_cast<float>((1 << BITS) - 1);
   uint32_t u[8];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -115,10 +136,10 @@ __device__ __forceinline__ uint32_t ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2
     u[2 * e] = __float_as_uint(c.x);
     u[2 * e + 1] = __float_as_uint(c.y);
   }
-  return pack8(u);
+  pack_codes<BITS>(u, out);
 }
 
-template <bool ROPE>
+template <bool ROPE, int BITS>
 __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int T, int hq, int hkv,
@@ -126,6 +147,7 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
     const float* __restrict__ rsin, int max_pos, __nv_bfloat16* __restrict__ q_out,
     uint8_t* __restrict__ k_cache, float* __restrict__ k_scale, uint8_t* __restrict__ k_zero,
     uint8_t* __restrict__ v_cache, float* __restrict__ v_scale, uint8_t* __restrict__ v_zero) {
+  constexpr int RB = D * BITS / 8;               // cache bytes per head vector
   const int nq = 4 * hq, nk = 4 * hkv;           // lanes per token pair
   const int items = nq + 2 * nk;
   const int lane = threadIdx.x & 31;
@@ -146,7 +168,7 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
       s = it & 1;
       if (tok >= T) continue;                    // both lanes of a vector leave together
       if (kind == 2) {
-        // V: 64 consecutive values, asymmetric 4-bit
+        // V: 64 consecutive values, asymmetric BITS-bit
         const int64_t g = static_cast<int64_t>(tok) * hkv + head;
         float x[64];
         load32_bf16(v + g * D + s * 64, x);
@@ -158,19 +180,21 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
           mx = fmaxf(mx, x[i]);
         }
         float scale, zero;
-        asym_params2(mn, mx, pmask, scale, zero);
+        asym_params2<BITS>(mn, mx, pmask, scale, zero);
         const float rs = __frcp_rn(scale);
         const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
-        uint32_t w[8];
+        constexpr int WPG = BITS / 4;            // words per 8 codes
+        uint32_t w[8 * WPG];
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
           const f2 xs[4] = {f2{x[8 * n], x[8 * n + 1]}, f2{x[8 * n + 2], x[8 * n + 3]},
                             f2{x[8 * n + 4], x[8 * n + 5]}, f2{x[8 * n + 6], x[8 * n + 7]}};
-          w[n] = ucodes8_div(xs, r2, sn2, z2);
+          ucodes8_div<BITS>(xs, r2, sn2, z2, w + WPG * n);
         }
-        uint4* dst = reinterpret_cast<uint4*>(v_cache + g * (D / 2) + s * 32);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        uint4* dst = reinterpret_cast<uint4*>(v_cache + g * RB + s * (RB / 2));
+#pragma unroll
+        for (int j = 0; j < 2 * WPG; ++j)
+          dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         if (s == 0) {
           v_scale[g] = scale;
           v_zero[g] = static_cast<uint8_t>(zero);
@@ -263,23 +287,29 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
           mx = fmaxf(mx, fmaxf(w[i].x, w[i].y));
         }
         float scale, zero;
-        asym_params2(mn * kNorm, mx * kNorm, pmask, scale, zero);
+        asym_params2<BITS>(mn * kNorm, mx * kNorm, pmask, scale, zero);
         const float kq = kNorm * __frcp_rn(scale);
         const f2 k2{kq, kq}, z2{zero, zero};
-        uint32_t wl[4], wh[4];
+        constexpr int WPG = BITS / 4;            // words per 8 codes
+        uint32_t wl[4 * WPG], wh[4 * WPG];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
           const f2 xl[4] = {f2{w[8 * n].x, w[8 * n + 1].x}, f2{w[8 * n + 2].x, w[8 * n + 3].x},
                             f2{w[8 * n + 4].x, w[8 * n + 5].x}, f2{w[8 * n + 6].x, w[8 * n + 7].x}};
           const f2 xh[4] = {f2{w[8 * n].y, w[8 * n + 1].y}, f2{w[8 * n + 2].y, w[8 * n + 3].y},
                             f2{w[8 * n + 4].y, w[8 * n + 5].y}, f2{w[8 * n + 6].y, w[8 * n + 7].y}};
-          wl[n] = ucodes8(xl, k2, z2);
-          wh[n] = ucodes8(xh, k2, z2);
+          ucodes8<BITS>(xl, k2, z2, wl + WPG * n);
+          ucodes8<BITS>(xh, k2, z2, wh + WPG * n);
         }
+        // elements s*32 .. s*32 + 31 and 64 + s*32 .. 64 + s*32 + 31
         const int64_t g = static_cast<int64_t>(tok) * hkv + head;
-        uint8_t* dst = k_cache + g * (D / 2);
-        *reinterpret_cast<uint4*>(dst + s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        *reinterpret_cast<uint4*>(dst + 32 + s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        uint4* dl = reinterpret_cast<uint4*>(k_cache + g * RB + s * (RB / 4));
+        uint4* dh = reinterpret_cast<uint4*>(k_cache + g * RB + RB / 2 + s * (RB / 4));
+#pragma unroll
+        for (int j = 0; j < WPG; ++j) {
+          dl[j] = make_uint4(wl[4 * j], wl[4 * j + 1], wl[4 * j + 2], wl[4 * j + 3]);
+          dh[j] = make_uint4(wh[4 * j], wh[4 * j + 1], wh[4 * j + 2], wh[4 * j + 3]);
+        }
         if (s == 0) {
           k_scale[g] = scale;
           k_zero[g] = static_cast<uint8_t>(zero);
@@ -290,6 +320,7 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
 }
 
 // out = bf16((code - zero) * scale); one thread per 16 codes.
+template <int BITS>
 __global__ void __launch_bounds__(256) kv_dequant_kernel(const uint8_t* __restrict__ cache,
                                                          const float* __restrict__ scale,
                                                          const uint8_t* __restrict__ zero,
@@ -299,13 +330,21 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const uint8_t* __restri
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t g = i >> 3;
-    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(cache) + i);
     const float s = __ldg(scale + g), z = static_cast<float>(__ldg(zero + g));
     float v[16];
+    if (BITS == 4) {
+      const uint2 w = __ldcs(reinterpret_cast<const uint2*>(cache) + i);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      v[e] = (static_cast<float>((w.x >> (4 * e)) & 0xFu) - z) * s;
-      v[8 + e] = (static_cast<float>((w.y >> (4 * e)) & 0xFu) - z) * s;
+      for (int e = 0; e < 8; ++e) {
+        v[e] = (static_cast<float>((w.x >> (4 * e)) & 0xFu) - z) * s;
+        v[8 + e] = (static_cast<float>((w.y >> (4 * e)) & 0xFu) - z) * s;
+      }
+    } else {
+      const uint4 w = __ldcs(reinterpret_cast<const uint4*>(cache) + i);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        v[e] = (static_cast<float>((ws[e >> 2] >> (8 * (e & 3))) & 0xFFu) - z) * s;
     }
     store16_bf16(out + i * 16, v);
   }
@@ -331,7 +370,7 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
                            int hkv, const int32_t* pos, const float* cos, const float* sin,
                            int max_pos, void* q_out, uint8_t* k_cache, float* k_scale,
                            uint8_t* k_zero, uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
-                           cudaStream_t stream) {
+                           int bits, cudaStream_t stream) {
   const int items = 4 * hq + 8 * hkv;            // lanes per pair of tokens
   const int threads = items >= 256 ? 256 : ((items + 31) & ~31);
   const int64_t pairs = (T + 1) / 2;
@@ -341,27 +380,26 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
   auto kp = static_cast<const __nv_bfloat16*>(k);
   auto vp = static_cast<const __nv_bfloat16*>(v);
   auto qo = static_cast<__nv_bfloat16*>(q_out);
-  if (cos)
-    kv_rotate_quant_kernel<true><<<grid, threads, 0, stream>>>(
-        qp, kp, vp, static_cast<int>(T), hq, hkv, pos, cos, sin, max_pos, qo, k_cache, k_scale,
-        k_zero, v_cache, v_scale, v_zero);
-  else
-    kv_rotate_quant_kernel<false><<<grid, threads, 0, stream>>>(
-        qp, kp, vp, static_cast<int>(T), hq, hkv, pos, cos, sin, max_pos, qo, k_cache, k_scale,
-        k_zero, v_cache, v_scale, v_zero);
+  auto kern = cos ? (bits == 8 ? kv_rotate_quant_kernel<true, 8> : kv_rotate_quant_kernel<true, 4>)
+                  : (bits == 8 ? kv_rotate_quant_kernel<false, 8>
+                               : kv_rotate_quant_kernel<false, 4>);
+  kern<<<grid, threads, 0, stream>>>(qp, kp, vp, static_cast<int>(T), hq, hkv, pos, cos, sin,
+                                     max_pos, qo, k_cache, k_scale, k_zero, v_cache, v_scale,
+                                     v_zero);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("kv_rotate_quant launch", e);
 }
 
 sq_status run_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero, int64_t T,
-                      int h, void* out, cudaStream_t stream) {
+                      int h, void* out, int bits, cudaStream_t stream) {
   const int64_t groups = T * h;
   const int64_t threads_needed = groups * 8;
   const int64_t cap = static_cast<int64_t>(host::num_sms()) * 16;
   int64_t grid = (threads_needed + 255) / 256;
   if (grid > cap) grid = cap;
-  kv_dequant_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(
-      cache, scale, zero, groups, static_cast<__nv_bfloat16*>(out));
+  auto kern = bits == 8 ? kv_dequant_kernel<8> : kv_dequant_kernel<4>;
+  kern<<<static_cast<int>(grid), 256, 0, stream>>>(cache, scale, zero, groups,
+                                                   static_cast<__nv_bfloat16*>(out));
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("kv_dequant launch", e);
 }

@@ -1,9 +1,11 @@
-// Decode attention over the asymmetric 4-bit KV caches, sm_100a tensor cores.
+// Decode attention over the asymmetric 4-bit (or 8-bit) KV caches, sm_100a
+// tensor cores.
 //
 // "SpinQuant, Reproduced", Q5: R3, the head-wise Hadamard on Q and K after
 // RoPE, is orthonormal, so q' k'^T = q k^T and a decode step can attend over
 // the rotated K cache as it was written; SpinQuant abstract: the KV cache is
-// 4-bit.  For query head h of sequence b (KV head kh = h / G, G = hq / hkv = 4):
+// 4-bit ("SpinQuant, Reproduced", Q7: 8-bit in the W4A8KV8 setting).  For
+// query head h of sequence b (KV head kh = h / G, G = hq / hkv = 4):
 //     o = sum_s softmax_s(q'[b][h] . k_hat[r][kh] / sqrt(128)) v_hat[r][kh],
 //     r = b * S_max + s, s < lengths[b],  x_hat = (code - zero) * scale.
 // With the zero points factored out, q . k_hat = scale_k (q . code - zero_k
@@ -15,7 +17,9 @@
 // tensor cores (tcgen05.mma kind::f16, f32 accumulation) with the 4-bit codes
 // as exact operands: a code c read as an f16 bit pattern is the subnormal
 // c * 2^-24, so eight packed codes become a 16-byte f16 operand chunk with two
-// masks and four byte permutes, and the products are exact.
+// masks and four byte permutes, and the products are exact.  8-bit codes
+// (at most 255) widen the same way, four byte permutes per 8 codes, and stay
+// exact: c * 2^-24 with c < 1024 is an f16 subnormal.
 //   scores:  D_S[t][h] = sum_d code_k[t][d] q[h][d]   (M = 128 tokens, N = 16:
 //            the 4 heads and 12 zero rows, K = 128 dims; A = the tile's K codes,
 //            K-major, B = the queries as f16, exact for bf16 queries in f16's
@@ -111,12 +115,22 @@ __device__ __forceinline__ float warp_max(float v) {
   return r;
 }
 
+// The 8 byte codes of two words as the f16 bit patterns 0..255.
+__device__ __forceinline__ uint4 codes8_f16(uint32_t w0, uint32_t w1) {
+  return make_uint4(prmt(w0, 0u, 0x4140u), prmt(w0, 0u, 0x4342u), prmt(w1, 0u, 0x4140u),
+                    prmt(w1, 0u, 0x4342u));
+}
+
+// One token row of a head: BITS * 8 bytes of K codes, as many of V.
+template <int BITS>
 struct Row {
-  uint4 k[4], v[4];
+  uint4 k[BITS], v[BITS];
   float sk, zk, sv, zv;
 };
 
-__global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
+template <int BITS>
+__global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
+  constexpr int RB = D * BITS / 8;         // cache bytes per token and head
   extern __shared__ uint8_t kvd_smem_raw[];
   uint8_t* smem = kvd_smem_raw + ((1024u - (smem_u32(kvd_smem_raw) & 1023u)) & 1023u);
   uint8_t* At = smem;
@@ -138,16 +152,16 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
   const int per = (len + P.nsplit - 1) / P.nsplit;
   const int t0 = split * per, t1 = min(len, t0 + per);
   const int ntiles = t1 > t0 ? (t1 - t0 + TILE - 1) / TILE : 0;
-  const int64_t row_stride = static_cast<int64_t>(P.hkv) * (D / 2);
+  const int64_t row_stride = static_cast<int64_t>(P.hkv) * RB;
   const int64_t row0 = static_cast<int64_t>(b) * P.S_max;
 
-  auto load_row = [&](int tok, Row& r) {
+  auto load_row = [&](int tok, Row<BITS>& r) {
     if (tok < t1) {
-      const int64_t off = (row0 + tok) * row_stride + kh * (D / 2);
+      const int64_t off = (row0 + tok) * row_stride + kh * RB;
       const uint4* kp = reinterpret_cast<const uint4*>(P.kc + off);
       const uint4* vp = reinterpret_cast<const uint4*>(P.vc + off);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < BITS; ++i) {
         r.k[i] = __ldg(kp + i);
         r.v[i] = __ldg(vp + i);
       }
@@ -158,12 +172,12 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
       r.zv = static_cast<float>(__ldg(P.vz + g));
     } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) r.k[i] = r.v[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < BITS; ++i) r.k[i] = r.v[i] = make_uint4(0u, 0u, 0u, 0u);
       r.sk = r.zk = r.sv = r.zv = 0.f;
     }
   };
   // the first tile's rows go out before the setup below
-  Row cur;
+  Row<BITS> cur;
   if (ntiles > 0) load_row(t0 + tid, cur);
 
   // queries as f16 (rows 0..3 of Bq; rows 4..15 zero), their sums per head,
@@ -218,13 +232,18 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
     qsum[h] = red2[h] + red2[8 + h] + red2[16 + h] + red2[24 + h];
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
 
-  auto store_codes = [&](const uint4 (&w)[4]) {
+  auto store_codes = [&](const uint4 (&w)[BITS]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < BITS; ++i) {
       const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+      if (BITS == 4) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        *reinterpret_cast<uint4*>(At + sw_off(tid, 4 * i + e, A_ATOM)) = codes_f16(ws[e]);
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(At + sw_off(tid, 4 * i + e, A_ATOM)) = codes_f16(ws[e]);
+      } else {
+        *reinterpret_cast<uint4*>(At + sw_off(tid, 2 * i, A_ATOM)) = codes8_f16(ws[0], ws[1]);
+        *reinterpret_cast<uint4*>(At + sw_off(tid, 2 * i + 1, A_ATOM)) = codes8_f16(ws[2], ws[3]);
+      }
     }
   };
 
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
   for (int it = 0; it < ntiles && ok; ++it) {
     const int tok = t0 + it * TILE + tid;
     const bool valid = tok < t1;
-    Row nxt;
+    Row<BITS> nxt;
     if (it + 1 < ntiles) load_row(tok + TILE, nxt);
     // scores: K codes of the tile, then the product with the queries
     store_codes(cur.k);
@@ -273,7 +292,25 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
       const float mx = warp_max(sc[h]);
       if (lane == 0) red[warp * 4 + h] = mx;
     }
+    {
+      const float svm = warp_max(cur.sv);  // scales are >= 0; rows past the end hold 0
+      if (lane == 0) red2[warp * 8] = svm;
+    }
     __syncthreads();
+    // The tile's weights p * scale_v (p <= 1) go to the tensor cores times a
+    // power of two 2^E that puts the largest just under 2^15, f16's top
+    // binade, so the f16 pair hi + lo keeps 22 bits of every weight down to
+    // 2^-29 of the largest instead of losing them in f16's subnormal range;
+    // the products are scaled back by 2^-E, exactly.
+    float up, down;
+    {
+      const float svmax = fmaxf(fmaxf(red2[0], red2[8]), fmaxf(red2[16], red2[24]));
+      // svmax < 2^e with e = biased exponent - 126 (normal, non-negative svmax)
+      const int e = static_cast<int>((__float_as_uint(svmax) >> 23) & 0xFFu) - 126;
+      const int E = svmax > 0.f ? min(max(15 - e, -100), 100) : 0;
+      up = __uint_as_float(static_cast<uint32_t>(127 + E) << 23);
+      down = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);
+    }
     float alpha[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -283,11 +320,11 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
       m[h] = mn;
       const float p = valid ? exp2f(sc[h] - mn) : 0.f;
       lsum[h] = lsum[h] * alpha[h] + p;
-      // weight times the value scale as an f16 pair hi + lo
-      const float pv = p * cur.sv;
+      // weight times the value scale (times 2^E) as an f16 pair hi + lo
+      const float pv = p * (cur.sv * up);
       const __half hi = __float2half_rn(pv);
       const __half lo = __float2half_rn(pv - __half2float(hi));
-      zsum[h] = zsum[h] * alpha[h] + (__half2float(hi) + __half2float(lo)) * cur.zv;
+      zsum[h] = zsum[h] * alpha[h] + (__half2float(hi) + __half2float(lo)) * down * cur.zv;
       const int byte = (tid & 7) * 2;
       *reinterpret_cast<__half*>(Bp + sw_off(h, tid >> 3, BP_ATOM) + byte) = hi;
       *reinterpret_cast<__half*>(Bp + sw_off(16 + h, tid >> 3, BP_ATOM) + byte) = lo;
@@ -309,10 +346,10 @@ __global__ void __launch_bounds__(THREADS) kv4_decode_tc_kernel(Params P) {
     uint32_t o32[32];
     tmem_ld32(lane_addr + 32, o32);
     tmem_ld_wait();
+    const float back = kTwo24 * down;
 #pragma unroll
     for (int h = 0; h < G; ++h)
-      o[h] = o[h] * alpha[h] +
-             (__uint_as_float(o32[h]) + __uint_as_float(o32[16 + h])) * kTwo24;
+      o[h] = o[h] * alpha[h] + (__uint_as_float(o32[h]) + __uint_as_float(o32[16 + h])) * back;
     tc_fence_before();
     cur = nxt;
     ok = __syncthreads_and(ok) != 0;       // leave together if a wait gave up
@@ -428,7 +465,8 @@ size_t workspace_bytes(int64_t B, int64_t S_max, int hkv, int num_sms) {
 sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const uint8_t* k_zero,
               const uint8_t* v_cache, const float* v_scale, const uint8_t* v_zero,
               const int32_t* lengths, int64_t B, int64_t S_max, int hq, int hkv, void* out,
-              void* workspace, size_t workspace_bytes_given, int num_sms, cudaStream_t stream) {
+              void* workspace, size_t workspace_bytes_given, int num_sms, int bits,
+              cudaStream_t stream) {
   Params P;
   P.q = static_cast<const __nv_bfloat16*>(q);
   P.kc = k_cache;
@@ -453,12 +491,12 @@ sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const
   (void)hq;
   P.spin_limit = host::spin_limit();
   const int64_t grid = B * hkv * ns;
-  cudaError_t ea = cudaFuncSetAttribute(kv4_decode_tc_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(kv4_decode)", ea);
-  kv4_decode_tc_kernel<<<static_cast<unsigned>(grid), THREADS, SMEM, stream>>>(P);
+  auto kern = bits == 8 ? kv_decode_tc_kernel<8> : kv_decode_tc_kernel<4>;
+  cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(kv_decode)", ea);
+  kern<<<static_cast<unsigned>(grid), THREADS, SMEM, stream>>>(P);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SQ_OK : host::cuda_fail("kv4_decode launch", e);
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("kv_decode launch", e);
 }
 
 }  // namespace kvd

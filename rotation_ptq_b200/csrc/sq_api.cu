@@ -252,12 +252,13 @@ size_t sq_kv4_decode_workspace_bytes(int64_t B, int64_t S_max, int hq, int hkv) 
   return sq::kvd::workspace_bytes(B, S_max, hkv, sq::host::num_sms());
 }
 
-sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
-                                  const uint8_t* k_zero, const uint8_t* v_cache,
-                                  const float* v_scale, const uint8_t* v_zero,
-                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
-                                  int hkv, int d, void* out, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+static sq_status kv_decode_attention(const void* q, const uint8_t* k_cache,
+                                     const float* k_scale, const uint8_t* k_zero,
+                                     const uint8_t* v_cache, const float* v_scale,
+                                     const uint8_t* v_zero, const int32_t* lengths, int64_t B,
+                                     int64_t S_max, int hq, int hkv, int d, void* out,
+                                     void* workspace, size_t workspace_bytes, int bits,
+                                     void* stream) {
   if (B < 0 || S_max < 1 || hq < 1 || hkv < 1) {
     set_error("bad sizes B=%lld S_max=%lld hq=%d hkv=%d", (long long)B, (long long)S_max, hq,
               hkv);
@@ -283,7 +284,27 @@ sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const f
   if (st != SQ_OK) return st;
   return sq::kvd::run(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, B, S_max,
                       hq, hkv, out, workspace, workspace ? workspace_bytes : 0,
-                      sq::host::num_sms(), static_cast<cudaStream_t>(stream));
+                      sq::host::num_sms(), bits, static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_kv4_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
+                                  const uint8_t* k_zero, const uint8_t* v_cache,
+                                  const float* v_scale, const uint8_t* v_zero,
+                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
+                                  int hkv, int d, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return kv_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, B,
+                             S_max, hq, hkv, d, out, workspace, workspace_bytes, 4, stream);
+}
+
+sq_status sq_kv8_decode_attention(const void* q, const uint8_t* k_cache, const float* k_scale,
+                                  const uint8_t* k_zero, const uint8_t* v_cache,
+                                  const float* v_scale, const uint8_t* v_zero,
+                                  const int32_t* lengths, int64_t B, int64_t S_max, int hq,
+                                  int hkv, int d, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return kv_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, B,
+                             S_max, hq, hkv, d, out, workspace, workspace_bytes, 8, stream);
 }
 
 size_t sq_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -368,12 +389,12 @@ sq_status sq_w4a8_linear(const int8_t* a_q, const float* a_scale, const uint8_t*
                           sq::host::spin_limit(), sq::host::num_sms());
 }
 
-sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
-                             int hkv, int d, const int32_t* pos, const float* rope_cos,
-                             const float* rope_sin, int max_pos, void* q_out,
-                             uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
-                             uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
-                             void* stream) {
+static sq_status kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
+                                 int hkv, int d, const int32_t* pos, const float* rope_cos,
+                                 const float* rope_sin, int max_pos, void* q_out,
+                                 uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                                 uint8_t* v_cache, float* v_scale, uint8_t* v_zero, int bits,
+                                 void* stream) {
   if (T < 0 || hq < 1 || hkv < 1) {
     set_error("bad sizes T=%lld hq=%d hkv=%d", (long long)T, hq, hkv);
     return SQ_ERR_INVALID_ARG;
@@ -410,11 +431,31 @@ sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_
   if (st != SQ_OK) return st;
   return sq::kv::run_rotate_quant(q, k, v, T, hq, hkv, pos, rope_cos, rope_sin, max_pos, q_out,
                                   k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
-                                  static_cast<cudaStream_t>(stream));
+                                  bits, static_cast<cudaStream_t>(stream));
 }
 
-sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
-                        int64_t T, int h, int d, void* out_bf16, void* stream) {
+sq_status sq_kv_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
+                             int hkv, int d, const int32_t* pos, const float* rope_cos,
+                             const float* rope_sin, int max_pos, void* q_out,
+                             uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                             uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                             void* stream) {
+  return kv_rotate_quant(q, k, v, T, hq, hkv, d, pos, rope_cos, rope_sin, max_pos, q_out, k_cache,
+                         k_scale, k_zero, v_cache, v_scale, v_zero, 4, stream);
+}
+
+sq_status sq_kv_rotate_quant8(const void* q, const void* k, const void* v, int64_t T, int hq,
+                              int hkv, int d, const int32_t* pos, const float* rope_cos,
+                              const float* rope_sin, int max_pos, void* q_out,
+                              uint8_t* k_cache, float* k_scale, uint8_t* k_zero,
+                              uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
+                              void* stream) {
+  return kv_rotate_quant(q, k, v, T, hq, hkv, d, pos, rope_cos, rope_sin, max_pos, q_out, k_cache,
+                         k_scale, k_zero, v_cache, v_scale, v_zero, 8, stream);
+}
+
+static sq_status kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                            int64_t T, int h, int d, void* out_bf16, int bits, void* stream) {
   if (T < 0 || h < 1) {
     set_error("bad sizes T=%lld h=%d", (long long)T, h);
     return SQ_ERR_INVALID_ARG;
@@ -434,8 +475,18 @@ sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t*
   }
   sq_status st = precheck_device();
   if (st != SQ_OK) return st;
-  return sq::kv::run_dequant(cache, scale, zero, T, h, out_bf16,
+  return sq::kv::run_dequant(cache, scale, zero, T, h, out_bf16, bits,
                              static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_kv_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                        int64_t T, int h, int d, void* out_bf16, void* stream) {
+  return kv_dequant(cache, scale, zero, T, h, d, out_bf16, 4, stream);
+}
+
+sq_status sq_kv8_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
+                         int64_t T, int h, int d, void* out_bf16, void* stream) {
+  return kv_dequant(cache, scale, zero, T, h, d, out_bf16, 8, stream);
 }
 
 sq_status sq_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,

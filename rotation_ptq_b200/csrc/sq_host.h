@@ -87,10 +87,12 @@ namespace kvd {
 // when it runs unsplit).
 int choose_splits(int64_t B, int64_t S_max, int hkv, int num_sms);
 size_t workspace_bytes(int64_t B, int64_t S_max, int hkv, int num_sms);
+// bits = 4 or 8: the caches' code width (as kv::run_dequant).
 sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const uint8_t* k_zero,
               const uint8_t* v_cache, const float* v_scale, const uint8_t* v_zero,
               const int32_t* lengths, int64_t B, int64_t S_max, int hq, int hkv, void* out,
-              void* workspace, size_t workspace_bytes, int num_sms, cudaStream_t stream);
+              void* workspace, size_t workspace_bytes, int num_sms, int bits,
+              cudaStream_t stream);
 }  // namespace kvd
 
 namespace kv {
@@ -98,9 +100,10 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
                            int hkv, const int32_t* pos, const float* cos, const float* sin,
                            int max_pos, void* q_out, uint8_t* k_cache, float* k_scale,
                            uint8_t* k_zero, uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
-                           cudaStream_t stream);
+                           int bits, cudaStream_t stream);
+// bits = 4: packed nibbles [T][h][64]; bits = 8: bytes [T][h][128].
 sq_status run_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero, int64_t T,
-                      int h, void* out, cudaStream_t stream);
+                      int h, void* out, int bits, cudaStream_t stream);
 sq_status run_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,
                           cudaStream_t stream);
 }  // namespace kv

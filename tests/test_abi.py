@@ -35,6 +35,7 @@ def test_header_declares_the_hot_path_calls():
     for n in ["sq_rotate_quant", "sq_swiglu_rotate_quant", "sq_w4a4_linear",
               "sq_kv4_decode_attention", "sq_kv4_decode_workspace_bytes",
               "sq_kv_rotate_quant", "sq_kv_dequant",
+              "sq_kv_rotate_quant8", "sq_kv8_dequant", "sq_kv8_decode_attention",
               "sq_status_string", "sq_w4a4_workspace_bytes", "sq_device_status"]:
         assert n in names
 
@@ -92,6 +93,15 @@ def test_validation_happens_before_any_launch(sq):
     assert lib.sq_kv4_decode_attention(*args, 2, 16, 16, 8, 128, None, None, 0, None) == 2
     assert lib.sq_kv4_decode_attention(*args, 2, 0, 32, 8, 128, None, None, 0, None) == 1
     assert lib.sq_kv4_decode_attention(*args, 0, 16, 32, 8, 128, None, None, 0, None) == 0
+    # the 8-bit KV entries share the 4-bit ones' rules
+    assert lib.sq_kv_rotate_quant8(None, None, None, 4, 32, 8, 64, None, None, None, 0,
+                                   None, None, None, None, None, None, None, None) == 2
+    assert lib.sq_kv_rotate_quant8(None, None, None, 0, 32, 8, 128, None, None, None, 0,
+                                   None, None, None, None, None, None, None, None) == 0
+    assert lib.sq_kv8_dequant(None, None, None, 4, 8, 64, None, None) == 2
+    assert lib.sq_kv8_dequant(None, None, None, 4, 8, 128, None, None) == 1
+    assert lib.sq_kv8_decode_attention(*args, 2, 16, 16, 8, 128, None, None, 0, None) == 2
+    assert lib.sq_kv8_decode_attention(*args, 0, 16, 32, 8, 128, None, None, 0, None) == 0
 
 
 def test_product_paley_matches_oracle():

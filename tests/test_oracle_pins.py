@@ -561,6 +561,28 @@ def test_kv8_composition_uses_rope_and_r3():
     assert e8 < e4 / 8                           # 17x finer grid
 
 
+def test_kv8_decode_uniform_keys_average_values():
+    # equal K codes, scales and zero points make every score equal: the
+    # softmax is uniform and the output the mean of the read-back values
+    rng = np.random.default_rng(103)
+    B, S, hkv, d = 2, 5, 1, 128
+    q = rng.standard_normal((B, 4, d))
+    kc = np.full((B * S, hkv, d), 77, np.uint8)
+    ks = np.full((B * S, hkv), 0.02, np.float32)
+    kz = np.full((B * S, hkv), 128, np.uint8)
+    vc = rng.integers(0, 256, (B * S, hkv, d), dtype=np.uint8)
+    vs = (0.01 + 0.02 * rng.random((B * S, hkv))).astype(np.float32)
+    vz = rng.integers(100, 156, (B * S, hkv)).astype(np.uint8)
+    lengths = np.array([5, 2])
+    o = O.kv8_decode_attention(q, kc, ks, kz, vc, vs, vz, lengths, S)
+    for b in range(B):
+        rows = range(b * S, b * S + lengths[b])
+        mean = sum((vc[r, 0].astype(np.float64) - float(vz[r, 0])) * float(vs[r, 0])
+                   for r in rows) / lengths[b]
+        for h in range(4):
+            assert np.allclose(o[b, h], mean, rtol=1e-12, atol=1e-15)
+
+
 # --------------------------------------------------------------------------
 # SwiGLU ahead of down_proj (fused SwiGLU + R4)
 # --------------------------------------------------------------------------

@@ -284,3 +284,31 @@ def kv4_decode(B: int = 16, S_max: int = 4096, hq: int = N_HEADS, hkv: int = N_K
     return DecodeWorkload("kv4_decode_B%d_S%d_hq%d_hkv%d" % (B, S_max, hq, hkv), _bf16(q),
                           t(kc), t(ks), t(kz), t(vc), t(vs), t(vz),
                           t(lengths.astype(np.int32)), S_max)
+
+
+def kv8_decode(B: int = 16, S_max: int = 4096, hq: int = N_HEADS, hkv: int = N_KV_HEADS,
+               d: int = 128, seed: int = SEED_BASE + 8, ragged: bool = False) -> DecodeWorkload:
+    """Decode step over 8-bit caches (the W4A8KV8 setting), same sizes as kv4_decode.
+
+    Codes are uniform 8-bit values [T, hkv, d]; scales and zero points take the
+    range that quantizing unit-variance head vectors to 0..255 gives (scale ~
+    0.018..0.03, zero ~ 100..155); queries ~ N(0, 1).
+    """
+    rng = np.random.default_rng(seed)
+    T = B * S_max
+    q = rng.standard_normal((B, hq, d))
+    kc = rng.integers(0, 256, (T, hkv, d), dtype=np.uint8)
+    vc = rng.integers(0, 256, (T, hkv, d), dtype=np.uint8)
+    ks = (0.018 + 0.012 * rng.random((T, hkv))).astype(np.float32)
+    vs = (0.018 + 0.012 * rng.random((T, hkv))).astype(np.float32)
+    kz = rng.integers(100, 156, (T, hkv)).astype(np.uint8)
+    vz = rng.integers(100, 156, (T, hkv)).astype(np.uint8)
+    if ragged:
+        lengths = rng.integers(1, S_max + 1, B)
+        lengths[0], lengths[-1] = S_max, 1
+    else:
+        lengths = np.full(B, S_max)
+    t = torch.from_numpy
+    return DecodeWorkload("kv8_decode_B%d_S%d_hq%d_hkv%d" % (B, S_max, hq, hkv), _bf16(q),
+                          t(kc), t(ks), t(kz), t(vc), t(vs), t(vz),
+                          t(lengths.astype(np.int32)), S_max)
