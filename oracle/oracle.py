@@ -483,6 +483,104 @@ def kv8_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
 
 
 # ---------------------------------------------------------------------------
+# Cayley SGD for the head-wise rotation R2 ("SpinQuant, Reproduced", Q6).
+# The pages give the transform R' = (I - a/2 Y)^-1 (I + a/2 Y) R with a skew
+# Y, a straight-through estimator through the quantizers, and the objective:
+# one layer's own W4A4 output error, weights frozen, R2 shared by all heads.
+# Readings where they are silent:
+#   * Y = R G^T - G R^T from the Euclidean gradient G of the loss at R, so
+#     that R' = R - a (G - R G^T R) + O(a^2), a descent step;
+#   * the layer is o_proj: R2 rotates its input (the attention output, H
+#     heads of d channels) head-wise, and its weight's input dimension by the
+#     same R, so x' w'^T = x w^T at full precision; activations are quantized
+#     per token and weights per output channel with quant_sym_int4;
+#   * the loss is ||y - y0||^2 / ||y0||^2 with y0 = x w^T and y the W4A4
+#     output; the straight-through estimator passes the gradient of each
+#     quantizer's output to its input unchanged;
+#   * a random Hadamard is diag(s) H_d / sqrt(d) with random signs s (the
+#     signs act first: H_d diag(s) would only flip the signs of the rotated
+#     channels, which no symmetric quantizer sees).
+# ---------------------------------------------------------------------------
+
+
+def cayley_skew(R: np.ndarray, G: np.ndarray) -> np.ndarray:
+    """Y = R G^T - G R^T (skew-symmetric), float64."""
+    R = np.asarray(R, np.float64)
+    G = np.asarray(G, np.float64)
+    return R @ G.T - G @ R.T
+
+
+def cayley_update(R: np.ndarray, G: np.ndarray, alpha: float) -> np.ndarray:
+    """R' = (I - alpha/2 Y)^-1 (I + alpha/2 Y) R with Y = cayley_skew(R, G)."""
+    R = np.asarray(R, np.float64)
+    n = R.shape[0]
+    Y = cayley_skew(R, G)
+    eye = np.eye(n)
+    return np.linalg.solve(eye - 0.5 * alpha * Y, (eye + 0.5 * alpha * Y) @ R)
+
+
+def orth_error(R: np.ndarray) -> float:
+    """||R^T R - I||_F."""
+    R = np.asarray(R, np.float64)
+    return float(np.linalg.norm(R.T @ R - np.eye(R.shape[0])))
+
+
+def random_hadamard(signs: np.ndarray) -> np.ndarray:
+    """diag(signs) H_d / sqrt(d) for a sign vector of length d (a power of 2)."""
+    s = np.asarray(signs, np.float64)
+    d = s.shape[0]
+    return s[:, None] * sylvester(d) / math.sqrt(d)
+
+
+def headwise(x: np.ndarray, R: np.ndarray) -> np.ndarray:
+    """Each row's consecutive groups of d = R.shape[0] channels times R."""
+    x = np.asarray(x, np.float64)
+    d = R.shape[0]
+    rows, K = x.shape
+    return (x.reshape(rows, K // d, d) @ np.asarray(R, np.float64)).reshape(rows, K)
+
+
+def r2_loss_grad(x: np.ndarray, w: np.ndarray, R: np.ndarray, want_grad: bool = True):
+    """W4A4 output error of y = x w^T with the input rotated head-wise by R,
+    and its straight-through gradient with respect to R.
+
+    x [T, H*d] activations, w [N, H*d] weights, R [d, d].  Rotations in
+    float64, each rounded to float32 before its quantizer decides (as the
+    rotate-and-quantize path does).  Returns (loss, G [d, d] or None).
+    """
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w, np.float64)
+    d = R.shape[0]
+    ca, sa, _ = quant_sym_int4(headwise(x, R).astype(F32))
+    cw, sw, _ = quant_sym_int4(headwise(w, R).astype(F32))
+    qa = ca.astype(np.float64) * sa.astype(np.float64)[:, None]
+    qw = cw.astype(np.float64) * sw.astype(np.float64)[:, None]
+    y0 = x @ w.T
+    E = qa @ qw.T - y0
+    den = float(np.sum(y0 * y0))
+    loss = float(np.sum(E * E)) / den
+    if not want_grad:
+        return loss, None
+    g_xr = (2.0 / den) * (E @ qw)          # d loss / d (x R), through the quantizer
+    g_wr = (2.0 / den) * (E.T @ qa)        # d loss / d (w R)
+    G = x.reshape(-1, d).T @ g_xr.reshape(-1, d) + w.reshape(-1, d).T @ g_wr.reshape(-1, d)
+    return loss, G
+
+
+def r2_cayley_learn(x, w, R0, alpha: float, iters: int):
+    """iters Cayley SGD steps from R0.  Returns (R, losses): losses[i] is the
+    loss at the i-th iterate (losses[iters] at the result)."""
+    R = np.asarray(R0, np.float64)
+    losses = []
+    for _ in range(iters):
+        loss, G = r2_loss_grad(x, w, R)
+        losses.append(loss)
+        R = cayley_update(R, G, alpha)
+    losses.append(r2_loss_grad(x, w, R, want_grad=False)[0])
+    return R, losses
+
+
+# ---------------------------------------------------------------------------
 # Statistics ("SpinQuant, Reproduced", Q3: kurtosis across channels within a
 # token, averaged over tokens; 3 is a Gaussian).
 # ---------------------------------------------------------------------------

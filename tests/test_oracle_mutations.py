@@ -195,10 +195,53 @@ def _asym8_clamp_15(x):
     return np.minimum(c, 15).astype(np.uint8), s, z, vv
 
 
+def _skew_ascent(R, G):
+    R = np.asarray(R, np.float64)
+    G = np.asarray(G, np.float64)
+    return G @ R.T - R @ G.T
+
+
+def _cayley_full_alpha(R, G, alpha):
+    R = np.asarray(R, np.float64)
+    n = R.shape[0]
+    Y = _orig["cayley_skew"](R, G)
+    eye = np.eye(n)
+    return np.linalg.solve(eye - alpha * Y, (eye + alpha * Y) @ R)
+
+
+def _r2_grad_no_weight_term(x, w, R, want_grad=True):
+    loss, G = _orig["r2_loss_grad"](x, w, R, want_grad)
+    if G is None:
+        return loss, G
+    xf = np.asarray(x, np.float64)
+    wf = np.asarray(w, np.float64)
+    d = R.shape[0]
+    ca, sa, _ = O.quant_sym_int4(O.headwise(xf, R).astype(np.float32))
+    cw, sw, _ = O.quant_sym_int4(O.headwise(wf, R).astype(np.float32))
+    qa = ca * sa.astype(np.float64)[:, None]
+    qw = cw * sw.astype(np.float64)[:, None]
+    y0 = xf @ wf.T
+    E = qa @ qw.T - y0
+    g_xr = (2.0 / np.sum(y0 * y0)) * (E @ qw)
+    return loss, xf.reshape(-1, d).T @ g_xr.reshape(-1, d)
+
+
+def _r2_grad_transposed(x, w, R, want_grad=True):
+    loss, G = _orig["r2_loss_grad"](x, w, R, want_grad)
+    return loss, (None if G is None else G.T)
+
+
+def _random_hadamard_signs_after(signs):
+    s = np.asarray(signs, np.float64)
+    d = s.shape[0]
+    return O.sylvester(d) * s[None, :] / np.sqrt(d)
+
+
 _orig = {name: getattr(O, name) for name in
          ["paley1", "kron", "rotate", "quant_sym_int4", "pack_int4", "rope",
           "quant_asym_uint4", "dequant", "sylvester", "silu", "round_bf16", "swiglu_bf16",
-          "decode_attention", "quant_sym_int8", "quant_asym_uint8"]}
+          "decode_attention", "quant_sym_int8", "quant_asym_uint8", "cayley_skew",
+          "r2_loss_grad"]}
 
 MUTATIONS = {
     "paley_transposed": ("paley1", _transposed_paley),
@@ -227,6 +270,11 @@ MUTATIONS = {
     "quant8_round_half_up": ("quant_sym_int8", _quant8_round_half_up),
     "asym8_divisor_256": ("quant_asym_uint8", _asym8_div256),
     "asym8_4bit_clamp": ("quant_asym_uint8", _asym8_clamp_15),
+    "cayley_skew_ascends": ("cayley_skew", _skew_ascent),
+    "cayley_alpha_not_halved": ("cayley_update", _cayley_full_alpha),
+    "r2_grad_drops_weight_term": ("r2_loss_grad", _r2_grad_no_weight_term),
+    "r2_grad_transposed": ("r2_loss_grad", _r2_grad_transposed),
+    "random_hadamard_signs_on_columns": ("random_hadamard", _random_hadamard_signs_after),
 }
 
 PIN_TESTS = [
@@ -265,6 +313,13 @@ PIN_TESTS = [
     P.test_rotate_quant8_is_rotation_then_quant8,
     P.test_asym8_bruteforce_and_bounds,
     P.test_asym8_constant_and_zero_rows,
+    P.test_cayley_2x2_is_a_plane_rotation,
+    P.test_cayley_keeps_orthogonality_and_first_order_step,
+    P.test_cayley_step_descends,
+    P.test_random_hadamard_is_orthogonal_with_signed_rows,
+    P.test_headwise_rotation_is_invisible_at_full_precision,
+    P.test_r2_loss_at_identity_is_the_plain_w4a4_error,
+    P.test_r2_ste_gradient_is_the_frozen_noise_derivative,
 ]
 
 

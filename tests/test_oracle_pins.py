@@ -584,6 +584,127 @@ def test_kv8_decode_uniform_keys_average_values():
 
 
 # --------------------------------------------------------------------------
+# Cayley SGD for R2
+# --------------------------------------------------------------------------
+
+def _rand_orth(rng, n):
+    q, r = np.linalg.qr(rng.standard_normal((n, n)))
+    return q * np.sign(np.diag(r))[None, :]
+
+
+def test_cayley_2x2_is_a_plane_rotation():
+    # R = I and G with G^T - G = [[0, -t], [t, 0]]: the Cayley transform of
+    # S = a/2 Y is the rotation by 2 atan(a t / 2)
+    for a, t in ((0.3, 1.0), (2.0, -0.7), (5.0, 3.0)):
+        G = np.array([[0.0, t / 2], [-t / 2, 0.0]])
+        Rn = O.cayley_update(np.eye(2), G, a)
+        phi = 2 * math.atan(a * t / 2)
+        want = np.array([[math.cos(phi), -math.sin(phi)], [math.sin(phi), math.cos(phi)]])
+        assert np.allclose(Rn, want, atol=1e-14)
+
+
+def test_cayley_keeps_orthogonality_and_first_order_step():
+    rng = np.random.default_rng(111)
+    R = _rand_orth(rng, 16)
+    G = rng.standard_normal((16, 16))
+    Y = O.cayley_skew(R, G)
+    assert np.allclose(Y, -Y.T, atol=0)
+    for a in (0.01, 1.0, 50.0):
+        assert O.orth_error(O.cayley_update(R, G, a)) < 1e-12
+    # R' = R - a (G - R G^T R) + O(a^2): the projected (Riemannian) descent step
+    a = 1e-5
+    step = (O.cayley_update(R, G, a) - R) / a
+    want = -(G - R @ G.T @ R)
+    assert np.linalg.norm(step - want) <= 1e-3 * np.linalg.norm(want)
+    assert np.array_equal(O.cayley_update(R, G, 0.0), R) or \
+        np.abs(O.cayley_update(R, G, 0.0) - R).max() < 1e-15
+    assert np.abs(O.cayley_update(R, np.zeros_like(G), 1.0) - R).max() < 1e-15
+
+
+def test_cayley_step_descends():
+    # f(R) = -tr(A^T R) has gradient -A; a small step must lower it
+    rng = np.random.default_rng(112)
+    R = _rand_orth(rng, 8)
+    A = rng.standard_normal((8, 8))
+    f = lambda M: -np.trace(A.T @ M)  # noqa: E731
+    for a in (1e-3, 1e-2):
+        assert f(O.cayley_update(R, -A, a)) < f(R)
+
+
+def test_random_hadamard_is_orthogonal_with_signed_rows():
+    rng = np.random.default_rng(113)
+    s = np.where(rng.random(128) < 0.5, -1, 1)
+    R = O.random_hadamard(s)
+    assert O.orth_error(R) < 1e-12
+    assert np.allclose(np.abs(R), 1 / math.sqrt(128))
+    # row i is s_i times row i of the Sylvester matrix (the signs act first)
+    H = O.sylvester(128)
+    assert np.allclose(R * math.sqrt(128), s[:, None] * H)
+
+
+def test_headwise_rotation_is_invisible_at_full_precision():
+    rng = np.random.default_rng(114)
+    x = rng.standard_normal((6, 4 * 16))
+    w = rng.standard_normal((5, 4 * 16))
+    R = _rand_orth(rng, 16)
+    assert np.allclose(O.headwise(x, R) @ O.headwise(w, R).T, x @ w.T, atol=1e-12)
+    # head h of the result only reads head h of the input
+    x2 = x.copy()
+    x2[:, 16:32] = 0
+    assert np.allclose(O.headwise(x2, R)[:, 16:32], 0)
+    assert np.allclose(O.headwise(x2, R)[:, :16], x[:, :16] @ R)
+
+
+def test_r2_loss_at_identity_is_the_plain_w4a4_error():
+    rng = np.random.default_rng(115)
+    x = rng.standard_normal((8, 256)).astype(np.float32)
+    w = (0.1 * rng.standard_normal((16, 256))).astype(np.float32)
+    loss, _ = O.r2_loss_grad(x, w, np.eye(128), want_grad=False)
+    ca, sa, _ = O.quant_sym_int4(x)
+    cw, sw, _ = O.quant_sym_int4(w)
+    y = O.dequant(O.gemm_int(ca, cw), sa, sw)
+    y0 = x.astype(np.float64) @ w.T.astype(np.float64)
+    assert math.isclose(loss, np.sum((y - y0) ** 2) / np.sum(y0 ** 2), rel_tol=1e-6)
+
+
+def test_r2_ste_gradient_is_the_frozen_noise_derivative():
+    # the straight-through gradient is the exact gradient of the loss with the
+    # rounding noise Q(z) - z of both quantizers frozen at R0
+    rng = np.random.default_rng(116)
+    d, H = 16, 3
+    x = rng.standard_normal((10, H * d))
+    w = rng.standard_normal((7, H * d))
+    R0 = _rand_orth(rng, d)
+    _, G = O.r2_loss_grad(x, w, R0)
+    ca, sa, _ = O.quant_sym_int4(O.headwise(x, R0).astype(np.float32))
+    cw, sw, _ = O.quant_sym_int4(O.headwise(w, R0).astype(np.float32))
+    na = ca * sa.astype(np.float64)[:, None] - O.headwise(x, R0)
+    nw = cw * sw.astype(np.float64)[:, None] - O.headwise(w, R0)
+    y0 = x @ w.T
+    den = np.sum(y0 ** 2)
+
+    def surrogate(R):
+        e = (O.headwise(x, R) + na) @ (O.headwise(w, R) + nw).T - y0
+        return np.sum(e ** 2) / den
+
+    for _ in range(4):
+        D = rng.standard_normal((d, d))
+        eps = 1e-6
+        fd = (surrogate(R0 + eps * D) - surrogate(R0 - eps * D)) / (2 * eps)
+        assert math.isclose(fd, np.sum(G * D), rel_tol=1e-6, abs_tol=1e-12)
+
+
+def test_r2_learner_beats_random_hadamards_and_stays_orthogonal():
+    wl = W.o_proj_layer(T=256, H=4, N=512)
+    draws = [O.r2_loss_grad(wl.x, wl.w, O.random_hadamard(s), want_grad=False)[0]
+             for s in wl.signs]
+    R, losses = O.r2_cayley_learn(wl.x, wl.w, O.random_hadamard(wl.signs[0]), 0.3, 120)
+    assert losses[-1] < min(draws)
+    assert losses[-1] < losses[0]
+    assert O.orth_error(R) < 1e-12
+
+
+# --------------------------------------------------------------------------
 # SwiGLU ahead of down_proj (fused SwiGLU + R4)
 # --------------------------------------------------------------------------
 

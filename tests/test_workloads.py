@@ -29,3 +29,12 @@ def test_kv_and_linear_generators():
     lin = W.tiny_linear()
     assert lin.x.shape[1] == lin.w.shape[1]
     assert np.array_equal(W.random_int8(1, 2, 128), W.random_int8(1, 2, 128))
+
+
+def test_o_proj_layer_generator():
+    wl = W.o_proj_layer(T=16, H=2, d=128, N=64, n_draws=4, seed=3)
+    assert wl.x.shape == (16, 256) and wl.x.dtype == np.float32
+    assert wl.w.shape == (64, 256) and wl.w.dtype == np.float32
+    assert wl.signs.shape == (4, 128) and set(np.unique(wl.signs)) <= {-1, 1}
+    again = W.o_proj_layer(T=16, H=2, d=128, N=64, n_draws=4, seed=3)
+    assert np.array_equal(wl.x, again.x) and np.array_equal(wl.signs, again.signs)

@@ -26,6 +26,8 @@ from __future__ import annotations
 
 import dataclasses
 
+import math
+
 import numpy as np
 import torch
 
@@ -312,3 +314,36 @@ def kv8_decode(B: int = 16, S_max: int = 4096, hq: int = N_HEADS, hkv: int = N_K
     return DecodeWorkload("kv8_decode_B%d_S%d_hq%d_hkv%d" % (B, S_max, hq, hkv), _bf16(q),
                           t(kc), t(ks), t(kz), t(vc), t(vs), t(vz),
                           t(lengths.astype(np.int32)), S_max)
+
+
+class OProjWorkload:
+    """Calibration activations and frozen weights of one o_proj linear, plus
+    the sign vectors of the random Hadamards the learned rotation is compared
+    with (rotation = diag(s) H_d / sqrt(d))."""
+
+    def __init__(self, name, x, w, signs, d):
+        self.name, self.x, self.w, self.signs, self.d = name, x, w, signs, d
+
+
+def o_proj_layer(T: int = 2048, H: int = N_HEADS, d: int = 128, N: int = HIDDEN,
+                 n_draws: int = 32, seed: int = SEED_BASE + 9) -> OProjWorkload:
+    """o_proj of a Qwen3-8B layer: x [T, H*d] (the attention output of 8
+    sequences x 256 tokens), w [N, H*d].
+
+    Each head's channels are Student-t(3) values with a per-channel scale
+    drawn log-uniform over a factor of 4, and 2 outlier channels per head at
+    12x; weights ~ N(0, 0.02) with a per-input-channel scale over a factor of
+    2.  float32 arrays; signs is int8 [n_draws, d] of +-1.
+    """
+    rng = np.random.default_rng(seed)
+    K = H * d
+    ch = np.exp(rng.uniform(0.0, math.log(4.0), K))
+    for h in range(H):
+        out = rng.choice(d, 2, replace=False)
+        ch[h * d + out] *= 12.0
+    x = (rng.standard_t(3, (T, K)) * ch[None, :] * 0.05).astype(np.float32)
+    wc = np.exp(rng.uniform(0.0, math.log(2.0), K))
+    w = (rng.standard_normal((N, K)) * 0.02 * wc[None, :]).astype(np.float32)
+    signs = np.where(rng.random((n_draws, d)) < 0.5, -1, 1).astype(np.int8)
+    return OProjWorkload("o_proj_T%d_H%d_d%d_N%d" % (T, H, d, N), x, w, signs, d)
+
