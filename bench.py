@@ -46,6 +46,18 @@ KV_T, KV_HQ, KV_HKV = 16 * 4096, 32, 8
 DECODE_BYTES = 2 * KV_T * KV_HKV * (64 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
 # ... of sq_kv8_decode_attention: one byte per code
 DECODE8_BYTES = 2 * KV_T * KV_HKV * (128 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
+# Cayley R2 learner on the o_proj layer (2048 tokens, 32 heads of 128, 4096
+# outputs): float32 FLOPs of one loss-and-gradient evaluation (head-wise
+# rotations of x and w, the two straight-through gradient products, and G)
+# and the INT4 tensor-core product
+R2_T, R2_H, R2_D, R2_N = 2048, 32, 128, 4096
+R2_K = R2_H * R2_D
+R2_F32_FLOPS = (2 * (R2_T + R2_N) * R2_K * R2_D + 2 * 2 * R2_T * R2_N * R2_K
+                + 2 * (R2_T + R2_N) * R2_H * R2_D * R2_D)
+R2_INT_OPS = 2 * R2_T * R2_N * R2_K
+R2_ALPHA = 0.3
+# CUDA-core float32 peak: 148 SMs x 128 FP32 lanes x 2 FLOP x 1.965 GHz
+F32_PEAK = 148 * 128 * 2 * 1.965e9 / 1e12
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
@@ -358,10 +370,50 @@ def run_ours(args, rank, world, local_rank):
                            "frac_of_hbm": DECODE8_BYTES / (mde * 1e-3) / 1e9 / load_peaks()[0]}
         del t8, dout
 
+    # Cayley SGD for R2 on one o_proj layer: loss-and-gradient evaluations and
+    # whole learner steps (loss, gradient and the float64 Cayley update)
+    r2_info = None
+    if not args.no_kv:
+        ow = W.o_proj_layer()
+        prob = sq.R2Problem(torch.from_numpy(ow.x).to(dev), torch.from_numpy(ow.w).to(dev), R2_H)
+        starts = sq.r2_random_hadamard(torch.from_numpy(ow.signs).to(dev))   # [32, d, d]
+        R0 = starts[0].contiguous()
+        R32 = R0.float()
+        prob.loss_grad(R32)
+        torch.cuda.synchronize()
+        tlg, tlearn = [], []
+        iters = 10
+        for _ in range(max(3, args.steps)):
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            prob.loss_grad(R32)
+            e1.record(stream)
+            prob.learn(R0, R2_ALPHA, iters)
+            e2.record(stream)
+            tlg.append((e0, e1))
+            tlearn.append((e1, e2))
+        torch.cuda.synchronize()
+        mlg, mlearn = ms(tlg), ms(tlearn)
+        # the learner as the page runs it: 120 steps from the first draw,
+        # against all 32 draws
+        draws = torch.cat([prob.loss_grad(starts[i].float(), grad=False)[0]
+                           for i in range(starts.shape[0])]).cpu()
+        R, losses = prob.learn(R0, R2_ALPHA, 120)
+        L = losses.cpu()
+        orth = float(sq.orth_error(R)[0])
+        r2_info = {"workload": ow.name, "alpha": R2_ALPHA,
+                   "loss_grad_us": mlg * 1e3,
+                   "loss_grad_f32_TFLOPs": R2_F32_FLOPS / (mlg * 1e-3) / 1e12,
+                   "learner_step_us": mlearn * 1e3 / iters,
+                   "loss_first_draw": float(L[0]), "loss_after_120": float(L[-1]),
+                   "best_of_32_draws": float(draws.min()), "worst_of_32_draws": float(draws.max()),
+                   "orth_error_after_120": orth}
+        del prob, starts
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
-                clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info, a8=a8_info)
+                clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info, a8=a8_info,
+                r2=r2_info)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -411,7 +463,8 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
                  "decode_gemm_m1", "decode_gemm_m16", "decode_gemm_m64", "rotate_quant_r4",
                  "kv_rotate_quant",
-                 "swiglu_rotate_quant_r4", "kv4_decode", "kv8_decode", "kv_rotate_quant8")
+                 "swiglu_rotate_quant_r4", "kv4_decode", "kv8_decode", "kv_rotate_quant8",
+                 "r2_loss_grad")
 
 
 def run_profile_case(case, steps, warmup):
@@ -447,6 +500,11 @@ def run_profile_case(case, steps, warmup):
                                 dw.v_zero, dw.lengths)]
         o = sq.kv4_decode_attention(*t, dw.S_max)
         fn = lambda: sq.kv4_decode_attention(*t, dw.S_max, out=o)  # noqa: E731
+    elif case == "r2_loss_grad":
+        ow = W.o_proj_layer()
+        prob = sq.R2Problem(torch.from_numpy(ow.x).cuda(), torch.from_numpy(ow.w).cuda(), R2_H)
+        R32 = sq.r2_random_hadamard(torch.from_numpy(ow.signs[:1]).cuda())[0].float()
+        fn = lambda: prob.loss_grad(R32)  # noqa: E731
     elif case == "kv8_decode":
         dw = W.kv8_decode()
         t = [x.cuda() for x in (dw.q, dw.k_cache, dw.k_scale, dw.k_zero, dw.v_cache, dw.v_scale,
@@ -655,6 +713,9 @@ def main():
             "w4a8": (dict(r["a8"], rotate_quant8_frac_of_hbm=r["a8"]["rotate_quant8_GB/s"] / hbm,
                           gemm_frac_of_int8_peak=r["a8"]["gemm_TOPS"] / int8_peak)
                      if r["a8"] else None),
+            "r2_cayley_learner": (dict(r["r2"], bound="alu", f32_peak_TFLOPs=F32_PEAK,
+                                       frac_of_f32_peak=r["r2"]["loss_grad_f32_TFLOPs"] / F32_PEAK)
+                                  if r["r2"] else None),
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,

@@ -312,6 +312,84 @@ sq_status sq_kv_rotate_quant8(const void* q, const void* k, const void* v, int64
 sq_status sq_kv8_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero,
                          int64_t T, int h, int d, void* out_bf16, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Cayley SGD for the head-wise rotation R2.
+ *
+ * Source: "SpinQuant, Reproduced", Q6.  R2 (d x d, one matrix shared by the
+ * heads) is learned against one layer's own W4A4 output error with the
+ * weights frozen, by the Cayley transform R' = (I - a/2 Y)^-1 (I + a/2 Y) R
+ * of a skew-symmetric Y, with a straight-through estimator through the
+ * quantizers.  The page leaves open how Y comes from the gradient and which
+ * linear is measured; this library takes Y = R G^T - G R^T (G the Euclidean
+ * gradient, a descent step) and the o_proj linear with its input rotated
+ * head-wise:
+ *     loss = ||Q(x R) Q(w R)^T - x w^T||_F^2 / ||x w^T||_F^2
+ * where x R rotates each group of d consecutive channels of every row by R,
+ * Q is per-row symmetric INT4 (scale = max|row| / 7, code = clamp(rint(v /
+ * scale), -8, 7)) per token of x and per output channel of w, and the
+ * gradient G passes each quantizer's output gradient to its input.
+ * ------------------------------------------------------------------------- */
+
+/* sq_r2_workspace_bytes -- device scratch of one (x, w) problem: T tokens,
+ * H heads of d channels, N outputs.  0 for an unsupported shape (d == 128,
+ * T and N multiples of 16, H * d <= 65536) or without a device. */
+size_t sq_r2_workspace_bytes(int64_t T, int H, int d, int64_t N);
+
+/* sq_r2_prepare -- compute y0 = x w^T and ||y0||^2 into the workspace; call
+ * once per (x, w) before sq_r2_loss_grad.  x device float32 [T][H d], w
+ * device float32 [N][H d], 16-byte aligned, owned by the caller and left
+ * unchanged.  The workspace (16-byte aligned, at least
+ * sq_r2_workspace_bytes()) belongs to this problem until the caller frees
+ * it; one call at a time per workspace. */
+sq_status sq_r2_prepare(const float* x, const float* w, int64_t T, int H, int d, int64_t N,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* sq_r2_loss_grad -- the loss above at R (device float32 [d][d]) into *loss
+ * (device float64), and, when grad is not NULL, its straight-through gradient
+ * with respect to R into grad (device float64 [d][d]).  x, w and the
+ * workspace as given to sq_r2_prepare.  Errors: shape and pointer checks as
+ * sq_r2_prepare; a device-side wait that runs out is reported by
+ * sq_device_status(). */
+sq_status sq_r2_loss_grad(const float* x, const float* w, const float* R, int64_t T, int H, int d,
+                          int64_t N, double* loss, double* grad, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* sq_r2_cayley_learn -- `iters` Cayley SGD steps R <- cayley(R, grad at R,
+ * alpha) from R0 (device float64 [d][d], orthogonal), the loss and gradient
+ * as sq_r2_loss_grad.  R (device float64 [d][d]; may be R0) receives the
+ * result; losses (device float64 [iters + 1]) the loss at each iterate, the
+ * last at the result.  The workspace must have been through sq_r2_prepare
+ * for (x, w).  iters >= 0. */
+sq_status sq_r2_cayley_learn(const float* x, const float* w, const double* R0, int64_t T, int H,
+                             int d, int64_t N, double alpha, int iters, double* R,
+                             double* losses, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* sq_cayley_workspace_bytes -- device scratch of sq_cayley_update (0 for
+ * n outside 1..128 or batch < 1). */
+size_t sq_cayley_workspace_bytes(int n, int batch);
+
+/* sq_cayley_update -- for each of `batch` n x n matrices (row-major, float64,
+ * device, 16-byte aligned):
+ *     Y = R G^T - G R^T,  R_out = (I - alpha/2 Y)^-1 (I + alpha/2 Y) R
+ * in float64 (Gauss-Jordan elimination; I - alpha/2 Y has symmetric part I,
+ * so no pivoting is needed).  R_out may be R.  R_out_f32, if not NULL,
+ * receives a float32 copy.  1 <= n <= 128; batch == 0 is a no-op. */
+sq_status sq_cayley_update(const double* R, const double* G, double alpha, int n, int batch,
+                           double* R_out, float* R_out_f32, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* sq_r2_random_hadamard -- the random Hadamards the learner starts from and
+ * is compared with: R_b = diag(s_b) H_d / sqrt(d) (Sylvester H_d, entry
+ * (i, j) = (-1)^popcount(i & j)) for each sign vector s_b of `signs`
+ * (device int8 [batch][d], negative means -1), into R (device float64
+ * [batch][d][d]).  d a power of 2, 1 <= d <= 128. */
+sq_status sq_r2_random_hadamard(const int8_t* signs, int d, int batch, double* R, void* stream);
+
+/* sq_orth_error -- out[b] = ||R_b^T R_b - I||_F (float64, device) for each
+ * of `batch` n x n float64 matrices; 1 <= n <= 128. */
+sq_status sq_orth_error(const double* R, int n, int batch, double* out, void* stream);
+
 /* sq_rope_tables -- the cos/sin tables the KV call reads:
  *     angle(p, i) = p * theta^(-2i/d),  cos[p][i] = float(cos(angle)),
  *     sin[p][i] = float(sin(angle)),  evaluated in double precision on the

@@ -11,11 +11,17 @@ Entry points (same names as the C ABI without the ``sq_`` prefix):
   w4a4_workspace_bytes, kv_rotate_quant,
   kv_dequant, kv4_decode_attention, kv4_decode_workspace_bytes, rope_tables,
   kv_rotate_quant8, kv8_dequant, kv8_decode_attention,
+  R2Problem (sq_r2_prepare / sq_r2_loss_grad / sq_r2_cayley_learn), cayley_update,
+  r2_random_hadamard, orth_error,
   device_status, debug_set_spin_limit.
 """
 from __future__ import annotations
 
 from .binding import (  # noqa: F401
+    R2Problem,
+    cayley_update,
+    orth_error,
+    r2_random_hadamard,
     SQ_IN_BF16,
     SQ_IN_F32,
     SQ_OUT_BF16,

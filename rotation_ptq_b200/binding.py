@@ -65,6 +65,25 @@ for _f in (lib.sq_kv_rotate_quant, lib.sq_kv_rotate_quant8):
 for _f in (lib.sq_kv_dequant, lib.sq_kv8_dequant):
     _f.restype = _i32
     _f.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]
+lib.sq_r2_workspace_bytes.restype = ctypes.c_size_t
+lib.sq_r2_workspace_bytes.argtypes = [_i64, _i32, _i32, _i64]
+lib.sq_r2_prepare.restype = _i32
+lib.sq_r2_prepare.argtypes = [_vp, _vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_size_t, _vp]
+lib.sq_r2_loss_grad.restype = _i32
+lib.sq_r2_loss_grad.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i64, _vp, _vp, _vp,
+                                ctypes.c_size_t, _vp]
+lib.sq_r2_cayley_learn.restype = _i32
+lib.sq_r2_cayley_learn.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i64, ctypes.c_double, _i32,
+                                   _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.sq_cayley_workspace_bytes.restype = ctypes.c_size_t
+lib.sq_cayley_workspace_bytes.argtypes = [_i32, _i32]
+lib.sq_cayley_update.restype = _i32
+lib.sq_cayley_update.argtypes = [_vp, _vp, ctypes.c_double, _i32, _i32, _vp, _vp, _vp,
+                                 ctypes.c_size_t, _vp]
+lib.sq_r2_random_hadamard.restype = _i32
+lib.sq_r2_random_hadamard.argtypes = [_vp, _i32, _i32, _vp, _vp]
+lib.sq_orth_error.restype = _i32
+lib.sq_orth_error.argtypes = [_vp, _i32, _i32, _vp, _vp]
 lib.sq_rope_tables.restype = _i32
 lib.sq_rope_tables.argtypes = [ctypes.c_double, _i32, _i32, _vp, _vp, _vp]
 lib.sq_device_status.restype = _i32
@@ -427,6 +446,104 @@ def kv8_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, ou
     st = lib.sq_kv8_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, d,
                             out.data_ptr(), _stream(cache))
     _check(st, "sq_kv8_dequant")
+    return out
+
+
+class R2Problem:
+    """One o_proj layer for the Cayley R2 learner: x float32 [T, H*d], w
+    float32 [N, H*d] on the GPU, and the prepared workspace
+    (``sq_r2_prepare``)."""
+
+    def __init__(self, x: torch.Tensor, w: torch.Tensor, H: int, d: int = 128):
+        _need_cuda(x, w)
+        if x.dtype != torch.float32 or w.dtype != torch.float32:
+            raise ValueError("x and w must be float32")
+        self.x, self.w = x.contiguous(), w.contiguous()
+        self.T, self.N, self.H, self.d = x.shape[0], w.shape[0], H, d
+        need = int(lib.sq_r2_workspace_bytes(self.T, H, d, self.N))
+        if need == 0:
+            raise ValueError("unsupported R2 problem shape T=%d H=%d d=%d N=%d"
+                             % (self.T, H, d, self.N))
+        self.ws = torch.empty((need,), dtype=torch.uint8, device=x.device)
+        st = lib.sq_r2_prepare(self.x.data_ptr(), self.w.data_ptr(), self.T, H, d, self.N,
+                               self.ws.data_ptr(), need, _stream(x))
+        _check(st, "sq_r2_prepare")
+
+    def loss_grad(self, R: torch.Tensor, grad: bool = True):
+        """Loss (device float64 [1]) and, with grad, G (device float64 [d, d]) at R
+        (float32 [d, d]) (``sq_r2_loss_grad``)."""
+        _need_cuda(R)
+        R = R.to(torch.float32).contiguous()
+        loss = torch.empty((1,), dtype=torch.float64, device=R.device)
+        G = torch.empty((self.d, self.d), dtype=torch.float64, device=R.device) if grad else None
+        st = lib.sq_r2_loss_grad(self.x.data_ptr(), self.w.data_ptr(), R.data_ptr(), self.T,
+                                 self.H, self.d, self.N, loss.data_ptr(), _ptr(G),
+                                 self.ws.data_ptr(), self.ws.numel(), _stream(R))
+        _check(st, "sq_r2_loss_grad")
+        return loss, G
+
+    def learn(self, R0: torch.Tensor, alpha: float, iters: int):
+        """iters Cayley SGD steps from R0 (float64 [d, d]) (``sq_r2_cayley_learn``).
+        Returns (R float64 [d, d], losses float64 [iters + 1]) on the device."""
+        _need_cuda(R0)
+        R0 = R0.to(torch.float64).contiguous()
+        R = torch.empty_like(R0)
+        losses = torch.empty((iters + 1,), dtype=torch.float64, device=R0.device)
+        st = lib.sq_r2_cayley_learn(self.x.data_ptr(), self.w.data_ptr(), R0.data_ptr(), self.T,
+                                    self.H, self.d, self.N, float(alpha), int(iters),
+                                    R.data_ptr(), losses.data_ptr(), self.ws.data_ptr(),
+                                    self.ws.numel(), _stream(R0))
+        _check(st, "sq_r2_cayley_learn")
+        return R, losses
+
+
+def cayley_update(R: torch.Tensor, G: torch.Tensor, alpha: float, out: torch.Tensor = None,
+                  out_f32: torch.Tensor = None):
+    """(I - alpha/2 Y)^-1 (I + alpha/2 Y) R with Y = R G^T - G R^T, float64, for
+    R, G [n, n] or [batch, n, n] (``sq_cayley_update``)."""
+    _need_cuda(R, G)
+    if R.dtype != torch.float64 or G.dtype != torch.float64 or R.shape != G.shape:
+        raise ValueError("R and G must be float64 of the same shape")
+    R, G = R.contiguous(), G.contiguous()
+    n = R.shape[-1]
+    batch = R.numel() // (n * n)
+    if out is None:
+        out = torch.empty_like(R)
+    need = int(lib.sq_cayley_workspace_bytes(n, max(batch, 1)))
+    ws = torch.empty((max(need, 16),), dtype=torch.uint8, device=R.device)
+    st = lib.sq_cayley_update(R.data_ptr(), G.data_ptr(), float(alpha), n, batch, out.data_ptr(),
+                              _ptr(out_f32), ws.data_ptr(), ws.numel(), _stream(R))
+    _check(st, "sq_cayley_update")
+    return out
+
+
+def r2_random_hadamard(signs: torch.Tensor) -> torch.Tensor:
+    """diag(s) H_d / sqrt(d) (float64) for signs int8 [d] or [batch, d]
+    (``sq_r2_random_hadamard``)."""
+    _need_cuda(signs)
+    if signs.dtype != torch.int8:
+        raise ValueError("signs must be int8")
+    signs = signs.contiguous()
+    d = signs.shape[-1]
+    batch = signs.numel() // d
+    R = torch.empty(tuple(signs.shape[:-1]) + (d, d), dtype=torch.float64, device=signs.device)
+    st = lib.sq_r2_random_hadamard(signs.data_ptr(), d, batch, R.data_ptr(), _stream(signs))
+    _check(st, "sq_r2_random_hadamard")
+    return R
+
+
+def orth_error(R: torch.Tensor) -> torch.Tensor:
+    """||R^T R - I||_F per matrix of R [n, n] or [batch, n, n] (float64)
+    (``sq_orth_error``)."""
+    _need_cuda(R)
+    if R.dtype != torch.float64:
+        raise ValueError("R must be float64")
+    R = R.contiguous()
+    n = R.shape[-1]
+    batch = R.numel() // (n * n)
+    out = torch.empty((batch,), dtype=torch.float64, device=R.device)
+    st = lib.sq_orth_error(R.data_ptr(), n, batch, out.data_ptr(), _stream(R))
+    _check(st, "sq_orth_error")
     return out
 
 

@@ -1,0 +1,695 @@
+// Cayley SGD for the head-wise rotation R2, sm_100a.
+//
+// "SpinQuant, Reproduced", Q6: R2 (d x d, d = 128, one matrix shared by all
+// heads) is learned against one layer's own W4A4 output error with the
+// weights frozen.  The update is the Cayley transform
+//     R' = (I - a/2 Y)^-1 (I + a/2 Y) R,   Y^T = -Y,
+// which keeps R orthogonal, and round() passes the gradient straight through
+// (a straight-through estimator).  Readings of what the page leaves open:
+// Y = R G^T - G R^T from the Euclidean gradient G, so that
+// R' = R - a (G - R G^T R) + O(a^2) is a descent step; the layer is o_proj,
+// whose input x [T][H d] and weight w [N][H d] are both rotated head-wise by
+// R (x' w'^T = x w^T at full precision):
+//     loss = ||Q(x R) Q(w R)^T - x w^T||^2 / ||x w^T||^2,
+//     E = Q(xR) Q(wR)^T - x w^T,  g_xr = 2/den E Q(wR),  g_wr = 2/den E^T Q(xR),
+//     G = sum_h x_h^T g_xr,h + w_h^T g_wr,h.
+// Q is per-row symmetric INT4: scale = max|row| / 7, code = clamp(rint(v /
+// scale), -8, 7), per token for activations, per output channel for weights.
+//
+// One loss-and-gradient evaluation on the device:
+//   xr = x_s R, wr = w_s R          fp32 GEMM (x_s = x viewed as [T H][d])
+//   quantize the rows of xr, wr     packed codes, scales, dequantized values
+//   acc = codes_a codes_w^T         INT4 tensor-core GEMM, exact int32 sums
+//   E = acc sa sw - y0, sum E^2     elementwise, fixed-order partial sums
+//   g_xr = E qw, g_wr = E^T qa      fp32 GEMMs (into the xr, wr buffers)
+//   G = x_s^T g_xr,s + w_s^T g_wr,s fp32 split-K GEMMs, partials summed in f64
+// The Cayley step runs in float64: A = I - a/2 (R G^T - G R^T) and
+// B = (I + a/2 Y) R = 2R - A R, then Gauss-Jordan elimination of A with B as
+// right-hand side in one CTA.  A's symmetric part is I, and so is at least
+// that of every Schur complement, so each pivot is >= 1: no pivoting needed.
+//
+// The fp32 GEMM is a CUDA-core kernel (128 x 128 tiles, 8 x 8 outputs per
+// thread, double-buffered shared memory): these products are float by float
+// and the page's probe needs float accuracy, not a low-precision format.
+#include <math.h>
+
+#include "sq_device.cuh"
+#include "sq_host.h"
+
+namespace sq {
+namespace r2 {
+
+// ---------------------------------------------------------------- fp32 GEMM
+
+constexpr int GM = 128, GN = 128, GK = 16, GT = 256, GPAD = 4;
+
+// C[m][n] = alpha sum_k A(m, k) B(k, n) + beta C[m][n] over k in this CTA's
+// chunk [z kchunk, (z + 1) kchunk); with more than one chunk each writes its
+// raw sums to C + z * part_stride (alpha 1, beta 0).
+//   TA = false: A(m, k) = A[m lda + k];  TA = true: A(m, k) = A[k lda + m].
+//   TB = false: B(k, n) = B[k ldb + n];  TB = true: B(k, n) = B[n ldb + k].
+// Requirements (checked by the host): K chunk a multiple of 16; lda, ldb,
+// ldc multiples of 4 and 16-byte aligned bases; M % 4 == 0 when TA, N % 4
+// == 0.  Rows and columns past M and N are read as zero and not written.
+template <bool TA, bool TB>
+__global__ void __launch_bounds__(GT, 2) sgemm_kernel(int M, int N, int K, const float* __restrict__ A,
+                                                   int64_t lda, const float* __restrict__ B,
+                                                   int64_t ldb, float* __restrict__ C, int64_t ldc,
+                                                   float alpha, float beta, int kchunk,
+                                                   int64_t part_stride) {
+  __shared__ __align__(16) float As[2][GK][GM + GPAD];
+  __shared__ __align__(16) float Bs[2][GK][GN + GPAD];
+  const int tid = threadIdx.x;
+  const int m0 = blockIdx.y * GM, n0 = blockIdx.x * GN;
+  const int kb0 = blockIdx.z * kchunk;
+  const int kb1 = min(K, kb0 + kchunk);
+  if (gridDim.z > 1) C += blockIdx.z * part_stride;
+  const int nk = (kb1 - kb0) / GK;
+
+  float4 ra[2], rb[2];
+  auto load_a = [&](int kb) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int idx = tid + GT * i;
+      if (!TA) {
+        const int row = idx >> 2, kq = idx & 3;
+        ra[i] = m0 + row < M ? __ldg(reinterpret_cast<const float4*>(
+                                   A + static_cast<int64_t>(m0 + row) * lda + kb + 4 * kq))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const int kr = idx >> 5, mq = idx & 31;
+        ra[i] = m0 + 4 * mq < M ? __ldg(reinterpret_cast<const float4*>(
+                                      A + static_cast<int64_t>(kb + kr) * lda + m0 + 4 * mq))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  auto load_b = [&](int kb) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int idx = tid + GT * i;
+      if (!TB) {
+        const int kr = idx >> 5, nq = idx & 31;
+        rb[i] = n0 + 4 * nq < N ? __ldg(reinterpret_cast<const float4*>(
+                                      B + static_cast<int64_t>(kb + kr) * ldb + n0 + 4 * nq))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const int row = idx >> 2, kq = idx & 3;
+        rb[i] = n0 + row < N ? __ldg(reinterpret_cast<const float4*>(
+                                   B + static_cast<int64_t>(n0 + row) * ldb + kb + 4 * kq))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int idx = tid + GT * i;
+      if (!TA) {
+        const int row = idx >> 2, kq = idx & 3;
+        As[buf][4 * kq + 0][row] = ra[i].x;
+        As[buf][4 * kq + 1][row] = ra[i].y;
+        As[buf][4 * kq + 2][row] = ra[i].z;
+        As[buf][4 * kq + 3][row] = ra[i].w;
+      } else {
+        const int kr = idx >> 5, mq = idx & 31;
+        *reinterpret_cast<float4*>(&As[buf][kr][4 * mq]) = ra[i];
+      }
+      if (!TB) {
+        const int kr = idx >> 5, nq = idx & 31;
+        *reinterpret_cast<float4*>(&Bs[buf][kr][4 * nq]) = rb[i];
+      } else {
+        const int row = idx >> 2, kq = idx & 3;
+        Bs[buf][4 * kq + 0][row] = rb[i].x;
+        Bs[buf][4 * kq + 1][row] = rb[i].y;
+        Bs[buf][4 * kq + 2][row] = rb[i].z;
+        Bs[buf][4 * kq + 3][row] = rb[i].w;
+      }
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int ty = tid >> 4, tx = tid & 15;
+  if (nk > 0) {
+    load_a(kb0);
+    load_b(kb0);
+    store(0);
+  }
+  __syncthreads();
+  for (int kt = 0; kt < nk; ++kt) {
+    const int cur = kt & 1;
+    if (kt + 1 < nk) {
+      load_a(kb0 + (kt + 1) * GK);
+      load_b(kb0 + (kt + 1) * GK);
+    }
+#pragma unroll
+    for (int kk = 0; kk < GK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][kk][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][kk][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][kk][64 + 4 * tx]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    if (kt + 1 < nk) store(cur ^ 1);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    if (m >= M) continue;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int n = n0 + 64 * h + 4 * tx;
+      if (n >= N) continue;
+      float* cp = C + static_cast<int64_t>(m) * ldc + n;
+      float4 v = make_float4(alpha * acc[i][4 * h], alpha * acc[i][4 * h + 1],
+                             alpha * acc[i][4 * h + 2], alpha * acc[i][4 * h + 3]);
+      if (beta != 0.f) {
+        const float4 o = *reinterpret_cast<const float4*>(cp);
+        v.x += beta * o.x;
+        v.y += beta * o.y;
+        v.z += beta * o.z;
+        v.w += beta * o.w;
+      }
+      *reinterpret_cast<float4*>(cp) = v;
+    }
+  }
+}
+
+// out[i] = sum_p part[p * n + i] in float64, partials in order.
+__global__ void sum_partials_kernel(const float* __restrict__ part, int P, int64_t n,
+                                    double* __restrict__ out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += static_cast<double>(__ldg(part + p * n + i));
+    out[i] = s;
+  }
+}
+
+// ------------------------------------------------------------ quantization
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < (blockDim.x >> 5); ++i) r = fmaxf(r, red[i]);
+  __syncthreads();
+  return r;
+}
+
+// Per-row symmetric INT4 of src [rows][K] (K % 8 == 0): scale = max|row| / 7
+// (1 for an all-zero row), code = clamp(rint(v / scale), -8, 7) with the
+// quotient rounded as IEEE float32 division.  Writes the packed codes
+// [rows][K/2] (element 2j in the low nibble of byte j), the scales, and the
+// dequantized values code * scale [rows][K].  One CTA per row.
+__global__ void __launch_bounds__(256) quant_rows_kernel(const float* __restrict__ src,
+                                                         int64_t rows, int K,
+                                                         uint8_t* __restrict__ packed,
+                                                         float* __restrict__ scale_out,
+                                                         float* __restrict__ deq) {
+  __shared__ float red[8];
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float* row = src + r * K;
+    float mx = 0.f;
+    for (int k = 4 * threadIdx.x; k < K; k += 4 * blockDim.x) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + k));
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    mx = block_max(mx, red);
+    float s = __fdiv_rn(mx, 7.0f);
+    if (s == 0.f) s = 1.0f;
+    if (threadIdx.x == 0) scale_out[r] = s;
+    for (int k = 8 * threadIdx.x; k < K; k += 8 * blockDim.x) {
+      const float4 v0 = __ldg(reinterpret_cast<const float4*>(row + k));
+      const float4 v1 = __ldg(reinterpret_cast<const float4*>(row + k + 4));
+      const float xv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float dv[8];
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float c = fminf(fmaxf(rintf(__fdiv_rn(xv[e], s)), -8.f), 7.f);
+        dv[e] = c * s;
+        word |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * e);
+      }
+      *reinterpret_cast<uint32_t*>(packed + r * (K / 2) + k / 2) = word;
+      float4* dp = reinterpret_cast<float4*>(deq + r * K + k);
+      dp[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+      dp[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+    }
+  }
+}
+
+// ------------------------------------------------------------- loss terms
+
+__device__ __forceinline__ double block_sum_d(double v, double* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  double r = 0.0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < (blockDim.x >> 5); ++i) r += red[i];
+  return r;                                   // valid in thread 0
+}
+
+// E = acc sa[t] sw[n] - y0[t][n] written as float over the int32 sums, and
+// this block's sum of E^2 (float64; a fixed grid gives a fixed order).
+// N % 4 == 0.
+__global__ void __launch_bounds__(256) r2_error_kernel(int32_t* __restrict__ acc,
+                                                       const float* __restrict__ sa,
+                                                       const float* __restrict__ sw,
+                                                       const float* __restrict__ y0, int64_t T,
+                                                       int N, double* __restrict__ part) {
+  __shared__ double red[8];
+  const int64_t n4 = T * N / 4;
+  double s = 0.0;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = (4 * i) / N;
+    const int n = static_cast<int>(4 * i - t * N);
+    const int4 a = reinterpret_cast<const int4*>(acc)[i];
+    const float4 y = __ldg(reinterpret_cast<const float4*>(y0) + i);
+    const float4 w = __ldg(reinterpret_cast<const float4*>(sw + n));
+    const float st = __ldg(sa + t);
+    float4 e;
+    e.x = static_cast<float>(a.x) * st * w.x - y.x;
+    e.y = static_cast<float>(a.y) * st * w.y - y.y;
+    e.z = static_cast<float>(a.z) * st * w.z - y.z;
+    e.w = static_cast<float>(a.w) * st * w.w - y.w;
+    reinterpret_cast<float4*>(acc)[i] = e;
+    s += static_cast<double>(e.x) * e.x + static_cast<double>(e.y) * e.y +
+         static_cast<double>(e.z) * e.z + static_cast<double>(e.w) * e.w;
+  }
+  s = block_sum_d(s, red);
+  if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+
+// This block's sum of x^2 over x [n4 * 4] (float64).
+__global__ void __launch_bounds__(256) sumsq_kernel(const float* __restrict__ x, int64_t n4,
+                                                    double* __restrict__ part) {
+  __shared__ double red[8];
+  double s = 0.0;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(x) + i);
+    s += static_cast<double>(v.x) * v.x + static_cast<double>(v.y) * v.y +
+         static_cast<double>(v.z) * v.z + static_cast<double>(v.w) * v.w;
+  }
+  s = block_sum_d(s, red);
+  if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+
+// out = sum_p part[p] (in order), divided by *den when den is given.
+__global__ void finish_kernel(const double* __restrict__ part, int P, const double* den,
+                              double* out) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  double s = 0.0;
+  for (int p = 0; p < P; ++p) s += part[p];
+  *out = den ? s / *den : s;
+}
+
+// G[i] = 2 / den * sum_p part[p * n + i] (float64, partials in order).
+__global__ void grad_sum_kernel(const float* __restrict__ part, int P, int64_t n,
+                                const double* __restrict__ den, double* __restrict__ G) {
+  const double f = 2.0 / *den;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += static_cast<double>(__ldg(part + p * n + i));
+    G[i] = f * s;
+  }
+}
+
+// ------------------------------------------------------------ Cayley step
+
+// A = I - h (R G^T - G R^T) for each of the batch's n x n matrices (h =
+// alpha / 2); each off-diagonal pair is computed once and written with both
+// signs, so A - I is exactly skew-symmetric.
+__global__ void cayley_a_kernel(const double* __restrict__ R, const double* __restrict__ G,
+                                double h, int n, double* __restrict__ A) {
+  const int64_t off = static_cast<int64_t>(blockIdx.y) * n * n;
+  R += off;
+  G += off;
+  A += off;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n * n;
+       idx += gridDim.x * blockDim.x) {
+    const int i = idx / n, j = idx - i * n;
+    if (i == j) {
+      A[idx] = 1.0;
+    } else if (i < j) {
+      double y = 0.0;
+      for (int l = 0; l < n; ++l) y += R[i * n + l] * G[j * n + l] - G[i * n + l] * R[j * n + l];
+      A[idx] = -h * y;
+      A[j * n + i] = h * y;
+    }
+  }
+}
+
+// B = (I + h Y) R = 2 R - A R.
+__global__ void cayley_b_kernel(const double* __restrict__ A, const double* __restrict__ R, int n,
+                                double* __restrict__ B) {
+  const int64_t off = static_cast<int64_t>(blockIdx.y) * n * n;
+  R += off;
+  A += off;
+  B += off;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n * n;
+       idx += gridDim.x * blockDim.x) {
+    const int i = idx / n, j = idx - i * n;
+    double s = 2.0 * R[idx];
+    for (int l = 0; l < n; ++l) s -= A[i * n + l] * R[l * n + j];
+    B[idx] = s;
+  }
+}
+
+constexpr int SOLVE_THREADS = 1024;
+constexpr int MAX_N = 128;
+
+// R_out = A^-1 B by Gauss-Jordan elimination, one CTA per matrix (n <= 128):
+// A in shared memory (row stride n + 1), B in registers, thread t holding
+// column t % 128 of rows t / 128 + 8 r.  Pivots are >= 1 (see the top).
+__global__ void __launch_bounds__(SOLVE_THREADS) cayley_solve_kernel(
+    const double* __restrict__ Ain, const double* __restrict__ Bin, int n,
+    double* __restrict__ R_out, float* __restrict__ R32) {
+  extern __shared__ double cs_smem[];
+  const int64_t off = static_cast<int64_t>(blockIdx.x) * n * n;
+  const int ld = n + 1;
+  double* As = cs_smem;
+  double* colk = As + n * ld;
+  double* pivB = colk + n;
+  const int t = threadIdx.x, j = t & (MAX_N - 1), rg = t >> 7;
+  const bool live = j < n;
+  double bv[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int i = rg + 8 * r;
+    bv[r] = 0.0;
+    if (live && i < n) {
+      bv[r] = Bin[off + i * n + j];
+      As[i * ld + j] = Ain[off + i * n + j];
+    }
+  }
+  __syncthreads();
+  for (int k = 0; k < n; ++k) {
+    if (j == k) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int i = rg + 8 * r;
+        if (i < n) colk[i] = As[i * ld + k];
+      }
+    }
+    __syncthreads();
+    const double piv = colk[k];
+    if (live && rg == (k & 7)) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        if (r == (k >> 3)) {
+          As[k * ld + j] = As[k * ld + j] / piv;
+          bv[r] = bv[r] / piv;
+          pivB[j] = bv[r];
+        }
+      }
+    }
+    __syncthreads();
+    if (live) {
+      const double akj = As[k * ld + j], bkj = pivB[j];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int i = rg + 8 * r;
+        if (i < n && i != k) {
+          const double f = colk[i];
+          As[i * ld + j] -= f * akj;
+          bv[r] -= f * bkj;
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int i = rg + 8 * r;
+    if (live && i < n) {
+      R_out[off + i * n + j] = bv[r];
+      if (R32) R32[off + i * n + j] = static_cast<float>(bv[r]);
+    }
+  }
+}
+
+// out[b] = ||R_b^T R_b - I||_F (float64), one CTA per matrix.
+__global__ void __launch_bounds__(SOLVE_THREADS) orth_error_kernel(const double* __restrict__ R,
+                                                                   int n, double* __restrict__ out) {
+  __shared__ double red[32];
+  R += static_cast<int64_t>(blockIdx.x) * n * n;
+  double s = 0.0;
+  for (int idx = threadIdx.x; idx < n * n; idx += blockDim.x) {
+    const int i = idx / n, j = idx - i * n;
+    double p = i == j ? -1.0 : 0.0;
+    for (int l = 0; l < n; ++l) p += R[l * n + i] * R[l * n + j];
+    s += p * p;
+  }
+  s = block_sum_d(s, red);
+  if (threadIdx.x == 0) out[blockIdx.x] = sqrt(s);
+}
+
+// R_b = diag(s_b) H_d / sqrt(d) for each sign vector s_b (d a power of 2):
+// entry (i, j) is s_i (-1)^popcount(i & j) / sqrt(d) (Sylvester order).
+__global__ void random_hadamard_kernel(const int8_t* __restrict__ signs, int d, int batch,
+                                       double* __restrict__ R) {
+  const int64_t n = static_cast<int64_t>(batch) * d * d;
+  const double inv = 1.0 / sqrt(static_cast<double>(d));
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = idx / (static_cast<int64_t>(d) * d);
+    const int rem = static_cast<int>(idx - b * d * d);
+    const int i = rem / d, j = rem - i * d;
+    const double h = (__popc(i & j) & 1) ? -inv : inv;
+    R[idx] = signs[b * d + i] < 0 ? -h : h;
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+size_t cayley_workspace_bytes(int n, int batch);
+
+__global__ void to_f32_kernel(const double* __restrict__ src, int64_t n, float* __restrict__ dst) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = static_cast<float>(src[i]);
+}
+
+namespace {
+
+constexpr int LOSS_BLOCKS = 1024;          // fixed grid of the loss sums
+constexpr int GRAD_CHUNK = 1024;           // K chunk of the split-K gradient GEMMs
+
+size_t al(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+struct Layout {
+  size_t y0, E, xr, qa, aq, sa, wr, qw, wq, sw, gpart, lpart, den, gws, gws_bytes, r32, g64, cay,
+      total;
+  int Px, Pw;
+};
+
+Layout layout(int64_t T, int H, int d, int64_t N, int num_sms) {
+  const int64_t K = static_cast<int64_t>(H) * d;
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += al(bytes);
+    return at;
+  };
+  L.Px = static_cast<int>((T * H + GRAD_CHUNK - 1) / GRAD_CHUNK);
+  L.Pw = static_cast<int>((N * H + GRAD_CHUNK - 1) / GRAD_CHUNK);
+  L.y0 = take(T * N * 4);
+  L.E = take(T * N * 4);
+  L.xr = take(T * K * 4);
+  L.qa = take(T * K * 4);
+  L.aq = take(T * K / 2);
+  L.sa = take(T * 4);
+  L.wr = take(N * K * 4);
+  L.qw = take(N * K * 4);
+  L.wq = take(N * K / 2);
+  L.sw = take(N * 4);
+  L.gpart = take(static_cast<size_t>(L.Px + L.Pw) * d * d * 4);
+  L.lpart = take(LOSS_BLOCKS * 8);
+  L.den = take(8);
+  const size_t g1 = gemm::workspace_bytes(T, N, K, num_sms);
+  const size_t g2 = gemm::tail_workspace_bytes(T, N, K, num_sms);
+  L.gws_bytes = g1 > g2 ? g1 : g2;
+  L.gws = take(L.gws_bytes);
+  L.r32 = take(static_cast<size_t>(d) * d * 4);       // the learner's float32 R
+  L.g64 = take(static_cast<size_t>(d) * d * 8);       // ... its gradient
+  L.cay = take(cayley_workspace_bytes(d, 1));        // ... its Cayley scratch
+  L.total = o;
+  return L;
+}
+
+template <bool TA, bool TB>
+cudaError_t sgemm(int64_t M, int64_t N, int64_t K, const float* A, int64_t lda, const float* B,
+                  int64_t ldb, float* C, int64_t ldc, float alpha, float beta, int splits,
+                  int kchunk, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((N + GN - 1) / GN), static_cast<unsigned>((M + GM - 1) / GM),
+                  static_cast<unsigned>(splits));
+  sgemm_kernel<TA, TB><<<grid, GT, 0, s>>>(static_cast<int>(M), static_cast<int>(N),
+                                           static_cast<int>(K), A, lda, B, ldb, C, ldc, alpha, beta,
+                                           kchunk, M * ldc);
+  return cudaGetLastError();
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+size_t workspace_bytes(int64_t T, int H, int d, int64_t N, int num_sms) {
+  return layout(T, H, d, N, num_sms).total;
+}
+
+sq_status prepare(const float* x, const float* w, int64_t T, int H, int d, int64_t N, void* ws,
+                  int num_sms, cudaStream_t s) {
+  const Layout L = layout(T, H, d, N, num_sms);
+  const int64_t K = static_cast<int64_t>(H) * d;
+  float* y0 = at<float>(ws, L.y0);
+  cudaError_t e = sgemm<false, true>(T, N, K, x, K, w, K, y0, N, 1.f, 0.f, 1, static_cast<int>(K), s);
+  if (e != cudaSuccess) return host::cuda_fail("r2 y0 GEMM", e);
+  sumsq_kernel<<<LOSS_BLOCKS, 256, 0, s>>>(y0, T * N / 4, at<double>(ws, L.lpart));
+  finish_kernel<<<1, 32, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, nullptr,
+                                 at<double>(ws, L.den));
+  if (L.gws_bytes) {
+    e = cudaMemsetAsync(at<uint8_t>(ws, L.gws), 0, L.gws_bytes, s);
+    if (e != cudaSuccess) return host::cuda_fail("r2 workspace clear", e);
+  }
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("r2 prepare", e);
+}
+
+sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, int H, int d,
+                    int64_t N, double* loss, double* G, void* ws, int num_sms, uint32_t spin_limit,
+                    cudaStream_t s) {
+  const Layout L = layout(T, H, d, N, num_sms);
+  const int64_t K = static_cast<int64_t>(H) * d;
+  float* xr = at<float>(ws, L.xr);
+  float* wr = at<float>(ws, L.wr);
+  float* qa = at<float>(ws, L.qa);
+  float* qw = at<float>(ws, L.qw);
+  float* sa = at<float>(ws, L.sa);
+  float* sw = at<float>(ws, L.sw);
+  uint8_t* aq = at<uint8_t>(ws, L.aq);
+  uint8_t* wq = at<uint8_t>(ws, L.wq);
+  int32_t* acc = at<int32_t>(ws, L.E);
+  float* E = at<float>(ws, L.E);
+  const double* den = at<double>(ws, L.den);
+  cudaError_t e;
+  // head-wise rotations: [T H][d] x R and [N H][d] x R
+  if ((e = sgemm<false, false>(T * H, d, d, x, d, R, d, xr, d, 1.f, 0.f, 1, d, s)) != cudaSuccess ||
+      (e = sgemm<false, false>(N * H, d, d, w, d, R, d, wr, d, 1.f, 0.f, 1, d, s)) != cudaSuccess)
+    return host::cuda_fail("r2 rotation GEMM", e);
+  const int qgrid_a = static_cast<int>(T < 8 * num_sms ? T : 8 * num_sms);
+  const int qgrid_w = static_cast<int>(N < 8 * num_sms ? N : 8 * num_sms);
+  quant_rows_kernel<<<qgrid_a, 256, 0, s>>>(xr, T, static_cast<int>(K), aq, sa, qa);
+  quant_rows_kernel<<<qgrid_w, 256, 0, s>>>(wr, N, static_cast<int>(K), wq, sw, qw);
+  if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 quantize", e);
+  // exact integer products on the tensor cores
+  sq_status st = gemm::run(aq, sa, wq, sw, T, N, K, acc, 1, L.gws_bytes ? at<void>(ws, L.gws) : nullptr,
+                           L.gws_bytes, s, spin_limit, num_sms, nullptr);
+  if (st != SQ_OK) return st;
+  r2_error_kernel<<<LOSS_BLOCKS, 256, 0, s>>>(acc, sa, sw, at<float>(ws, L.y0), T,
+                                              static_cast<int>(N), at<double>(ws, L.lpart));
+  finish_kernel<<<1, 32, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, den, loss);
+  if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 loss", e);
+  if (!G) return SQ_OK;
+  // straight-through gradients of the rotated operands (the 2 / den factor
+  // is applied to G), into the rotation buffers
+  if ((e = sgemm<false, false>(T, K, N, E, N, qw, K, xr, K, 1.f, 0.f, 1, static_cast<int>(N), s)) !=
+          cudaSuccess ||
+      (e = sgemm<true, false>(N, K, T, E, N, qa, K, wr, K, 1.f, 0.f, 1, static_cast<int>(T), s)) !=
+          cudaSuccess)
+    return host::cuda_fail("r2 gradient GEMM", e);
+  // G = x_s^T g_xr,s + w_s^T g_wr,s, split over the long reduction
+  float* gp = at<float>(ws, L.gpart);
+  if ((e = sgemm<true, false>(d, d, T * H, x, d, xr, d, gp, d, 1.f, 0.f, L.Px, GRAD_CHUNK, s)) !=
+          cudaSuccess ||
+      (e = sgemm<true, false>(d, d, N * H, w, d, wr, d, gp + static_cast<int64_t>(L.Px) * d * d, d,
+                              1.f, 0.f, L.Pw, GRAD_CHUNK, s)) != cudaSuccess)
+    return host::cuda_fail("r2 G GEMM", e);
+  grad_sum_kernel<<<(d * d + 255) / 256, 256, 0, s>>>(gp, L.Px + L.Pw,
+                                                       static_cast<int64_t>(d) * d, den, G);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("r2 gradient sum", e);
+}
+
+size_t cayley_workspace_bytes(int n, int batch) {
+  return 2 * static_cast<size_t>(batch) * n * n * sizeof(double);
+}
+
+sq_status cayley_update(const double* R, const double* G, double alpha, int n, int batch,
+                        double* R_out, float* R32, void* ws, cudaStream_t s) {
+  double* A = static_cast<double*>(ws);
+  double* B = A + static_cast<int64_t>(batch) * n * n;
+  const dim3 grid((n * n + 255) / 256, batch);
+  cayley_a_kernel<<<grid, 256, 0, s>>>(R, G, 0.5 * alpha, n, A);
+  cayley_b_kernel<<<grid, 256, 0, s>>>(A, R, n, B);
+  const int smem = (n * (n + 1) + 2 * n) * static_cast<int>(sizeof(double));
+  cudaError_t e = cudaFuncSetAttribute(cayley_solve_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(cayley_solve)", e);
+  cayley_solve_kernel<<<batch, SOLVE_THREADS, smem, s>>>(A, B, n, R_out, R32);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("cayley launch", e);
+}
+
+sq_status learn(const float* x, const float* w, const double* R0, int64_t T, int H, int d,
+                int64_t N, double alpha, int iters, double* R, double* losses, void* ws,
+                int num_sms, uint32_t spin_limit, cudaStream_t s) {
+  const Layout L = layout(T, H, d, N, num_sms);
+  float* R32 = at<float>(ws, L.r32);
+  double* G = at<double>(ws, L.g64);
+  const int64_t nn = static_cast<int64_t>(d) * d;
+  cudaError_t e = cudaSuccess;
+  if (R != R0) e = cudaMemcpyAsync(R, R0, nn * sizeof(double), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return host::cuda_fail("r2 learn copy", e);
+  to_f32_kernel<<<(nn + 255) / 256, 256, 0, s>>>(R, nn, R32);
+  for (int i = 0; i < iters; ++i) {
+    sq_status st = loss_grad(x, w, R32, T, H, d, N, losses + i, G, ws, num_sms, spin_limit, s);
+    if (st != SQ_OK) return st;
+    st = cayley_update(R, G, alpha, d, 1, R, R32, at<void>(ws, L.cay), s);
+    if (st != SQ_OK) return st;
+  }
+  return loss_grad(x, w, R32, T, H, d, N, losses + iters, nullptr, ws, num_sms, spin_limit, s);
+}
+
+sq_status random_hadamard(const int8_t* signs, int d, int batch, double* R, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(batch) * d * d;
+  const int64_t grid = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+  random_hadamard_kernel<<<static_cast<int>(grid), 256, 0, s>>>(signs, d, batch, R);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("random_hadamard launch", e);
+}
+
+sq_status orth_error(const double* R, int n, int batch, double* out, cudaStream_t s) {
+  orth_error_kernel<<<batch, SOLVE_THREADS, 0, s>>>(R, n, out);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("orth_error launch", e);
+}
+
+}  // namespace r2
+}  // namespace sq

@@ -489,6 +489,168 @@ sq_status sq_kv8_dequant(const uint8_t* cache, const float* scale, const uint8_t
   return kv_dequant(cache, scale, zero, T, h, d, out_bf16, 8, stream);
 }
 
+// ------------------------------------------------------- Cayley R2 learner
+
+static sq_status check_r2_shape(int64_t T, int H, int d, int64_t N) {
+  if (T < 0 || H < 1 || d < 1 || N < 1) {
+    set_error("bad sizes T=%lld H=%d d=%d N=%lld", (long long)T, H, d, (long long)N);
+    return SQ_ERR_INVALID_ARG;
+  }
+  const int64_t K = static_cast<int64_t>(H) * d;
+  if (d != 128 || T % 16 != 0 || T < 16 || N % 16 != 0 || K > 65536 || T * K > (1LL << 31) ||
+      N * K > (1LL << 31) || T * N > (1LL << 31)) {
+    set_error("unsupported shape T=%lld H=%d d=%d N=%lld (need d == 128, T and N multiples "
+              "of 16, H * d <= 65536)", (long long)T, H, d, (long long)N);
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  return SQ_OK;
+}
+
+size_t sq_r2_workspace_bytes(int64_t T, int H, int d, int64_t N) {
+  if (check_r2_shape(T, H, d, N) != SQ_OK) return 0;
+  if (sq::host::current_device() < 0) return 0;
+  return sq::r2::workspace_bytes(T, H, d, N, sq::host::num_sms());
+}
+
+sq_status sq_r2_prepare(const float* x, const float* w, int64_t T, int H, int d, int64_t N,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  sq_status st = check_r2_shape(T, H, d, N);
+  if (st != SQ_OK) return st;
+  if (!x || !w || !workspace) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(w) || !aligned16(workspace)) {
+    set_error("x, w and the workspace must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  st = precheck_device();
+  if (st != SQ_OK) return st;
+  if (workspace_bytes < sq::r2::workspace_bytes(T, H, d, N, sq::host::num_sms())) {
+    set_error("workspace of %zu bytes is smaller than sq_r2_workspace_bytes()", workspace_bytes);
+    return SQ_ERR_INVALID_ARG;
+  }
+  return sq::r2::prepare(x, w, T, H, d, N, workspace, sq::host::num_sms(),
+                         static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_r2_loss_grad(const float* x, const float* w, const float* R, int64_t T, int H, int d,
+                          int64_t N, double* loss, double* grad, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  sq_status st = check_r2_shape(T, H, d, N);
+  if (st != SQ_OK) return st;
+  if (!x || !w || !R || !loss || !workspace) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(w) || !aligned16(R) || !aligned16(workspace)) {
+    set_error("x, w, R and the workspace must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  st = precheck_device();
+  if (st != SQ_OK) return st;
+  if (workspace_bytes < sq::r2::workspace_bytes(T, H, d, N, sq::host::num_sms())) {
+    set_error("workspace of %zu bytes is smaller than sq_r2_workspace_bytes()", workspace_bytes);
+    return SQ_ERR_INVALID_ARG;
+  }
+  return sq::r2::loss_grad(x, w, R, T, H, d, N, loss, grad, workspace, sq::host::num_sms(),
+                           sq::host::spin_limit(), static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_r2_cayley_learn(const float* x, const float* w, const double* R0, int64_t T, int H,
+                             int d, int64_t N, double alpha, int iters, double* R,
+                             double* losses, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  sq_status st = check_r2_shape(T, H, d, N);
+  if (st != SQ_OK) return st;
+  if (iters < 0 || !(alpha == alpha)) {
+    set_error("bad learner arguments iters=%d alpha=%g", iters, alpha);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!x || !w || !R0 || !R || !losses || !workspace) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(w) || !aligned16(R0) || !aligned16(R) ||
+      !aligned16(workspace)) {
+    set_error("x, w, R0, R and the workspace must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  st = precheck_device();
+  if (st != SQ_OK) return st;
+  if (workspace_bytes < sq::r2::workspace_bytes(T, H, d, N, sq::host::num_sms())) {
+    set_error("workspace of %zu bytes is smaller than sq_r2_workspace_bytes()", workspace_bytes);
+    return SQ_ERR_INVALID_ARG;
+  }
+  return sq::r2::learn(x, w, R0, T, H, d, N, alpha, iters, R, losses, workspace,
+                       sq::host::num_sms(), sq::host::spin_limit(),
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t sq_cayley_workspace_bytes(int n, int batch) {
+  if (n < 1 || n > 128 || batch < 1) return 0;
+  return sq::r2::cayley_workspace_bytes(n, batch);
+}
+
+sq_status sq_cayley_update(const double* R, const double* G, double alpha, int n, int batch,
+                           double* R_out, float* R_out_f32, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (n < 1 || n > 128 || batch < 0 || batch > 65535 || !(alpha == alpha)) {
+    set_error("bad Cayley arguments n=%d batch=%d alpha=%g (need 1 <= n <= 128)", n, batch,
+              alpha);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (batch == 0) return SQ_OK;
+  if (!R || !G || !R_out || !workspace) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < sq::r2::cayley_workspace_bytes(n, batch)) {
+    set_error("workspace of %zu bytes is smaller than sq_cayley_workspace_bytes()",
+              workspace_bytes);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(R) || !aligned16(G) || !aligned16(R_out) || !aligned16(workspace) ||
+      (R_out_f32 && !aligned16(R_out_f32))) {
+    set_error("device pointers must be 16-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::r2::cayley_update(R, G, alpha, n, batch, R_out, R_out_f32, workspace,
+                               static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_r2_random_hadamard(const int8_t* signs, int d, int batch, double* R, void* stream) {
+  if (d < 1 || d > 128 || (d & (d - 1)) || batch < 0) {
+    set_error("bad sizes d=%d batch=%d (need d a power of 2 <= 128)", d, batch);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (batch == 0) return SQ_OK;
+  if (!signs || !R) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::r2::random_hadamard(signs, d, batch, R, static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_orth_error(const double* R, int n, int batch, double* out, void* stream) {
+  if (n < 1 || n > 128 || batch < 0 || batch > 65535) {
+    set_error("bad sizes n=%d batch=%d (need 1 <= n <= 128)", n, batch);
+    return SQ_ERR_INVALID_ARG;
+  }
+  if (batch == 0) return SQ_OK;
+  if (!R || !out) {
+    set_error("null pointer argument");
+    return SQ_ERR_INVALID_ARG;
+  }
+  sq_status st = precheck_device();
+  if (st != SQ_OK) return st;
+  return sq::r2::orth_error(R, n, batch, out, static_cast<cudaStream_t>(stream));
+}
+
 sq_status sq_rope_tables(double theta, int max_pos, int d, float* cos, float* sin,
                          void* stream) {
   if (!(theta > 1.0) || max_pos < 1 || d < 2 || d > 1024 || (d & 1)) {

@@ -95,6 +95,26 @@ sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const
               cudaStream_t stream);
 }  // namespace kvd
 
+namespace r2 {
+// Cayley SGD for the head-wise rotation R2 (see cayley.cu).
+size_t workspace_bytes(int64_t T, int H, int d, int64_t N, int num_sms);
+sq_status prepare(const float* x, const float* w, int64_t T, int H, int d, int64_t N, void* ws,
+                  int num_sms, cudaStream_t s);
+sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, int H, int d,
+                    int64_t N, double* loss, double* G, void* ws, int num_sms, uint32_t spin_limit,
+                    cudaStream_t s);
+size_t cayley_workspace_bytes(int n, int batch);
+sq_status cayley_update(const double* R, const double* G, double alpha, int n, int batch,
+                        double* R_out, float* R32, void* ws, cudaStream_t s);
+sq_status orth_error(const double* R, int n, int batch, double* out, cudaStream_t s);
+sq_status random_hadamard(const int8_t* signs, int d, int batch, double* R, cudaStream_t s);
+// iters Cayley steps from R0 into R (may be R0); losses[i] is the loss at the
+// i-th iterate, losses[iters] at the result.  ws prepared by prepare().
+sq_status learn(const float* x, const float* w, const double* R0, int64_t T, int H, int d,
+                int64_t N, double alpha, int iters, double* R, double* losses, void* ws,
+                int num_sms, uint32_t spin_limit, cudaStream_t s);
+}  // namespace r2
+
 namespace kv {
 sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t T, int hq,
                            int hkv, const int32_t* pos, const float* cos, const float* sin,

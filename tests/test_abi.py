@@ -36,6 +36,8 @@ def test_header_declares_the_hot_path_calls():
               "sq_kv4_decode_attention", "sq_kv4_decode_workspace_bytes",
               "sq_kv_rotate_quant", "sq_kv_dequant",
               "sq_kv_rotate_quant8", "sq_kv8_dequant", "sq_kv8_decode_attention",
+              "sq_r2_workspace_bytes", "sq_r2_prepare", "sq_r2_loss_grad", "sq_r2_cayley_learn",
+              "sq_cayley_update", "sq_cayley_workspace_bytes", "sq_orth_error",
               "sq_status_string", "sq_w4a4_workspace_bytes", "sq_device_status"]:
         assert n in names
 
@@ -102,6 +104,20 @@ def test_validation_happens_before_any_launch(sq):
     assert lib.sq_kv8_dequant(None, None, None, 4, 8, 128, None, None) == 1
     assert lib.sq_kv8_decode_attention(*args, 2, 16, 16, 8, 128, None, None, 0, None) == 2
     assert lib.sq_kv8_decode_attention(*args, 0, 16, 32, 8, 128, None, None, 0, None) == 0
+    # Cayley R2 learner: d == 128, T and N multiples of 16; n <= 128
+    assert lib.sq_r2_workspace_bytes(2048, 32, 64, 4096) == 0
+    assert lib.sq_r2_prepare(None, None, 2048, 32, 64, 4096, None, 0, None) == 2
+    assert lib.sq_r2_prepare(None, None, 2040, 32, 128, 4096, None, 0, None) == 2
+    assert lib.sq_r2_prepare(None, None, 2048, 32, 128, 4096, None, 0, None) == 1
+    assert lib.sq_r2_loss_grad(None, None, None, 2048, 32, 128, 4008, None, None, None, 0,
+                               None) == 2
+    assert lib.sq_r2_cayley_learn(None, None, None, 64, 4, 128, 256, 0.3, -1, None, None, None,
+                                  0, None) == 1
+    assert lib.sq_cayley_update(None, None, 0.1, 129, 1, None, None, None, 0, None) == 1
+    assert lib.sq_cayley_update(None, None, 0.1, 16, 0, None, None, None, 0, None) == 0
+    assert lib.sq_cayley_update(None, None, 0.1, 16, 1, None, None, None, 0, None) == 1
+    assert lib.sq_cayley_workspace_bytes(128, 2) == 2 * 2 * 128 * 128 * 8
+    assert lib.sq_orth_error(None, 0, 1, None, None) == 1
 
 
 def test_product_paley_matches_oracle():
