@@ -47,17 +47,16 @@ DECODE_BYTES = 2 * KV_T * KV_HKV * (64 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
 # ... of sq_kv8_decode_attention: one byte per code
 DECODE8_BYTES = 2 * KV_T * KV_HKV * (128 + 4 + 1) + 2 * (16 * KV_HQ * 128 * 2)
 # Cayley R2 learner on the o_proj layer (2048 tokens, 32 heads of 128, 4096
-# outputs): float32 FLOPs of one loss-and-gradient evaluation (head-wise
-# rotations of x and w, the two straight-through gradient products, and G)
-# and the INT4 tensor-core product
+# outputs).  Algorithmic work of one loss-and-gradient evaluation: the INT4
+# product Q(xR) Q(wR)^T, the two straight-through gradient products E Q(wR)
+# and E^T Q(xR) (tensor cores, float operand as two bf16 halves, so executed
+# twice), and the float32 rotations and G
 R2_T, R2_H, R2_D, R2_N = 2048, 32, 128, 4096
 R2_K = R2_H * R2_D
-R2_F32_FLOPS = (2 * (R2_T + R2_N) * R2_K * R2_D + 2 * 2 * R2_T * R2_N * R2_K
-                + 2 * (R2_T + R2_N) * R2_H * R2_D * R2_D)
 R2_INT_OPS = 2 * R2_T * R2_N * R2_K
+R2_GRAD_FLOPS = 2 * 2 * R2_T * R2_N * R2_K
+R2_F32_FLOPS = 2 * (R2_T + R2_N) * R2_K * R2_D + 2 * (R2_T + R2_N) * R2_H * R2_D * R2_D
 R2_ALPHA = 0.3
-# CUDA-core float32 peak: 148 SMs x 128 FP32 lanes x 2 FLOP x 1.965 GHz
-F32_PEAK = 148 * 128 * 2 * 1.965e9 / 1e12
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
@@ -403,7 +402,9 @@ def run_ours(args, rank, world, local_rank):
         orth = float(sq.orth_error(R)[0])
         r2_info = {"workload": ow.name, "alpha": R2_ALPHA,
                    "loss_grad_us": mlg * 1e3,
-                   "loss_grad_f32_TFLOPs": R2_F32_FLOPS / (mlg * 1e-3) / 1e12,
+                   "loss_grad_work": {"int4_gop": R2_INT_OPS / 1e9,
+                                      "grad_products_gflop": R2_GRAD_FLOPS / 1e9,
+                                      "f32_gflop": R2_F32_FLOPS / 1e9},
                    "learner_step_us": mlearn * 1e3 / iters,
                    "loss_first_draw": float(L[0]), "loss_after_120": float(L[-1]),
                    "best_of_32_draws": float(draws.min()), "worst_of_32_draws": float(draws.max()),
@@ -713,9 +714,7 @@ def main():
             "w4a8": (dict(r["a8"], rotate_quant8_frac_of_hbm=r["a8"]["rotate_quant8_GB/s"] / hbm,
                           gemm_frac_of_int8_peak=r["a8"]["gemm_TOPS"] / int8_peak)
                      if r["a8"] else None),
-            "r2_cayley_learner": (dict(r["r2"], bound="alu", f32_peak_TFLOPs=F32_PEAK,
-                                       frac_of_f32_peak=r["r2"]["loss_grad_f32_TFLOPs"] / F32_PEAK)
-                                  if r["r2"] else None),
+            "r2_cayley_learner": r["r2"],
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,

@@ -31,6 +31,7 @@
 // The fp32 GEMM is a CUDA-core kernel (128 x 128 tiles, 8 x 8 outputs per
 // thread, double-buffered shared memory): these products are float by float
 // and the page's probe needs float accuracy, not a low-precision format.
+#include <cuda_bf16.h>
 #include <math.h>
 
 #include "sq_device.cuh"
@@ -217,12 +218,13 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // (1 for an all-zero row), code = clamp(rint(v / scale), -8, 7) with the
 // quotient rounded as IEEE float32 division.  Writes the packed codes
 // [rows][K/2] (element 2j in the low nibble of byte j), the scales, and the
-// dequantized values code * scale [rows][K].  One CTA per row.
+// codes again as bf16 [rows][K] (exact), the tensor-core operand of the
+// gradient products.  One CTA per row.
 __global__ void __launch_bounds__(256) quant_rows_kernel(const float* __restrict__ src,
                                                          int64_t rows, int K,
                                                          uint8_t* __restrict__ packed,
                                                          float* __restrict__ scale_out,
-                                                         float* __restrict__ deq) {
+                                                         uint16_t* __restrict__ codes_bf16) {
   __shared__ float red[8];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const float* row = src + r * K;
@@ -239,18 +241,17 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const float* __restrict
       const float4 v0 = __ldg(reinterpret_cast<const float4*>(row + k));
       const float4 v1 = __ldg(reinterpret_cast<const float4*>(row + k + 4));
       const float xv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float dv[8];
+      uint32_t hv[4] = {0u, 0u, 0u, 0u};
       uint32_t word = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float c = fminf(fmaxf(rintf(__fdiv_rn(xv[e], s)), -8.f), 7.f);
-        dv[e] = c * s;
         word |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * e);
+        // a small integer is exact in bf16: the top half of its float32 bits
+        hv[e >> 1] |= (__float_as_uint(c) >> 16) << (16 * (e & 1));
       }
       *reinterpret_cast<uint32_t*>(packed + r * (K / 2) + k / 2) = word;
-      float4* dp = reinterpret_cast<float4*>(deq + r * K + k);
-      dp[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
-      dp[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+      *reinterpret_cast<uint4*>(codes_bf16 + r * K + k) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
   }
 }
@@ -316,13 +317,15 @@ __global__ void __launch_bounds__(256) sumsq_kernel(const float* __restrict__ x,
   if (threadIdx.x == 0) part[blockIdx.x] = s;
 }
 
-// out = sum_p part[p] (in order), divided by *den when den is given.
-__global__ void finish_kernel(const double* __restrict__ part, int P, const double* den,
-                              double* out) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// out = sum_p part[p], divided by *den when den is given: one block, each
+// thread a fixed stride of the partials, then a fixed tree (deterministic).
+__global__ void __launch_bounds__(1024) finish_kernel(const double* __restrict__ part, int P,
+                                                      const double* den, double* out) {
+  __shared__ double red[32];
   double s = 0.0;
-  for (int p = 0; p < P; ++p) s += part[p];
-  *out = den ? s / *den : s;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) s += part[p];
+  s = block_sum_d(s, red);
+  if (threadIdx.x == 0) *out = den ? s / *den : s;
 }
 
 // G[i] = 2 / den * sum_p part[p * n + i] (float64, partials in order).
@@ -332,94 +335,335 @@ __global__ void grad_sum_kernel(const float* __restrict__ part, int P, int64_t n
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     double s = 0.0;
+#pragma unroll 8
     for (int p = 0; p < P; ++p) s += static_cast<double>(__ldg(part + p * n + i));
     G[i] = f * s;
   }
 }
 
-// ------------------------------------------------------------ Cayley step
+// ------------------------------------------- gradient products on tensor cores
 
-// A = I - h (R G^T - G R^T) for each of the batch's n x n matrices (h =
-// alpha / 2); each off-diagonal pair is computed once and written with both
-// signs, so A - I is exactly skew-symmetric.
-__global__ void cayley_a_kernel(const double* __restrict__ R, const double* __restrict__ G,
-                                double h, int n, double* __restrict__ A) {
-  const int64_t off = static_cast<int64_t>(blockIdx.y) * n * n;
-  R += off;
-  G += off;
-  A += off;
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n * n;
-       idx += gridDim.x * blockDim.x) {
-    const int i = idx / n, j = idx - i * n;
-    if (i == j) {
-      A[idx] = 1.0;
-    } else if (i < j) {
-      double y = 0.0;
-      for (int l = 0; l < n; ++l) y += R[i * n + l] * G[j * n + l] - G[i * n + l] * R[j * n + l];
-      A[idx] = -h * y;
-      A[j * n + i] = h * y;
+// v as bf16 hi + lo (hi = RN(v), lo = RN(v - hi); v - hi is exact in float32),
+// so hi + lo keeps about 17 bits of v.
+__device__ __forceinline__ void split_bf16(float v, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+  hi = __bfloat16_as_ushort(h);
+  lo = __bfloat16_as_ushort(l);
+}
+
+// From E [T][N] (float32): A1 = E diag(sw) [T][N] and A2 = (diag(sa) E)^T
+// [N][T], each as bf16 hi and lo halves: the float operands of
+// g_xr = E Q(wR) = A1 codes_w and g_wr = E^T Q(xR) = A2 codes_a, with each
+// quantizer's scale moved onto the reduction side.  32 x 32 tiles through
+// shared memory, so both writes are coalesced.
+__global__ void __launch_bounds__(256) split_error_kernel(
+    const float* __restrict__ E, const float* __restrict__ sa, const float* __restrict__ sw,
+    int T, int N, uint16_t* __restrict__ a1h, uint16_t* __restrict__ a1l,
+    uint16_t* __restrict__ a2h, uint16_t* __restrict__ a2l) {
+  __shared__ float tile[32][33];
+  const int t0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 32 x 8
+  for (int r = ty; r < 32; r += 8) {
+    const int t = t0 + r, n = n0 + tx;
+    float e = 0.f;
+    if (t < T && n < N) {
+      e = E[static_cast<int64_t>(t) * N + n];
+      uint16_t h, l;
+      split_bf16(e * __ldg(sw + n), h, l);
+      a1h[static_cast<int64_t>(t) * N + n] = h;
+      a1l[static_cast<int64_t>(t) * N + n] = l;
+    }
+    tile[r][tx] = e;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int n = n0 + r, t = t0 + tx;
+    if (t < T && n < N) {
+      uint16_t h, l;
+      split_bf16(tile[tx][r] * __ldg(sa + t), h, l);
+      a2h[static_cast<int64_t>(n) * T + t] = h;
+      a2l[static_cast<int64_t>(n) * T + t] = l;
     }
   }
 }
 
-// B = (I + h Y) R = 2 R - A R.
-__global__ void cayley_b_kernel(const double* __restrict__ A, const double* __restrict__ R, int n,
-                                double* __restrict__ B) {
+// D[m][n] = sum_k (Ahi[m][k] + Alo[m][k]) B[k][n] on the tensor cores
+// (tcgen05.mma kind::f16, bf16 operands, float32 accumulation in TMEM): Ahi,
+// Alo bf16 [M][Kr] (K-major), B bf16 [Kr][Nn] (read MN-major), D float32
+// [M][ldd].  One 128 x 128 output tile per CTA; warp 0 issues the TMA copies
+// (4 stages of A hi, A lo and B, 48 KB each), warp 1 the MMAs (two per 16-deep
+// step, hi and lo into the same accumulator), warps 2..5 the epilogue (TMEM
+// lane quadrant = warp % 4).  The copy engine zero-fills rows and columns past
+// M, Nn and Kr.  Every wait is bounded; one that runs out marks the tile
+// aborted, leaves D unwritten and records SQ_ERR_TIMEOUT.
+constexpr int CG_BM = 128, CG_BN = 128, CG_BK = 64, CG_ST = 4, CG_THREADS = 192;
+constexpr int CG_A = CG_BM * CG_BK * 2;                 // 16 KB: 128 rows x 128 B
+constexpr int CG_B = CG_BK * CG_BN * 2;                 // 16 KB: two MN atoms of 64 x 128 B
+constexpr int CG_STAGE = 2 * CG_A + CG_B;
+constexpr int CG_BAR = CG_ST * CG_STAGE;
+constexpr int CG_SMEM = CG_BAR + (2 * CG_ST + 1) * 8 + 16 + 1024;
+constexpr uint32_t CG_IDESC = idesc_bf16(128, 128, false, true);
+static_assert(CG_STAGE % 1024 == 0 && CG_A % 1024 == 0 && CG_B % 2048 == 0,
+              "swizzle atoms need 1 KB alignment");
+
+__global__ void __launch_bounds__(CG_THREADS, 1) codes_gemm_kernel(
+    const __grid_constant__ CUtensorMap mapAh, const __grid_constant__ CUtensorMap mapAl,
+    const __grid_constant__ CUtensorMap mapB, int M, int Nn, int Kr, float* __restrict__ D,
+    int64_t ldd, uint32_t spin_limit) {
+  extern __shared__ uint8_t cg_raw[];
+  uint8_t* smem = cg_raw + ((1024u - (smem_u32(cg_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + CG_BAR);
+  uint64_t* empty = full + CG_ST;
+  uint64_t* done = empty + CG_ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * CG_BM, n0 = blockIdx.x * CG_BN;
+  const int nk = (Kr + CG_BK - 1) / CG_BK;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < CG_ST; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (; it < nk; ++it) {
+        const int st = it % CG_ST;
+        const uint32_t ph = (it / CG_ST) & 1;
+        if (!mbar_wait(&empty[st], ph ^ 1, spin_limit) || *abort_flag) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* dst = smem + st * CG_STAGE;
+        mbar_arrive_expect_tx(&full[st], CG_STAGE);
+        tma_load_2d(dst, &mapAh, it * CG_BK, m0, &full[st]);
+        tma_load_2d(dst + CG_A, &mapAl, it * CG_BK, m0, &full[st]);
+        tma_load_2d(dst + 2 * CG_A, &mapB, n0, it * CG_BK, &full[st]);
+        tma_load_2d(dst + 2 * CG_A + CG_B / 2, &mapB, n0 + 64, it * CG_BK, &full[st]);
+      }
+      // every copy this CTA issued lands before it exits
+      for (int j = it > CG_ST ? it - CG_ST : 0; j < it; ++j)
+        mbar_wait(&full[j % CG_ST], (j / CG_ST) & 1, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int it = 0; it < nk; ++it) {
+        const int st = it % CG_ST;
+        const uint32_t ph = (it / CG_ST) & 1;
+        if (!mbar_wait(&full[st], ph, spin_limit) || *abort_flag) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + st * CG_STAGE);
+        const uint32_t b = a + 2 * CG_A;
+#pragma unroll
+        for (int kk = 0; kk < CG_BK / 16; ++kk) {
+          const uint64_t db = desc_sw128_mn(b + kk * 2048, CG_B / 2, 1024);
+          mma_bf16(tmem, desc_sw128(a + kk * 32), db, CG_IDESC, (it | kk) ? 1u : 0u);
+          mma_bf16(tmem, desc_sw128(a + CG_A + kk * 32), db, CG_IDESC, 1u);
+        }
+        mma_commit(&empty[st]);
+      }
+      mma_commit(done);                    // completes once every issued MMA has
+    }
+  } else {
+    ok = mbar_wait(done, 0, spin_limit) && !*abort_flag;
+    tc_fence_after();
+    const int q = warp & 3;
+    const int row = m0 + 32 * q + lane;
+#pragma unroll 1
+    for (int c = 0; c < CG_BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * c, v);
+      tmem_ld_wait();
+      const int col = n0 + 32 * c;
+      if (ok && row < M && col < Nn) {
+        float* dst = D + static_cast<int64_t>(row) * ldd + col;
+        if (col + 32 <= Nn) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            reinterpret_cast<float4*>(dst)[j] =
+                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < Nn - col) dst[j] = __uint_as_float(v[j]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+  if (!ok && lane == 0) record_status(SQ_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------ Cayley step
+
+// A = I - h (R G^T - G R^T) for each of the batch's n x n matrices (h =
+// alpha / 2), in 32 x 32 tiles through shared memory.  Only tiles on or above
+// the diagonal are computed, and each off-diagonal pair once, written with
+// both signs, so A - I is exactly skew-symmetric.  Block (bi, bj) with
+// bi <= bj; 256 threads, 4 outputs each.
+constexpr int CT = 32;
+__global__ void __launch_bounds__(256) cayley_a_kernel(const double* __restrict__ R,
+                                                       const double* __restrict__ G, double h,
+                                                       int n, double* __restrict__ A) {
+  __shared__ double Ri[CT][CT + 1], Gi[CT][CT + 1], Rj[CT][CT + 1], Gj[CT][CT + 1];
+  const int nt = (n + CT - 1) / CT;
+  // blockIdx.x enumerates the pairs bi <= bj
+  int bi = 0, rem = blockIdx.x;
+  while (rem >= nt - bi) {
+    rem -= nt - bi;
+    ++bi;
+  }
+  const int bj = bi + rem;
+  const int64_t off = static_cast<int64_t>(blockIdx.y) * n * n;
+  R += off;
+  G += off;
+  A += off;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int i0 = bi * CT, j0 = bj * CT;
+  double y[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int l0 = 0; l0 < n; l0 += CT) {
+    for (int r = ty; r < CT; r += 8) {
+      const int l = l0 + tx;
+      const bool lok = l < n;
+      Ri[r][tx] = (lok && i0 + r < n) ? R[(i0 + r) * n + l] : 0.0;
+      Gi[r][tx] = (lok && i0 + r < n) ? G[(i0 + r) * n + l] : 0.0;
+      Rj[r][tx] = (lok && j0 + r < n) ? R[(j0 + r) * n + l] : 0.0;
+      Gj[r][tx] = (lok && j0 + r < n) ? G[(j0 + r) * n + l] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int l = 0; l < CT; ++l) {
+      const double rj = Rj[tx][l], gj = Gj[tx][l];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = ty + 8 * q;
+        y[q] += Ri[r][l] * gj - Gi[r][l] * rj;
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = i0 + ty + 8 * q, j = j0 + tx;
+    if (i >= n || j >= n) continue;
+    if (i == j) {
+      A[i * n + j] = 1.0;
+    } else if (i < j) {
+      A[i * n + j] = -h * y[q];
+      A[j * n + i] = h * y[q];
+    }
+  }
+}
+
+// B = (I + h Y) R = 2 R - A R, in 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256) cayley_b_kernel(const double* __restrict__ A,
+                                                       const double* __restrict__ R, int n,
+                                                       double* __restrict__ B) {
+  __shared__ double At[CT][CT + 1], Rt[CT][CT + 1];
+  const int nt = (n + CT - 1) / CT;
+  const int bi = blockIdx.x / nt, bj = blockIdx.x - bi * nt;
   const int64_t off = static_cast<int64_t>(blockIdx.y) * n * n;
   R += off;
   A += off;
   B += off;
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n * n;
-       idx += gridDim.x * blockDim.x) {
-    const int i = idx / n, j = idx - i * n;
-    double s = 2.0 * R[idx];
-    for (int l = 0; l < n; ++l) s -= A[i * n + l] * R[l * n + j];
-    B[idx] = s;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int i0 = bi * CT, j0 = bj * CT;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int l0 = 0; l0 < n; l0 += CT) {
+    for (int r = ty; r < CT; r += 8) {
+      At[r][tx] = (i0 + r < n && l0 + tx < n) ? A[(i0 + r) * n + l0 + tx] : 0.0;
+      Rt[r][tx] = (l0 + r < n && j0 + tx < n) ? R[(l0 + r) * n + j0 + tx] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int l = 0; l < CT; ++l) {
+      const double rv = Rt[l][tx];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] += At[ty + 8 * q][l] * rv;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = i0 + ty + 8 * q, j = j0 + tx;
+    if (i < n && j < n) B[i * n + j] = 2.0 * R[i * n + j] - acc[q];
   }
 }
 
-constexpr int SOLVE_THREADS = 1024;
+constexpr int SOLVE_THREADS = 512;
+constexpr int ORTH_THREADS = 1024;
 constexpr int MAX_N = 128;
+constexpr int SOLVE_RG = SOLVE_THREADS / MAX_N;        // row groups
+constexpr int SOLVE_RPT = MAX_N / SOLVE_RG;            // rows per thread (in registers)
 
 // R_out = A^-1 B by Gauss-Jordan elimination, one CTA per matrix (n <= 128):
 // A in shared memory (row stride n + 1), B in registers, thread t holding
-// column t % 128 of rows t / 128 + 8 r.  Pivots are >= 1 (see the top).
-__global__ void __launch_bounds__(SOLVE_THREADS) cayley_solve_kernel(
+// column t % 128 of rows t / 128 + 4 r (32 rows, 64 registers).  Pivots are
+// >= 1 (see the top).
+__global__ void __launch_bounds__(SOLVE_THREADS, 1) cayley_solve_kernel(
     const double* __restrict__ Ain, const double* __restrict__ Bin, int n,
     double* __restrict__ R_out, float* __restrict__ R32) {
   extern __shared__ double cs_smem[];
   const int64_t off = static_cast<int64_t>(blockIdx.x) * n * n;
   const int ld = n + 1;
   double* As = cs_smem;
-  double* colk = As + n * ld;
-  double* pivB = colk + n;
-  const int t = threadIdx.x, j = t & (MAX_N - 1), rg = t >> 7;
+  double* colbuf = As + n * ld;            // [2][n]: pivot columns, double-buffered
+  double* pivB = colbuf + 2 * n;
+  const int t = threadIdx.x, j = t & (MAX_N - 1), rg = t / MAX_N;
   const bool live = j < n;
-  double bv[16];
+  double bv[SOLVE_RPT];
 #pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    const int i = rg + 8 * r;
+  for (int r = 0; r < SOLVE_RPT; ++r) {
+    const int i = rg + SOLVE_RG * r;
     bv[r] = 0.0;
     if (live && i < n) {
       bv[r] = Bin[off + i * n + j];
       As[i * ld + j] = Ain[off + i * n + j];
     }
   }
+  if (j == 0) {
+#pragma unroll
+    for (int r = 0; r < SOLVE_RPT; ++r) {
+      const int i = rg + SOLVE_RG * r;
+      if (i < n) colbuf[i] = As[i * ld];
+    }
+  }
   __syncthreads();
   for (int k = 0; k < n; ++k) {
-    if (j == k) {
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int i = rg + 8 * r;
-        if (i < n) colk[i] = As[i * ld + k];
-      }
-    }
-    __syncthreads();
+    // colk = column k of A before step k, staged at the end of step k - 1
+    const double* colk = colbuf + (k & 1) * n;
+    double* coln = colbuf + ((k + 1) & 1) * n;
     const double piv = colk[k];
-    if (live && rg == (k & 7)) {
+    if (live && rg == k % SOLVE_RG) {
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        if (r == (k >> 3)) {
+      for (int r = 0; r < SOLVE_RPT; ++r) {
+        if (r == k / SOLVE_RG) {
           As[k * ld + j] = As[k * ld + j] / piv;
           bv[r] = bv[r] / piv;
           pivB[j] = bv[r];
@@ -430,20 +674,23 @@ __global__ void __launch_bounds__(SOLVE_THREADS) cayley_solve_kernel(
     if (live) {
       const double akj = As[k * ld + j], bkj = pivB[j];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int i = rg + 8 * r;
+      for (int r = 0; r < SOLVE_RPT; ++r) {
+        const int i = rg + SOLVE_RG * r;
         if (i < n && i != k) {
           const double f = colk[i];
           As[i * ld + j] -= f * akj;
           bv[r] -= f * bkj;
         }
+        // the owner of column k + 1 stages it for the next step (row k was
+        // normalised by this same thread above)
+        if (j == k + 1 && i < n) coln[i] = As[i * ld + j];
       }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    const int i = rg + 8 * r;
+  for (int r = 0; r < SOLVE_RPT; ++r) {
+    const int i = rg + SOLVE_RG * r;
     if (live && i < n) {
       R_out[off + i * n + j] = bv[r];
       if (R32) R32[off + i * n + j] = static_cast<float>(bv[r]);
@@ -452,7 +699,7 @@ __global__ void __launch_bounds__(SOLVE_THREADS) cayley_solve_kernel(
 }
 
 // out[b] = ||R_b^T R_b - I||_F (float64), one CTA per matrix.
-__global__ void __launch_bounds__(SOLVE_THREADS) orth_error_kernel(const double* __restrict__ R,
+__global__ void __launch_bounds__(ORTH_THREADS) orth_error_kernel(const double* __restrict__ R,
                                                                    int n, double* __restrict__ out) {
   __shared__ double red[32];
   R += static_cast<int64_t>(blockIdx.x) * n * n;
@@ -496,13 +743,13 @@ __global__ void to_f32_kernel(const double* __restrict__ src, int64_t n, float* 
 namespace {
 
 constexpr int LOSS_BLOCKS = 1024;          // fixed grid of the loss sums
-constexpr int GRAD_CHUNK = 1024;           // K chunk of the split-K gradient GEMMs
+constexpr int GRAD_CHUNK = 512;            // K chunk of the split-K G GEMMs (~2.6 CTAs per SM)
 
 size_t al(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t y0, E, xr, qa, aq, sa, wr, qw, wq, sw, gpart, lpart, den, gws, gws_bytes, r32, g64, cay,
-      total;
+  size_t y0, E, xr, qa, aq, sa, wr, qw, wq, sw, a1h, a1l, a2h, a2l, gpart, lpart, den, gws,
+      gws_bytes, r32, g64, cay, total;
   int Px, Pw;
 };
 
@@ -520,13 +767,17 @@ Layout layout(int64_t T, int H, int d, int64_t N, int num_sms) {
   L.y0 = take(T * N * 4);
   L.E = take(T * N * 4);
   L.xr = take(T * K * 4);
-  L.qa = take(T * K * 4);
+  L.qa = take(T * K * 2);                           // activation codes, bf16
   L.aq = take(T * K / 2);
   L.sa = take(T * 4);
   L.wr = take(N * K * 4);
-  L.qw = take(N * K * 4);
+  L.qw = take(N * K * 2);                           // weight codes, bf16
   L.wq = take(N * K / 2);
   L.sw = take(N * 4);
+  L.a1h = take(T * N * 2);
+  L.a1l = take(T * N * 2);
+  L.a2h = take(T * N * 2);
+  L.a2l = take(T * N * 2);
   L.gpart = take(static_cast<size_t>(L.Px + L.Pw) * d * d * 4);
   L.lpart = take(LOSS_BLOCKS * 8);
   L.den = take(8);
@@ -558,6 +809,50 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// 2-D bf16 tensor [outer][inner] (inner contiguous), boxes of 64 x box_outer
+// in the 128-byte swizzle.
+bool bf16_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int box_outer) {
+  auto encode = host::tensor_map_encoder();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    host::set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+// D [M][Nn] = (Ah + Al) [M][Kr] x B [Kr][Nn] on the tensor cores.
+sq_status codes_gemm(const uint16_t* Ah, const uint16_t* Al, const uint16_t* B, int64_t M,
+                     int64_t Nn, int64_t Kr, float* D, uint32_t spin_limit, cudaStream_t s) {
+  CUtensorMap mh, ml, mb;
+  if (!bf16_map(&mh, Ah, Kr, M, CG_BM) || !bf16_map(&ml, Al, Kr, M, CG_BM) ||
+      !bf16_map(&mb, B, Nn, Kr, CG_BK))
+    return SQ_ERR_CUDA;
+  static bool attr_done[64] = {};
+  const int dev = host::current_device();
+  if (dev < 0) return SQ_ERR_CUDA;
+  if (!attr_done[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(codes_gemm_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, CG_SMEM);
+    if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(codes_gemm)", e);
+    attr_done[dev & 63] = true;
+  }
+  const dim3 grid(static_cast<unsigned>((Nn + CG_BN - 1) / CG_BN),
+                  static_cast<unsigned>((M + CG_BM - 1) / CG_BM));
+  codes_gemm_kernel<<<grid, CG_THREADS, CG_SMEM, s>>>(mh, ml, mb, static_cast<int>(M),
+                                                      static_cast<int>(Nn), static_cast<int>(Kr),
+                                                      D, Nn, spin_limit);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("codes_gemm launch", e);
+}
+
 }  // namespace
 
 size_t workspace_bytes(int64_t T, int H, int d, int64_t N, int num_sms) {
@@ -572,7 +867,7 @@ sq_status prepare(const float* x, const float* w, int64_t T, int H, int d, int64
   cudaError_t e = sgemm<false, true>(T, N, K, x, K, w, K, y0, N, 1.f, 0.f, 1, static_cast<int>(K), s);
   if (e != cudaSuccess) return host::cuda_fail("r2 y0 GEMM", e);
   sumsq_kernel<<<LOSS_BLOCKS, 256, 0, s>>>(y0, T * N / 4, at<double>(ws, L.lpart));
-  finish_kernel<<<1, 32, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, nullptr,
+  finish_kernel<<<1, 1024, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, nullptr,
                                  at<double>(ws, L.den));
   if (L.gws_bytes) {
     e = cudaMemsetAsync(at<uint8_t>(ws, L.gws), 0, L.gws_bytes, s);
@@ -589,8 +884,8 @@ sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, i
   const int64_t K = static_cast<int64_t>(H) * d;
   float* xr = at<float>(ws, L.xr);
   float* wr = at<float>(ws, L.wr);
-  float* qa = at<float>(ws, L.qa);
-  float* qw = at<float>(ws, L.qw);
+  uint16_t* ca = at<uint16_t>(ws, L.qa);
+  uint16_t* cw = at<uint16_t>(ws, L.qw);
   float* sa = at<float>(ws, L.sa);
   float* sw = at<float>(ws, L.sw);
   uint8_t* aq = at<uint8_t>(ws, L.aq);
@@ -605,8 +900,8 @@ sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, i
     return host::cuda_fail("r2 rotation GEMM", e);
   const int qgrid_a = static_cast<int>(T < 8 * num_sms ? T : 8 * num_sms);
   const int qgrid_w = static_cast<int>(N < 8 * num_sms ? N : 8 * num_sms);
-  quant_rows_kernel<<<qgrid_a, 256, 0, s>>>(xr, T, static_cast<int>(K), aq, sa, qa);
-  quant_rows_kernel<<<qgrid_w, 256, 0, s>>>(wr, N, static_cast<int>(K), wq, sw, qw);
+  quant_rows_kernel<<<qgrid_a, 256, 0, s>>>(xr, T, static_cast<int>(K), aq, sa, ca);
+  quant_rows_kernel<<<qgrid_w, 256, 0, s>>>(wr, N, static_cast<int>(K), wq, sw, cw);
   if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 quantize", e);
   // exact integer products on the tensor cores
   sq_status st = gemm::run(aq, sa, wq, sw, T, N, K, acc, 1, L.gws_bytes ? at<void>(ws, L.gws) : nullptr,
@@ -614,16 +909,23 @@ sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, i
   if (st != SQ_OK) return st;
   r2_error_kernel<<<LOSS_BLOCKS, 256, 0, s>>>(acc, sa, sw, at<float>(ws, L.y0), T,
                                               static_cast<int>(N), at<double>(ws, L.lpart));
-  finish_kernel<<<1, 32, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, den, loss);
+  finish_kernel<<<1, 1024, 0, s>>>(at<double>(ws, L.lpart), LOSS_BLOCKS, den, loss);
   if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 loss", e);
   if (!G) return SQ_OK;
   // straight-through gradients of the rotated operands (the 2 / den factor
-  // is applied to G), into the rotation buffers
-  if ((e = sgemm<false, false>(T, K, N, E, N, qw, K, xr, K, 1.f, 0.f, 1, static_cast<int>(N), s)) !=
-          cudaSuccess ||
-      (e = sgemm<true, false>(N, K, T, E, N, qa, K, wr, K, 1.f, 0.f, 1, static_cast<int>(T), s)) !=
-          cudaSuccess)
-    return host::cuda_fail("r2 gradient GEMM", e);
+  // is applied to G), into the rotation buffers, on the tensor cores:
+  // g_xr = (E diag(sw)) codes_w and g_wr = (diag(sa) E)^T codes_a
+  uint16_t* a1h = at<uint16_t>(ws, L.a1h);
+  uint16_t* a1l = at<uint16_t>(ws, L.a1l);
+  uint16_t* a2h = at<uint16_t>(ws, L.a2h);
+  uint16_t* a2l = at<uint16_t>(ws, L.a2l);
+  split_error_kernel<<<dim3(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>((T + 31) / 32)),
+                       256, 0, s>>>(E, sa, sw, static_cast<int>(T), static_cast<int>(N), a1h, a1l,
+                                    a2h, a2l);
+  if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 error split", e);
+  if ((st = codes_gemm(a1h, a1l, cw, T, K, N, xr, spin_limit, s)) != SQ_OK ||
+      (st = codes_gemm(a2h, a2l, ca, N, K, T, wr, spin_limit, s)) != SQ_OK)
+    return st;
   // G = x_s^T g_xr,s + w_s^T g_wr,s, split over the long reduction
   float* gp = at<float>(ws, L.gpart);
   if ((e = sgemm<true, false>(d, d, T * H, x, d, xr, d, gp, d, 1.f, 0.f, L.Px, GRAD_CHUNK, s)) !=
@@ -645,10 +947,10 @@ sq_status cayley_update(const double* R, const double* G, double alpha, int n, i
                         double* R_out, float* R32, void* ws, cudaStream_t s) {
   double* A = static_cast<double*>(ws);
   double* B = A + static_cast<int64_t>(batch) * n * n;
-  const dim3 grid((n * n + 255) / 256, batch);
-  cayley_a_kernel<<<grid, 256, 0, s>>>(R, G, 0.5 * alpha, n, A);
-  cayley_b_kernel<<<grid, 256, 0, s>>>(A, R, n, B);
-  const int smem = (n * (n + 1) + 2 * n) * static_cast<int>(sizeof(double));
+  const int nt = (n + CT - 1) / CT;
+  cayley_a_kernel<<<dim3(nt * (nt + 1) / 2, batch), 256, 0, s>>>(R, G, 0.5 * alpha, n, A);
+  cayley_b_kernel<<<dim3(nt * nt, batch), 256, 0, s>>>(A, R, n, B);
+  const int smem = (n * (n + 1) + 3 * n) * static_cast<int>(sizeof(double));
   cudaError_t e = cudaFuncSetAttribute(cayley_solve_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(cayley_solve)", e);
@@ -686,7 +988,7 @@ sq_status random_hadamard(const int8_t* signs, int d, int batch, double* R, cuda
 }
 
 sq_status orth_error(const double* R, int n, int batch, double* out, cudaStream_t s) {
-  orth_error_kernel<<<batch, SOLVE_THREADS, 0, s>>>(R, n, out);
+  orth_error_kernel<<<batch, ORTH_THREADS, 0, s>>>(R, n, out);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("orth_error launch", e);
 }
