@@ -121,15 +121,23 @@ __device__ __forceinline__ uint4 codes8_f16(uint32_t w0, uint32_t w1) {
                     prmt(w1, 0u, 0x4342u));
 }
 
-// One token row of a head: BITS * 8 bytes of K codes, as many of V.
+// A thread's share of the next tile (its prefetch): BITS 16-byte chunks of K
+// codes and the scales and zero points of the token row it owns.  The code
+// chunks are loaded warp-cooperatively: warp w covers rows 32 w .. 32 w + 31,
+// and one load instruction of the warp reads 32 / CPR whole rows (CPR = RB /
+// 16 chunks per row), lane l taking chunk l % CPR of row l / CPR, so every
+// instruction reads full 128-byte lines (a row per thread would touch 32 lines
+// per instruction: consecutive tokens of a head are hkv * RB bytes apart).
+// V codes are loaded the same way at the start of their own tile, in flight
+// while the K codes are widened and the score product runs.
 template <int BITS>
 struct Row {
-  uint4 k[BITS], v[BITS];
+  uint4 k[BITS];
   float sk, zk, sv, zv;
 };
 
 template <int BITS>
-__global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
+__global__ void __launch_bounds__(THREADS, 4) kv_decode_tc_kernel(Params P) {
   constexpr int RB = D * BITS / 8;         // cache bytes per token and head
   extern __shared__ uint8_t kvd_smem_raw[];
   uint8_t* smem = kvd_smem_raw + ((1024u - (smem_u32(kvd_smem_raw) & 1023u)) & 1023u);
@@ -155,24 +163,30 @@ __global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
   const int64_t row_stride = static_cast<int64_t>(P.hkv) * RB;
   const int64_t row0 = static_cast<int64_t>(b) * P.S_max;
 
-  auto load_row = [&](int tok, Row<BITS>& r) {
-    if (tok < t1) {
-      const int64_t off = (row0 + tok) * row_stride + kh * RB;
-      const uint4* kp = reinterpret_cast<const uint4*>(P.kc + off);
-      const uint4* vp = reinterpret_cast<const uint4*>(P.vc + off);
+  constexpr int CPR = RB / 16;             // 16-byte chunks per row: 4 or 8
+  constexpr int RPI = 32 / CPR;            // rows per warp instruction: 8 or 4
+  static_assert(RPI * BITS == 32, "a warp's BITS instructions cover its 32 rows");
+  const int lane_row = lane / CPR, lane_chunk = lane % CPR;
+  // codes of the tile starting at token tt: chunk lane_chunk of rows
+  // 32 warp + RPI i + lane_row
+  auto load_codes = [&](const uint8_t* base, int tt, uint4 (&v)[BITS]) {
 #pragma unroll
-      for (int i = 0; i < BITS; ++i) {
-        r.k[i] = __ldg(kp + i);
-        r.v[i] = __ldg(vp + i);
-      }
+    for (int i = 0; i < BITS; ++i) {
+      const int tok = tt + 32 * warp + RPI * i + lane_row;
+      v[i] = tok < t1 ? __ldg(reinterpret_cast<const uint4*>(
+                            base + (row0 + tok) * row_stride + kh * RB) + lane_chunk)
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto load_row = [&](int tok, Row<BITS>& r) {
+    load_codes(P.kc, tok - tid, r.k);
+    if (tok < t1) {
       const int64_t g = (row0 + tok) * P.hkv + kh;
       r.sk = __ldg(P.ks + g);
       r.zk = static_cast<float>(__ldg(P.kz + g));
       r.sv = __ldg(P.vs + g);
       r.zv = static_cast<float>(__ldg(P.vz + g));
     } else {
-#pragma unroll
-      for (int i = 0; i < BITS; ++i) r.k[i] = r.v[i] = make_uint4(0u, 0u, 0u, 0u);
       r.sk = r.zk = r.sv = r.zv = 0.f;
     }
   };
@@ -232,17 +246,24 @@ __global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
     qsum[h] = red2[h] + red2[8 + h] + red2[16 + h] + red2[24 + h];
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
 
+  // widen this thread's chunks into the f16 tile: a 16-byte chunk c holds
+  // elements 32 c .. 32 c + 31 (4-bit) or 16 c .. 16 c + 15 (8-bit), i.e.
+  // f16 chunks 4 c .. 4 c + 3 or 2 c, 2 c + 1 of its row
   auto store_codes = [&](const uint4 (&w)[BITS]) {
 #pragma unroll
     for (int i = 0; i < BITS; ++i) {
+      const int row = 32 * warp + RPI * i + lane_row;
       const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
       if (BITS == 4) {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(At + sw_off(tid, 4 * i + e, A_ATOM)) = codes_f16(ws[e]);
+          *reinterpret_cast<uint4*>(At + sw_off(row, 4 * lane_chunk + e, A_ATOM)) =
+              codes_f16(ws[e]);
       } else {
-        *reinterpret_cast<uint4*>(At + sw_off(tid, 2 * i, A_ATOM)) = codes8_f16(ws[0], ws[1]);
-        *reinterpret_cast<uint4*>(At + sw_off(tid, 2 * i + 1, A_ATOM)) = codes8_f16(ws[2], ws[3]);
+        *reinterpret_cast<uint4*>(At + sw_off(row, 2 * lane_chunk, A_ATOM)) =
+            codes8_f16(ws[0], ws[1]);
+        *reinterpret_cast<uint4*>(At + sw_off(row, 2 * lane_chunk + 1, A_ATOM)) =
+            codes8_f16(ws[2], ws[3]);
       }
     }
   };
@@ -258,10 +279,12 @@ __global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
   for (int it = 0; it < ntiles && ok; ++it) {
     const int tok = t0 + it * TILE + tid;
     const bool valid = tok < t1;
-    Row<BITS> nxt;
-    if (it + 1 < ntiles) load_row(tok + TILE, nxt);
+    uint4 vcur[BITS];
+    load_codes(P.vc, tok - tid, vcur);
     // scores: K codes of the tile, then the product with the queries
     store_codes(cur.k);
+    Row<BITS> nxt;
+    if (it + 1 < ntiles) load_row(tok + TILE, nxt);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -280,7 +303,7 @@ __global__ void __launch_bounds__(THREADS) kv_decode_tc_kernel(Params P) {
     tmem_ld16(lane_addr, s16);
     tmem_ld_wait();
     // the tile buffer is free again: V codes
-    store_codes(cur.v);
+    store_codes(vcur);
     float sc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h)
