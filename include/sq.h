@@ -347,9 +347,10 @@ sq_status sq_r2_prepare(const float* x, const float* w, int64_t T, int H, int d,
 /* sq_r2_loss_grad -- the loss above at R (device float32 [d][d]) into *loss
  * (device float64), and, when grad is not NULL, its straight-through gradient
  * with respect to R into grad (device float64 [d][d]).  x, w and the
- * workspace as given to sq_r2_prepare.  Errors: shape and pointer checks as
- * sq_r2_prepare; a device-side wait that runs out is reported by
- * sq_device_status(). */
+ * workspace as given to sq_r2_prepare (a workspace that has not been through
+ * it gives meaningless values; nothing checks that on the device).  Errors:
+ * shape and pointer checks as sq_r2_prepare, loss and grad 8-byte aligned; a
+ * device-side wait that runs out is reported by sq_device_status(). */
 sq_status sq_r2_loss_grad(const float* x, const float* w, const float* R, int64_t T, int H, int d,
                           int64_t N, double* loss, double* grad, void* workspace,
                           size_t workspace_bytes, void* stream);
@@ -387,7 +388,8 @@ sq_status sq_cayley_update(const double* R, const double* G, double alpha, int n
 sq_status sq_r2_random_hadamard(const int8_t* signs, int d, int batch, double* R, void* stream);
 
 /* sq_orth_error -- out[b] = ||R_b^T R_b - I||_F (float64, device) for each
- * of `batch` n x n float64 matrices; 1 <= n <= 128. */
+ * of `batch` n x n float64 matrices; 1 <= n <= 128.  R and out 8-byte
+ * aligned (SQ_ERR_MISALIGNED otherwise). */
 sq_status sq_orth_error(const double* R, int n, int batch, double* out, void* stream);
 
 /* sq_rope_tables -- the cos/sin tables the KV call reads:

@@ -93,6 +93,7 @@ using sq::host::set_error;
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 sq_status precheck_device() {
   if (sq::host::current_device() < 0) return SQ_ERR_CUDA;
@@ -543,8 +544,9 @@ sq_status sq_r2_loss_grad(const float* x, const float* w, const float* R, int64_
     set_error("null pointer argument");
     return SQ_ERR_INVALID_ARG;
   }
-  if (!aligned16(x) || !aligned16(w) || !aligned16(R) || !aligned16(workspace)) {
-    set_error("x, w, R and the workspace must be 16-byte aligned");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(R) || !aligned16(workspace) ||
+      !aligned8(loss) || (grad && !aligned8(grad))) {
+    set_error("x, w, R and the workspace must be 16-byte aligned, loss and grad 8-byte");
     return SQ_ERR_MISALIGNED;
   }
   st = precheck_device();
@@ -572,8 +574,8 @@ sq_status sq_r2_cayley_learn(const float* x, const float* w, const double* R0, i
     return SQ_ERR_INVALID_ARG;
   }
   if (!aligned16(x) || !aligned16(w) || !aligned16(R0) || !aligned16(R) ||
-      !aligned16(workspace)) {
-    set_error("x, w, R0, R and the workspace must be 16-byte aligned");
+      !aligned16(workspace) || !aligned8(losses)) {
+    set_error("x, w, R0, R and the workspace must be 16-byte aligned, losses 8-byte");
     return SQ_ERR_MISALIGNED;
   }
   st = precheck_device();
@@ -631,6 +633,10 @@ sq_status sq_r2_random_hadamard(const int8_t* signs, int d, int batch, double* R
     set_error("null pointer argument");
     return SQ_ERR_INVALID_ARG;
   }
+  if (!aligned8(R)) {
+    set_error("R must be 8-byte aligned");
+    return SQ_ERR_MISALIGNED;
+  }
   sq_status st = precheck_device();
   if (st != SQ_OK) return st;
   return sq::r2::random_hadamard(signs, d, batch, R, static_cast<cudaStream_t>(stream));
@@ -645,6 +651,10 @@ sq_status sq_orth_error(const double* R, int n, int batch, double* out, void* st
   if (!R || !out) {
     set_error("null pointer argument");
     return SQ_ERR_INVALID_ARG;
+  }
+  if (!aligned8(R) || !aligned8(out)) {
+    set_error("R and out must be 8-byte aligned");
+    return SQ_ERR_MISALIGNED;
   }
   sq_status st = precheck_device();
   if (st != SQ_OK) return st;

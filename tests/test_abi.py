@@ -118,6 +118,12 @@ def test_validation_happens_before_any_launch(sq):
     assert lib.sq_cayley_update(None, None, 0.1, 16, 1, None, None, None, 0, None) == 1
     assert lib.sq_cayley_workspace_bytes(128, 2) == 2 * 2 * 128 * 128 * 8
     assert lib.sq_orth_error(None, 0, 1, None, None) == 1
+    # float64 device pointers must be 8-byte aligned (checked before any launch)
+    assert lib.sq_orth_error(0x1004, 16, 1, 0x2000, None) == 3
+    assert lib.sq_r2_random_hadamard(0x1000, 128, 1, 0x2004, None) == 3
+    assert lib.sq_r2_random_hadamard(0x1000, 96, 1, 0x2000, None) == 1      # not a power of 2
+    assert lib.sq_r2_loss_grad(0x1000, 0x2000, 0x3000, 64, 4, 128, 256, 0x4004, None,
+                               0x5000, 1 << 30, None) == 3
 
 
 def test_product_paley_matches_oracle():
