@@ -419,21 +419,24 @@ def run_ours(args, rank, world, local_rank):
 
 # ------------------------------------------------------------ oracle arm
 
-def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
+def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None, prepared=None):
     """Time the CPU oracle on rows x cols of the workload; extrapolate one full step.
 
     The oracle's step is rotate+quant of x (cost per row) then the integer GEMM
     and dequant (cost per row x column).  Weight codes are prepared offline and
-    not timed, as on the GPU side.
+    not timed, as on the GPU side; `prepared` (the result's "prepared" entry)
+    reuses them.
     """
-    import numpy as np
     from oracle import oracle as O
     from workloads import synthetic as W
 
-    wl = W.down_proj(M=rows, K=K, N=cols, seed=1001)
-    x = wl.x.double().numpy()
-    wp, ws, _ = O.quantize_weights(wl.w.double().numpy(), N_SMALL, N_POW2)
-    O.rotate_quant(x[:2], N_SMALL, N_POW2)          # builds and caches the dense H
+    if prepared is None:
+        wl = W.down_proj(M=rows, K=K, N=cols, seed=1001)
+        x = wl.x.double().numpy()
+        wp, ws, _ = O.quantize_weights(wl.w.double().numpy(), N_SMALL, N_POW2)
+        O.rotate_quant(x[:2], N_SMALL, N_POW2)      # builds and caches the dense H
+        prepared = (x, wp, ws)
+    x, wp, ws = prepared
     t_rot, t_gemm, n = 0.0, 0.0, 0
     t_start = time.perf_counter()
     while True:
@@ -458,7 +461,8 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None):
     return {"value": OPS / full_s / 1e12, "unit": "TOPS", "cores": int(cores), "kind": "oracle",
             "sample": "%d rows x %d cols of the workload, %d repetitions (%.1f s), extrapolated "
                       "to one full step (rotation cost per row, GEMM cost per row x col)"
-                      % (rows, cols, n, t_rot + t_gemm), "full_step_s": full_s}
+                      % (rows, cols, n, t_rot + t_gemm), "full_step_s": full_s,
+            "prepared": prepared}
 
 
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
@@ -686,6 +690,15 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample()
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        # the same sample on one host thread (the BLAS pool limited to 1)
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                one = oracle_sample(min_seconds=5.0, prepared=cb["prepared"])
+            cpu["one_thread"] = {"value": one["value"], "unit": "TOPS", "cores": 1,
+                                 "sample": one["sample"]}
+        except ImportError:
+            pass
     from rotation_ptq_b200.shard import job_rate
     # whole job: every rank's M tokens over the slowest rank's step time
     tops_job = job_rate(world * OPS, r["ms_step"] * 1e-3) / 1e12
