@@ -16,7 +16,7 @@ Citations name the page and section they restate:
   * "SpinQuant, Reproduced", Q1-Q13: the third-party reproduction page.
   * "SpinQuant abstract": the arXiv abstract reproduced on several pages.
 
-Readings of points the pages leave open (each listed in the design doc):
+Readings of points the pages leave open:
   * Hadamard matrices: Sylvester H_{2^k}[a][b] = (-1)^popcount(a&b) in natural
     order; Paley-I H12 from the quadratic residues mod 11; H12 (x) H_{2^k} with
     H12 on the outer channel index; row-vector convention y = x H.
@@ -35,6 +35,11 @@ Readings of points the pages leave open (each listed in the design doc):
   * Decode attention over the 4-bit caches: query head h reads KV head
     h // (hq / hkv); softmax(q k^T / sqrt(d)) v over the first lengths[b]
     cache rows b * S_max + s of sequence b.
+  * 8-bit KV cache: the asymmetric 4-bit rule on the grid 0..255.
+  * Cayley SGD for R2: Y = R G^T - G R^T from the Euclidean gradient; the
+    objective is o_proj's W4A4 output error with its input rotated head-wise;
+    the straight-through estimator passes each quantizer's output gradient to
+    its input; a random Hadamard is diag(s) H_d / sqrt(d).
 
 Parity pins: every function below is checked in tests/test_oracle_pins.py
 against closed forms, brute force or invariants that do not reuse it.
