@@ -14,6 +14,23 @@
  * all data layouts are readings of points the pages leave open; each is
  * stated below at the call that uses it.
  *
+ * Entry points, by group
+ *   - W4A4 path: sq_rotate_quant (online R4 + per-token INT4),
+ *     sq_swiglu_rotate_quant (the SwiGLU product fused in front of it),
+ *     sq_w4a4_linear (+ _workspace_bytes, _tail_workspace_bytes, _noalloc).
+ *   - KV path: sq_rope_tables, sq_kv_rotate_quant (RoPE + R3 + 4-bit caches),
+ *     sq_kv_dequant, sq_kv4_decode_attention (+ _workspace_bytes).
+ *   - W4A8KV8 ("SpinQuant, Reproduced", Q7): sq_rotate_quant8,
+ *     sq_w4a8_linear, sq_kv_rotate_quant8, sq_kv8_dequant,
+ *     sq_kv8_decode_attention.
+ *   - R2 learner ("SpinQuant, Reproduced", Q6; offline): sq_r2_prepare,
+ *     sq_r2_loss_grad, sq_r2_cayley_learn (+ sq_r2_workspace_bytes),
+ *     sq_cayley_update (+ _workspace_bytes), sq_orth_error,
+ *     sq_r2_random_hadamard.  Their float64 pointers need only 8-byte
+ *     alignment.
+ *   - Status: sq_version, sq_status_string, sq_last_error, sq_device_status, and test
+ *     hooks sq_debug_set_spin_limit, sq_debug_set_gemm_path.
+ *
  * Conventions for every call
  *   - Plain C; nothing throws across the ABI.
  *   - Every tensor pointer is caller-owned DEVICE memory unless the argument
