@@ -231,6 +231,18 @@ def _r2_grad_transposed(x, w, R, want_grad=True):
     return loss, (None if G is None else G.T)
 
 
+def _orth_error_max_abs(R):
+    R = np.asarray(R, np.float64)
+    return float(np.abs(R.T @ R - np.eye(R.shape[0])).max())
+
+
+def _headwise_transposed(x, R):
+    x = np.asarray(x, np.float64)
+    d = R.shape[0]
+    rows, K = x.shape
+    return (x.reshape(rows, K // d, d) @ np.asarray(R, np.float64).T).reshape(rows, K)
+
+
 def _random_hadamard_signs_after(signs):
     s = np.asarray(signs, np.float64)
     d = s.shape[0]
@@ -275,6 +287,8 @@ MUTATIONS = {
     "r2_grad_drops_weight_term": ("r2_loss_grad", _r2_grad_no_weight_term),
     "r2_grad_transposed": ("r2_loss_grad", _r2_grad_transposed),
     "random_hadamard_signs_on_columns": ("random_hadamard", _random_hadamard_signs_after),
+    "orth_error_max_abs": ("orth_error", _orth_error_max_abs),
+    "headwise_uses_transpose": ("headwise", _headwise_transposed),
 }
 
 PIN_TESTS = [
@@ -320,6 +334,7 @@ PIN_TESTS = [
     P.test_headwise_rotation_is_invisible_at_full_precision,
     P.test_r2_loss_at_identity_is_the_plain_w4a4_error,
     P.test_r2_ste_gradient_is_the_frozen_noise_derivative,
+    P.test_orth_error_closed_forms,
 ]
 
 

@@ -642,6 +642,15 @@ def test_random_hadamard_is_orthogonal_with_signed_rows():
     assert np.allclose(R * math.sqrt(128), s[:, None] * H)
 
 
+def test_orth_error_closed_forms():
+    # ||R^T R - I||_F = sqrt(sum (sigma_i^2 - 1)^2): diag(2, 1) gives 3, and
+    # [[1, 2], [0, 1]] (R^T R = [[1, 2], [2, 5]]) gives sqrt(24)
+    assert math.isclose(O.orth_error(np.diag([2.0, 1.0])), 3.0, rel_tol=1e-15)
+    assert math.isclose(O.orth_error(np.array([[1.0, 2.0], [0.0, 1.0]])), math.sqrt(24.0),
+                        rel_tol=1e-15)
+    assert O.orth_error(np.eye(7)) == 0.0
+
+
 def test_headwise_rotation_is_invisible_at_full_precision():
     rng = np.random.default_rng(114)
     x = rng.standard_normal((6, 4 * 16))
