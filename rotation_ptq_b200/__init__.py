@@ -29,6 +29,7 @@ from .binding import (  # noqa: F401
     SqError,
     debug_set_gemm_path,
     debug_set_spin_limit,
+    SPIN_FAIL_AT_ONCE,
     device_status,
     kv4_decode_attention,
     kv4_decode_workspace_bytes,

@@ -125,6 +125,36 @@ def _need_cuda(*ts):
             raise ValueError("rotation_ptq_b200 takes CUDA tensors (no CPU path)")
 
 
+SQ_ERR_TIMEOUT = 5
+
+
+def _expect(t, name, dtype, shape):
+    """Reject a tensor whose dtype, shape or layout the C entry point would
+    misread (a short or mistyped buffer would be read or written past its end
+    on the device)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _same_device(*ts):
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError("all tensors must be on one device, got %s" % sorted(map(str, devs)))
+
+
+def _expect_workspace(ws):
+    if ws is None:
+        return
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor")
+
+
 def rotate_quant(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float = 1.0,
                  a_q: torch.Tensor = None, a_scale: torch.Tensor = None):
     """Online rotation + per-token INT4 (``sq_rotate_quant``).
@@ -132,7 +162,6 @@ def rotate_quant(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float =
     x: CUDA [M, K] bf16 or float32 (unit stride along K).  had_small: None or a
     host +-1 int8 matrix [n, n].  Returns (a_q uint8 [M, K/2], a_scale f32 [M]).
     """
-    _need_cuda(x)
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit stride along K")
     if x.dtype == torch.bfloat16:
@@ -150,10 +179,18 @@ def rotate_quant(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float =
         if hs.shape != (n_small, n_small):
             raise ValueError("had_small must be square")
         hs_ptr = hs.ctypes.data
+    if K % 2:
+        raise ValueError("K must be even")
+    if a_q is not None:
+        _expect(a_q, "a_q", torch.uint8, (M, K // 2))
+    if a_scale is not None:
+        _expect(a_scale, "a_scale", torch.float32, (M,))
+    _same_device(x, a_q, a_scale)
     if a_q is None:
         a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if a_scale is None:
         a_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need_cuda(x, a_q, a_scale)
     st = lib.sq_rotate_quant(x.data_ptr(), dt, M, K, x.stride(0), hs_ptr, n_small, n_pow2,
                              float(clip), a_q.data_ptr(), a_scale.data_ptr(), _stream(x))
     _check(st, "sq_rotate_quant")
@@ -176,7 +213,6 @@ def rotate_quant8(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float 
 
     x: CUDA [M, K] bf16 or float32.  Returns (a_q int8 [M, K], a_scale f32 [M]).
     """
-    _need_cuda(x)
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit stride along K")
     if x.dtype == torch.bfloat16:
@@ -187,6 +223,12 @@ def rotate_quant8(x: torch.Tensor, had_small=None, n_pow2: int = 1, clip: float 
         raise ValueError("x must be bf16 or float32")
     M, K = x.shape
     hs, n_small, hs_ptr = _small_hadamard(had_small)
+    if a_q is not None:
+        _expect(a_q, "a_q", torch.int8, (M, K))
+    if a_scale is not None:
+        _expect(a_scale, "a_scale", torch.float32, (M,))
+    _same_device(x, a_q, a_scale)
+    _need_cuda(x, a_q, a_scale)
     if a_q is None:
         a_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if a_scale is None:
@@ -206,14 +248,19 @@ def swiglu_rotate_quant(gate_up: torch.Tensor, had_small=None, n_pow2: int = 1,
     half its width (gate = columns [0, K), up = [K, 2K)).  Returns
     (a_q uint8 [M, K/2], a_scale f32 [M]).
     """
-    _need_cuda(gate_up)
     if gate_up.dim() != 2 or gate_up.stride(1) != 1 or gate_up.dtype != torch.bfloat16:
         raise ValueError("gate_up must be a 2-D bf16 tensor with unit stride along columns")
     M, W2 = gate_up.shape
-    if W2 % 2:
-        raise ValueError("gate_up width must be even ([gate | up])")
+    if W2 % 4:
+        raise ValueError("gate_up width must be 2K with K even ([gate | up])")
     K = W2 // 2
     hs, n_small, hs_ptr = _small_hadamard(had_small)
+    if a_q is not None:
+        _expect(a_q, "a_q", torch.uint8, (M, K // 2))
+    if a_scale is not None:
+        _expect(a_scale, "a_scale", torch.float32, (M,))
+    _same_device(gate_up, a_q, a_scale)
+    _need_cuda(gate_up, a_q, a_scale)
     if a_q is None:
         a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=gate_up.device)
     if a_scale is None:
@@ -236,6 +283,20 @@ def quantize_weights(w: torch.Tensor, had_small=None, n_pow2: int = 1):
 
 _ws_lock = threading.Lock()
 _ws_cache = {}
+
+
+def _reset_workspaces(device_index: int) -> None:
+    """Zero every cached workspace of a device.  The library leaves a
+    workspace zero after each call that completes; a call whose device waits
+    ran out (SQ_ERR_TIMEOUT) can leave partial sums and arrival counters in
+    it, which the next call would otherwise add to."""
+    with _ws_lock:
+        bufs = [b for (d, _), b in _ws_cache.items() if d == device_index]
+    if bufs:
+        torch.cuda.synchronize(device_index)
+        for b in bufs:
+            b.zero_()
+        torch.cuda.synchronize(device_index)
 
 
 def _workspace(device: torch.device, stream: int, nbytes: int) -> torch.Tensor:
@@ -265,10 +326,20 @@ def w4a4_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
     a_q [M, K/2], a_scale [M], w_q [N, K/2], w_scale [N] on one CUDA device.
     Returns bf16 [M, N] (or int32 accumulators with out_int32=True).
     """
-    _need_cuda(a_q, a_scale, w_q, w_scale)
+    if a_q.dim() != 2 or w_q.dim() != 2:
+        raise ValueError("a_q must be [M, K/2] and w_q [N, K/2]")
     M, Kh = a_q.shape
     N = w_q.shape[0]
     K = 2 * Kh
+    _expect(a_q, "a_q", torch.uint8, (M, Kh))
+    _expect(a_scale, "a_scale", torch.float32, (M,))
+    _expect(w_q, "w_q", torch.uint8, (N, Kh))
+    _expect(w_scale, "w_scale", torch.float32, (N,))
+    if out is not None:
+        _expect(out, "out", torch.int32 if out_int32 else torch.bfloat16, (M, N))
+    _expect_workspace(workspace)
+    _same_device(a_q, a_scale, w_q, w_scale, out, workspace)
+    _need_cuda(a_q, a_scale, w_q, w_scale, out, workspace)
     if out is None:
         out = torch.empty((M, N), dtype=torch.int32 if out_int32 else torch.bfloat16,
                           device=a_q.device)
@@ -319,14 +390,26 @@ def kv8_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.
 
 def _kv_decode(fn, name, q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, S_max,
                out, workspace):
-    _need_cuda(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths)
+    if q.dim() != 3 or k_scale.dim() != 2:
+        raise ValueError("q must be [B, hq, d] and the scales [B * S_max, hkv]")
     B, hq, d = q.shape
     hkv = k_scale.shape[1]
-    for t, dt in ((q, torch.bfloat16), (k_cache, torch.uint8), (v_cache, torch.uint8),
-                  (k_scale, torch.float32), (v_scale, torch.float32), (k_zero, torch.uint8),
-                  (v_zero, torch.uint8), (lengths, torch.int32)):
-        if t.dtype != dt or not t.is_contiguous():
-            raise ValueError("decode attention inputs must be contiguous with the documented dtypes")
+    rows = B * S_max
+    row_bytes = k_cache.shape[-1] if k_cache.dim() == 3 else -1
+    _expect(q, "q", torch.bfloat16, (B, hq, d))
+    for nm, c, sc, z in (("k", k_cache, k_scale, k_zero), ("v", v_cache, v_scale, v_zero)):
+        _expect(c, nm + "_cache", torch.uint8, (rows, hkv, row_bytes))
+        _expect(sc, nm + "_scale", torch.float32, (rows, hkv))
+        _expect(z, nm + "_zero", torch.uint8, (rows, hkv))
+    if row_bytes != (d // 2 if fn is lib.sq_kv4_decode_attention else d):
+        raise ValueError("cache rows must hold %s bytes per head vector"
+                         % ("d/2" if fn is lib.sq_kv4_decode_attention else "d"))
+    _expect(lengths, "lengths", torch.int32, (B,))
+    if out is not None:
+        _expect(out, "out", torch.bfloat16, (B, hq, d))
+    _expect_workspace(workspace)
+    _same_device(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, out, workspace)
+    _need_cuda(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero, lengths, out, workspace)
     if out is None:
         out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=q.device)
     stream = _stream(q)
@@ -350,13 +433,21 @@ def w4a8_linear(a_q: torch.Tensor, a_scale: torch.Tensor, w_q: torch.Tensor,
     a_q: int8 [M, K] (from rotate_quant8); w_q: uint8 [N, K/2].  Returns bf16
     (or, with out_i32, the exact int32 sums) [M, N].
     """
-    _need_cuda(a_q, a_scale, w_q, w_scale)
-    if a_q.dtype != torch.int8 or w_q.dtype != torch.uint8:
+    if a_q.dim() != 2 or w_q.dim() != 2:
         raise ValueError("a_q must be int8 [M, K] and w_q uint8 [N, K/2]")
     M, K = a_q.shape
     N = w_q.shape[0]
-    if w_q.shape[1] * 2 != K:
-        raise ValueError("w_q must be [N, K/2]")
+    if K % 2:
+        raise ValueError("K must be even")
+    _expect(a_q, "a_q", torch.int8, (M, K))
+    _expect(a_scale, "a_scale", torch.float32, (M,))
+    _expect(w_q, "w_q", torch.uint8, (N, K // 2))
+    _expect(w_scale, "w_scale", torch.float32, (N,))
+    if out is not None:
+        _expect(out, "out", torch.int32 if out_i32 else torch.bfloat16, (M, N))
+    _expect_workspace(workspace)
+    _same_device(a_q, a_scale, w_q, w_scale, out, workspace)
+    _need_cuda(a_q, a_scale, w_q, w_scale, out, workspace)
     if out is None:
         out = torch.empty((M, N), dtype=torch.int32 if out_i32 else torch.bfloat16,
                           device=a_q.device)
@@ -403,10 +494,34 @@ def kv_rotate_quant8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: tor
 
 
 def _kv_rotate_quant(fn, name, per_byte, q, k, v, pos, cos, sin, out):
-    _need_cuda(q, k, v, pos, cos, sin)
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q must be [T, hq, d] and k, v [T, hkv, d]")
     T, hq, d = q.shape
     hkv = k.shape[1]
+    _expect(q, "q", torch.bfloat16, (T, hq, d))
+    _expect(k, "k", torch.bfloat16, (T, hkv, d))
+    _expect(v, "v", torch.bfloat16, (T, hkv, d))
+    _expect(pos, "pos", torch.int32, (T,))
+    if (cos is None) != (sin is None):
+        raise ValueError("cos and sin must both be given or both be None")
+    if cos is not None:
+        if cos.dim() != 2:
+            raise ValueError("cos must be [max_pos, d/2]")
+        _expect(cos, "cos", torch.float32, (cos.shape[0], d // 2))
+        _expect(sin, "sin", torch.float32, tuple(cos.shape))
     dev = q.device
+    if out is not None:
+        shapes = dict(q_out=((T, hq, d), torch.bfloat16),
+                      k_cache=((T, hkv, d // per_byte), torch.uint8),
+                      k_scale=((T, hkv), torch.float32), k_zero=((T, hkv), torch.uint8),
+                      v_cache=((T, hkv, d // per_byte), torch.uint8),
+                      v_scale=((T, hkv), torch.float32), v_zero=((T, hkv), torch.uint8))
+        for key, (shp, dt) in shapes.items():
+            if key not in out:
+                raise ValueError("out is missing %s" % key)
+            _expect(out[key], "out[%s]" % key, dt, shp)
+    _same_device(q, k, v, pos, cos, sin, *(out.values() if out is not None else ()))
+    _need_cuda(q, k, v, pos, cos, sin, *(out.values() if out is not None else ()))
     if out is None:
         out = dict(
             q_out=torch.empty_like(q),
@@ -427,8 +542,16 @@ def _kv_rotate_quant(fn, name, per_byte, q, k, v, pos, cos, sin, out):
 
 def kv_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out=None):
     """Packed asymmetric cache [T, h, 64] -> bf16 [T, h, 128] (``sq_kv_dequant``)."""
-    _need_cuda(cache, scale, zero)
+    if cache.dim() != 3:
+        raise ValueError("cache must be [T, h, 64]")
     T, h, dh = cache.shape
+    _expect(cache, "cache", torch.uint8, (T, h, dh))
+    _expect(scale, "scale", torch.float32, (T, h))
+    _expect(zero, "zero", torch.uint8, (T, h))
+    if out is not None:
+        _expect(out, "out", torch.bfloat16, (T, h, 2 * dh))
+    _same_device(cache, scale, zero, out)
+    _need_cuda(cache, scale, zero, out)
     if out is None:
         out = torch.empty((T, h, 2 * dh), dtype=torch.bfloat16, device=cache.device)
     st = lib.sq_kv_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, 2 * dh,
@@ -439,8 +562,16 @@ def kv_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out
 
 def kv8_dequant(cache: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, out=None):
     """8-bit asymmetric cache [T, h, 128] -> bf16 [T, h, 128] (``sq_kv8_dequant``)."""
-    _need_cuda(cache, scale, zero)
+    if cache.dim() != 3:
+        raise ValueError("cache must be [T, h, 128]")
     T, h, d = cache.shape
+    _expect(cache, "cache", torch.uint8, (T, h, d))
+    _expect(scale, "scale", torch.float32, (T, h))
+    _expect(zero, "zero", torch.uint8, (T, h))
+    if out is not None:
+        _expect(out, "out", torch.bfloat16, (T, h, d))
+    _same_device(cache, scale, zero, out)
+    _need_cuda(cache, scale, zero, out)
     if out is None:
         out = torch.empty((T, h, d), dtype=torch.bfloat16, device=cache.device)
     st = lib.sq_kv8_dequant(cache.data_ptr(), scale.data_ptr(), zero.data_ptr(), T, h, d,
@@ -548,16 +679,29 @@ def orth_error(R: torch.Tensor) -> torch.Tensor:
 
 
 def device_status(device=None) -> int:
-    """Synchronise the current stream and return (and clear) the device status word."""
+    """Synchronise the current stream and return (and clear) the device status word.
+
+    After SQ_ERR_TIMEOUT every cached workspace of the device is zeroed again
+    (a kernel that gave up may have left partial sums in it)."""
     dev = torch.device("cuda") if device is None else torch.device(device)
-    return int(lib.sq_device_status(torch.cuda.current_stream(dev).cuda_stream))
+    st = int(lib.sq_device_status(torch.cuda.current_stream(dev).cuda_stream))
+    if st == SQ_ERR_TIMEOUT:
+        idx = dev.index if dev.index is not None else torch.cuda.current_device()
+        _reset_workspaces(idx)
+    return st
+
+
+SPIN_FAIL_AT_ONCE = 0xFFFFFFFF
 
 
 def debug_set_spin_limit(polls: int) -> None:
+    """Test hook: polls per bounded device wait (0: the default bound;
+    SPIN_FAIL_AT_ONCE: every bounded wait gives up before its first poll)."""
     lib.sq_debug_set_spin_limit(int(polls))
 
 
 def debug_set_gemm_path(path: int) -> None:
     """0 = automatic, 1 = one-CTA tiles, 2 = CTA-pair tiles with both operands
-    widened in shared memory, 3 = CTA-pair tiles with A in tensor memory."""
+    widened in shared memory, 3 = CTA-pair tiles with A in tensor memory,
+    4 = the CUDA-core GEMV for M <= 8."""
     lib.sq_debug_set_gemm_path(int(path))

@@ -483,6 +483,9 @@ __global__ void __launch_bounds__(CG_THREADS, 1) codes_gemm_kernel(
         mma_commit(&empty[st]);
       }
       mma_commit(done);                    // completes once every issued MMA has
+      // finished writing tensor memory; the CTA frees it only after that,
+      // also when the epilogue's own wait gave up
+      mbar_wait(done, 0, 0);
     }
   } else {
     ok = mbar_wait(done, 0, spin_limit) && !*abort_flag;

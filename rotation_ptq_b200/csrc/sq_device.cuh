@@ -90,9 +90,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Default bound of a device wait: this many nanoseconds of polling.
 constexpr uint64_t kWaitNs = 2000000000ull;
 
+// A limit of kWaitFailAtOnce (a test setting) makes every bounded wait give
+// up before its first poll, so that a kernel's abort path runs from its very
+// first wait.  Waits given limit 0 (a CTA waiting for its own copies and
+// MMAs before it exits) are unaffected.
+constexpr uint32_t kWaitFailAtOnce = 0xFFFFFFFFu;
+
 // Poll an mbarrier phase.  Gives up after `limit` polls (when limit != 0) or
 // kWaitNs of wall time, records SQ_ERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  if (limit == kWaitFailAtOnce) {
+    record_status(SQ_ERR_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t polls = 1;; ++polls) {
@@ -336,6 +346,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // As mbar_wait, with cluster-scope acquire (arrivals come from the peer CTA).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  if (limit == kWaitFailAtOnce) {
+    record_status(SQ_ERR_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait_cluster(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t polls = 1;; ++polls) {
