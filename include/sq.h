@@ -154,18 +154,20 @@ sq_status sq_rotate_quant8(const void* x, sq_in_dtype x_dtype, int64_t M, int64_
  * For every row m and channel k < K:
  *     g = gate_up[m][k],  u = gate_up[m][K + k]              (gate half first)
  *     h[m][k] = bf16_round_nearest_even(silu(g) * u),  silu(g) = g / (1 + e^-g)
- * evaluated in float32; then exactly sq_rotate_quant on x = h (bf16).  h is
- * never written to memory.
+ * the exact product rounded once; then exactly sq_rotate_quant on x = h
+ * (bf16).  h is never written to memory.
  *
  * gate_up   device, bf16 [M][ld] (ld >= 2K, ld * 2 a multiple of 16 bytes),
  *           16-byte aligned; read only.
  * had_small, n_small, n_pow2, clip_ratio, a_q, a_scale: as sq_rotate_quant
  *           (a_q [M][K/2] packed codes, a_scale [M] float32, both written).
  * Shape rules and errors as sq_rotate_quant, with ld >= 2K; M == 0 is a
- * no-op.  The SwiGLU is evaluated with hardware exponential and reciprocal
- * approximations (a few float32 ulps), so h can differ from a correctly
- * rounded product in its last bf16 bit where the product lies next to a
- * rounding midpoint.
+ * no-op.  The product is evaluated in float32 with the hardware exponential
+ * and reciprocal approximations; where that value lies within their error
+ * bound of a bf16 rounding midpoint, or |g| > 60, it is recomputed in double
+ * precision before the single rounding, so h is the correctly rounded product
+ * except where the exact one lies within double-precision error of a
+ * midpoint.
  * ------------------------------------------------------------------------- */
 sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int64_t ld,
                                  const int8_t* had_small, int n_small, int n_pow2,
@@ -199,6 +201,10 @@ sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int6
  *           less, that wave runs whole.  Results are identical either way.
  * Shape rules: M >= 0 (0 is a no-op), N % 16 == 0, N >= 16, K % 128 == 0,
  * 128 <= K <= 65536 (so |acc| < 2^31).
+ * Ordering: for 5 <= M <= 32 the kernel is launched as a programmatic
+ * dependent (CUDA's programmatic stream serialization): it may set up while
+ * the preceding kernel of the stream finishes, and waits for that kernel's
+ * completion before it reads or writes any operand.
  * ------------------------------------------------------------------------- */
 sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
                          const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
@@ -283,6 +289,10 @@ sq_status sq_w4a8_linear(const int8_t* a_q, const float* a_scale, const uint8_t*
  *     lo = min(min x, 0), hi = max(max x, 0), scale = (hi - lo) / 15 (1 if 0),
  *     zero = clamp(rint(-lo / scale), 0, 15),
  *     code = clamp(rint(x / scale) + zero, 0, 15)      (float32, unsigned codes)
+ *   Precision: Q is rotated in float32.  K is rotated in double precision and
+ *   rounded once to float32, so y_k is the exact rotation rounded to float32
+ *   (but for double-precision near-ties); every quotient x / scale is the
+ *   correctly rounded float32 quotient.
  *
  * q         device, [T][hq][d] bf16.        k, v: device, [T][hkv][d] bf16.
  * pos       device, [T] int32, 0 <= pos < max_pos (out-of-range positions set
@@ -425,16 +435,26 @@ sq_status sq_device_status(void* stream);
 
 /* sq_debug_set_spin_limit -- test hook: the number of polls a device wait
  * makes before giving up (0 restores the default, which is a few seconds of
- * polling).  Applies to kernels launched afterwards from any thread. */
+ * polling).  SQ_SPIN_FAIL_AT_ONCE makes every bounded wait give up before
+ * its first poll, so that a kernel's abort path runs from its first wait;
+ * the waits with which a CTA lets its own copies and MMAs finish before it
+ * exits keep their default bound.  A kernel that gives up records
+ * SQ_ERR_TIMEOUT (read by sq_device_status); its outputs are then undefined,
+ * and a caller workspace it used must be zeroed again before reuse.
+ * Applies to kernels launched afterwards from any thread. */
+#define SQ_SPIN_FAIL_AT_ONCE 0xFFFFFFFFu
 void sq_debug_set_spin_limit(uint32_t polls);
 
-/* sq_debug_set_gemm_path -- test hook: which sq_w4a4_linear kernel large-M
- * shapes use.  0 = automatic (default), 1 = one-CTA 128-row tiles,
- * 2 = two-CTA 256-row tiles with both operands in shared memory (M >= 256
- * and N >= 256 only; smaller shapes keep
- * their automatic kernel), 3 = two-CTA tiles with the widened A operand in
- * tensor memory (the automatic choice for those shapes).  Results are
- * identical; only speed differs.
+/* sq_debug_set_gemm_path -- test hook: which sq_w4a4_linear kernel a shape
+ * uses.  0 = automatic (default: the CUDA-core GEMV for M <= 4, the
+ * persistent decode kernel for 5 <= M <= 32, the one-CTA kernel for
+ * 32 < M <= 128, CTA pairs above), 1 = one-CTA
+ * 128-row tiles, 2 = two-CTA 256-row tiles with both operands in shared
+ * memory (M >= 256 and N >= 256 only; smaller shapes keep their automatic
+ * kernel), 3 = two-CTA tiles with the widened A operand in tensor memory (the
+ * automatic choice for those shapes), 4 = the CUDA-core GEMV for M <= 8 (the
+ * one-CTA kernel for larger M below 129).  Results are identical; only speed
+ * differs.
  * Applies to calls made afterwards from any thread. */
 void sq_debug_set_gemm_path(int path);
 

@@ -9,23 +9,27 @@
 // bytes of packed nibbles (element 2j in the low nibble of byte j) at 4 bits,
 // [T][h][128] bytes at 8.
 //
-// Thread layout (rotate/quant): a CTA takes two tokens per iteration; each
-// head vector of 128 values is owned by 2 adjacent lanes.  Items are ordered
-// [Q of token 0 | Q of token 1 | K of both | V of both], so with 8 | hq and
-// 8 | hkv no warp mixes item kinds.  For Q and K the lane with sub-index s
-// holds elements s*32 + t and 64 + s*32 + t (t < 32) as float pairs: each
-// RoPE pair (i, i + 64) sits in one pair, the butterfly bits j0..j4 run
-// across the thread's pairs (f32x2), j6 inside each pair, and j5 = s takes
-// one shuffle with the partner lane.  V lanes hold 64 consecutive values.
+// Thread layout (rotate/quant): a CTA takes two tokens per iteration.  Items
+// are ordered [Q of token 0 | Q of token 1 | K of both | V of both], so with
+// 8 | hq and 8 | hkv no warp mixes item kinds.  A Q vector of 128 values is
+// owned by 2 adjacent lanes: the lane with sub-index s holds elements
+// s*32 + t and 64 + s*32 + t (t < 32) as float pairs, so each RoPE pair
+// (i, i + 64) sits in one pair, the butterfly bits j0..j4 run across the
+// thread's pairs (f32x2), j6 inside each pair, and j5 = s takes one shuffle
+// with the partner lane.  V lanes (2 per vector) hold 64 consecutive values.
+//
+// K is rotated in double precision, so that its codes are those of the exact
+// rotation rounded once to float32: 4 lanes per vector, lane s holding the
+// RoPE pairs i = 16 s + t (t < 16).  With P = c + s and M = c - s of the
+// RoPE tables, the Hadamard bit j6 folds into RoPE:
+//     A_i = r_i + r_{i+64} = x_i P_i + x_{i+64} M_i,
+//     B_i = r_i - r_{i+64} = x_i M_i - x_{i+64} P_i,
+// and the outputs y_c (c < 64) and y_{c+64} are H64 of A and of B; bits
+// j0..j3 run in-thread, j4 and j5 across the 4 lanes.
 //
 // Quantization follows the pinned asymmetric rule, with one division per
-// group for the scale and the zero point.  V codes use the exactly rounded
-// quotient x / scale (raw bf16 inputs meet exact .5 ties often); K codes are
-// clamp(rint(x * k + zero), 0, top) with k = norm / scale in float32, K being
-// rotated without the 1/sqrt(128) factor (its float32 rotation already
-// differs from the exact one in the last bits, so the codes can differ from
-// the oracle's only at a rounding tie); K's scale and zero point come from
-// the normalised extremes.
+// group for the scale and the zero point and the exactly rounded quotient
+// x / scale for every code.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -53,6 +57,21 @@ __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, float* v) {
   }
 }
 
+// 16 bf16 (32 bytes, 16-byte aligned) -> 16 floats.
+__device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* v) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint4 w = __ldcs(q + h);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[h * 8 + 2 * e] = __uint_as_float(ws[e] << 16);
+      v[h * 8 + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -67,15 +86,18 @@ __device__ __forceinline__ void store16_bf16(__nv_bfloat16* p, const float* v) {
   q[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// Asymmetric parameters of a group from its (normalised) extremes, with the
-// group's other lane: scale = (max' - min') / (2^BITS - 1),
-// zero = rint(-min' / scale).
-template <int BITS>
-__device__ __forceinline__ void asym_params2(float lo, float hi, unsigned pmask, float& scale,
-                                             float& zero) {
+// Asymmetric parameters of a group from its extremes, combined over the
+// group's LANES lanes (2 or 4 adjacent lanes in `pmask`):
+// scale = (max' - min') / (2^BITS - 1), zero = rint(-min' / scale).
+template <int BITS, int LANES = 2>
+__device__ __forceinline__ void asym_params(float lo, float hi, unsigned pmask, float& scale,
+                                            float& zero) {
   const float top = static_cast<float>((1 << BITS) - 1);
-  lo = fminf(lo, __shfl_xor_sync(pmask, lo, 1));
-  hi = fmaxf(hi, __shfl_xor_sync(pmask, hi, 1));
+#pragma unroll
+  for (int o = 1; o < LANES; o <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(pmask, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(pmask, hi, o));
+  }
   lo = fminf(lo, 0.f);
   hi = fmaxf(hi, 0.f);
   scale = __fdiv_rn(hi - lo, top);
@@ -95,28 +117,8 @@ __device__ __forceinline__ void pack_codes(const uint32_t (&u)[8], uint32_t* out
   }
 }
 
-// 8 unsigned codes clamp(rint(x k + zero), 0, 2^BITS - 1), packed; x given
-// as 4 float pairs.  For operands whose quotient by the scale must round
-// exactly as float32 division does (raw bf16 values meet exact .5 ties
-// often), see ucodes8_div.
-template <int BITS>
-__device__ __forceinline__ void ucodes8(const f2* x, f2 k2, f2 z2, uint32_t* out) {
-  const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
-  const float top = static_cast<float>((1 << BITS) - 1);
-  uint32_t u[8];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    f2 c = fma2(x[e], k2, z2);
-    c.x = fminf(fmaxf(c.x, 0.f), top);
-    c.y = fminf(fmaxf(c.y, 0.f), top);
-    c = add2(c, magic);
-    u[2 * e] = __float_as_uint(c.x);
-    u[2 * e + 1] = __float_as_uint(c.y);
-  }
-  pack_codes<BITS>(u, out);
-}
-
-// As ucodes8 with the quotient x / scale rounded exactly like IEEE float32
+// 8 unsigned codes clamp(rint(x / scale) + zero, 0, 2^BITS - 1), packed; x
+// given as 4 float pairs.  The quotient is rounded exactly like IEEE float32
 // division: q = x r, e = x - q s, q' = q + e r with r = RN(1 / s), the
 // one-step fma correction of Markstein ("IA-64 and Elementary Functions",
 // 2000), which yields the correctly rounded quotient when r is the correctly
@@ -139,8 +141,76 @@ __device__ __forceinline__ void ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2 z2,
   pack_codes<BITS>(u, out);
 }
 
+// One K head vector rotated in double precision (4 lanes per vector, see the
+// file comment): returns this lane's 32 outputs rounded once to float32,
+// ya[t] = y_{16 s + t} and yb[t] = y_{64 + 16 s + t}.
+template <bool ROPE>
+__device__ __forceinline__ void k_rotate_exact(const __nv_bfloat16* src, const float* rc,
+                                               const float* rs, int s, unsigned pmask, float* ya,
+                                               float* yb) {
+  float lo[16], hi[16];
+  load16_bf16(src + 16 * s, lo);
+  load16_bf16(src + 64 + 16 * s, hi);
+  double a[16], b[16];
+  if (ROPE) {
+    const float4* c4 = reinterpret_cast<const float4*>(rc + 16 * s);
+    const float4* s4 = reinterpret_cast<const float4*>(rs + 16 * s);
+#pragma unroll
+    for (int qd = 0; qd < 4; ++qd) {
+      const float4 c = __ldg(c4 + qd), sn = __ldg(s4 + qd);
+      const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {sn.x, sn.y, sn.z, sn.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 4 * qd + e;
+        const double P = static_cast<double>(cc[e]) + static_cast<double>(ss[e]);
+        const double Mn = static_cast<double>(cc[e]) - static_cast<double>(ss[e]);
+        const double xl = lo[t], xh = hi[t];
+        a[t] = fma(xl, P, xh * Mn);
+        b[t] = fma(xl, Mn, -(xh * P));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      a[t] = static_cast<double>(lo[t]) + static_cast<double>(hi[t]);
+      b[t] = static_cast<double>(lo[t]) - static_cast<double>(hi[t]);
+    }
+  }
+  // H64 over i = 16 s + t: bits j0..j3 in-thread
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      if ((t & h) == 0) {
+        const double a0 = a[t], a1 = a[t + h], b0 = b[t], b1 = b[t + h];
+        a[t] = a0 + a1;
+        a[t + h] = a0 - a1;
+        b[t] = b0 + b1;
+        b[t + h] = b0 - b1;
+      }
+    }
+  }
+  // bits j4, j5 across the vector's lanes: the lane with the bit set keeps
+  // partner - own, the other own + partner
+#pragma unroll
+  for (int m = 1; m < 4; m <<= 1) {
+    const double sg = (s & m) ? -1.0 : 1.0;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      a[t] = fma(sg, a[t], __shfl_xor_sync(pmask, a[t], m));
+      b[t] = fma(sg, b[t], __shfl_xor_sync(pmask, b[t], m));
+    }
+  }
+  constexpr double kNormD = 0.088388347648318440550;   // 1/sqrt(128)
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    ya[t] = static_cast<float>(a[t] * kNormD);
+    yb[t] = static_cast<float>(b[t] * kNormD);
+  }
+}
+
 template <bool ROPE, int BITS>
-__global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
+__global__ void __launch_bounds__(224) kv_rotate_quant_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int T, int hq, int hkv,
     const int32_t* __restrict__ pos, const float* __restrict__ rcos,
@@ -148,10 +218,10 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
     uint8_t* __restrict__ k_cache, float* __restrict__ k_scale, uint8_t* __restrict__ k_zero,
     uint8_t* __restrict__ v_cache, float* __restrict__ v_scale, uint8_t* __restrict__ v_zero) {
   constexpr int RB = D * BITS / 8;               // cache bytes per head vector
-  const int nq = 4 * hq, nk = 4 * hkv;           // lanes per token pair
-  const int items = nq + 2 * nk;
+  constexpr int WPG = BITS / 4;                  // code words per 8 codes
+  const int nq = 4 * hq, nk = 8 * hkv, nv = 4 * hkv;   // lanes per token pair
+  const int items = nq + nk + nv;
   const int lane = threadIdx.x & 31;
-  const unsigned pmask = 0x3u << (lane & 30);    // this vector's 2 lanes
   for (int t0 = 2 * blockIdx.x; t0 < T; t0 += 2 * gridDim.x) {
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
       int kind, tok, head, s;
@@ -159,14 +229,23 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
         kind = 0;
         tok = t0 + it / (2 * hq);
         head = (it % (2 * hq)) >> 1;
+        s = it & 1;
+      } else if (it < nq + nk) {
+        const int j = it - nq;
+        kind = 1;
+        tok = t0 + j / (4 * hkv);
+        head = (j % (4 * hkv)) >> 2;
+        s = j & 3;
       } else {
-        const int j = it < nq + nk ? it - nq : it - nq - nk;
-        kind = it < nq + nk ? 1 : 2;
+        const int j = it - nq - nk;
+        kind = 2;
         tok = t0 + j / (2 * hkv);
         head = (j % (2 * hkv)) >> 1;
+        s = j & 1;
       }
-      s = it & 1;
-      if (tok >= T) continue;                    // both lanes of a vector leave together
+      if (tok >= T) continue;                    // all lanes of a vector leave together
+      // this vector's 2 (Q, V) or 4 (K) lanes; nq and nq + nk are multiples of 4
+      const unsigned pmask = kind == 1 ? 0xFu << (lane & 28) : 0x3u << (lane & 30);
       if (kind == 2) {
         // V: 64 consecutive values, asymmetric BITS-bit
         const int64_t g = static_cast<int64_t>(tok) * hkv + head;
@@ -180,10 +259,9 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
           mx = fmaxf(mx, x[i]);
         }
         float scale, zero;
-        asym_params2<BITS>(mn, mx, pmask, scale, zero);
+        asym_params<BITS>(mn, mx, pmask, scale, zero);
         const float rs = __frcp_rn(scale);
         const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
-        constexpr int WPG = BITS / 4;            // words per 8 codes
         uint32_t w[8 * WPG];
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
@@ -209,9 +287,49 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
           continue;
         }
       }
-      const bool is_q = kind == 0;
-      const __nv_bfloat16* src = is_q ? q + (static_cast<int64_t>(tok) * hq + head) * D
-                                      : k + (static_cast<int64_t>(tok) * hkv + head) * D;
+      if (kind == 1) {
+        // K: exact rotation, then the asymmetric quantizer on its float32 values
+        const int64_t g = static_cast<int64_t>(tok) * hkv + head;
+        float ya[16], yb[16];
+        k_rotate_exact<ROPE>(k + g * D, rcos + static_cast<int64_t>(p) * 64,
+                             rsin + static_cast<int64_t>(p) * 64, s, pmask, ya, yb);
+        float mn = ya[0], mx = ya[0];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          mn = fminf(mn, fminf(ya[t], yb[t]));
+          mx = fmaxf(mx, fmaxf(ya[t], yb[t]));
+        }
+        float scale, zero;
+        asym_params<BITS, 4>(mn, mx, pmask, scale, zero);
+        const float rs = __frcp_rn(scale);
+        const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
+        uint32_t wl[2 * WPG], wh[2 * WPG];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          const f2 xl[4] = {f2{ya[8 * n], ya[8 * n + 1]}, f2{ya[8 * n + 2], ya[8 * n + 3]},
+                            f2{ya[8 * n + 4], ya[8 * n + 5]}, f2{ya[8 * n + 6], ya[8 * n + 7]}};
+          const f2 xh[4] = {f2{yb[8 * n], yb[8 * n + 1]}, f2{yb[8 * n + 2], yb[8 * n + 3]},
+                            f2{yb[8 * n + 4], yb[8 * n + 5]}, f2{yb[8 * n + 6], yb[8 * n + 7]}};
+          ucodes8_div<BITS>(xl, r2, sn2, z2, wl + WPG * n);
+          ucodes8_div<BITS>(xh, r2, sn2, z2, wh + WPG * n);
+        }
+        // elements 16 s .. 16 s + 15 and 64 + 16 s .. 64 + 16 s + 15
+        uint8_t* row = k_cache + g * RB;
+        if (BITS == 4) {
+          *reinterpret_cast<uint2*>(row + 8 * s) = make_uint2(wl[0], wl[1]);
+          *reinterpret_cast<uint2*>(row + 32 + 8 * s) = make_uint2(wh[0], wh[1]);
+        } else {
+          *reinterpret_cast<uint4*>(row + 16 * s) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          *reinterpret_cast<uint4*>(row + 64 + 16 * s) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        }
+        if (s == 0) {
+          k_scale[g] = scale;
+          k_zero[g] = static_cast<uint8_t>(zero);
+        }
+        continue;
+      }
+      // Q: float32 RoPE and rotation, bf16 out
+      const __nv_bfloat16* src = q + (static_cast<int64_t>(tok) * hq + head) * D;
       // w[t] = (element s*32 + t, element 64 + s*32 + t)
       f2 w[32];
       {
@@ -260,60 +378,21 @@ __global__ void __launch_bounds__(256) kv_rotate_quant_kernel(
           w[i] = fma2(s2, w[i], o);
         }
       }
-      if (is_q) {
-        const f2 n2{kNorm, kNorm};
-        __nv_bfloat16* dst = q_out + (static_cast<int64_t>(tok) * hq + head) * D;
-        uint32_t lo_w[16], hi_w[16];
+      const f2 n2{kNorm, kNorm};
+      __nv_bfloat16* dst = q_out + (static_cast<int64_t>(tok) * hq + head) * D;
+      uint32_t lo_w[16], hi_w[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const f2 a = mul2(w[i], n2), b = mul2(w[i + 1], n2);
-          lo_w[i / 2] = bf16x2(a.x, b.x);
-          hi_w[i / 2] = bf16x2(a.y, b.y);
-        }
-        uint4* dl = reinterpret_cast<uint4*>(dst + s * 32);
-        uint4* dh = reinterpret_cast<uint4*>(dst + 64 + s * 32);
+      for (int i = 0; i < 32; i += 2) {
+        const f2 a = mul2(w[i], n2), b = mul2(w[i + 1], n2);
+        lo_w[i / 2] = bf16x2(a.x, b.x);
+        hi_w[i / 2] = bf16x2(a.y, b.y);
+      }
+      uint4* dl = reinterpret_cast<uint4*>(dst + s * 32);
+      uint4* dh = reinterpret_cast<uint4*>(dst + 64 + s * 32);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          __stcs(dl + j, make_uint4(lo_w[4 * j], lo_w[4 * j + 1], lo_w[4 * j + 2], lo_w[4 * j + 3]));
-          __stcs(dh + j, make_uint4(hi_w[4 * j], hi_w[4 * j + 1], hi_w[4 * j + 2], hi_w[4 * j + 3]));
-        }
-      } else {
-        // K: extremes of the unnormalised values; scale and zero from the
-        // normalised ones
-        float mn = w[0].x, mx = w[0].x;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          mn = fminf(mn, fminf(w[i].x, w[i].y));
-          mx = fmaxf(mx, fmaxf(w[i].x, w[i].y));
-        }
-        float scale, zero;
-        asym_params2<BITS>(mn * kNorm, mx * kNorm, pmask, scale, zero);
-        const float kq = kNorm * __frcp_rn(scale);
-        const f2 k2{kq, kq}, z2{zero, zero};
-        constexpr int WPG = BITS / 4;            // words per 8 codes
-        uint32_t wl[4 * WPG], wh[4 * WPG];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          const f2 xl[4] = {f2{w[8 * n].x, w[8 * n + 1].x}, f2{w[8 * n + 2].x, w[8 * n + 3].x},
-                            f2{w[8 * n + 4].x, w[8 * n + 5].x}, f2{w[8 * n + 6].x, w[8 * n + 7].x}};
-          const f2 xh[4] = {f2{w[8 * n].y, w[8 * n + 1].y}, f2{w[8 * n + 2].y, w[8 * n + 3].y},
-                            f2{w[8 * n + 4].y, w[8 * n + 5].y}, f2{w[8 * n + 6].y, w[8 * n + 7].y}};
-          ucodes8<BITS>(xl, k2, z2, wl + WPG * n);
-          ucodes8<BITS>(xh, k2, z2, wh + WPG * n);
-        }
-        // elements s*32 .. s*32 + 31 and 64 + s*32 .. 64 + s*32 + 31
-        const int64_t g = static_cast<int64_t>(tok) * hkv + head;
-        uint4* dl = reinterpret_cast<uint4*>(k_cache + g * RB + s * (RB / 4));
-        uint4* dh = reinterpret_cast<uint4*>(k_cache + g * RB + RB / 2 + s * (RB / 4));
-#pragma unroll
-        for (int j = 0; j < WPG; ++j) {
-          dl[j] = make_uint4(wl[4 * j], wl[4 * j + 1], wl[4 * j + 2], wl[4 * j + 3]);
-          dh[j] = make_uint4(wh[4 * j], wh[4 * j + 1], wh[4 * j + 2], wh[4 * j + 3]);
-        }
-        if (s == 0) {
-          k_scale[g] = scale;
-          k_zero[g] = static_cast<uint8_t>(zero);
-        }
+      for (int j = 0; j < 4; ++j) {
+        __stcs(dl + j, make_uint4(lo_w[4 * j], lo_w[4 * j + 1], lo_w[4 * j + 2], lo_w[4 * j + 3]));
+        __stcs(dh + j, make_uint4(hi_w[4 * j], hi_w[4 * j + 1], hi_w[4 * j + 2], hi_w[4 * j + 3]));
       }
     }
   }
@@ -371,18 +450,26 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
                            int max_pos, void* q_out, uint8_t* k_cache, float* k_scale,
                            uint8_t* k_zero, uint8_t* v_cache, float* v_scale, uint8_t* v_zero,
                            int bits, cudaStream_t stream) {
-  const int items = 4 * hq + 8 * hkv;            // lanes per pair of tokens
-  const int threads = items >= 256 ? 256 : ((items + 31) & ~31);
+  const int items = 4 * hq + 12 * hkv;           // lanes per pair of tokens
+  const int threads = items >= 224 ? 224 : ((items + 31) & ~31);   // the launch bound
+  auto kern = cos ? (bits == 8 ? kv_rotate_quant_kernel<true, 8> : kv_rotate_quant_kernel<true, 4>)
+                  : (bits == 8 ? kv_rotate_quant_kernel<false, 8>
+                               : kv_rotate_quant_kernel<false, 4>);
+  // persistent grid: the resident CTAs stride over the token pairs, so no
+  // partial last wave
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess ||
+      per_sm < 1) {
+    (void)cudaGetLastError();
+    per_sm = 1;
+  }
   const int64_t pairs = (T + 1) / 2;
-  const int64_t cap = static_cast<int64_t>(host::num_sms()) * 8;
+  const int64_t cap = static_cast<int64_t>(host::num_sms()) * per_sm;
   const int grid = static_cast<int>(pairs < cap ? pairs : cap);
   auto qp = static_cast<const __nv_bfloat16*>(q);
   auto kp = static_cast<const __nv_bfloat16*>(k);
   auto vp = static_cast<const __nv_bfloat16*>(v);
   auto qo = static_cast<__nv_bfloat16*>(q_out);
-  auto kern = cos ? (bits == 8 ? kv_rotate_quant_kernel<true, 8> : kv_rotate_quant_kernel<true, 4>)
-                  : (bits == 8 ? kv_rotate_quant_kernel<false, 8>
-                               : kv_rotate_quant_kernel<false, 4>);
   kern<<<grid, threads, 0, stream>>>(qp, kp, vp, static_cast<int>(T), hq, hkv, pos, cos, sin,
                                      max_pos, qo, k_cache, k_scale, k_zero, v_cache, v_scale,
                                      v_zero);

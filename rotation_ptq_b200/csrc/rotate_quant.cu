@@ -77,6 +77,63 @@ __device__ __forceinline__ float row_scale8(float absmax, float clip) {
   return s == 0.f ? 1.0f : s;
 }
 
+// ------------------------------------------------------------------- SwiGLU
+
+// h = bf16(silu(g) * u), silu(g) = g / (1 + e^-g), the product rounded once.
+// The fast evaluation is (g * u) * rcp(1 + e^-g) in float32 with the hardware
+// approximations.  By their published error bounds (__expf: 2 +
+// floor(1.173 |x|) ulp; rcp.approx: 1 ulp; the add and the two multiplies:
+// half an ulp each) its relative error is below (4.5 + 1.2 |g|) * 2^-23, at
+// most 9 + 2.4 |g| float32 ulps of h.  Rounding the fast value to bf16
+// therefore gives the correctly rounded product unless its low 16 bits lie
+// within that many ulps of 0x8000, the bf16 rounding midpoint; the test below
+// uses 12 + 2.5 |g|.  Those products are recomputed in double precision and
+// rounded once.  Past |g| = 88 the bound is not needed: for g > 88,
+// e^-g flushes to 0 and the fast value is the exact product g * u, which
+// differs from h only if g * u falls exactly on a midpoint; for g < -88, e^-g
+// overflows, the fast value is 0 and the exact product is below 1e-36 |u|,
+// far below any quantization step.  So h is the correctly rounded product
+// except at those two measure-zero edges and where the exact value lies
+// within double-precision error of a midpoint (never exactly on one:
+// silu(g) is transcendental for g != 0).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));   // PTX: at most 1 ulp
+  return r;
+}
+
+// 2^23 + (low 16 bits of h), exactly: the bits of h with 0x4B00 on top.
+__device__ __forceinline__ float lo16_as_float(float h) {
+  return __uint_as_float(__byte_perm(__float_as_uint(h), 0x4B000000u, 0x7610));
+}
+
+// Whether h may round to the other side of a bf16 midpoint than the exact
+// product, given the gate magnitude `ga` that bounds its error.
+__device__ __forceinline__ bool near_bf16_midpoint(float h, float ga) {
+  return fabsf(lo16_as_float(h) - 8421376.0f) <= fmaf(2.5f, ga, 12.0f);   // 2^23 + 0x8000
+}
+
+// silu(g) * u in double precision (the same order as the definition: the
+// quotient, then the product), rounded to 8 significant bits with ties to
+// even straight from the double (no intermediate float rounding); returns the
+// bf16 bit pattern.
+__device__ __noinline__ uint32_t swiglu_exact_bits(float g, float u) {
+  const double gd = static_cast<double>(g);
+  const double h = gd / (1.0 + exp(-gd)) * static_cast<double>(u);
+  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(h));
+  b = (b + 0xFFFFFFFFFFFull + ((b >> 45) & 1ull)) & ~0x1FFFFFFFFFFFull;
+  const float f = static_cast<float>(__longlong_as_double(static_cast<long long>(b)));   // exact
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ float swiglu_bf16(float g, float u) {
+  const float h = g * u * rcp_approx(1.0f + __expf(-g));
+  const uint32_t b = near_bf16_midpoint(h, fabsf(g))
+                         ? swiglu_exact_bits(g, u)
+                         : static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(h)));
+  return __uint_as_float(b << 16);
+}
+
 // ------------------------------------------------------------------ generic
 
 // One CTA per row (grid-stride).  The row is staged in shared memory as
@@ -84,10 +141,6 @@ __device__ __forceinline__ float row_scale8(float absmax, float clip) {
 // contiguous blocks of n_pow2 channels, then each thread applies the small
 // Hadamard to the n_small values (i * n_pow2 + j, i < n_small) of one
 // (group, j), then the row is normalised, reduced and quantized.
-// h = bf16(silu(g) * u), silu(g) = g / (1 + e^-g), in float32.
-__device__ __forceinline__ float swiglu_bf16(float g, float u) {
-  return __bfloat162float(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u));
-}
 
 // With SWIGLU the row is the SwiGLU product of x[m][0, K) (gate) and
 // x[m][K, 2K) (up), rounded to bf16 as it is staged.  BITS 8 writes one
@@ -226,12 +279,13 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
 // two identically swizzled copies, and h is formed element by element in
 // place of the gate row (the operation is elementwise, so the swizzle does
 // not matter).  A row is 1,536 chunks of 16 bytes: warp 11, which otherwise
-// idles, takes chunks [0, 672), and each of the three warps of the group
-// that will rotate the row three rows later takes 288 more (they form them
-// before waiting for their current row's accumulator, so the MMA of row
-// r + 3 overlaps their work on row r).  The split evens out the instructions
-// per SM sub-partition: the group's warps also run the butterflies.  The MMA
-// waits for all four parts instead of the TMA.
+// idles, takes the first TC_AUX_CHUNKS (96), and each of the three warps of
+// the group that will rotate the row three rows later takes 480 more (they
+// form them before waiting for their current row's accumulator, so the MMA
+// of row r + 3 overlaps their work on row r).  Warp 11 works on every row
+// and the group warps on every third, so its share is the smaller one; 96
+// was the fastest of the shares measured.  The MMA waits for all four parts
+// instead of the TMA.
 constexpr int TC_NBUF = 3;                         // TMEM accumulators = row groups
 constexpr int TC_THREADS = 32 * 4 * TC_NBUF;       // 384
 constexpr int TC_ROW_BYTES = 12288 * 2;
@@ -243,12 +297,14 @@ constexpr int TC_TMA_WARP = 3;
 constexpr int TC_MMA_WARP = 7;
 constexpr int TC_AUX_WARP = 11;
 #ifndef SQ_TC_AUX_CHUNKS
-#define SQ_TC_AUX_CHUNKS 288
+#define SQ_TC_AUX_CHUNKS 96
 #endif
 constexpr int TC_AUX_CHUNKS = SQ_TC_AUX_CHUNKS;     // SwiGLU chunks of warp 11 per row
 constexpr int TC_GROUP_CHUNKS = (TC_ROW_BYTES / 16 - TC_AUX_CHUNKS) / 3;   // ... of each group warp
 static_assert(TC_AUX_CHUNKS + 3 * TC_GROUP_CHUNKS == TC_ROW_BYTES / 16,
               "the SwiGLU split covers the row");
+
+constexpr int TC_QCAP = 32;                        // queued SwiGLU products per warp
 
 // Shared-memory plan: the constant operand, then STAGES row slots, then the
 // barriers (slot full, slot free, h ready; accumulator full / read; drain).
@@ -259,43 +315,126 @@ struct TcCfg {
   static constexpr int BAR_OFF = TC_A_BYTES + STAGES * SLOT;
   static constexpr int NBARS = 3 * STAGES + 2 * TC_NBUF + 1;
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
-  static constexpr int SMEM = MISC_OFF + 16 + 4 * TC_NBUF * 2 * 3 + 1024;
+  // per-warp queues of ambiguous SwiGLU products (12 warps x TC_QCAP)
+  static constexpr int QUEUE_OFF = MISC_OFF + 128;
+  static constexpr int SMEM = QUEUE_OFF + (SWIGLU ? 12 * TC_QCAP * 4 : 0) + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 static_assert(TC_A_BYTES % 1024 == 0 && TC_ROW_BYTES % 1024 == 0 && TC_BOX_BYTES % 1024 == 0,
               "swizzle atoms need 1 KB alignment");
 
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));   // PTX: at most 1 ulp
-  return r;
+// The fast SwiGLU of one 16-byte chunk (8 elements): gate words gw, up
+// words uw -> bf16 product words hw, multiplies and adds on float pairs.
+// MASK: return which elements lie near a bf16 rounding midpoint (bit e);
+// otherwise only whether any does (one predicate chain, for the hot loop).
+// Both forms compute h identically.
+template <bool MASK>
+__device__ __forceinline__ uint32_t swiglu_chunk8(const uint32_t (&gw)[4], const uint32_t (&uw)[4],
+                                                 uint32_t (&hw)[4]) {
+  const f2 one{1.0f, 1.0f};
+  uint32_t near = 0u;
+  bool any = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const f2 g{__uint_as_float(gw[e] << 16), __uint_as_float(gw[e] & 0xFFFF0000u)};
+    const f2 u{__uint_as_float(uw[e] << 16), __uint_as_float(uw[e] & 0xFFFF0000u)};
+    const f2 d = add2(one, f2{__expf(-g.x), __expf(-g.y)});
+    const f2 h = mul2(mul2(g, u), f2{rcp_approx(d.x), rcp_approx(d.y)});
+    // one error bound for the pair, from the larger gate; the distances of
+    // both products to their midpoints on a float pair
+    const float t = fmaf(2.5f, fmaxf(fabsf(g.x), fabsf(g.y)), 12.0f);
+    const f2 dm = sub2(f2{lo16_as_float(h.x), lo16_as_float(h.y)}, f2{8421376.0f, 8421376.0f});
+    if (MASK) {
+      near |= (static_cast<uint32_t>(fabsf(dm.x) <= t) << (2 * e)) |
+              (static_cast<uint32_t>(fabsf(dm.y) <= t) << (2 * e + 1));
+    } else {
+      any = any || fabsf(dm.x) <= t || fabsf(dm.y) <= t;
+    }
+    __nv_bfloat162 hb = __floats2bfloat162_rn(h.x, h.y);
+    hw[e] = *reinterpret_cast<uint32_t*>(&hb);
+  }
+  return MASK ? near : static_cast<uint32_t>(any);
+}
+
+// The chunks of one warp's range that held an ambiguous product (bit i of
+// `cmask`: chunk c0 + lane + 32 i; the hot loop left them unwritten): redo
+// each with the fast evaluation, queue its ambiguous elements (byte offset,
+// gate bits) and recompute those in double precision, up to TC_QCAP at a
+// time with every lane of the warp taking one.  Out of line, so that its code
+// stays out of the hot loop.
+__device__ __noinline__ void swiglu_fixup(uint8_t* gbase, int c0, int lane, uint32_t cmask,
+                                          uint32_t* queue) {
+  const uint8_t* ubase = gbase + TC_ROW_BYTES;
+  int nq = 0;                                      // warp-uniform
+  auto flush = [&]() {
+    __syncwarp();
+    for (int i = lane; i < nq; i += 32) {
+      const uint32_t e = queue[i];
+      const uint32_t off = e & 0xFFFFu;
+      const float g = __uint_as_float(e & 0xFFFF0000u);
+      const float u = __uint_as_float(static_cast<uint32_t>(
+                          *reinterpret_cast<const uint16_t*>(ubase + off)) << 16);
+      *reinterpret_cast<uint16_t*>(gbase + off) = static_cast<uint16_t>(swiglu_exact_bits(g, u));
+    }
+    __syncwarp();
+    nq = 0;
+  };
+  while (__any_sync(0xffffffffu, cmask != 0u)) {
+    uint32_t near = 0u, gw[4] = {0u, 0u, 0u, 0u};
+    int c = 0;
+    if (cmask) {
+      c = c0 + lane + 32 * (__ffs(cmask) - 1);
+      cmask &= cmask - 1u;
+      const uint4 g4 = *reinterpret_cast<const uint4*>(gbase + 16 * c);
+      const uint4 u4 = *reinterpret_cast<const uint4*>(ubase + 16 * c);
+      gw[0] = g4.x;
+      gw[1] = g4.y;
+      gw[2] = g4.z;
+      gw[3] = g4.w;
+      const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+      uint32_t hw[4];
+      near = swiglu_chunk8<true>(gw, uw, hw);
+      *reinterpret_cast<uint4*>(gbase + 16 * c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+    while (__any_sync(0xffffffffu, near != 0u)) {
+      const uint32_t want = __ballot_sync(0xffffffffu, near != 0u);
+      if (nq + __popc(want) > TC_QCAP) flush();
+      if (near) {
+        const int e = __ffs(near) - 1;
+        near &= near - 1u;
+        const uint32_t word = e < 2 ? gw[0] : (e < 4 ? gw[1] : (e < 6 ? gw[2] : gw[3]));
+        const uint32_t gbits = (e & 1) ? (word & 0xFFFF0000u) : (word << 16);
+        queue[nq + __popc(want & ((1u << lane) - 1u))] = gbits | static_cast<uint32_t>(16 * c + 2 * e);
+      }
+      nq += __popc(want);
+    }
+  }
+  if (nq > 0) flush();
 }
 
 // Chunks [c0, c1) of a row's SwiGLU product, in place: lane l takes 16-byte
 // chunks c0 + l, c0 + l + 32, ... (8 bf16 of gate and of up each);
-// h = bf16(g * u * (1 / (1 + e^-g))) = bf16(silu(g) * u) in float32, the
-// multiplies and adds on float pairs.
-__device__ __forceinline__ void swiglu_chunks(uint8_t* slot, int c0, int c1, int lane) {
+// h = bf16(silu(g) * u) by the fast evaluation; a chunk holding an ambiguous
+// product is left as it is and redone by swiglu_fixup (see swiglu_bf16).
+__device__ __forceinline__ void swiglu_chunks(uint8_t* slot, int c0, int c1, int lane,
+                                              uint32_t* queue) {
   uint8_t* gbase = slot;
   const uint8_t* ubase = gbase + TC_ROW_BYTES;
-  const f2 one{1.0f, 1.0f};
+  uint32_t cmask = 0u;                             // bit i: chunk c0 + lane + 32 i
+  int i = 0;
 #pragma unroll 4
-  for (int c = c0 + lane; c < c1; c += 32) {
+  for (int c = c0 + lane; c < c1; c += 32, ++i) {
     const uint4 g4 = *reinterpret_cast<const uint4*>(gbase + 16 * c);
     const uint4 u4 = *reinterpret_cast<const uint4*>(ubase + 16 * c);
     const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w}, uw[4] = {u4.x, u4.y, u4.z, u4.w};
     uint32_t hw[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const f2 g{__uint_as_float(gw[e] << 16), __uint_as_float(gw[e] & 0xFFFF0000u)};
-      const f2 u{__uint_as_float(uw[e] << 16), __uint_as_float(uw[e] & 0xFFFF0000u)};
-      const f2 d = add2(one, f2{__expf(-g.x), __expf(-g.y)});
-      const f2 h = mul2(mul2(g, u), f2{rcp_approx(d.x), rcp_approx(d.y)});
-      __nv_bfloat162 hb = __floats2bfloat162_rn(h.x, h.y);
-      hw[e] = *reinterpret_cast<uint32_t*>(&hb);
+    if (swiglu_chunk8<false>(gw, uw, hw)) {
+      cmask |= 1u << i;
+    } else {
+      *reinterpret_cast<uint4*>(gbase + 16 * c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     }
-    *reinterpret_cast<uint4*>(gbase + 16 * c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   }
+  if (__any_sync(0xffffffffu, cmask != 0u)) swiglu_fixup(gbase, c0, lane, cmask, queue);
   fence_proxy_async_smem();          // h is read by the tensor core (async proxy)
 }
 
@@ -321,6 +460,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
   float* red = reinterpret_cast<float*>(smem + C::MISC_OFF + 16);   // [group][parity][3]
+  uint32_t* wqueue = reinterpret_cast<uint32_t*>(smem + C::QUEUE_OFF) + (threadIdx.x >> 5) * TC_QCAP;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int nrows = M > static_cast<int>(blockIdx.x)
@@ -436,7 +576,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         *abort_flag = 1;
         break;
       }
-      swiglu_chunks(stage + s * C::SLOT, 0, TC_AUX_CHUNKS, lane);
+      swiglu_chunks(stage + s * C::SLOT, 0, TC_AUX_CHUNKS, lane, wqueue);
       __syncwarp();
       if (lane == 0) mbar_arrive(&hready[s]);
     }
@@ -451,7 +591,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int s = rr % TC_STAGES;
       if (!mbar_wait(&sfull[s], (rr / TC_STAGES) & 1, spin_limit)) return false;
       const int c0 = TC_AUX_CHUNKS + q * TC_GROUP_CHUNKS;
-      swiglu_chunks(stage + s * C::SLOT, c0, c0 + TC_GROUP_CHUNKS, lane);
+      swiglu_chunks(stage + s * C::SLOT, c0, c0 + TC_GROUP_CHUNKS, lane, wqueue);
       __syncwarp();
       if (lane == 0) mbar_arrive(&hready[s]);
       return true;

@@ -1,20 +1,13 @@
 """GPU parity of sq_swiglu_rotate_quant (SwiGLU + online rotation + INT4) against the oracle.
 
 The oracle forms h = bf16(silu(gate) * up) from the float64 product.  The
-kernel evaluates it in float32 as gate * up * rcp(1 + e^-gate) with the
-hardware approximations; by the published bounds (__expf: 2 + floor(1.173 |x|)
-ulp; rcp.approx: 1 ulp; one add and two multiplies: 0.5 ulp each) its
-relative error is below (6 + 1.2 |gate|) * 2^-23, so h can differ from the
-oracle's only by one bf16 ulp, and only where the product lies that close to
-a bf16 rounding midpoint.
-For each row the test bounds what such elements can do to a rotated value
-(the sum of their ulps over a rotation group, divided by sqrt(group)) and
-widens, for that row only, the scale tolerance and the +-1 tie window of the
-standard rule by that bound (a moved row maximum moves every value of the
-row through the scale, so the mismatch-rate cap does not apply to those
-rows; each of their mismatches must still lie inside the widened window).
-Rows without such elements are graded exactly as sq_rotate_quant's outputs
-are.
+kernel evaluates the product in float32 with the hardware approximations and,
+wherever that value lies within its error bound of a bf16 rounding midpoint
+(or the gate is large), recomputes it in double precision before the single
+bf16 rounding.  Its h is then the oracle's h, and the codes are graded by the
+same rule as sq_rotate_quant's: equal, or +-1 only at a rounding boundary of
+the oracle's pre-round value, with a mismatch rate of at most 1e-5, and scales
+within 1e-5 relative.
 """
 import numpy as np
 import pytest
@@ -27,46 +20,14 @@ from workloads import synthetic as W
 pytestmark = pytest.mark.gpu
 
 
-def _ambiguity_bound(gu64, K, G):
-    """Per row: the largest change of a rotated value that bf16 roundings of
-    near-midpoint SwiGLU products can cause (0 for most rows)."""
-    g = gu64[:, :K]
-    p = O.silu(g) * gu64[:, K:2 * K]
-    m, e = np.frexp(p)
-    ulp = np.ldexp(1.0, e - 8)
-    frac = np.abs(m) * 256.0
-    dist = np.abs(frac - np.floor(frac) - 0.5) * ulp            # to the nearest midpoint
-    eps = (6.0 + 1.2 * np.abs(g)) * 2.0 ** -23
-    amb = np.where(dist <= eps * np.abs(p) + 1e-300, ulp, 0.0)
-    per_group = amb.reshape(amb.shape[0], K // G, G).sum(axis=2) / np.sqrt(G)
-    return per_group.max(axis=1)
-
-
-def _check(aq, asc, gu64, K, ns, np2, clip=1.0):
+def _check(aq, asc, gu64, K, ns, np2, clip=1.0, what="swiglu codes"):
     ref_p, ref_s, ref_c, ref_v = O.swiglu_rotate_quant(gu64, K, ns, np2, clip)
-    B = _ambiguity_bound(gu64, K, ns * np2)
-    # scale = clip * absmax / 7: an absmax moves by at most B
-    rel = np.abs(asc.astype(np.float64) - ref_s) / ref_s
-    assert (rel <= P.SCALE_RTOL + clip * B / 7.0 / ref_s).all(), rel.max()
+    P.check_scales(asc, ref_s, what="swiglu scale")
     got = O.unpack_int4(aq).astype(np.int64)
-    bad = got != ref_c
-    clean = B == 0
-    # rows whose SwiGLU products are all unambiguous: the standard rule
-    P.check_codes(got[clean], ref_c[clean], ref_v[clean])
-    # the other rows: a moved row maximum moves the scale and with it every
-    # value of the row, so any code may flip by one, but only within the
-    # widened window around a rounding boundary
-    if bad[~clean].any():
-        b = bad[~clean]
-        assert np.abs(got[~clean] - ref_c[~clean])[b].max() == 1
-        v = ref_v[~clean].astype(np.float64)
-        # v = y / scale moves by at most B / scale + |v| * dscale / scale
-        window = P.TIE_WINDOW + (B[~clean] / ref_s[~clean]) * (1.0 + 7.5 * clip / 7.0)
-        dist = np.abs(v - (np.floor(v) + 0.5))
-        assert (dist <= window[:, None])[b].all(), "mismatch away from a rounding boundary"
+    n_bad = P.check_codes(got, ref_c, ref_v, what=what)
     same = (got == ref_c).reshape(got.shape[0], -1, 2).all(axis=2)
     assert np.array_equal(aq[same], ref_p[same])     # packing of equal codes is exact
-    return int(bad.sum()), int((B > 0).sum())
+    return n_bad
 
 
 def _run(sq, gu, ns, np2, clip=1.0):
@@ -76,12 +37,19 @@ def _run(sq, gu, ns, np2, clip=1.0):
     return a_q.cpu().numpy(), a_s.cpu().numpy()
 
 
-def test_r4_full_size_sampled_rows(cuda_ok):
+def test_r4_full_size_all_rows(cuda_ok):
+    # every row of the gate_up output of the down_proj workload (M 4096,
+    # [gate | up] of 2 x 12,288), graded in row blocks against the oracle
     import rotation_ptq_b200 as sq
-    gu = W.gate_up_out()                               # M 4096, [gate | up] of 2 x 12,288
+    gu = W.gate_up_out()
     aq, asc = _run(sq, gu, 12, 1024)
-    rows = P.sample_rows(gu.shape[0], 64, seed=21)
-    _check(aq[rows], asc[rows], gu[torch.from_numpy(rows)].double().numpy(), 12288, 12, 1024)
+    n_bad, n = 0, 0
+    for r0 in range(0, gu.shape[0], 512):
+        r1 = min(r0 + 512, gu.shape[0])
+        n_bad += _check(aq[r0:r1], asc[r0:r1], gu[r0:r1].double().numpy(), 12288, 12, 1024)
+        n += (r1 - r0) * 12288
+    assert n_bad <= P.MAX_MISMATCH_RATE * n
+    print("swiglu R4 full size: %d code mismatches at rounding ties of %d codes" % (n_bad, n))
 
 
 @pytest.mark.parametrize("M", [1, 5, 149, 300])
