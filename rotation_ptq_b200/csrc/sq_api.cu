@@ -126,7 +126,7 @@ void sq_debug_set_spin_limit(uint32_t polls) {
 }
 
 void sq_debug_set_gemm_path(int path) {
-  sq::host::g_gemm_path.store(path >= 1 && path <= 3 ? path : 0, std::memory_order_relaxed);
+  sq::host::g_gemm_path.store(path >= 1 && path <= 4 ? path : 0, std::memory_order_relaxed);
 }
 
 sq_status sq_device_status(void* stream) {

@@ -42,6 +42,16 @@ size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 size_t tail_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 }  // namespace gemm
 
+namespace dec {
+// W4A4 linear for 5 <= M <= 32 tokens on the tensor cores (w4a4_decode.cu):
+// a persistent grid streaming the packed weights once.
+bool eligible(int64_t M);
+size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, const float* w_scale,
+              int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
+              size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms);
+}  // namespace dec
+
 namespace gemv {
 // Decode-sized W4A4 linear on CUDA cores: M <= 8 and the widened activation
 // codes (M rounded to 1/2/4/8, times K bytes) fit in 96 KB of shared memory.

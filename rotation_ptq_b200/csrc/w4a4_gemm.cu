@@ -1489,6 +1489,8 @@ size_t tail_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 
 size_t workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K < BK) return 0;
+  if (host::gemm_path() == 0 && dec::eligible(M)) return dec::workspace_bytes(M, N, K, num_sms);
+  if (host::gemm_path() == 0 && M <= 4 && gemv::eligible(M, K)) return 0;   // the GEMV splits nothing
   if (use_pair(M, N)) return 0;
   Plan pl = plan_gemm(M, N, K, true, num_sms);
   if (pl.splits <= 1) return 0;
@@ -1528,7 +1530,11 @@ sq_status run(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q, cons
               int64_t M, int64_t N, int64_t K, void* out, int out_i32, void* ws,
               size_t ws_bytes, cudaStream_t stream, uint32_t spin_limit, int num_sms,
               const Plan* forced) {
-  if (!forced && host::gemm_path() == 0 && gemv::eligible(M, K))
+  if (!forced && host::gemm_path() == 0 && dec::eligible(M))
+    return dec::run(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32, ws, ws_bytes, stream,
+                    spin_limit, num_sms);
+  if (!forced && (host::gemm_path() == 4 || (host::gemm_path() == 0 && M <= 4)) &&
+      gemv::eligible(M, K))
     return gemv::run(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32, num_sms, spin_limit,
                      stream);
   if (!forced && use_pair(M, N)) {

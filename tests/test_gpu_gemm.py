@@ -66,7 +66,7 @@ def test_no_workspace_path_matches(cuda_ok):
 
 def test_workspace_left_zero_and_repeatable(cuda_ok):
     import rotation_ptq_b200 as sq
-    M, N, K = 4, 4096, 12288
+    M, N, K = 12, 4096, 12288
     nbytes = sq.w4a4_workspace_bytes(M, N, K)
     assert nbytes > 0
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
@@ -93,31 +93,47 @@ def test_extreme_codes_full_k(cuda_ok):
     assert np.all(got[:, 0] == 64 * K) and np.all(got[:, 1] == -56 * K)
 
 
-def test_down_proj_full_size_sampled_rows(cuda_ok):
+def _check_rows(acc_dev, a, w, rows=None, block=1024):
+    """int32 accumulators of the given rows (all by default) against the
+    oracle's exact integer GEMM, one block of rows at a time."""
+    wc = O.unpack_int4(w).astype(np.float64)          # converted once for every block
+    rows = np.arange(a.shape[0]) if rows is None else rows
+    for i in range(0, len(rows), block):
+        r = rows[i:i + block]
+        got = acc_dev[torch.from_numpy(r).cuda()].cpu().numpy().astype(np.int64)
+        ref = O.gemm_int(O.unpack_int4(a[r]), wc)
+        assert np.array_equal(got, ref), "rows %d.. differ" % r[0]
+
+
+def test_down_proj_full_size_all_rows(cuda_ok):
+    # every output of the down_proj GEMM (M 4096, N 4096, K 12288): int32
+    # bit-exact, bf16 within one rounding of the oracle's float64 dequant
     import rotation_ptq_b200 as sq
     M, N, K = 4096, 4096, 12288
     a, w, sa, sw = _operands(M, N, K, 2024)
     da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
-    acc = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True).cpu().numpy()
-    out = sq.w4a4_linear(da, dsa, dw, dsw).float().cpu().numpy()
-    rows = P.sample_rows(M, 48, seed=5)
-    wc = O.unpack_int4(w)
-    ref_acc = O.gemm_int(O.unpack_int4(a[rows]), wc)
-    assert np.array_equal(acc[rows].astype(np.int64), ref_acc)
-    P.check_fro(out[rows], O.dequant(ref_acc, sa[rows], sw))
+    acc = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+    out = sq.w4a4_linear(da, dsa, dw, dsw)
+    assert sq.device_status() == 0
+    _check_rows(acc, a, w)
+    acc64 = acc.cpu().numpy().astype(np.int64)
+    ref = O.dequant(acc64, sa, sw)
+    got = out.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-30)
+    P.check_fro(got, ref)
 
 
 @pytest.mark.parametrize("M", [1, 4, 16, 64, 256, 1024, 4096, 16384])
 @pytest.mark.parametrize("shape", ["down_proj", "gate_up"])
-def test_m_sweep_int32_sampled(cuda_ok, M, shape):
+def test_m_sweep_int32(cuda_ok, M, shape):
+    # every row up to M = 4096, 2048 seeded rows at M = 16384
     import rotation_ptq_b200 as sq
     N, K = (4096, 12288) if shape == "down_proj" else (24576, 4096)
     a, w, sa, sw = _operands(M, N, K, 9000 + M)
     acc = sq.w4a4_linear(_dev(a), _dev(sa), _dev(w), _dev(sw), out_int32=True)
-    rows = P.sample_rows(M, 16, seed=M)
-    got = acc[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.int64)
-    ref = O.gemm_int(O.unpack_int4(a[rows]), O.unpack_int4(w))
-    assert np.array_equal(got, ref)
+    assert sq.device_status() == 0
+    rows = None if M <= 4096 else P.sample_rows(M, 2048, seed=M)
+    _check_rows(acc, a, w, rows)
 
 
 def test_forced_timeout_reports_status_and_recovers(cuda_ok):
@@ -209,17 +225,58 @@ def test_few_tile_k_split_matches_whole_tiles(cuda_ok, M, N, K):
     P.check_fro(bf[torch.from_numpy(rows).cuda()].float().cpu().numpy(), O.dequant(ref, sa[rows], sw))
 
 
+@pytest.mark.parametrize("M,N,K", [(5, 128, 128), (6, 16, 384), (5, 1040, 12416), (8, 272, 640),
+                                   (9, 4096, 12288), (17, 24576, 4096), (24, 4096, 1152),
+                                   (31, 528, 4096), (32, 4096, 12288)])
+def test_decode_kernel_matches_other_paths(cuda_ok, M, N, K):
+    # 5 <= M <= 32 runs the persistent decode kernel (work ranges that start
+    # and end inside row tiles, parts added in the workspace); the one-CTA
+    # kernel (debug path 1) and, for M <= 8, the CUDA-core GEMV (path 4) give
+    # identical int32 and bf16 results; with no workspace the decode kernel
+    # takes whole row tiles per CTA, again identical; the int32 sums equal
+    # the oracle's exactly and the workspace is left zero.
+    import rotation_ptq_b200 as sq
+    a, w, sa, sw = _operands(M, N, K, 1300 + M)
+    da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
+    nbytes = sq.w4a4_workspace_bytes(M, N, K)
+    assert nbytes > 0
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    gi = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True, workspace=ws)
+    gb = sq.w4a4_linear(da, dsa, dw, dsw, workspace=ws)
+    wi = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True, use_workspace=False)
+    wb = sq.w4a4_linear(da, dsa, dw, dsw, use_workspace=False)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) == 0
+    others = [1, 4] if M <= 8 else [1]
+    for path in others:
+        sq.debug_set_gemm_path(path)
+        try:
+            ti = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+            tb = sq.w4a4_linear(da, dsa, dw, dsw)
+        finally:
+            sq.debug_set_gemm_path(0)
+        assert torch.equal(gi, ti) and torch.equal(gb, tb), path
+    assert sq.device_status() == 0
+    assert torch.equal(gi, wi) and torch.equal(gb, wb)
+    ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
+    assert np.array_equal(gi.cpu().numpy().astype(np.int64), ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 272, 12288), (2, 4096, 4096), (3, 1040, 12288),
                                    (7, 4096, 12288), (8, 24576, 4096)])
 def test_decode_gemv_matches_tensor_path(cuda_ok, M, N, K):
-    # M <= 8 runs on the CUDA-core GEMV (dp4a); the one-CTA tensor-core
-    # kernel (forced with debug path 1) must give identical int32 and bf16
-    # results, and the int32 sums equal the oracle's exactly.
+    # the CUDA-core GEMV (dp4a; debug path 4, M <= 8) and the one-CTA
+    # tensor-core kernel (path 1) give identical int32 and bf16 results, and
+    # the int32 sums equal the oracle's exactly
     import rotation_ptq_b200 as sq
     a, w, sa, sw = _operands(M, N, K, 1200 + M)
     da, dw, dsa, dsw = _dev(a), _dev(w), _dev(sa), _dev(sw)
-    gi = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
-    gb = sq.w4a4_linear(da, dsa, dw, dsw)
+    sq.debug_set_gemm_path(4)
+    try:
+        gi = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
+        gb = sq.w4a4_linear(da, dsa, dw, dsw)
+    finally:
+        sq.debug_set_gemm_path(0)
     sq.debug_set_gemm_path(1)
     try:
         ti = sq.w4a4_linear(da, dsa, dw, dsw, out_int32=True)
