@@ -410,11 +410,18 @@ def run_ours(args, rank, world, local_rank):
                    "best_of_32_draws": float(draws.min()), "worst_of_32_draws": float(draws.max()),
                    "orth_error_after_120": orth}
         del prob, starts
+    # the R1-folded projections (M 8192, K 4096, N 4096 / 1024 / 12288) and
+    # the decode-to-prefill M sweep, timed alone for the record
+    r1_info = sweep_info = None
+    if not args.no_kv:
+        r1_info = r1_folded_record(dev, flush, args.steps)
+        recs, peaks = sweep_records(min(args.steps, 10), 3)
+        sweep_info = {"peaks": peaks, "points": recs}
     # max over ranks
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
                 clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info, a8=a8_info,
-                r2=r2_info)
+                r2=r2_info, r1=r1_info, sweep=sweep_info)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -462,7 +469,7 @@ def oracle_sample(rows=64, cols=512, min_seconds=10.0, max_steps=None, prepared=
             "sample": "%d rows x %d cols of the workload, %d repetitions (%.1f s), extrapolated "
                       "to one full step (rotation cost per row, GEMM cost per row x col)"
                       % (rows, cols, n, t_rot + t_gemm), "full_step_s": full_s,
-            "prepared": prepared}
+            "repetitions": n, "timed_s": t_rot + t_gemm, "prepared": prepared}
 
 
 PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
@@ -544,8 +551,8 @@ SWEEP_M = (1, 4, 16, 64, 256, 1024, 4096, 16384)
 SWEEP_SHAPES = (("down_proj", 12288, 4096), ("gate_up", 4096, 24576))
 
 
-def run_sweep(steps, warmup):
-    """The decode-to-prefill M sweep of the W4A4 GEMM (one JSON line per point).
+def sweep_records(steps, warmup):
+    """The decode-to-prefill M sweep of the W4A4 GEMM: one record per point.
 
     Operands are seeded random packed codes of the configuration's shapes;
     each point is timed with CUDA events over `steps` launches after `warmup`,
@@ -554,15 +561,18 @@ def run_sweep(steps, warmup):
     events bracket the kernel alone.  Bytes are the algorithmic
     operand + output bytes (packed weights N*K/2, packed activations M*K/2,
     scales 4(M+N), bf16 output 2MN); the roofline is the slower of the
-    measured-HBM and int8-tensor times.
+    measured-HBM and int8-tensor times.  For M <= 64 the point is also timed
+    as eight launches back to back in a CUDA graph, each on its own copy of
+    the weights (8 copies exceed the L2), so that neither launch overhead nor
+    a warm L2 enters the per-launch time.
     """
     import torch
     import rotation_ptq_b200 as sq
     from workloads import synthetic as W
     hbm, bf16, _, peak_src = load_peaks()
     int8_peak = 2.0 * bf16
-    torch.cuda.set_device(0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    recs = []
     for name, K, N in SWEEP_SHAPES:
         w = torch.from_numpy(W.random_packed(21, N, K)).cuda()
         sw = torch.from_numpy(W.random_scales(22, N)).cuda()
@@ -576,8 +586,6 @@ def run_sweep(steps, warmup):
             times = []
             for _ in range(steps):
                 flush.zero_()
-                # keep the device busy while the host prepares the launch, so
-                # that the events bracket the kernel and not host overhead
                 torch.cuda._sleep(200000)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
@@ -588,9 +596,6 @@ def run_sweep(steps, warmup):
             if sq.device_status() != 0:
                 raise SystemExit("device status set")
             t = statistics.median(times)
-            # small M: eight launches back to back in a CUDA graph, each on
-            # its own copy of the weights (8 copies exceed the L2), so neither
-            # launch overhead nor a warm L2 enters the per-launch time
             t_graph = None
             if m <= 64:
                 copies = [w.clone() for _ in range(8)]
@@ -618,16 +623,86 @@ def run_sweep(steps, warmup):
             ops = 2.0 * m * N * K
             nbytes = N * K // 2 + m * K // 2 + 4 * (m + N) + 2 * m * N
             t_roof = max(nbytes / (hbm * 1e9), ops / (int8_peak * 1e12))
-            print(json.dumps({
+            recs.append({
                 "sweep": name, "M": m, "K": K, "N": N, "us": t * 1e6,
                 "TOPS": ops / t / 1e12, "GB/s": nbytes / t / 1e9,
                 "bound": "hbm" if nbytes / (hbm * 1e9) >= ops / (int8_peak * 1e12) else "tensor",
                 "roofline_us": t_roof * 1e6, "frac": t_roof / t,
                 "graph_us": t_graph * 1e6 if t_graph else None,
-                "graph_frac": t_roof / t_graph if t_graph else None,
-                "peaks": "%s HBM %.1f GB/s, int8 %.0f TOPS" % (peak_src, hbm, int8_peak)}),
-                flush=True)
+                "graph_frac": t_roof / t_graph if t_graph else None})
             del a, sa, out
+        del w, sw
+    del flush
+    return recs, "%s HBM %.1f GB/s, int8 %.0f TOPS" % (peak_src, hbm, int8_peak)
+
+
+def run_sweep(steps, warmup):
+    """--sweep: the M sweep alone, one JSON line per point."""
+    import torch
+    torch.cuda.set_device(0)
+    recs, peaks = sweep_records(steps, warmup)
+    for r in recs:
+        print(json.dumps(dict(r, peaks=peaks)), flush=True)
+
+
+def r1_folded_record(dev, flush, steps):
+    """The R1-folded projections at hidden 4096 (M 8192 tokens, K 4096): the
+    quant-only sq_rotate_quant of the activations (no online rotation: R1 is
+    folded into the weights), then the W4A4 GEMM for N = 4096 (q, o), 1024
+    (k, v) and 12288 (gate, up), weights folded and quantized offline."""
+    import torch
+    import rotation_ptq_b200 as sq
+    from workloads import synthetic as W
+    hbm, bf16, _, _ = load_peaks()
+    int8_peak = 2.0 * bf16
+    wls = W.r1_folded()
+    x = wls[0].x.to(dev)
+    Mr, Kr = x.shape
+    a_q = torch.empty((Mr, Kr // 2), dtype=torch.uint8, device=dev)
+    a_s = torch.empty((Mr,), dtype=torch.float32, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    sq.rotate_quant(x, None, 1, 1.0, a_q=a_q, a_scale=a_s)
+    torch.cuda.synchronize()
+    tq = []
+    for _ in range(max(3, steps)):
+        flush.zero_()
+        e0, e1 = ev(), ev()
+        e0.record()
+        sq.rotate_quant(x, None, 1, 1.0, a_q=a_q, a_scale=a_s)
+        e1.record()
+        tq.append((e0, e1))
+    torch.cuda.synchronize()
+    mq = sum(a.elapsed_time(b) for a, b in tq) / len(tq)
+    q_bytes = Mr * (2 * Kr + Kr // 2 + 4)
+    rec = {"workload": "r1_folded_M%d_K%d" % (Mr, Kr),
+           "rotate_quant": {"us": mq * 1e3, "GB/s": q_bytes / (mq * 1e-3) / 1e9,
+                            "frac_of_hbm": q_bytes / (mq * 1e-3) / 1e9 / hbm, "bytes": q_bytes},
+           "gemm": []}
+    for wl in wls:
+        wq, ws = sq.quantize_weights(wl.w.to(dev), None, 1)
+        out = torch.empty((Mr, wl.N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            sq.w4a4_linear(a_q, a_s, wq, ws, out=out)
+        torch.cuda.synchronize()
+        tg = []
+        for _ in range(max(3, steps)):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record()
+            sq.w4a4_linear(a_q, a_s, wq, ws, out=out)
+            e1.record()
+            tg.append((e0, e1))
+        torch.cuda.synchronize()
+        mg = sum(a.elapsed_time(b) for a, b in tg) / len(tg)
+        ops = 2.0 * Mr * wl.N * Kr
+        tops = ops / (mg * 1e-3) / 1e12
+        rec["gemm"].append({"N": wl.N, "us": mg * 1e3, "TOPS": tops,
+                            "frac_of_int8_peak": tops / int8_peak})
+        del wq, ws, out
+    if sq.device_status() != 0:
+        raise RuntimeError("device status set in the R1-folded record")
+    del x, a_q, a_s, wls
+    return rec
 
 
 def main():
@@ -669,7 +744,12 @@ def main():
                 "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N},
                 "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
                 "e2e": {"value": cb["value"], "unit": "TOPS", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
+                        "d2h_bytes_per_step": 0},
+                # no full step is timed: ms_per_step is the sample's cost scaled
+                # to one step, not a measured region
+                "extrapolated": True,
+                "timed": {"repetitions": cb["repetitions"], "seconds": cb["timed_s"],
+                          "rows": 64, "cols": 512}}
         print(json.dumps(line), flush=True)
         return
 
@@ -728,6 +808,8 @@ def main():
                           gemm_frac_of_int8_peak=r["a8"]["gemm_TOPS"] / int8_peak)
                      if r["a8"] else None),
             "r2_cayley_learner": r["r2"],
+            "r1_folded": r["r1"],
+            "m_sweep": r["sweep"],
         },
         "roofline": {"bound": "tensor", "achieved": tops_gemm, "peak": int8_peak,
                      "unit": "TOPS", "frac": tops_gemm / int8_peak, "traffic": GEMM_TRAFFIC,
