@@ -721,21 +721,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // --------------------------------------------------------------- quant only
 
 // No rotation: each of K/32 threads holds 32 consecutive values of the row.
+// A persistent grid strides over the rows, and each thread requests its part
+// of the next row before it reduces and quantizes the current one, so that a
+// row's loads are in flight while the previous row is worked on.
+template <typename T>
+struct RowPart {
+  static constexpr int WORDS = sizeof(T) == 2 ? 4 : 8;   // 16-byte loads per thread
+  uint4 w[WORDS];
+};
+
+template <typename T>
+__device__ __forceinline__ void load_part(const T* xr, RowPart<T>& r) {
+  const uint4* p = reinterpret_cast<const uint4*>(xr);
+#pragma unroll
+  for (int q = 0; q < RowPart<T>::WORDS; ++q) r.w[q] = __ldcs(p + q);
+}
+
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, int64_t ldx, int M,
                                                       float clip, uint8_t* __restrict__ aq,
                                                       float* __restrict__ ascale) {
   __shared__ float red[NT / 32];
   constexpr int K = NT * 32;
-  for (int m = blockIdx.x; m < M; m += gridDim.x) {
+  int m = blockIdx.x;
+  if (m >= M) return;
+  RowPart<T> next;
+  load_part(x + static_cast<int64_t>(m) * ldx + threadIdx.x * 32, next);
+  for (; m < M; m += gridDim.x) {
+    const RowPart<T> cur = next;
+    if (m + static_cast<int>(gridDim.x) < M)
+      load_part(x + static_cast<int64_t>(m + gridDim.x) * ldx + threadIdx.x * 32, next);
     float v[32];
-    const T* xr = x + static_cast<int64_t>(m) * ldx + threadIdx.x * 32;
     if constexpr (sizeof(T) == 2) {
-      const uint4* p = reinterpret_cast<const uint4*>(xr);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint4 w = __ldcs(p + q);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t ws[4] = {cur.w[q].x, cur.w[q].y, cur.w[q].z, cur.w[q].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           v[q * 8 + 2 * e] = bf16lo(ws[e]);
@@ -743,14 +763,12 @@ __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, i
         }
       }
     } else {
-      const float4* p = reinterpret_cast<const float4*>(xr);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const float4 w = __ldcs(p + q);
-        v[4 * q] = w.x;
-        v[4 * q + 1] = w.y;
-        v[4 * q + 2] = w.z;
-        v[4 * q + 3] = w.w;
+        v[4 * q] = __uint_as_float(cur.w[q].x);
+        v[4 * q + 1] = __uint_as_float(cur.w[q].y);
+        v[4 * q + 2] = __uint_as_float(cur.w[q].z);
+        v[4 * q + 3] = __uint_as_float(cur.w[q].w);
       }
     }
     float amax = 0.f;
@@ -758,13 +776,28 @@ __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, i
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = block_max<NT>(amax, red);
     const float s = row_scale(amax, clip);
+    // codes clamp(rint(y / s), -8, 7) with the correctly rounded quotient
+    // (q = y r, e = y - q s, q' = q + e r, r = RN(1 / s): Markstein's one-step
+    // correction), clamped, then rounded to nearest even by the 1.5 * 2^23
+    // magic addition; the low nibble of each float holds the code.
+    const float r = __frcp_rn(s);
+    const f2 r2{r, r}, sn2{-s, -s}, lo2{-8.f, -8.f}, hi2{7.f, 7.f};
+    const f2 magic{12582912.f, 12582912.f};
     uint32_t words[4];
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      uint32_t word = 0;
+      uint32_t u8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) word |= code_of(v[w * 8 + e], s) << (4 * e);
-      words[w] = word;
+      for (int e = 0; e < 4; ++e) {
+        const f2 y{v[w * 8 + 2 * e], v[w * 8 + 2 * e + 1]};
+        const f2 q = mul2(y, r2);
+        f2 c = fma2(fma2(q, sn2, y), r2, q);
+        c = f2{fminf(fmaxf(c.x, lo2.x), hi2.x), fminf(fmaxf(c.y, lo2.y), hi2.y)};
+        c = add2(c, magic);
+        u8[2 * e] = __float_as_uint(c.x);
+        u8[2 * e + 1] = __float_as_uint(c.y);
+      }
+      words[w] = pack8(u8);
     }
     uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * (K / 2)) + threadIdx.x;
     *dst = make_uint4(words[0], words[1], words[2], words[3]);
@@ -790,16 +823,30 @@ static sq_status launch_generic(const T* x, int64_t ldx, int M, int K, const Sma
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_generic launch", e);
 }
 
+// Persistent grid: as many CTAs as fit on the SMs at once.
+template <typename T, int NT>
+static sq_status launch_quant_k(const T* x, int64_t ldx, int M, float clip, uint8_t* aq,
+                                float* as, cudaStream_t st) {
+  auto kfn = rq_quant_kernel<T, NT>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NT, 0) != cudaSuccess ||
+      per_sm < 1) {
+    (void)cudaGetLastError();
+    per_sm = 1;
+  }
+  const int cap = per_sm * host::num_sms();
+  kfn<<<M < cap ? M : cap, NT, 0, st>>>(x, ldx, M, clip, aq, as);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_quant launch", e);
+}
+
 template <typename T>
 static sq_status launch_quant(const T* x, int64_t ldx, int M, int K, float clip, uint8_t* aq,
                               float* as, cudaStream_t st) {
-  const int grid = M < 16 * host::num_sms() ? M : 16 * host::num_sms();
-  cudaError_t e = cudaSuccess;
   switch (K) {
-#define SQ_RQ_CASE(KK)                                                             \
-  case KK:                                                                         \
-    rq_quant_kernel<T, KK / 32><<<grid, KK / 32, 0, st>>>(x, ldx, M, clip, aq, as); \
-    break;
+#define SQ_RQ_CASE(KK) \
+  case KK:             \
+    return launch_quant_k<T, KK / 32>(x, ldx, M, clip, aq, as, st);
     SQ_RQ_CASE(1024)
     SQ_RQ_CASE(2048)
     SQ_RQ_CASE(4096)
@@ -812,8 +859,6 @@ static sq_status launch_quant(const T* x, int64_t ldx, int M, int K, float clip,
     default:
       return SQ_ERR_UNSUPPORTED_SHAPE;
   }
-  e = cudaGetLastError();
-  return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_quant launch", e);
 }
 
 static bool is_paley12(const int8_t* h) {
