@@ -38,8 +38,9 @@ Readings of points the pages leave open:
   * 8-bit KV cache: the asymmetric 4-bit rule on the grid 0..255.
   * Cayley SGD for R2: Y = R G^T - G R^T from the Euclidean gradient; the
     objective is o_proj's W4A4 output error with its input rotated head-wise;
-    the straight-through estimator passes each quantizer's output gradient to
-    its input; a random Hadamard is diag(s) H_d / sqrt(d).
+    the straight-through estimator takes round()'s derivative as 1 and
+    differentiates the quantizer's scale max|z| / 7 as it is; a random
+    Hadamard is diag(s) H_d / sqrt(d).
 
 Parity pins: every function below is checked in tests/test_oracle_pins.py
 against closed forms, brute force or invariants that do not reuse it.
@@ -500,8 +501,14 @@ def kv8_decode_attention(q, k_cache, k_scale, k_zero, v_cache, v_scale, v_zero,
 #     same R, so x' w'^T = x w^T at full precision; activations are quantized
 #     per token and weights per output channel with quant_sym_int4;
 #   * the loss is ||y - y0||^2 / ||y0||^2 with y0 = x w^T and y the W4A4
-#     output; the straight-through estimator passes the gradient of each
-#     quantizer's output to its input unchanged;
+#     output.  The straight-through estimator replaces the derivative of
+#     round() by 1 and differentiates the rest of each quantizer as it is:
+#     Q(z) = s(z) round(z / s(z)) with the row scale s(z) = max_k |z_k| / 7
+#     gives dQ_j/dz_i = delta_ij + ds/dz_i (code_j - z_j / s), where ds/dz_i
+#     = sign(z_i) / 7 at the row's largest magnitude and 0 elsewhere.  (The
+#     pages say round() alone has no useful gradient; the scale is an
+#     ordinary function of z.  Passing dL/dQ through unchanged would drop
+#     the only path by which a rotation changes the quantization step.)
 #   * a random Hadamard is diag(s) H_d / sqrt(d) with random signs s (the
 #     signs act first: H_d diag(s) would only flip the signs of the rotated
 #     channels, which no symmetric quantizer sees).
@@ -545,6 +552,25 @@ def headwise(x: np.ndarray, R: np.ndarray) -> np.ndarray:
     return (x.reshape(rows, K // d, d) @ np.asarray(R, np.float64)).reshape(rows, K)
 
 
+def ste_backward(gq: np.ndarray, z32: np.ndarray, codes: np.ndarray, scale: np.ndarray,
+                 v: np.ndarray) -> np.ndarray:
+    """Straight-through backward of quant_sym_int4 (clip 1) over float32 rows
+    z32, given dL/dQ = gq and the quantizer's codes, scales and quotients v.
+
+    dL/dz_i = gq_i + [i = the row's first largest |z|] sign(z_i) / 7
+    sum_j gq_j (code_j - v_j); an all-zero row passes gq unchanged.
+    """
+    g = np.array(gq, dtype=np.float64, copy=True)
+    z = np.asarray(z32, dtype=F32)
+    res = np.asarray(codes, np.float64) - np.asarray(v, np.float64)
+    coef = np.sum(np.asarray(gq, np.float64) * res, axis=1)
+    rows = np.arange(z.shape[0])
+    im = np.argmax(np.abs(z), axis=1)
+    top = z[rows, im].astype(np.float64)
+    g[rows, im] += np.where(top != 0.0, coef * np.sign(top) / 7.0, 0.0)
+    return g
+
+
 def r2_loss_grad(x: np.ndarray, w: np.ndarray, R: np.ndarray, want_grad: bool = True):
     """W4A4 output error of y = x w^T with the input rotated head-wise by R,
     and its straight-through gradient with respect to R.
@@ -556,8 +582,10 @@ def r2_loss_grad(x: np.ndarray, w: np.ndarray, R: np.ndarray, want_grad: bool = 
     x = np.asarray(x, np.float64)
     w = np.asarray(w, np.float64)
     d = R.shape[0]
-    ca, sa, _ = quant_sym_int4(headwise(x, R).astype(F32))
-    cw, sw, _ = quant_sym_int4(headwise(w, R).astype(F32))
+    za = headwise(x, R).astype(F32)
+    zw = headwise(w, R).astype(F32)
+    ca, sa, va = quant_sym_int4(za)
+    cw, sw, vw = quant_sym_int4(zw)
     qa = ca.astype(np.float64) * sa.astype(np.float64)[:, None]
     qw = cw.astype(np.float64) * sw.astype(np.float64)[:, None]
     y0 = x @ w.T
@@ -566,8 +594,9 @@ def r2_loss_grad(x: np.ndarray, w: np.ndarray, R: np.ndarray, want_grad: bool = 
     loss = float(np.sum(E * E)) / den
     if not want_grad:
         return loss, None
-    g_xr = (2.0 / den) * (E @ qw)          # d loss / d (x R), through the quantizer
-    g_wr = (2.0 / den) * (E.T @ qa)        # d loss / d (w R)
+    # d loss / d (x R) and d loss / d (w R) through the quantizers
+    g_xr = ste_backward((2.0 / den) * (E @ qw), za, ca, sa, va)
+    g_wr = ste_backward((2.0 / den) * (E.T @ qa), zw, cw, sw, vw)
     G = x.reshape(-1, d).T @ g_xr.reshape(-1, d) + w.reshape(-1, d).T @ g_wr.reshape(-1, d)
     return loss, G
 

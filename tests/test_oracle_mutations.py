@@ -209,21 +209,52 @@ def _cayley_full_alpha(R, G, alpha):
     return np.linalg.solve(eye - alpha * Y, (eye + alpha * Y) @ R)
 
 
-def _r2_grad_no_weight_term(x, w, R, want_grad=True):
-    loss, G = _orig["r2_loss_grad"](x, w, R, want_grad)
-    if G is None:
-        return loss, G
+def _r2_parts(x, w, R):
+    # the two straight-through terms of G, recomputed with the oracle's own
+    # pieces: (x part, w part, loss)
     xf = np.asarray(x, np.float64)
     wf = np.asarray(w, np.float64)
     d = R.shape[0]
-    ca, sa, _ = O.quant_sym_int4(O.headwise(xf, R).astype(np.float32))
-    cw, sw, _ = O.quant_sym_int4(O.headwise(wf, R).astype(np.float32))
+    za = O.headwise(xf, R).astype(np.float32)
+    zw = O.headwise(wf, R).astype(np.float32)
+    ca, sa, va = O.quant_sym_int4(za)
+    cw, sw, vw = O.quant_sym_int4(zw)
     qa = ca * sa.astype(np.float64)[:, None]
     qw = cw * sw.astype(np.float64)[:, None]
     y0 = xf @ wf.T
     E = qa @ qw.T - y0
-    g_xr = (2.0 / np.sum(y0 * y0)) * (E @ qw)
+    den = np.sum(y0 * y0)
+    return xf, wf, d, za, zw, ca, sa, va, cw, sw, vw, qa, qw, E, den
+
+
+def _r2_grad_no_weight_term(x, w, R, want_grad=True):
+    loss, G = _orig["r2_loss_grad"](x, w, R, want_grad)
+    if G is None:
+        return loss, G
+    xf, wf, d, za, zw, ca, sa, va, cw, sw, vw, qa, qw, E, den = _r2_parts(x, w, R)
+    g_xr = O.ste_backward((2.0 / den) * (E @ qw), za, ca, sa, va)
     return loss, xf.reshape(-1, d).T @ g_xr.reshape(-1, d)
+
+
+def _r2_grad_identity_ste(x, w, R, want_grad=True):
+    # dL/dQ passed through unchanged: no path through the scales
+    loss, G = _orig["r2_loss_grad"](x, w, R, want_grad)
+    if G is None:
+        return loss, G
+    xf, wf, d, za, zw, ca, sa, va, cw, sw, vw, qa, qw, E, den = _r2_parts(x, w, R)
+    g_xr = (2.0 / den) * (E @ qw)
+    g_wr = (2.0 / den) * (E.T @ qa)
+    return loss, xf.reshape(-1, d).T @ g_xr.reshape(-1, d) + wf.reshape(-1, d).T @ g_wr.reshape(-1, d)
+
+
+def _ste_term_sign_flipped(gq, z32, codes, scale, v):
+    g = np.array(gq, dtype=np.float64, copy=True)
+    z = np.asarray(z32, np.float32)
+    coef = np.sum(np.asarray(gq, np.float64) * (codes - np.asarray(v, np.float64)), axis=1)
+    rows = np.arange(z.shape[0])
+    im = np.argmax(np.abs(z), axis=1)
+    g[rows, im] -= coef * np.sign(z[rows, im]) / 7.0
+    return g
 
 
 def _r2_grad_transposed(x, w, R, want_grad=True):
@@ -286,6 +317,8 @@ MUTATIONS = {
     "cayley_alpha_not_halved": ("cayley_update", _cayley_full_alpha),
     "r2_grad_drops_weight_term": ("r2_loss_grad", _r2_grad_no_weight_term),
     "r2_grad_transposed": ("r2_loss_grad", _r2_grad_transposed),
+    "r2_grad_identity_ste": ("r2_loss_grad", _r2_grad_identity_ste),
+    "ste_scale_term_sign_flipped": ("ste_backward", _ste_term_sign_flipped),
     "random_hadamard_signs_on_columns": ("random_hadamard", _random_hadamard_signs_after),
     "orth_error_max_abs": ("orth_error", _orth_error_max_abs),
     "headwise_uses_transpose": ("headwise", _headwise_transposed),
@@ -333,7 +366,8 @@ PIN_TESTS = [
     P.test_random_hadamard_is_orthogonal_with_signed_rows,
     P.test_headwise_rotation_is_invisible_at_full_precision,
     P.test_r2_loss_at_identity_is_the_plain_w4a4_error,
-    P.test_r2_ste_gradient_is_the_frozen_noise_derivative,
+    P.test_r2_ste_gradient_is_the_frozen_residual_derivative,
+    P.test_r2_ste_scale_term_sits_on_the_row_maximum,
     P.test_orth_error_closed_forms,
 ]
 
