@@ -56,7 +56,7 @@ R2_K = R2_H * R2_D
 R2_INT_OPS = 2 * R2_T * R2_N * R2_K
 R2_GRAD_FLOPS = 2 * 2 * R2_T * R2_N * R2_K
 R2_F32_FLOPS = 2 * (R2_T + R2_N) * R2_K * R2_D + 2 * (R2_T + R2_N) * R2_H * R2_D * R2_D
-R2_ALPHA = 0.3
+R2_ALPHA = 3.0      # step size: of 0.3, 1, 3 and 10 on this layer, 3 and 10 end lowest
 METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200; % of int8/HBM roofline"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels (profiles/w4a4_gemm_pair_ts_*.md, profiles/rotate_quant_h12x1024_tc_*.md);
@@ -408,6 +408,7 @@ def run_ours(args, rank, world, local_rank):
                    "learner_step_us": mlearn * 1e3 / iters,
                    "loss_first_draw": float(L[0]), "loss_after_120": float(L[-1]),
                    "best_of_32_draws": float(draws.min()), "worst_of_32_draws": float(draws.max()),
+                   "learned_vs_best_draw": float(L[-1]) / float(draws.min()) - 1.0,
                    "orth_error_after_120": orth}
         del prob, starts
     # the R1-folded projections (M 8192, K 4096, N 4096 / 1024 / 12288) and

@@ -353,8 +353,10 @@ sq_status sq_kv8_dequant(const uint8_t* cache, const float* scale, const uint8_t
  *     loss = ||Q(x R) Q(w R)^T - x w^T||_F^2 / ||x w^T||_F^2
  * where x R rotates each group of d consecutive channels of every row by R,
  * Q is per-row symmetric INT4 (scale = max|row| / 7, code = clamp(rint(v /
- * scale), -8, 7)) per token of x and per output channel of w, and the
- * gradient G passes each quantizer's output gradient to its input.
+ * scale), -8, 7)) per token of x and per output channel of w.  The
+ * straight-through estimator takes round()'s derivative as 1 and
+ * differentiates the rest of Q as it is: dL/dz = dL/dQ plus, at each row's
+ * first largest |z|, sign(z) / 7 * sum_j dL/dQ_j (code_j - z_j / scale).
  * ------------------------------------------------------------------------- */
 
 /* sq_r2_workspace_bytes -- device scratch of one (x, w) problem: T tokens,

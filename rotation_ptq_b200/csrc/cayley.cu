@@ -5,23 +5,29 @@
 // weights frozen.  The update is the Cayley transform
 //     R' = (I - a/2 Y)^-1 (I + a/2 Y) R,   Y^T = -Y,
 // which keeps R orthogonal, and round() passes the gradient straight through
-// (a straight-through estimator).  Readings of what the page leaves open:
+// (a straight-through estimator: round()'s derivative is taken as 1, the rest
+// of the quantizer, its scale max|z| / 7 included, is differentiated as it
+// is).  Readings of what the page leaves open:
 // Y = R G^T - G R^T from the Euclidean gradient G, so that
 // R' = R - a (G - R G^T R) + O(a^2) is a descent step; the layer is o_proj,
 // whose input x [T][H d] and weight w [N][H d] are both rotated head-wise by
 // R (x' w'^T = x w^T at full precision):
 //     loss = ||Q(x R) Q(w R)^T - x w^T||^2 / ||x w^T||^2,
-//     E = Q(xR) Q(wR)^T - x w^T,  g_xr = 2/den E Q(wR),  g_wr = 2/den E^T Q(xR),
+//     E = Q(xR) Q(wR)^T - x w^T,  dL/dQ(xR) = 2/den E Q(wR),
+//     dL/dQ(wR) = 2/den E^T Q(xR),  g = dL/dQ + scale term (below),
 //     G = sum_h x_h^T g_xr,h + w_h^T g_wr,h.
 // Q is per-row symmetric INT4: scale = max|row| / 7, code = clamp(rint(v /
 // scale), -8, 7), per token for activations, per output channel for weights.
+// Through the scale, dL/dz gains sign(z) / 7 sum_j dL/dQ_j (code_j - z_j /
+// scale) at each row's largest |z|.
 //
 // One loss-and-gradient evaluation on the device:
 //   xr = x_s R, wr = w_s R          fp32 GEMM (x_s = x viewed as [T H][d])
 //   quantize the rows of xr, wr     packed codes, scales, dequantized values
 //   acc = codes_a codes_w^T         INT4 tensor-core GEMM, exact int32 sums
 //   E = acc sa sw - y0, sum E^2     elementwise, fixed-order partial sums
-//   g_xr = E qw, g_wr = E^T qa      fp32 GEMMs (into the xr, wr buffers)
+//   dL/dQ: E qw, E^T qa             tensor cores (bf16 hi + lo of the float side)
+//   g = dL/dQ + scale term          one CTA per row
 //   G = x_s^T g_xr,s + w_s^T g_wr,s fp32 split-K GEMMs, partials summed in f64
 // The Cayley step runs in float64: A = I - a/2 (R G^T - G R^T) and
 // B = (I + a/2 Y) R = 2R - A R, then Gauss-Jordan elimination of A with B as
@@ -253,6 +259,84 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const float* __restrict
       *reinterpret_cast<uint32_t*>(packed + r * (K / 2) + k / 2) = word;
       *reinterpret_cast<uint4*>(codes_bf16 + r * K + k) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
+  }
+}
+
+// The straight-through backward of the row quantizer above, in place on
+// g = dL/dQ [rows][K] given the quantizer's input z: round()'s derivative is
+// taken as 1 and the scale s = max|z| / 7 is differentiated as it is, so
+// dL/dz = g plus, at the row's first largest |z|, sign(z) / 7 * sum_j g_j
+// (code_j - z_j / s) (the rounding residuals are exact in float32; the sum
+// is float64).  An all-zero row is left as it is.  One CTA per row.
+__global__ void __launch_bounds__(256) ste_scale_kernel(const float* __restrict__ z, int64_t rows,
+                                                        int K, float* __restrict__ g) {
+  __shared__ float red_v[8];
+  __shared__ int red_i[8];
+  __shared__ double red_d[8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float* zr = z + r * K;
+    float* gr = g + r * K;
+    // the largest |z| and its first index
+    float bv = -1.f;
+    int bi = 0;
+    for (int k = 4 * threadIdx.x; k < K; k += 4 * blockDim.x) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(zr + k));
+      const float a[4] = {fabsf(v.x), fabsf(v.y), fabsf(v.z), fabsf(v.w)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (a[e] > bv) {                   // indices rise within a thread
+          bv = a[e];
+          bi = k + e;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      red_v[w] = bv;
+      red_i[w] = bi;
+    }
+    __syncthreads();
+    float mx = red_v[0];
+    int im = red_i[0];
+    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i)
+      if (red_v[i] > mx || (red_v[i] == mx && red_i[i] < im)) {
+        mx = red_v[i];
+        im = red_i[i];
+      }
+    __syncthreads();                       // red_* are reused below
+    if (mx == 0.f) continue;               // uniform: every thread read the same mx
+    const float s = __fdiv_rn(mx, 7.0f);
+    double acc = 0.0;
+    for (int k = 4 * threadIdx.x; k < K; k += 4 * blockDim.x) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(zr + k));
+      const float4 gv = *reinterpret_cast<const float4*>(gr + k);
+      const float zz[4] = {v.x, v.y, v.z, v.w}, gg[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float q = __fdiv_rn(zz[e], s);
+        const float c = fminf(fmaxf(rintf(q), -8.f), 7.f);
+        acc += static_cast<double>(gg[e]) * static_cast<double>(c - q);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red_d[w] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double coef = 0.0;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) coef += red_d[i];
+      const double sg = zr[im] < 0.f ? -1.0 : 1.0;
+      gr[im] = static_cast<float>(static_cast<double>(gr[im]) + coef * sg / 7.0);
+    }
+    __syncthreads();                       // red_d is reused by the next row
   }
 }
 
@@ -751,7 +835,8 @@ constexpr int GRAD_CHUNK = 512;            // K chunk of the split-K G GEMMs (~2
 size_t al(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t y0, E, xr, qa, aq, sa, wr, qw, wq, sw, a1h, a1l, a2h, a2l, gpart, lpart, den, gws,
+  size_t y0, E, xr, qa, aq, sa, wr, qw, wq, sw, gxr, gwr, a1h, a1l, a2h, a2l, gpart, lpart, den,
+      gws,
       gws_bytes, r32, g64, cay, total;
   int Px, Pw;
 };
@@ -777,6 +862,8 @@ Layout layout(int64_t T, int H, int d, int64_t N, int num_sms) {
   L.qw = take(N * K * 2);                           // weight codes, bf16
   L.wq = take(N * K / 2);
   L.sw = take(N * 4);
+  L.gxr = take(T * K * 4);                          // dL/d(x R), dL/d(w R)
+  L.gwr = take(N * K * 4);
   L.a1h = take(T * N * 2);
   L.a1l = take(T * N * 2);
   L.a2h = take(T * N * 2);
@@ -916,8 +1003,8 @@ sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, i
   if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 loss", e);
   if (!G) return SQ_OK;
   // straight-through gradients of the rotated operands (the 2 / den factor
-  // is applied to G), into the rotation buffers, on the tensor cores:
-  // g_xr = (E diag(sw)) codes_w and g_wr = (diag(sa) E)^T codes_a
+  // is applied to G), on the tensor cores: dL/dQ_a = (E diag(sw)) codes_w and
+  // dL/dQ_w = (diag(sa) E)^T codes_a, then each quantizer's scale term
   uint16_t* a1h = at<uint16_t>(ws, L.a1h);
   uint16_t* a1l = at<uint16_t>(ws, L.a1l);
   uint16_t* a2h = at<uint16_t>(ws, L.a2h);
@@ -926,14 +1013,19 @@ sq_status loss_grad(const float* x, const float* w, const float* R, int64_t T, i
                        256, 0, s>>>(E, sa, sw, static_cast<int>(T), static_cast<int>(N), a1h, a1l,
                                     a2h, a2l);
   if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 error split", e);
-  if ((st = codes_gemm(a1h, a1l, cw, T, K, N, xr, spin_limit, s)) != SQ_OK ||
-      (st = codes_gemm(a2h, a2l, ca, N, K, T, wr, spin_limit, s)) != SQ_OK)
+  float* gxr = at<float>(ws, L.gxr);
+  float* gwr = at<float>(ws, L.gwr);
+  if ((st = codes_gemm(a1h, a1l, cw, T, K, N, gxr, spin_limit, s)) != SQ_OK ||
+      (st = codes_gemm(a2h, a2l, ca, N, K, T, gwr, spin_limit, s)) != SQ_OK)
     return st;
+  ste_scale_kernel<<<qgrid_a, 256, 0, s>>>(xr, T, static_cast<int>(K), gxr);
+  ste_scale_kernel<<<qgrid_w, 256, 0, s>>>(wr, N, static_cast<int>(K), gwr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return host::cuda_fail("r2 scale term", e);
   // G = x_s^T g_xr,s + w_s^T g_wr,s, split over the long reduction
   float* gp = at<float>(ws, L.gpart);
-  if ((e = sgemm<true, false>(d, d, T * H, x, d, xr, d, gp, d, 1.f, 0.f, L.Px, GRAD_CHUNK, s)) !=
+  if ((e = sgemm<true, false>(d, d, T * H, x, d, gxr, d, gp, d, 1.f, 0.f, L.Px, GRAD_CHUNK, s)) !=
           cudaSuccess ||
-      (e = sgemm<true, false>(d, d, N * H, w, d, wr, d, gp + static_cast<int64_t>(L.Px) * d * d, d,
+      (e = sgemm<true, false>(d, d, N * H, w, d, gwr, d, gp + static_cast<int64_t>(L.Px) * d * d, d,
                               1.f, 0.f, L.Pw, GRAD_CHUNK, s)) != cudaSuccess)
     return host::cuda_fail("r2 G GEMM", e);
   grad_sum_kernel<<<(d * d + 255) / 256, 256, 0, s>>>(gp, L.Px + L.Pw,

@@ -151,15 +151,18 @@ def test_r2_learner_follows_the_oracle(cuda_ok):
     assert float(sq.orth_error(R)[0]) <= 1e-11
 
 
-def test_r2_learner_full_size_descends_and_stays_orthogonal(cuda_ok):
+def test_r2_learner_full_size_beats_the_draws_and_stays_orthogonal(cuda_ok):
     import rotation_ptq_b200 as sq
     wl = W.o_proj_layer()
     prob = sq.R2Problem(torch.from_numpy(wl.x).cuda(), torch.from_numpy(wl.w).cuda(), 32)
-    R0 = sq.r2_random_hadamard(torch.from_numpy(wl.signs[:1]).cuda())[0]
-    R, losses = prob.learn(R0, 0.3, 120)
+    starts = sq.r2_random_hadamard(torch.from_numpy(wl.signs).cuda())
+    draws = [float(prob.loss_grad(starts[i].float(), grad=False)[0][0]) for i in range(32)]
+    R, losses = prob.learn(starts[0], 0.3, 120)
     assert sq.device_status() == 0
     L = losses.cpu().numpy()
     assert L[-1] < L[0]
+    # from the first draw to below the best of all 32
+    assert L[-1] < min(draws)
     assert float(sq.orth_error(R)[0]) <= 1e-11
     # the last iterate's loss is the loss of the returned rotation
     again, _ = prob.loss_grad(R.float(), grad=False)
