@@ -477,7 +477,7 @@ PROFILE_CASES = ("down_proj_gemm", "down_proj_gemm_1cta", "down_proj_gemm_pair",
                  "decode_gemm_m1", "decode_gemm_m16", "decode_gemm_m64", "rotate_quant_r4",
                  "kv_rotate_quant",
                  "swiglu_rotate_quant_r4", "kv4_decode", "kv8_decode", "kv_rotate_quant8",
-                 "r2_loss_grad")
+                 "r2_loss_grad", "quant_only_r1", "kv_rotate_quant_t16k", "kv_rotate_quant8_t16k")
 
 
 def run_profile_case(case, steps, warmup):
@@ -501,6 +501,12 @@ def run_profile_case(case, steps, warmup):
         a_q = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
         a_s = torch.empty((M,), dtype=torch.float32, device="cuda")
         fn = lambda: sq.rotate_quant(x, hs, N_POW2, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
+    elif case == "quant_only_r1":
+        # the R1-folded projections' input: M 8192, K 4096, no online rotation
+        x = W.r1_folded(Ns=(16,))[0].x.cuda()
+        a_q = torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device="cuda")
+        a_s = torch.empty((x.shape[0],), dtype=torch.float32, device="cuda")
+        fn = lambda: sq.rotate_quant(x, None, 1, 1.0, a_q=a_q, a_scale=a_s)  # noqa: E731
     elif case == "swiglu_rotate_quant_r4":
         gu = W.gate_up_out(M=M, K=K).cuda()
         hs = sq.paley_h12()
@@ -524,14 +530,14 @@ def run_profile_case(case, steps, warmup):
                                 dw.v_zero, dw.lengths)]
         o = sq.kv8_decode_attention(*t, dw.S_max)
         fn = lambda: sq.kv8_decode_attention(*t, dw.S_max, out=o)  # noqa: E731
-    elif case == "kv_rotate_quant8":
-        kw = W.kv_path()
+    elif case in ("kv_rotate_quant8", "kv_rotate_quant8_t16k"):
+        kw = W.kv_path(batch=16 if case == "kv_rotate_quant8" else 4)
         q, k, v, pos = kw.q.cuda(), kw.k.cuda(), kw.v.cuda(), kw.pos.cuda()
         cos, sin = sq.rope_tables(kw.theta, kw.max_pos, 128)
         o = sq.kv_rotate_quant8(q, k, v, pos, cos, sin)
         fn = lambda: sq.kv_rotate_quant8(q, k, v, pos, cos, sin, out=o)  # noqa: E731
-    elif case == "kv_rotate_quant":
-        kvw = W.kv_path()
+    elif case in ("kv_rotate_quant", "kv_rotate_quant_t16k"):
+        kvw = W.kv_path(batch=16 if case == "kv_rotate_quant" else 4)
         q, k, v, pos = kvw.q.cuda(), kvw.k.cuda(), kvw.v.cuda(), kvw.pos.cuda()
         cos, sin = sq.rope_tables(kvw.theta, kvw.max_pos, 128)
         o = sq.kv_rotate_quant(q, k, v, pos, cos, sin)

@@ -117,6 +117,10 @@ int sq_version(void);
  * K % g == 0.
  * The same call quantizes weights offline: pass W [N][K] as x (float32) to
  * get per-output-channel codes and scales with the rotation folded in.
+ * Range: the bf16 H12 x H1024 path (K = 12288) forms its first factor on the
+ * tensor cores, which treat float32-subnormal inputs and sums (|v| < 2^-126)
+ * as zero, so rows of that magnitude (scale below ~1e-38) are outside its
+ * range; the other paths follow the rule for every finite input.
  * ------------------------------------------------------------------------- */
 sq_status sq_rotate_quant(const void* x, sq_in_dtype x_dtype, int64_t M, int64_t K,
                           int64_t ld_x, const int8_t* had_small, int n_small, int n_pow2,

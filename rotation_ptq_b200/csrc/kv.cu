@@ -123,15 +123,20 @@ __device__ __forceinline__ void pack_codes(const uint32_t (&u)[8], uint32_t* out
 // one-step fma correction of Markstein ("IA-64 and Elementary Functions",
 // 2000), which yields the correctly rounded quotient when r is the correctly
 // rounded reciprocal.  Then rint(q') + zero, clamped to [0, 2^BITS - 1].
+// x and s enter scaled by the same power of two u2 (2^64 for a subnormal
+// scale, whose reciprocal would overflow, else 1): exact scalings that leave
+// the quotient unchanged; s2neg is -s u.
 template <int BITS>
-__device__ __forceinline__ void ucodes8_div(const f2* x, f2 r2, f2 s2neg, f2 z2, uint32_t* out) {
+__device__ __forceinline__ void ucodes8_div(const f2* x, f2 u2, f2 r2, f2 s2neg, f2 z2,
+                                            uint32_t* out) {
   const f2 magic{12582912.f, 12582912.f};       // 1.5 * 2^23: nearest even
   const float lo = 12582912.f, hi = 12582912.f + static_cast<float>((1 << BITS) - 1);
   uint32_t u[8];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const f2 q = mul2(x[e], r2);
-    const f2 er = fma2(q, s2neg, x[e]);
+    const f2 xs = mul2(x[e], u2);
+    const f2 q = mul2(xs, r2);
+    const f2 er = fma2(q, s2neg, xs);
     f2 c = add2(add2(fma2(er, r2, q), magic), z2);   // magic + rint(q') + zero, exact
     c.x = fminf(fmaxf(c.x, lo), hi);
     c.y = fminf(fmaxf(c.y, lo), hi);
@@ -260,14 +265,17 @@ __global__ void __launch_bounds__(224) kv_rotate_quant_kernel(
         }
         float scale, zero;
         asym_params<BITS>(mn, mx, pmask, scale, zero);
-        const float rs = __frcp_rn(scale);
-        const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
+        // scale and inputs times 2^64 when the scale is subnormal (see ucodes8_div)
+        const float up = scale < 1.17549435e-38f ? 18446744073709551616.0f : 1.0f;
+        const float su = scale * up;
+        const float rs = __frcp_rn(su);
+        const f2 u2{up, up}, r2{rs, rs}, sn2{-su, -su}, z2{zero, zero};
         uint32_t w[8 * WPG];
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
           const f2 xs[4] = {f2{x[8 * n], x[8 * n + 1]}, f2{x[8 * n + 2], x[8 * n + 3]},
                             f2{x[8 * n + 4], x[8 * n + 5]}, f2{x[8 * n + 6], x[8 * n + 7]}};
-          ucodes8_div<BITS>(xs, r2, sn2, z2, w + WPG * n);
+          ucodes8_div<BITS>(xs, u2, r2, sn2, z2, w + WPG * n);
         }
         uint4* dst = reinterpret_cast<uint4*>(v_cache + g * RB + s * (RB / 2));
 #pragma unroll
@@ -301,8 +309,11 @@ __global__ void __launch_bounds__(224) kv_rotate_quant_kernel(
         }
         float scale, zero;
         asym_params<BITS, 4>(mn, mx, pmask, scale, zero);
-        const float rs = __frcp_rn(scale);
-        const f2 r2{rs, rs}, sn2{-scale, -scale}, z2{zero, zero};
+        // scale and inputs times 2^64 when the scale is subnormal (see ucodes8_div)
+        const float up = scale < 1.17549435e-38f ? 18446744073709551616.0f : 1.0f;
+        const float su = scale * up;
+        const float rs = __frcp_rn(su);
+        const f2 u2{up, up}, r2{rs, rs}, sn2{-su, -su}, z2{zero, zero};
         uint32_t wl[2 * WPG], wh[2 * WPG];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
@@ -310,8 +321,8 @@ __global__ void __launch_bounds__(224) kv_rotate_quant_kernel(
                             f2{ya[8 * n + 4], ya[8 * n + 5]}, f2{ya[8 * n + 6], ya[8 * n + 7]}};
           const f2 xh[4] = {f2{yb[8 * n], yb[8 * n + 1]}, f2{yb[8 * n + 2], yb[8 * n + 3]},
                             f2{yb[8 * n + 4], yb[8 * n + 5]}, f2{yb[8 * n + 6], yb[8 * n + 7]}};
-          ucodes8_div<BITS>(xl, r2, sn2, z2, wl + WPG * n);
-          ucodes8_div<BITS>(xh, r2, sn2, z2, wh + WPG * n);
+          ucodes8_div<BITS>(xl, u2, r2, sn2, z2, wl + WPG * n);
+          ucodes8_div<BITS>(xh, u2, r2, sn2, z2, wh + WPG * n);
         }
         // elements 16 s .. 16 s + 15 and 64 + 16 s .. 64 + 16 s + 15
         uint8_t* row = k_cache + g * RB;

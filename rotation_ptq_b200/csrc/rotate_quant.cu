@@ -737,7 +737,7 @@ __device__ __forceinline__ void load_part(const T* xr, RowPart<T>& r) {
   for (int q = 0; q < RowPart<T>::WORDS; ++q) r.w[q] = __ldcs(p + q);
 }
 
-template <typename T, int NT>
+template <typename T, int NT, bool CLAMP>
 __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, int64_t ldx, int M,
                                                       float clip, uint8_t* __restrict__ aq,
                                                       float* __restrict__ ascale) {
@@ -771,33 +771,53 @@ __global__ void __launch_bounds__(NT) rq_quant_kernel(const T* __restrict__ x, i
         v[4 * q + 3] = __uint_as_float(cur.w[q].w);
       }
     }
-    float amax = 0.f;
+    // two independent three-input max chains
+    float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    amax = block_max<NT>(amax, red);
+    for (int i = 0; i < 32; i += 4) {
+      m0 = fmax3(m0, fabsf(v[i]), fabsf(v[i + 1]));
+      m1 = fmax3(m1, fabsf(v[i + 2]), fabsf(v[i + 3]));
+    }
+    const float amax = block_max<NT>(fmaxf(m0, m1), red);
     const float s = row_scale(amax, clip);
     // codes clamp(rint(y / s), -8, 7) with the correctly rounded quotient
     // (q = y r, e = y - q s, q' = q + e r, r = RN(1 / s): Markstein's one-step
-    // correction), clamped, then rounded to nearest even by the 1.5 * 2^23
-    // magic addition; the low nibble of each float holds the code.
-    const float r = __frcp_rn(s);
-    const f2 r2{r, r}, sn2{-s, -s}, lo2{-8.f, -8.f}, hi2{7.f, 7.f};
-    const f2 magic{12582912.f, 12582912.f};
+    // correction), then rounded to nearest even by the 1.5 * 2^23 magic
+    // addition; the low nibble of each float holds the code.  With clip >= 1
+    // (CLAMP false) |y| / s <= 7 (1 + 2^-23) < 7.5, so the clamp cannot change
+    // a code.  A row whose scale is subnormal (RN(1 / s) would overflow)
+    // divides element by element and clamps (uniform per row).
     uint32_t words[4];
+    if (s >= 1.17549435e-38f) {
+      const float r = __frcp_rn(s);
+      const f2 r2{r, r}, sn2{-s, -s};
+      const f2 magic{12582912.f, 12582912.f};
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t u8[8];
+      for (int w = 0; w < 4; ++w) {
+        uint32_t u8[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const f2 y{v[w * 8 + 2 * e], v[w * 8 + 2 * e + 1]};
-        const f2 q = mul2(y, r2);
-        f2 c = fma2(fma2(q, sn2, y), r2, q);
-        c = f2{fminf(fmaxf(c.x, lo2.x), hi2.x), fminf(fmaxf(c.y, lo2.y), hi2.y)};
-        c = add2(c, magic);
-        u8[2 * e] = __float_as_uint(c.x);
-        u8[2 * e + 1] = __float_as_uint(c.y);
+        for (int e = 0; e < 4; ++e) {
+          const f2 y{v[w * 8 + 2 * e], v[w * 8 + 2 * e + 1]};
+          const f2 q = mul2(y, r2);
+          f2 c = fma2(fma2(q, sn2, y), r2, q);
+          if (CLAMP) c = f2{fminf(fmaxf(c.x, -8.f), 7.f), fminf(fmaxf(c.y, -8.f), 7.f)};
+          c = add2(c, magic);
+          u8[2 * e] = __float_as_uint(c.x);
+          u8[2 * e + 1] = __float_as_uint(c.y);
+        }
+        words[w] = pack8(u8);
       }
-      words[w] = pack8(u8);
+    } else {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t u8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float c = fminf(fmaxf(rintf(__fdiv_rn(v[w * 8 + e], s)), -8.f), 7.f);
+          u8[e] = static_cast<uint32_t>(static_cast<int>(c));
+        }
+        words[w] = pack8(u8);
+      }
     }
     uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<int64_t>(m) * (K / 2)) + threadIdx.x;
     *dst = make_uint4(words[0], words[1], words[2], words[3]);
@@ -827,7 +847,7 @@ static sq_status launch_generic(const T* x, int64_t ldx, int M, int K, const Sma
 template <typename T, int NT>
 static sq_status launch_quant_k(const T* x, int64_t ldx, int M, float clip, uint8_t* aq,
                                 float* as, cudaStream_t st) {
-  auto kfn = rq_quant_kernel<T, NT>;
+  auto kfn = clip < 1.0f ? rq_quant_kernel<T, NT, true> : rq_quant_kernel<T, NT, false>;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NT, 0) != cudaSuccess ||
       per_sm < 1) {

@@ -64,6 +64,31 @@ def test_small_kv(cuda_ok, T, hq, hkv, rope):
         _check_dequant(sq, ref[name + "_cache"], ref[name + "_scale"], ref[name + "_zero"])
 
 
+def test_tiny_heads_subnormal_scales(cuda_ok):
+    # heads whose range gives a subnormal scale: the quantizer cannot use
+    # RN(1 / scale) (it overflows) and divides instead; codes, scales and
+    # zero points still follow the rule
+    import rotation_ptq_b200 as sq
+    wl = W.kv_path(batch=1, seq=16, hq=8, hkv=2, seed=431)
+    k = wl.k.double().clone()
+    v = wl.v.double().clone()
+    k[:, 0] *= 1e-39
+    v[:, 1] *= 3e-39
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    cos, sin = sq.rope_tables(wl.theta, wl.max_pos, 128)
+    rc, rs = O.rope_tables(wl.theta, wl.max_pos, 128)
+    out = sq.kv_rotate_quant(wl.q.cuda(), k.cuda(), v.cuda(), wl.pos.cuda(), cos, sin)
+    assert sq.device_status() == 0
+    r = {n: t.cpu() for n, t in out.items()}
+    r["q_out"] = r["q_out"].float()
+    r = {n: t.numpy() for n, t in r.items()}
+    ref = O.kv_rotate_quant(wl.q.double().numpy(), k.double().numpy(), v.float().numpy(),
+                            wl.pos.numpy(), rc, rs)
+    ref["v_in"] = v.float().numpy()
+    assert (ref["k_scale"][:, 0] < 1.17549435e-38).all() and (ref["v_scale"][:, 1] < 1.17549435e-38).all()
+    _compare(r, ref, np.arange(16))
+
+
 def _check_dequant(sq, cache, scale, zero):
     deq = sq.kv_dequant(torch.from_numpy(cache).cuda(), torch.from_numpy(scale).cuda(),
                         torch.from_numpy(zero).cuda()).float().cpu().numpy()

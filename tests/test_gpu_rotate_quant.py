@@ -84,6 +84,25 @@ def test_clip_ratio_clamps(cuda_ok):
     assert (codes == -8).any() or (codes == 7).sum() > 16
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quant_only_clip_and_tiny_rows(cuda_ok, dtype):
+    # the quant-only kernel skips its clamp only for clip >= 1 and a normal
+    # scale: clip < 1 must clamp, and rows whose scale is subnormal (largest
+    # magnitude ~1e-38 .. 1e-44) keep the clamp as well
+    import rotation_ptq_b200 as sq
+    rng = np.random.default_rng(91)
+    x = rng.standard_t(3, (64, 4096))
+    for i, mag in enumerate((1e-38, 5e-39, 3e-41, 2e-44)):
+        x[i] = np.sign(x[i]) * mag * np.abs(x[i]) / np.abs(x[i]).max()
+    xt = torch.from_numpy(x.astype(np.float32)).to(dtype)
+    x64 = xt.double().numpy()
+    for clip in (1.0, 0.8):
+        aq, asc = _run(sq, xt, 1, 1, clip=clip)
+        codes = _check(aq, asc, x64, 1, 1, clip=clip)
+        if clip < 1:
+            assert (codes[4:] == 7).sum() + (codes[4:] == -8).sum() > 64
+
+
 def test_zero_and_constant_rows(cuda_ok):
     import rotation_ptq_b200 as sq
     x = torch.zeros((4, 4096), dtype=torch.bfloat16)
