@@ -93,9 +93,9 @@ sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,
 }  // namespace rq
 
 namespace kvd {
-// Split count of the decode-attention kernel and the workspace it needs (0
-// when it runs unsplit).
-int choose_splits(int64_t B, int64_t S_max, int hkv, int num_sms);
+// Split count of the decode-attention kernel at ctas_per_sm resident CTAs,
+// and the workspace either code width needs (0 when both run unsplit).
+int choose_splits(int64_t B, int64_t S_max, int hkv, int num_sms, int ctas_per_sm);
 size_t workspace_bytes(int64_t B, int64_t S_max, int hkv, int num_sms);
 // bits = 4 or 8: the caches' code width (as kv::run_dequant).
 sq_status run(const void* q, const uint8_t* k_cache, const float* k_scale, const uint8_t* k_zero,
