@@ -409,34 +409,67 @@ __global__ void __launch_bounds__(224) kv_rotate_quant_kernel(
   }
 }
 
-// out = bf16((code - zero) * scale); one thread per 16 codes.
+// out = bf16((code - zero) * scale).  The unit is a chunk of 8 codes (16
+// bytes of output; a group of 128 codes has 16).  Each warp takes 64
+// consecutive chunks per step, lane l the chunks l and 32 + l, so every
+// store instruction of the warp writes 512 contiguous bytes and every code
+// load reads 128 (4-bit) or 256 (8-bit) contiguous bytes.  A code becomes a
+// float without a conversion instruction: the bits 0x4B000000 | c are
+// 2^23 + c, and subtracting 2^23 + zero leaves c - zero exactly; one
+// multiply by the scale then rounds once, as (code - zero) * scale does.
+template <int BITS>
+__device__ __forceinline__ uint4 dequant_chunk(const uint8_t* __restrict__ cache,
+                                               const float* __restrict__ scale,
+                                               const uint8_t* __restrict__ zero, int64_t c) {
+  const int64_t g = c >> 4;
+  const float s = __ldg(scale + g);
+  const float zb = 8388608.0f + static_cast<float>(__ldg(zero + g));
+  uint32_t t[8];
+  if (BITS == 4) {
+    const uint32_t w = __ldcs(reinterpret_cast<const uint32_t*>(cache) + c);
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    // element 2j sits in the low nibble of byte j
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      t[2 * j] = __byte_perm(lo, 0x4B000000u, 0x7440u + j);
+      t[2 * j + 1] = __byte_perm(hi, 0x4B000000u, 0x7440u + j);
+    }
+  } else {
+    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(cache) + c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      t[j] = __byte_perm(w.x, 0x4B000000u, 0x7440u + j);
+      t[4 + j] = __byte_perm(w.y, 0x4B000000u, 0x7440u + j);
+    }
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    o[e] = bf16x2((__uint_as_float(t[2 * e]) - zb) * s, (__uint_as_float(t[2 * e + 1]) - zb) * s);
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) kv_dequant_kernel(const uint8_t* __restrict__ cache,
                                                          const float* __restrict__ scale,
                                                          const uint8_t* __restrict__ zero,
                                                          int64_t groups,
                                                          __nv_bfloat16* __restrict__ out) {
-  const int64_t n = groups * 8;                  // 8 chunks of 16 codes per group
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t g = i >> 3;
-    const float s = __ldg(scale + g), z = static_cast<float>(__ldg(zero + g));
-    float v[16];
-    if (BITS == 4) {
-      const uint2 w = __ldcs(reinterpret_cast<const uint2*>(cache) + i);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[e] = (static_cast<float>((w.x >> (4 * e)) & 0xFu) - z) * s;
-        v[8 + e] = (static_cast<float>((w.y >> (4 * e)) & 0xFu) - z) * s;
-      }
-    } else {
-      const uint4 w = __ldcs(reinterpret_cast<const uint4*>(cache) + i);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        v[e] = (static_cast<float>((ws[e >> 2] >> (8 * (e & 3))) & 0xFFu) - z) * s;
+  const int64_t n = groups * 16;                 // chunks
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  uint4* dst = reinterpret_cast<uint4*>(out);
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 64;
+       base < n; base += warps * 64) {
+    const int64_t c0 = base + lane, c1 = base + 32 + lane;
+    if (c1 < n) {
+      const uint4 v0 = dequant_chunk<BITS>(cache, scale, zero, c0);
+      const uint4 v1 = dequant_chunk<BITS>(cache, scale, zero, c1);
+      __stcs(dst + c0, v0);
+      __stcs(dst + c1, v1);
+    } else if (c0 < n) {
+      __stcs(dst + c0, dequant_chunk<BITS>(cache, scale, zero, c0));
     }
-    store16_bf16(out + i * 16, v);
   }
 }
 
@@ -491,9 +524,9 @@ sq_status run_rotate_quant(const void* q, const void* k, const void* v, int64_t 
 sq_status run_dequant(const uint8_t* cache, const float* scale, const uint8_t* zero, int64_t T,
                       int h, void* out, int bits, cudaStream_t stream) {
   const int64_t groups = T * h;
-  const int64_t threads_needed = groups * 8;
-  const int64_t cap = static_cast<int64_t>(host::num_sms()) * 16;
-  int64_t grid = (threads_needed + 255) / 256;
+  // 8 warps per CTA, 64 chunks of 8 codes per warp and step
+  const int64_t cap = static_cast<int64_t>(host::num_sms()) * 8;
+  int64_t grid = (groups * 16 + 8 * 64 - 1) / (8 * 64);
   if (grid > cap) grid = cap;
   auto kern = bits == 8 ? kv_dequant_kernel<8> : kv_dequant_kernel<4>;
   kern<<<static_cast<int>(grid), 256, 0, stream>>>(cache, scale, zero, groups,
