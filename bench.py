@@ -198,6 +198,12 @@ def run_ours(args, rank, world, local_rank):
     ms_step, ms_rq, ms_gemm = ms(t_step), ms(t_rq), ms(t_gemm)
     status = sq.device_status()
 
+    # the R4 rotate+quant back to back over three copies of x (302 MB)
+    xs = [x] + [x.clone() for _ in range(2)]
+    us_rq_b2b = back_to_back_us([lambda xx=xx: sq.rotate_quant(xx, hs, N_POW2, 1.0, a_q=a_q,
+                                                               a_scale=a_s) for xx in xs])
+    del xs
+
     # e2e: pinned host input, H2D + path + D2H every step, device-timed
     x_host = x.cpu().pin_memory()
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
@@ -345,8 +351,18 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         mde = ms(tde)
         dec_bytes = DECODE_BYTES
+        # back to back over four copies of the caches (290 MB)
+        copies = [(dq, dkc, dks, dkz, dvc, dvs, dvz)] + \
+            [tuple(t.clone() for t in (dq, dkc, dks, dkz, dvc, dvs, dvz)) for _ in range(3)]
+        us_dec_b2b = back_to_back_us([
+            lambda c=c: sq.kv4_decode_attention(*c, dln, dw.S_max, out=dout) for c in copies])
+        del copies
         dec_info = {"workload": dw.name, "us": mde * 1e3,
-                    "GB/s": dec_bytes / (mde * 1e-3) / 1e9, "bytes": dec_bytes}
+                    "GB/s": dec_bytes / (mde * 1e-3) / 1e9, "bytes": dec_bytes,
+                    "back_to_back": {"us": us_dec_b2b,
+                                     "GB/s": dec_bytes / (us_dec_b2b * 1e-6) / 1e9,
+                                     "how": "8 launches over 4 copies of the caches (290 MB) "
+                                            "between one event pair"}}
         del dq, dkc, dks, dkz, dvc, dvs, dvz, dln, dout
         # the same step over 8-bit caches
         dw = W.kv8_decode()
@@ -422,7 +438,7 @@ def run_ours(args, rank, world, local_rank):
     ms_step, ms_rq, ms_gemm, ms_e2e = shard.max_over_ranks([ms_step, ms_rq, ms_gemm, ms_e2e])
     return dict(ms_step=ms_step, ms_rq=ms_rq, ms_gemm=ms_gemm, ms_e2e=ms_e2e, status=status,
                 clocks=clk.result, kv=kv_info, swiglu=sw_info, decode=dec_info, a8=a8_info,
-                r2=r2_info, r1=r1_info, sweep=sweep_info)
+                r2=r2_info, r1=r1_info, sweep=sweep_info, us_rq_b2b=us_rq_b2b)
 
 
 # ------------------------------------------------------------ oracle arm
@@ -558,6 +574,34 @@ SWEEP_M = (1, 4, 16, 64, 256, 1024, 4096, 16384)
 SWEEP_SHAPES = (("down_proj", 12288, 4096), ("gate_up", 4096, 24576))
 
 
+def back_to_back_us(calls, rounds=5):
+    """Average launch duration with the launches back to back: `calls` (one
+    per input copy, the copies together larger than the L2, so each launch
+    finds its input evicted by the others) run twice over between one pair
+    of CUDA events, after a 256 MB write; the median of `rounds` rounds.
+    Unlike the single-launch events it excludes the launch latency of an
+    idle stream, as in a model's forward, where kernels follow each other."""
+    import statistics
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(rounds):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _rep in range(2):
+            for c in calls:
+                c()
+        e1.record()
+        torch.cuda.synchronize()
+        per.append(e0.elapsed_time(e1) * 1e3 / (2 * len(calls)))
+    del flush
+    return statistics.median(per)
+
+
 def sweep_records(steps, warmup):
     """The decode-to-prefill M sweep of the W4A4 GEMM: one record per point.
 
@@ -681,9 +725,17 @@ def r1_folded_record(dev, flush, steps):
     torch.cuda.synchronize()
     mq = sum(a.elapsed_time(b) for a, b in tq) / len(tq)
     q_bytes = Mr * (2 * Kr + Kr // 2 + 4)
+    xs = [x] + [x.clone() for _ in range(3)]
+    us_b2b = back_to_back_us([lambda xx=xx: sq.rotate_quant(xx, None, 1, 1.0, a_q=a_q, a_scale=a_s)
+                              for xx in xs])
+    del xs
     rec = {"workload": "r1_folded_M%d_K%d" % (Mr, Kr),
            "rotate_quant": {"us": mq * 1e3, "GB/s": q_bytes / (mq * 1e-3) / 1e9,
-                            "frac_of_hbm": q_bytes / (mq * 1e-3) / 1e9 / hbm, "bytes": q_bytes},
+                            "frac_of_hbm": q_bytes / (mq * 1e-3) / 1e9 / hbm, "bytes": q_bytes,
+                            "back_to_back": {"us": us_b2b,
+                                             "frac_of_hbm": q_bytes / (us_b2b * 1e-6) / 1e9 / hbm,
+                                             "how": "8 launches over 4 copies of x (268 MB) "
+                                                    "between one event pair"}},
            "gemm": []}
     for wl in wls:
         wq, ws = sq.quantize_weights(wl.w.to(dev), None, 1)
@@ -803,7 +855,11 @@ def main():
                    "l2": "flushed (256 MB write) between timed steps"},
         "kernels": {
             "rotate_quant": {"us": r["ms_rq"] * 1e3, "GB/s": gbs_rq,
-                             "frac_of_hbm": gbs_rq / hbm, "bytes": RQ_BYTES},
+                             "frac_of_hbm": gbs_rq / hbm, "bytes": RQ_BYTES,
+                             "back_to_back": {"us": r["us_rq_b2b"],
+                                              "frac_of_hbm": RQ_BYTES / (r["us_rq_b2b"] * 1e-6) / 1e9 / hbm,
+                                              "how": "6 launches over 3 copies of x (302 MB) "
+                                                     "between one event pair"}},
             "w4a4_gemm": {"us": r["ms_gemm"] * 1e3, "TOPS": tops_gemm,
                           "frac_of_int8_peak": tops_gemm * 1e12 / (int8_peak * 1e12)},
             "kv_path": r["kv"],
