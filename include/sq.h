@@ -117,6 +117,8 @@ int sq_version(void);
  * K % g == 0.
  * The same call quantizes weights offline: pass W [N][K] as x (float32) to
  * get per-output-channel codes and scales with the rotation folded in.
+ * n_small = 12, n_pow2 = 1024 (K = 12288) with bf16 x takes the tensor-core
+ * kernel for any +-1 12 x 12 had_small (Paley's or another).
  * Range: the bf16 H12 x H1024 path (K = 12288) forms its first factor on the
  * tensor cores, which treat float32-subnormal inputs and sums (|v| < 2^-126)
  * as zero, so rows of that magnitude (scale below ~1e-38) are outside its

@@ -117,13 +117,15 @@ def hadamard(n_small: int, n_pow2: int) -> np.ndarray:
     return kron(small_hadamard(n_small), sylvester(n_pow2)).astype(np.float64)
 
 
-def rotate(x: np.ndarray, n_small: int, n_pow2: int) -> np.ndarray:
+def rotate(x: np.ndarray, n_small: int, n_pow2: int, h_small=None) -> np.ndarray:
     """Online rotation y = x H / sqrt(g), block-diagonal on each group of g channels.
 
     g = n_small * n_pow2; the row-vector convention y_c = sum_k x_k H[k][c] is
     used.  Computed in float64 by one dense matmul, returned in float32 (the
     precision in which the quantizer then decides).  With g = 1 this is the
-    identity (the R1-folded projections have no online rotation).
+    identity (the R1-folded projections have no online rotation).  h_small,
+    when given, is the +-1 n_small x n_small factor in place of the pinned
+    construction.
     """
     x = np.asarray(x, dtype=np.float64)
     M, K = x.shape
@@ -131,7 +133,10 @@ def rotate(x: np.ndarray, n_small: int, n_pow2: int) -> np.ndarray:
     assert K % g == 0
     if g == 1:
         return x.astype(F32)
-    H = hadamard(n_small, n_pow2)
+    if h_small is None:
+        H = hadamard(n_small, n_pow2)
+    else:
+        H = kron(np.asarray(h_small, np.int64), sylvester(n_pow2)).astype(np.float64)
     y = (x.reshape(M * (K // g), g) @ H) / math.sqrt(g)
     return y.reshape(M, K).astype(F32)
 
@@ -182,7 +187,7 @@ def unpack_int4(packed: np.ndarray, signed: bool = True) -> np.ndarray:
     return out.astype(np.int8 if signed else np.uint8)
 
 
-def rotate_quant(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
+def rotate_quant(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0, h_small=None):
     """Online rotation followed by per-token INT4 quantization and packing.
 
     "SpinQuant, Reproduced", Q5: R4 sits before down_proj and cannot be merged,
@@ -190,7 +195,7 @@ def rotate_quant(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
     quantized to 4 bits (SpinQuant abstract).
     Returns (packed uint8 [M, K/2], scale f32 [M], codes int8, v f32).
     """
-    y = rotate(x, n_small, n_pow2)
+    y = rotate(x, n_small, n_pow2, h_small)
     codes, scale, v = quant_sym_int4(y, clip)
     return pack_int4(codes), scale, codes, v
 
@@ -244,9 +249,9 @@ def swiglu_bf16(gate_up: np.ndarray, K: int) -> np.ndarray:
 
 
 def swiglu_rotate_quant(gate_up: np.ndarray, K: int, n_small: int, n_pow2: int,
-                        clip: float = 1.0):
+                        clip: float = 1.0, h_small=None):
     """SwiGLU product, then the online rotation and per-token INT4 (rotate_quant)."""
-    return rotate_quant(swiglu_bf16(gate_up, K), n_small, n_pow2, clip)
+    return rotate_quant(swiglu_bf16(gate_up, K), n_small, n_pow2, clip, h_small)
 
 
 # ---------------------------------------------------------------------------
@@ -304,9 +309,9 @@ def quant_sym_int8(y: np.ndarray, clip: float = 1.0):
     return codes, scale, v
 
 
-def rotate_quant8(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0):
+def rotate_quant8(x: np.ndarray, n_small: int, n_pow2: int, clip: float = 1.0, h_small=None):
     """Online rotation, then per-token INT8: returns (codes int8 [M, K], scale f32 [M], v f32)."""
-    return quant_sym_int8(rotate(x, n_small, n_pow2), clip)
+    return quant_sym_int8(rotate(x, n_small, n_pow2, h_small), clip)
 
 
 def w4a8_linear(a_codes, a_scale, w_packed, w_scale):

@@ -26,6 +26,10 @@ namespace rq {
 struct SmallH {
   int8_t h[32 * 32];   // row-major n_small x n_small, entries +-1
 };
+// The 12 x 12 factor of the tensor-core R4 path (row-major, entries +-1).
+struct H12 {
+  int8_t h[144];
+};
 
 template <typename T>
 __device__ __forceinline__ float to_f(T v);
@@ -210,20 +214,6 @@ __global__ void __launch_bounds__(256) rq_generic_kernel(const T* __restrict__ x
 
 // ------------------------------------------------------ H12 (x) H1024 (R4)
 
-// Paley construction I for q = 11, evaluated at compile time: row 0 all +1,
-// column 0 below the diagonal -1, and 1 + chi(j - i) in the 11 x 11 core,
-// chi the quadratic character mod 11 (Euler's criterion r^5 = 1 mod 11).
-__host__ __device__ constexpr int chi11(int r) {
-  r = ((r % 11) + 11) % 11;
-  if (r == 0) return 0;
-  int p = 1;
-  for (int e = 0; e < 5; ++e) p = (p * r) % 11;
-  return p == 1 ? 1 : -1;
-}
-__host__ __device__ constexpr int paley12(int i, int j) {
-  return i == j ? 1 : (i == 0 ? 1 : (j == 0 ? -1 : chi11((j - 1) - (i - 1))));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -250,7 +240,8 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool v) {
   return r != 0;
 }
 
-// R4 = H12 (x) H1024 with the Sylvester factor split as H8 (x) H128 (jt =
+// R4 = H12 (x) H1024, H12 the caller's +-1 12 x 12 factor (e.g. Paley's),
+// with the Sylvester factor split as H8 (x) H128 (jt =
 // j7..j9 outer, jl = j0..j6 inner).  Write row m as X[kappa][jl], kappa =
 // 8 i + jt (96 rows of 128 contiguous channels), and mu = 8 o + jt' for the
 // output block.  Then
@@ -441,8 +432,8 @@ __device__ __forceinline__ void swiglu_chunks(uint8_t* slot, int c0, int c1, int
 template <bool CLAMP, bool SWIGLU, bool A8>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     rq_h12x1024_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                          const __grid_constant__ CUtensorMap map_u, int M, float norm,
-                          float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
+                          const __grid_constant__ CUtensorMap map_u, const H12 h12, int M,
+                          float norm, float clip, uint32_t spin_limit, uint8_t* __restrict__ aq,
                           float* __restrict__ ascale) {
   using C = TcCfg<SWIGLU>;
   constexpr int TC_STAGES = C::STAGES;
@@ -477,7 +468,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (mu < 96 && c < 12) {
       const int o = mu >> 3, jtp = mu & 7;
-      const uint32_t neg = paley12(c, o) < 0 ? 0x80008000u : 0u;
+      const uint32_t neg = h12.h[c * 12 + o] < 0 ? 0x80008000u : 0u;
       uint32_t wd[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -881,13 +872,6 @@ static sq_status launch_quant(const T* x, int64_t ldx, int M, int K, float clip,
   }
 }
 
-static bool is_paley12(const int8_t* h) {
-  for (int i = 0; i < 12; ++i)
-    for (int j = 0; j < 12; ++j)
-      if (h[i * 12 + j] != paley12(i, j)) return false;
-  return true;
-}
-
 bool quant_fast_shape(int64_t K) {
   switch (K) {
     case 1024: case 2048: case 4096: case 8192: case 12288: case 16384: case 24576: case 32768:
@@ -918,8 +902,11 @@ static sq_status r4_map(CUtensorMap* map, const void* base, int64_t M, int64_t l
 }
 
 template <bool SWIGLU, bool A8 = false>
-static sq_status launch_r4(const void* x, const void* u, int64_t M, int64_t ld, float norm,
-                           float clip, uint8_t* a_q, float* a_scale, cudaStream_t stream) {
+static sq_status launch_r4(const void* x, const void* u, const int8_t* had_small, int64_t M,
+                           int64_t ld, float norm, float clip, uint8_t* a_q, float* a_scale,
+                           cudaStream_t stream) {
+  H12 h12;
+  for (int i = 0; i < 144; ++i) h12.h[i] = had_small[i];
   CUtensorMap map_x, map_u;
   sq_status st = r4_map(&map_x, x, M, ld);
   if (st != SQ_OK) return st;
@@ -936,14 +923,16 @@ static sq_status launch_r4(const void* x, const void* u, int64_t M, int64_t ld, 
   constexpr int smem = TcCfg<SWIGLU>::SMEM;
   cudaError_t ea = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (ea != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(rq_h12x1024)", ea);
-  kfn<<<grid, TC_THREADS, smem, stream>>>(map_x, map_u, m, norm, clip, host::spin_limit(), a_q,
-                                          a_scale);
+  kfn<<<grid, TC_THREADS, smem, stream>>>(map_x, map_u, h12, m, norm, clip, host::spin_limit(),
+                                          a_q, a_scale);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("rq_h12x1024 launch", e);
 }
 
-static bool is_r4(int n_small, int n_pow2, int64_t K, const int8_t* had_small) {
-  return n_small == 12 && n_pow2 == 1024 && K == 12288 && is_paley12(had_small);
+// H_small (x) H1024 with any +-1 12 x 12 H_small (the API has checked the
+// entries) over 12,288 channels: the tensor-core kernel
+static bool is_r4(int n_small, int n_pow2, int64_t K) {
+  return n_small == 12 && n_pow2 == 1024 && K == 12288;
 }
 
 sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
@@ -954,8 +943,8 @@ sq_status run(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const int G = n_small * n_pow2;
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   const int m = static_cast<int>(M), k = static_cast<int>(K);
-  if (x_bf16 && is_r4(n_small, n_pow2, K, had_small))
-    return launch_r4<false>(x, nullptr, M, ld_x, norm, clip, a_q, a_scale, stream);
+  if (x_bf16 && is_r4(n_small, n_pow2, K))
+    return launch_r4<false>(x, nullptr, had_small, M, ld_x, norm, clip, a_q, a_scale, stream);
   if (G == 1 && quant_fast_shape(K)) {
     return x_bf16 ? launch_quant(static_cast<const __nv_bfloat16*>(x), ld_x, m, k, clip, a_q,
                                  a_scale, stream)
@@ -977,8 +966,9 @@ sq_status run8(const void* x, int x_bf16, int64_t M, int64_t K, int64_t ld_x,
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   const int m = static_cast<int>(M), k = static_cast<int>(K);
   uint8_t* q8 = reinterpret_cast<uint8_t*>(a_q);
-  if (x_bf16 && is_r4(n_small, n_pow2, K, had_small))
-    return launch_r4<false, true>(x, nullptr, M, ld_x, norm, clip, q8, a_scale, stream);
+  if (x_bf16 && is_r4(n_small, n_pow2, K))
+    return launch_r4<false, true>(x, nullptr, had_small, M, ld_x, norm, clip, q8, a_scale,
+                                  stream);
   return x_bf16 ? launch_generic<__nv_bfloat16, false, 8>(static_cast<const __nv_bfloat16*>(x),
                                                           ld_x, m, k, hs, n_small, n_pow2, norm,
                                                           clip, q8, a_scale, stream)
@@ -995,8 +985,8 @@ sq_status run_swiglu(const void* gate_up, int64_t M, int64_t K, int64_t ld,
   const int G = n_small * n_pow2;
   const float norm = static_cast<float>(1.0 / sqrt(static_cast<double>(G)));
   auto gu = static_cast<const __nv_bfloat16*>(gate_up);
-  if (is_r4(n_small, n_pow2, K, had_small))
-    return launch_r4<true>(gu, gu + K, M, ld, norm, clip, a_q, a_scale, stream);
+  if (is_r4(n_small, n_pow2, K))
+    return launch_r4<true>(gu, gu + K, had_small, M, ld, norm, clip, a_q, a_scale, stream);
   return launch_generic<__nv_bfloat16, true>(gu, ld, static_cast<int>(M), static_cast<int>(K),
                                              hs, n_small, n_pow2, norm, clip, a_q, a_scale,
                                              stream);

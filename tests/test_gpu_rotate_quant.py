@@ -50,6 +50,47 @@ def test_down_proj_full_size_all_rows(cuda_ok):
         _check(aq[r0:r0 + 512], asc[r0:r0 + 512], x64, 12, 1024)
 
 
+def _other_h12():
+    # a +-1 12 x 12 factor that is not Paley's: rows permuted and signed,
+    # columns signed (still a Hadamard matrix)
+    rng = np.random.default_rng(12)
+    p = O.paley1(11)
+    h = p[rng.permutation(12)]
+    h = h * np.where(rng.random(12) < 0.5, -1, 1)[:, None] * np.where(rng.random(12) < 0.5, -1, 1)
+    assert not np.array_equal(h, p)
+    return h.astype(np.int8)
+
+
+@pytest.mark.parametrize("which", ["int4", "int8", "swiglu"])
+def test_r4_with_another_h12(cuda_ok, which):
+    # the tensor-core R4 path takes the caller's H12, not only Paley's
+    import rotation_ptq_b200 as sq
+    h = _other_h12()
+    if which == "swiglu":
+        gu = W.gate_up_out(M=64)
+        aq, asc = sq.swiglu_rotate_quant(gu.cuda(), h, 1024, 1.0)
+        assert sq.device_status() == 0
+        _, ref_s, ref_c, ref_v = O.swiglu_rotate_quant(gu.double().numpy(), 12288, 12, 1024, 1.0,
+                                                       h_small=h)
+        P.check_scales(asc.cpu().numpy(), ref_s)
+        P.check_codes(O.unpack_int4(aq.cpu().numpy()), ref_c, ref_v)
+        return
+    wl = W.down_proj(M=257, with_weights=False, seed=121)
+    x64 = wl.x.double().numpy()
+    if which == "int4":
+        aq, asc = sq.rotate_quant(wl.x.cuda(), h, 1024, 1.0)
+        assert sq.device_status() == 0
+        _, ref_s, ref_c, ref_v = O.rotate_quant(x64, 12, 1024, 1.0, h_small=h)
+        P.check_scales(asc.cpu().numpy(), ref_s)
+        P.check_codes(O.unpack_int4(aq.cpu().numpy()), ref_c, ref_v)
+    else:
+        aq, asc = sq.rotate_quant8(wl.x.cuda(), h, 1024, 1.0)
+        assert sq.device_status() == 0
+        ref_c, ref_s, ref_v = O.rotate_quant8(x64, 12, 1024, 1.0, h_small=h)
+        P.check_scales(asc.cpu().numpy(), ref_s)
+        P.check_codes(aq.cpu().numpy().astype(np.int64), ref_c, ref_v)
+
+
 @pytest.mark.parametrize("M", [1, 3, 33, 149, 300])
 def test_down_proj_ragged_m(cuda_ok, M):
     # 149 and 300 rows: some CTAs of the persistent grid take one row more

@@ -24,13 +24,14 @@ def _kron_swapped(A, B):
     return np.kron(B, A)
 
 
-def _rotate_unnormalised(x, n_small, n_pow2):
+def _rotate_unnormalised(x, n_small, n_pow2, h_small=None):
     x = np.asarray(x, np.float64)
     M, K = x.shape
     g = n_small * n_pow2
     if g == 1:
         return x.astype(F32)
-    H = O.hadamard(n_small, n_pow2)
+    H = O.hadamard(n_small, n_pow2) if h_small is None else \
+        O.kron(np.asarray(h_small, np.int64), O.sylvester(n_pow2)).astype(np.float64)
     return (x.reshape(-1, g) @ H).reshape(M, K).astype(F32)
 
 

@@ -135,6 +135,18 @@ def test_rotation_of_one_hot_is_scaled_row(ns, np2):
         assert np.allclose(y[0], H[k] / math.sqrt(g), rtol=0, atol=1e-7)
 
 
+def test_rotation_with_explicit_small_factor():
+    # an explicit h_small equal to the pinned construction gives the same
+    # rotation; another +-1 factor gives x (h (x) H_pow2) / sqrt(g) written out
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((3, 48))
+    p = O.paley1(11)
+    assert np.array_equal(O.rotate(x, 12, 4, h_small=p), O.rotate(x, 12, 4))
+    h = -p[::-1]
+    want = (x.reshape(3, 1, 48) @ np.kron(h, O.sylvester(4)) / np.sqrt(48)).reshape(3, 48)
+    assert np.allclose(O.rotate(x, 12, 4, h_small=h), want.astype(np.float32), rtol=1e-6, atol=1e-6)
+
+
 def test_rotation_is_row_vector_convention():
     # y = x H (not H x): with the non-symmetric Paley factor these differ.
     x = np.zeros((1, 12 * 2))
