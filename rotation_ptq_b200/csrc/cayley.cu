@@ -31,7 +31,7 @@
 //   G = x_s^T g_xr,s + w_s^T g_wr,s fp32 split-K GEMMs, partials summed in f64
 // The Cayley step runs in float64: A = I - a/2 (R G^T - G R^T) and
 // B = (I + a/2 Y) R = 2R - A R, then Gauss-Jordan elimination of A with B as
-// right-hand side in one CTA.  A's symmetric part is I, and so is at least
+// right-hand side over a cluster of 8 CTAs.  A's symmetric part is I, and so is at least
 // that of every Schur complement, so each pivot is >= 1: no pivoting needed.
 //
 // The fp32 GEMM is a CUDA-core kernel (128 x 128 tiles, 8 x 8 outputs per
@@ -703,84 +703,120 @@ __global__ void __launch_bounds__(256) cayley_b_kernel(const double* __restrict_
   }
 }
 
-constexpr int SOLVE_THREADS = 512;
 constexpr int ORTH_THREADS = 1024;
 constexpr int MAX_N = 128;
-constexpr int SOLVE_RG = SOLVE_THREADS / MAX_N;        // row groups
-constexpr int SOLVE_RPT = MAX_N / SOLVE_RG;            // rows per thread (in registers)
 
-// R_out = A^-1 B by Gauss-Jordan elimination, one CTA per matrix (n <= 128):
-// A in shared memory (row stride n + 1), B in registers, thread t holding
-// column t % 128 of rows t / 128 + 4 r (32 rows, 64 registers).  Pivots are
-// >= 1 (see the top).
-__global__ void __launch_bounds__(SOLVE_THREADS, 1) cayley_solve_kernel(
+// R_out = A^-1 B by Gauss-Jordan elimination over a cluster of CS_CLUSTER
+// CTAs per matrix (n <= 128).  CTA r of the cluster owns columns 32 r .. 32 r
+// + 31 of the augmented matrix [A | B] (A's n columns first, then B's); warp
+// w owns its columns 4 w .. 4 w + 3 and lane l rows 4 l .. 4 l + 3 of them,
+// in registers (x[j][q]: column 4 w + j, row 4 l + q).  Step k: the CTA
+// owning column k has staged that column, as it stands after step k - 1, in
+// its shared colbuf[k & 1]; after a cluster barrier 64 threads copy it from
+// there (distributed shared memory, one 16-byte load each) into this CTA's
+// colk, and after a CTA barrier every thread reads its four rows and the
+// pivot locally; the pivot row's values come from lane k / 4 by shuffles
+// (lanes 0..3 divide them by the pivot), and every thread updates its rows:
+// x[i] -= col_k[i] * prow, x[k] = prow.  The staging buffers alternate, so a
+// buffer is rewritten only after every CTA has passed the cluster barrier
+// that follows its last read.  Pivots are >= 1 (see the top): no pivoting.
+constexpr int CS_CLUSTER = 8;
+constexpr int CS_THREADS = 256;
+
+__device__ __forceinline__ void ld_cluster_f64x2(uint32_t addr, double& a, double& b) {
+  asm volatile("ld.shared::cluster.v2.f64 {%0, %1}, [%2];" : "=d"(a), "=d"(b) : "r"(addr) : "memory");
+}
+// v[sel] for sel in 0..3 by two selects (an indexed read would put v in local memory)
+__device__ __forceinline__ double pick4(const double (&v)[4], int sel) {
+  const double lo = (sel & 1) ? v[1] : v[0], hi = (sel & 1) ? v[3] : v[2];
+  return (sel & 2) ? hi : lo;
+}
+
+__global__ void __launch_bounds__(CS_THREADS, 1) cayley_solve_kernel(
     const double* __restrict__ Ain, const double* __restrict__ Bin, int n,
     double* __restrict__ R_out, float* __restrict__ R32) {
-  extern __shared__ double cs_smem[];
-  const int64_t off = static_cast<int64_t>(blockIdx.x) * n * n;
-  const int ld = n + 1;
-  double* As = cs_smem;
-  double* colbuf = As + n * ld;            // [2][n]: pivot columns, double-buffered
-  double* pivB = colbuf + 2 * n;
-  const int t = threadIdx.x, j = t & (MAX_N - 1), rg = t / MAX_N;
-  const bool live = j < n;
-  double bv[SOLVE_RPT];
+  __shared__ __align__(16) double colbuf[2][MAX_N];   // the pivot column this CTA stages
+  __shared__ __align__(16) double colk[MAX_N];        // this step's pivot column
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int64_t off = static_cast<int64_t>(blockIdx.x / CS_CLUSTER) * n * n;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int col0 = 32 * rank + 4 * w;                 // this warp's first column of [A | B]
+  double x[4][4];
 #pragma unroll
-  for (int r = 0; r < SOLVE_RPT; ++r) {
-    const int i = rg + SOLVE_RG * r;
-    bv[r] = 0.0;
-    if (live && i < n) {
-      bv[r] = Bin[off + i * n + j];
-      As[i * ld + j] = Ain[off + i * n + j];
+  for (int j = 0; j < 4; ++j) {
+    const int col = col0 + j;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = 4 * lane + q;
+      x[j][q] = 0.0;
+      if (col < 2 * n && i < n)
+        x[j][q] = col < n ? Ain[off + i * n + col] : Bin[off + i * n + (col - n)];
     }
   }
-  if (j == 0) {
+  // stage one of this warp's columns (j) into colbuf[buf]: 32 bytes a lane
+  auto stage = [&](int j, int buf) {
+    double v[4];
 #pragma unroll
-    for (int r = 0; r < SOLVE_RPT; ++r) {
-      const int i = rg + SOLVE_RG * r;
-      if (i < n) colbuf[i] = As[i * ld];
+    for (int q = 0; q < 4; ++q) {
+      const double c4[4] = {x[0][q], x[1][q], x[2][q], x[3][q]};
+      v[q] = pick4(c4, j);
     }
-  }
-  __syncthreads();
+    double2* dst = reinterpret_cast<double2*>(&colbuf[buf][4 * lane]);
+    dst[0] = make_double2(v[0], v[1]);
+    dst[1] = make_double2(v[2], v[3]);
+  };
+  if (rank == 0 && w == 0) stage(0, 0);               // column 0 for step 0
   for (int k = 0; k < n; ++k) {
-    // colk = column k of A before step k, staged at the end of step k - 1
-    const double* colk = colbuf + (k & 1) * n;
-    double* coln = colbuf + ((k + 1) & 1) * n;
+    cluster_sync();
+    if (threadIdx.x < MAX_N / 2) {
+      double a, b;
+      ld_cluster_f64x2(mapa_shared(smem_u32(&colbuf[k & 1][2 * threadIdx.x]), k >> 5), a, b);
+      reinterpret_cast<double2*>(colk)[threadIdx.x] = make_double2(a, b);
+    }
+    __syncthreads();
+    double ck[4];
+    {
+      const double2 c01 = reinterpret_cast<const double2*>(colk)[2 * lane];
+      const double2 c23 = reinterpret_cast<const double2*>(colk)[2 * lane + 1];
+      ck[0] = c01.x;
+      ck[1] = c01.y;
+      ck[2] = c23.x;
+      ck[3] = c23.y;
+    }
     const double piv = colk[k];
-    if (live && rg == k % SOLVE_RG) {
+    // pivot row: lane k / 4 holds row k of the warp's four columns; lane j
+    // takes column j's value and divides it by the pivot
+    double pr[4];
 #pragma unroll
-      for (int r = 0; r < SOLVE_RPT; ++r) {
-        if (r == k / SOLVE_RG) {
-          As[k * ld + j] = As[k * ld + j] / piv;
-          bv[r] = bv[r] / piv;
-          pivB[j] = bv[r];
-        }
+    for (int j = 0; j < 4; ++j) pr[j] = __shfl_sync(0xffffffffu, pick4(x[j], k & 3), k >> 2);
+    double mine = pick4(pr, lane & 3) / piv;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pr[j] = __shfl_sync(0xffffffffu, mine, j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = 4 * lane + q;
+        x[j][q] = i == k ? pr[j] : fma(-ck[q], pr[j], x[j][q]);
       }
     }
-    __syncthreads();
-    if (live) {
-      const double akj = As[k * ld + j], bkj = pivB[j];
-#pragma unroll
-      for (int r = 0; r < SOLVE_RPT; ++r) {
-        const int i = rg + SOLVE_RG * r;
-        if (i < n && i != k) {
-          const double f = colk[i];
-          As[i * ld + j] -= f * akj;
-          bv[r] -= f * bkj;
-        }
-        // the owner of column k + 1 stages it for the next step (row k was
-        // normalised by this same thread above)
-        if (j == k + 1 && i < n) coln[i] = As[i * ld + j];
-      }
-    }
-    __syncthreads();
+    // stage column k + 1 for the next step, as it stands now
+    const int kn = k + 1;
+    if (kn < n && rank == (kn >> 5) && w == ((kn & 31) >> 2)) stage(kn & 3, kn & 1);
   }
+  // no CTA leaves while another may still read its staging buffer
+  cluster_sync();
 #pragma unroll
-  for (int r = 0; r < SOLVE_RPT; ++r) {
-    const int i = rg + SOLVE_RG * r;
-    if (live && i < n) {
-      R_out[off + i * n + j] = bv[r];
-      if (R32) R32[off + i * n + j] = static_cast<float>(bv[r]);
+  for (int j = 0; j < 4; ++j) {
+    const int col = col0 + j;
+    if (col < n || col >= 2 * n) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = 4 * lane + q;
+      if (i < n) {
+        R_out[off + i * n + (col - n)] = x[j][q];
+        if (R32) R32[off + i * n + (col - n)] = static_cast<float>(x[j][q]);
+      }
     }
   }
 }
@@ -1045,12 +1081,22 @@ sq_status cayley_update(const double* R, const double* G, double alpha, int n, i
   const int nt = (n + CT - 1) / CT;
   cayley_a_kernel<<<dim3(nt * (nt + 1) / 2, batch), 256, 0, s>>>(R, G, 0.5 * alpha, n, A);
   cayley_b_kernel<<<dim3(nt * nt, batch), 256, 0, s>>>(A, R, n, B);
-  const int smem = (n * (n + 1) + 3 * n) * static_cast<int>(sizeof(double));
-  cudaError_t e = cudaFuncSetAttribute(cayley_solve_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return host::cuda_fail("cudaFuncSetAttribute(cayley_solve)", e);
-  cayley_solve_kernel<<<batch, SOLVE_THREADS, smem, s>>>(A, B, n, R_out, R32);
-  e = cudaGetLastError();
+  // one cluster of CS_CLUSTER CTAs per matrix
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS_CLUSTER;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(CS_CLUSTER * batch), 1, 1);
+  cfg.blockDim = dim3(CS_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, cayley_solve_kernel, static_cast<const double*>(A),
+                                     static_cast<const double*>(B), n, R_out, R32);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("cayley launch", e);
 }
 
