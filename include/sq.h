@@ -207,10 +207,12 @@ sq_status sq_swiglu_rotate_quant(const void* gate_up, int64_t M, int64_t K, int6
  *           less, that wave runs whole.  Results are identical either way.
  * Shape rules: M >= 0 (0 is a no-op), N % 16 == 0, N >= 16, K % 128 == 0,
  * 128 <= K <= 65536 (so |acc| < 2^31).
- * Ordering: for 5 <= M <= 32 the kernel is launched as a programmatic
- * dependent (CUDA's programmatic stream serialization): it may set up while
- * the preceding kernel of the stream finishes, and waits for that kernel's
- * completion before it reads or writes any operand.
+ * Ordering: for 5 <= M <= 32, and for M <= 4 when M rounded up to a power
+ * of two times K is at most 98,304, the kernel is launched as a programmatic
+ * dependent (CUDA's programmatic stream serialization): it may set up,
+ * and for M <= 4 ask the L2 to prefetch w_q (a hint that reads no values),
+ * while the preceding kernel of the stream finishes, and waits for that
+ * kernel's completion before it reads or writes any operand.
  * ------------------------------------------------------------------------- */
 sq_status sq_w4a4_linear(const uint8_t* a_q, const float* a_scale, const uint8_t* w_q,
                          const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
@@ -272,6 +274,9 @@ sq_status sq_w4a4_linear_noalloc(const uint8_t* a_q, const float* a_scale, const
  *           large-M tiles split by K; size it with
  *           sq_w4a4_tail_workspace_bytes).
  * Shape rules and errors as sq_w4a4_linear.
+ * Ordering: for M <= 8, when M rounded up to a power of two times K is at
+ * most 98,304, the kernel is launched as a programmatic dependent, as
+ * sq_w4a4_linear describes.
  * ------------------------------------------------------------------------- */
 sq_status sq_w4a8_linear(const int8_t* a_q, const float* a_scale, const uint8_t* w_q,
                          const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,

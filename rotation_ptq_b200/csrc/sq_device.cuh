@@ -293,6 +293,22 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, 
       : "memory");
 }
 
+// L2 prefetch hint.  It only asks the L2 to fetch lines; every store on the
+// GPU lands in the L2, so a prefetched line is never stale and a later load
+// after proper ordering sees the current data.  Address 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid (its memory
+// visible), and let the following grid be scheduled.  Both are no-ops in a
+// kernel not launched as a programmatic dependent.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 
 // ------------------------------------------------------------- clusters
 

@@ -135,13 +135,6 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// Programmatic dependent launch: wait for the preceding grid (its memory
-// visible), and let the following grid be scheduled.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // atomicAdd with acquire-release semantics at GPU scope (returns the old value).
 __device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
   unsigned old;

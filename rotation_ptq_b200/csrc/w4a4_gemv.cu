@@ -17,6 +17,14 @@
 // 2^31 for K <= 65,536.  The batch's activation codes are widened once per CTA
 // into shared memory as separate even-code and odd-code word arrays, so that
 // a warp's reads are contiguous.
+//
+// The kernel is launched as a programmatic dependent (programmatic stream
+// serialization).  The weights are never the preceding grid's output, so
+// before it waits for that grid each warp asks the L2 for every weight row it
+// will stream (a bulk prefetch hint, no read of the values), and it lets the
+// following grid be scheduled; the weight stream of back-to-back calls then
+// overlaps the end of the preceding call.  Every load and store comes after
+// the wait.
 #include <cuda_bf16.h>
 
 #include "sq_device.cuh"
@@ -54,6 +62,13 @@ __global__ void __launch_bounds__(NW * 32) w4a4_gemv_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_step = gridDim.x * NW * R;     // rows handled by all warps per pass
   int n0 = (blockIdx.x * NW + warp) * R;
+
+  if (lane < R) {
+    for (int n = n0 + lane; n < N; n += row_step)
+      prefetch_l2_bulk(w_q + static_cast<int64_t>(n) * (K / 2), static_cast<uint32_t>(K / 2));
+  }
+  griddep_launch_dependents();
+  griddep_wait();
 
   // the first rows' weight loads go out before the activations are staged
   uint4 wv[R][CPL];
@@ -198,8 +213,17 @@ static sq_status launch(const uint8_t* a_q, const float* a_scale, const uint8_t*
   const int64_t groups = (static_cast<int64_t>(N) + NW * R - 1) / (NW * R);
   const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
   const int grid = static_cast<int>(groups < cap ? groups : cap);
-  kfn<<<grid, NW * 32, smem, stream>>>(a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NW * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kfn, a_q, a_scale, w_q, w_scale, M, N, K, out, out_i32);
   return e == cudaSuccess ? SQ_OK : host::cuda_fail("w4a4_gemv launch", e);
 }
 
@@ -208,22 +232,26 @@ static sq_status run_t(const uint8_t* a_q, const float* a_scale, const uint8_t* 
                        const float* w_scale, int64_t M, int64_t N, int64_t K, void* out,
                        int out_i32, int num_sms, cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  // rows of at most 4 chunks per lane (K <= 4096) go several to a warp
+  // rows of at most 4 chunks per lane (K <= 4096) go several to a warp.  For
+  // longer rows, two rows per warp from M = 2 on: each lane's activation
+  // words, read from shared memory once per chunk, then serve two weight
+  // rows (at M = 4 with one row per warp those reads, 8 x the weight bytes,
+  // outlast the weight stream)
   const bool short_rows = K <= 4096;
 #define SQ_GEMV(MT, NW, CPL, R) \
   return launch<MT, NW, CPL, R, A8>(a_q, a_scale, w_q, w_scale, m, n, k, out, out_i32, num_sms, \
                                     stream)
   if (M <= 1) {
     if (short_rows) SQ_GEMV(1, 8, 4, 3);
-    SQ_GEMV(1, 16, 12, 1);
+    SQ_GEMV(1, 16, 6, 2);
   }
   if (M <= 2) {
     if (short_rows) SQ_GEMV(2, 8, 4, 3);
-    SQ_GEMV(2, 16, 12, 1);
+    SQ_GEMV(2, 8, 6, 2);
   }
   if (M <= 4) {
     if (short_rows) SQ_GEMV(4, 8, 4, 2);
-    SQ_GEMV(4, 8, 8, 1);
+    SQ_GEMV(4, 8, 4, 2);
   }
   if (short_rows) SQ_GEMV(8, 8, 4, 1);
   SQ_GEMV(8, 8, 8, 1);

@@ -287,3 +287,48 @@ def test_decode_gemv_matches_tensor_path(cuda_ok, M, N, K):
     assert torch.equal(gi, ti) and torch.equal(gb, tb)
     ref = O.gemm_int(O.unpack_int4(a), O.unpack_int4(w))
     assert np.array_equal(gi.cpu().numpy().astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_programmatic_launch_sees_operands_written_just_before(cuda_ok, M):
+    # The M <= 32 kernels start while the preceding kernel of the stream
+    # finishes and prefetch their weights into the L2 before waiting for it.
+    # Each call here follows a kernel that has just rewritten both operands
+    # (in place, the same buffers every time), eagerly and replayed in a
+    # graph; every result must be the product of the values written last.
+    import rotation_ptq_b200 as sq
+    N, K = 1024, 4096
+    sets = [_operands(M, N, K, 1500 + 10 * i + M) for i in range(3)]
+    dev = [(_dev(a), _dev(sa), _dev(w), _dev(sw)) for a, w, sa, sw in sets]
+    refs = [O.gemm_int(O.unpack_int4(a), O.unpack_int4(w)) for a, w, _, _ in sets]
+    da, dsa, dw, dsw = (torch.empty_like(t) for t in dev[0])
+    outs = [torch.empty((M, N), dtype=torch.int32, device="cuda") for _ in sets]
+    ws = torch.zeros(max(16, sq.w4a4_workspace_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+
+    def chain():
+        for (a, sa, w, sw), o in zip(dev, outs):
+            da.copy_(a)
+            dw.copy_(w)
+            sq.w4a4_linear(da, dsa, dw, dsw, out=o, out_int32=True, workspace=ws)
+
+    dsa.copy_(dev[0][1])
+    dsw.copy_(dev[0][3])
+    chain()
+    torch.cuda.synchronize()
+    for o, r in zip(outs, refs):
+        assert np.array_equal(o.cpu().numpy().astype(np.int64), r)
+    for o in outs:
+        o.zero_()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            chain()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    del g
+    assert sq.device_status() == 0
+    for o, r in zip(outs, refs):
+        assert np.array_equal(o.cpu().numpy().astype(np.int64), r)
