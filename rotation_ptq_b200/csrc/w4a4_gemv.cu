@@ -243,14 +243,14 @@ static sq_status run_t(const uint8_t* a_q, const float* a_scale, const uint8_t* 
                                     stream)
   if (M <= 1) {
     if (short_rows) SQ_GEMV(1, 8, 4, 3);
-    SQ_GEMV(1, 16, 6, 2);
+    SQ_GEMV(1, 4, 6, 2);
   }
   if (M <= 2) {
     if (short_rows) SQ_GEMV(2, 8, 4, 3);
     SQ_GEMV(2, 8, 6, 2);
   }
   if (M <= 4) {
-    if (short_rows) SQ_GEMV(4, 8, 4, 2);
+    if (short_rows) SQ_GEMV(4, 4, 4, 2);
     SQ_GEMV(4, 8, 4, 2);
   }
   if (short_rows) SQ_GEMV(8, 8, 4, 1);
